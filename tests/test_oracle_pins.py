@@ -1,0 +1,309 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each test checks the oracle against something it cannot agree with by
+construction: the worked examples printed on the pages (tests/golden), closed
+forms, invariants of the method, an independent library (numpy's binary16),
+and an independent brute force (oracle/bruteforce.py).  A plausible slip in the
+oracle -- a dropped term, a wrong sign or index, a transposed operand, a
+division where a multiplication belongs, the wrong rounding -- fails at least
+one of them.
+"""
+import json
+import math
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from awq_activation_aware_b200 import synth
+from oracle import bruteforce
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# binary16 rounding vs numpy (independent implementation)
+# ---------------------------------------------------------------------------
+
+def test_rn16_matches_numpy(oracle_mod):
+    rng = np.random.default_rng(1234)
+    vals = np.concatenate([
+        rng.standard_normal(3000) * 10.0 ** rng.integers(-9, 5, 3000),
+        np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, -65520.0, 1e9, 2.0 ** -24, 2.0 ** -25,
+                  3 * 2.0 ** -25, 2.0 ** -26, 2.0 ** -14, 2.0 ** -14 - 2.0 ** -25,
+                  1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2049.0, 2051.0]),
+    ])
+    for v in vals:
+        with np.errstate(over="ignore"):
+            ref = np.array([v]).astype(np.float16).view(np.uint16)[0]
+        got = oracle_mod.rn16_bits(v)
+        assert got == ref, (v, hex(got), hex(ref))
+    for b in [0, 1, 0x3FF, 0x400, 0x3C00, 0x7BFF, 0x8001, 0xFBFF, 0x7C00]:
+        assert oracle_mod.h2d(b) == float(np.array([b], dtype=np.uint16).view(np.float16)[0])
+
+
+# ---------------------------------------------------------------------------
+# Worked example of "AWQ: Activation-Aware Weight Quantization For On-Device
+# LLM Compression AND Acceleration", section "Measures"
+# ---------------------------------------------------------------------------
+
+def test_awq_note_example_primitives(oracle_mod):
+    g = _gold("awq_note_int3_example.json")
+    w = g["W"]
+    # symmetric absmax step for INT3: max|w| / (2^(b-1) - 1)
+    assert oracle_mod.absmax_step(w, g["bits"]) == pytest.approx(g["step"], rel=1e-15)
+    assert oracle_mod.absmax_step(g["overscaled_W"], g["bits"]) == pytest.approx(
+        g["overscaled_step"], rel=1e-15)
+    # the non-negative levels of the step-1/3 grid
+    levels = sorted({oracle_mod.round_to_step(v, g["step"]) for v in np.linspace(0, 1, 101)})
+    assert levels == pytest.approx(g["levels_nonnegative"], abs=1e-15)
+    x2 = g["activation_second"]
+    assert w[1] * x2 == pytest.approx(g["true_contribution"])
+    rtn = oracle_mod.round_to_step(w[1], g["step"]) * x2
+    scaled = oracle_mod.round_to_step(w[1] * g["s"], g["step"]) / g["s"] * x2
+    tol = 0.5 * 10.0 ** -g["printed_decimals"]
+    assert rtn == pytest.approx(g["rtn_output"], abs=tol)
+    assert scaled == pytest.approx(g["scaled_output"], abs=tol)
+
+
+def test_awq_note_example_through_group_quantizer(oracle_mod):
+    """The same example through the oracle's asymmetric group quantizer.
+
+    A group [1.0, 0.2, 0, 0] at w_bit = 2 has min 0 and max 1, so scale = 1/3
+    (stored in fp16) and the levels are the page's 0, 1/3, 2/3, 1.  Scaling the
+    second input channel by 2 keeps the group maximum and halves the effective
+    error; scaling it to 2.0 makes the step 2/3."""
+    g = _gold("awq_note_int3_example.json")
+    W = np.array([[1.0, 0.2, 0.0, 0.0]], dtype=np.float16)
+    ones = np.ones(4, dtype=np.float32)
+    # the page prints 3 decimals; the quantizer stores the step 1/3 in fp16 and
+    # rounds Ŵ to fp16: two roundings of at most 2^-11 relative each
+    def tol(v):
+        return 0.5 * 10.0 ** -g["printed_decimals"] + abs(v) * 2 * 2.0 ** -11
+    r0 = oracle_mod.quantize(W, ones, bits=2, group=4)
+    assert float(r0["sh"][0, 0]) == pytest.approx(g["step"], rel=2 ** -11)
+    assert float(r0["z"][0, 0]) == 0.0
+    assert float(r0["what"][0, 1]) * g["activation_second"] == pytest.approx(g["rtn_output"], abs=tol(g["rtn_output"]))
+    s = np.array([1.0, g["s"], 1.0, 1.0], dtype=np.float32)
+    r1 = oracle_mod.quantize(W, s, bits=2, group=4)
+    assert float(r1["sh"][0, 0]) == float(r0["sh"][0, 0])           # group max unchanged
+    assert float(r1["what"][0, 1]) * g["activation_second"] == pytest.approx(g["scaled_output"], abs=tol(g["scaled_output"]))
+    s2 = np.array([1.0, g["overscaled_W"][1] / float(W[0, 1]), 1.0, 1.0], dtype=np.float32)
+    r2 = oracle_mod.quantize(W, s2, bits=2, group=4)
+    assert float(r2["sh"][0, 0]) == pytest.approx(g["overscaled_step"], rel=2 ** -10)
+
+
+def test_notes52_example_through_group_quantizer(oracle_mod):
+    """"52 · AWQ, GPTQ và SmoothQuant" §3: step 0.125; 0.19 -> 0.25, and
+    0.38 -> 0.375 -> 0.1875 after halving.  Group [1.875, 0.19, 0, 0] at
+    w_bit = 4 has scale exactly 1.875 / 15 = 0.125."""
+    g = _gold("notes52_step0125_example.json")
+    W = np.array([[1.875, g["w"], 0.0, 0.0]], dtype=np.float16)
+    r0 = oracle_mod.quantize(W, np.ones(4, dtype=np.float32), bits=4, group=4)
+    assert float(r0["sh"][0, 0]) == g["step"]
+    assert float(r0["what"][0, 1]) == g["rtn"]
+    assert abs(g["rtn"] - g["w"]) / g["w"] * 100 == pytest.approx(g["rtn_rel_err_pct"], abs=0.5)
+    s = np.array([1.0, g["s"], 1.0, 1.0], dtype=np.float32)
+    r1 = oracle_mod.quantize(W, s, bits=4, group=4)
+    assert int(r1["q"][0, 1]) * g["step"] == g["scaled_rtn"]
+    assert float(r1["what"][0, 1]) == g["unscaled"]
+    assert abs(g["unscaled"] - g["w"]) / g["w"] * 100 == pytest.approx(g["unscaled_rel_err_pct"], abs=0.5)
+
+
+# ---------------------------------------------------------------------------
+# Closed forms and invariants
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (2, 64)])
+def test_round_trip_exact_codes(oracle_mod, bits, group):
+    """W built from chosen codes/scales/zeros (each group holds codes 0 and
+    qmax, scales powers of two) is recovered exactly at alpha = 0, and Ŵ = W."""
+    rng = np.random.default_rng(bits * 100 + group)
+    N, K = 6, 2 * group
+    qmax = (1 << bits) - 1
+    G = K // group
+    q = rng.integers(0, qmax + 1, size=(N, K))
+    for n in range(N):
+        for gi in range(G):
+            pos = rng.choice(group, 2, replace=False) + gi * group
+            q[n, pos[0]], q[n, pos[1]] = 0, qmax
+    z = rng.integers(0, qmax + 1, size=(N, G))
+    sh = 2.0 ** rng.integers(-9, -3, size=(N, G))
+    W = np.empty((N, K))
+    for n in range(N):
+        for gi in range(G):
+            sl = slice(gi * group, (gi + 1) * group)
+            W[n, sl] = (q[n, sl] - z[n, gi]) * sh[n, gi]
+    W16 = W.astype(np.float16)
+    assert np.array_equal(W16.astype(np.float64), W)
+    r = oracle_mod.quantize(W16, np.ones(K, dtype=np.float32), bits, group)
+    assert np.array_equal(r["q"], q)
+    assert np.array_equal(r["z"], z.astype(np.float32))
+    assert np.array_equal(r["sh"].astype(np.float64), sh)
+    assert np.array_equal(r["what"], W16)
+
+
+def test_ties_round_to_even(oracle_mod):
+    # scale = 15/15 = 1; the values k + 1/2 land exactly on ties
+    W = np.array([[0.0, 15.0, 0.5, 1.5, 2.5, 3.5, 10.5, 11.5]], dtype=np.float16)
+    r = oracle_mod.quantize(W, np.ones(8, dtype=np.float32), bits=4, group=8)
+    assert float(r["sh"][0, 0]) == 1.0 and float(r["z"][0, 0]) == 0.0
+    assert r["q"][0].tolist() == [0, 15, 0, 2, 2, 4, 10, 12]
+
+
+def test_alpha_zero_is_plain_rtn(oracle_mod):
+    """alpha = 0 gives s = 1 exactly, so the search's first candidate is plain
+    group RTN; the brute force's RTN (binary32 hardware ops) must agree bit
+    for bit."""
+    W, X, _ = synth.generate(synth.make_config(4, 256, 8, bits=4, group=128, seed=7))
+    a = oracle_mod.act_stats(X)
+    s = oracle_mod.scales(a, 0.0)
+    assert np.all(s == 1.0)
+    r = oracle_mod.quantize(W, s, 4, 128)
+    Wl = [[float(v) for v in row] for row in W.astype(np.float64)]
+    Q, SH, Z, WH = bruteforce.quantize(Wl, [np.float32(1.0)] * 256, 4, 128)
+    assert r["q"].tolist() == Q
+    assert r["z"].tolist() == Z
+    assert r["sh"].astype(np.float64).tolist() == SH
+    assert r["what"].astype(np.float64).tolist() == WH
+
+
+def test_scaling_is_identity_without_rounding(oracle_mod):
+    """Y = (W D)(D^-1 x): without the rounding step, scale-quantize-unscale
+    returns W up to binary32/binary16 rounding, so the loss is ~0."""
+    cfg = synth.make_config(16, 256, 64, bits=4, group=128, seed=3)
+    W, X, _ = synth.generate(cfg)
+    a = oracle_mod.act_stats(X)
+    alphas = synth.default_alphas()
+    ident = oracle_mod.search(W, X, a, 4, 128, alphas, no_round=True)["losses"]
+    real = oracle_mod.search(W, X, a, 4, 128, alphas)["losses"]
+    assert np.all(ident <= 1e-6 * real.min())
+    for al in alphas:
+        what = oracle_mod.quantize(W, oracle_mod.scales(a, float(al)), 4, 128, no_round=True)["what"]
+        # at most one fp16 ulp away from W
+        ulp = np.spacing(np.abs(W).astype(np.float16)).astype(np.float64)
+        assert np.all(np.abs(what.astype(np.float64) - W.astype(np.float64)) <= ulp)
+
+
+def test_power_of_two_scale_invariance(oracle_mod):
+    """s -> 2^k s multiplies every binary32/binary16 intermediate by 2^k and
+    divides it back out, so codes and Ŵ are bit-identical."""
+    cfg = synth.make_config(8, 256, 16, bits=4, group=128, seed=11)
+    W, X, _ = synth.generate(cfg)
+    s = oracle_mod.scales(oracle_mod.act_stats(X), 0.5)
+    r0 = oracle_mod.quantize(W, s, 4, 128)
+    for k in (-3, 1, 4):
+        r1 = oracle_mod.quantize(W, (s * np.float32(2.0 ** k)).astype(np.float32), 4, 128)
+        assert np.array_equal(r0["q"], r1["q"])
+        assert np.array_equal(r0["z"], r1["z"])
+        assert np.array_equal(r0["what"], r1["what"])
+
+
+def test_loss_identity_activations(oracle_mod):
+    """X = I_K (T = K): the output error is the Frobenius norm of Ŵ - W."""
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((3, 64)) * 0.02).astype(np.float16)
+    What = (W.astype(np.float64) + rng.integers(-3, 4, W.shape) * 2.0 ** -12).astype(np.float16)
+    X = np.eye(64, dtype=np.float16)
+    got = oracle_mod.output_error_sum(W, What, X)
+    d = What.astype(np.float64) - W.astype(np.float64)
+    for n in range(3):
+        assert got[n] == pytest.approx(sum(v * v for v in d[n]), rel=1e-13)
+
+
+def test_loss_rank_one_activations(oracle_mod):
+    """Every token equal to x: row error = T (ΔW_n · x)^2."""
+    rng = np.random.default_rng(6)
+    W = (rng.standard_normal((4, 128)) * 0.02).astype(np.float16)
+    What = (W.astype(np.float64) * 1.01).astype(np.float16)
+    x = rng.standard_normal(128).astype(np.float16)
+    T = 9
+    X = np.tile(x, (T, 1))
+    got = oracle_mod.output_error_sum(W, What, X)
+    for n in range(4):
+        dot = sum((float(What[n, k]) - float(W[n, k])) * float(x[k]) for k in range(128))
+        assert got[n] == pytest.approx(T * dot * dot, rel=1e-12)
+
+
+def test_act_stats_exact_mean(oracle_mod):
+    rng = np.random.default_rng(9)
+    X = (rng.standard_normal((37, 24)) * 10.0 ** rng.integers(-6, 2, (37, 24))).astype(np.float16)
+    X[:, 5] = 0
+    a = oracle_mod.act_stats(X)
+    for j in range(24):
+        tot = sum(Fraction(abs(float(v))) for v in X[:, j])
+        assert a[j] == np.float32(float(tot) / 37)
+    assert a[5] == 0.0
+
+
+def test_pack_codes_bit_layout(oracle_mod):
+    rng = np.random.default_rng(2)
+    for bits in (2, 3, 4):
+        q = rng.integers(0, 1 << bits, size=(3, 64)).astype(np.uint8)
+        codes = oracle_mod.pack_codes(q, bits)
+        c = 2 if bits == 2 else 4
+        per = 32 // c
+        for n in range(3):
+            for k in range(64):
+                word = int(codes[n, k // per])
+                assert (word >> (c * (k % per))) & ((1 << c) - 1) == q[n, k]
+
+
+def test_argmin_rules(oracle_mod):
+    assert oracle_mod.argmin([3.0, 1.0, 1.0, 2.0]) == 1
+    assert oracle_mod.argmin([float("nan"), 5.0, float("nan"), 4.0]) == 3
+    assert oracle_mod.argmin([float("nan"), float("nan")]) == 0
+    assert oracle_mod.argmin([float("inf"), 7.0]) == 1
+
+
+# ---------------------------------------------------------------------------
+# Brute force on tiny layers
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,T,bits,group,seed", [
+    (3, 128, 8, 4, 128, 21),
+    (2, 128, 6, 3, 64, 22),
+    (4, 64, 5, 2, 64, 23),
+    (2, 256, 4, 4, 128, 24),
+])
+def test_bruteforce_search(oracle_mod, N, K, T, bits, group, seed):
+    cfg = synth.make_config(N, K, T, bits=bits, group=group, seed=seed, outlier_frac=0.03)
+    W, X, _ = synth.generate(cfg)
+    alphas = synth.default_alphas()
+    bf = bruteforce.search(W, X, bits, group, alphas)
+    a = oracle_mod.act_stats(X)
+    assert np.array_equal(a, bf["a"])
+    orc = oracle_mod.search(W, X, a, bits, group, alphas)
+    np.testing.assert_allclose(orc["losses"], bf["losses"], rtol=1e-12, atol=0)
+    assert orc["best"] == bf["best"]
+    for i in (0, bf["best"], len(alphas) - 1):
+        Q, SH, Z, WH, s = bf["per_alpha"][i]
+        r = oracle_mod.quantize(W, oracle_mod.scales(a, float(alphas[i])), bits, group)
+        assert r["q"].tolist() == Q
+        assert r["z"].tolist() == Z
+        assert r["what"].astype(np.float64).tolist() == WH
+        assert oracle_mod.scales(a, float(alphas[i])).tolist() == [float(v) for v in s]
+
+
+# ---------------------------------------------------------------------------
+# Premise of the method (sanity, not a value pin)
+# ---------------------------------------------------------------------------
+
+def test_premise_activation_aware_beats_rtn(oracle_mod):
+    """With ~1% outlier channels the best alpha beats plain RTN (alpha = 0), and
+    the error is not monotone in alpha (it falls, then rises again: the note
+    "52 · AWQ, GPTQ và SmoothQuant" §3 observes error falling up to a point)."""
+    cfg = synth.make_config(64, 512, 128, bits=4, group=128, seed=0, lo=20.0, hi=20.0)
+    W, X, _ = synth.generate(cfg)
+    a = oracle_mod.act_stats(X)
+    r = oracle_mod.search(W, X, a, 4, 128, synth.default_alphas())
+    L = r["losses"]
+    assert r["best"] > 0 and L[r["best"]] < L[0]
+    assert not np.all(np.diff(L) >= 0)
