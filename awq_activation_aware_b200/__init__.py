@@ -1,0 +1,221 @@
+"""B200-native AWQ per-layer scale search: Python binding of ``libawq.so``.
+
+Every function here only marshals arguments (tensor pointers, sizes, the
+current CUDA stream) into the C ABI declared in ``include/awq.h``; all of the
+work runs in the library's sm_100a kernels.  There is no CPU fallback: if the
+library is missing or the device is not a B200-class (sm_100) GPU, calls raise.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+__all__ = [
+    "AWQError", "lib", "act_stats", "alpha_scales", "quant_dequant", "search_workspace_bytes",
+    "search_layer", "pack", "quantize_layer", "get_status", "set_wait_timeout_ms", "default_alphas",
+    "profile_next_search",
+    "LIB_PATH",
+]
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libawq.so"
+
+STATUS = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED", 3: "AWQ_ERR_CUDA",
+          4: "AWQ_ERR_TIMEOUT", 5: "AWQ_ERR_WORKSPACE"}
+
+
+class AWQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS.get(self.code, self.code)}")
+
+
+class QCfg(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("zero_point", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m awq_activation_aware_b200.build`")
+    L = ctypes.CDLL(str(LIB_PATH))
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    L.awq_act_stats.argtypes = [P, i64, i64, i64, P, P]
+    L.awq_alpha_scales.argtypes = [P, i64, P, i32, P, P]
+    L.awq_quant_dequant.argtypes = [P, i64, i64, P, QCfg, P, P]
+    L.awq_search_workspace_bytes.argtypes = [i64, i64, i64, QCfg, i32]
+    L.awq_search_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_search_layer.argtypes = [P, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P, ctypes.c_size_t, P]
+    L.awq_pack.argtypes = [P, i64, i64, P, QCfg, P, P, i32, P, P, P, P, P, P]
+    L.awq_get_status.argtypes = [P]
+    L.awq_set_wait_timeout_ms.argtypes = [ctypes.c_uint32]
+    L.awq_set_wait_timeout_ms.restype = None
+    L.awq_profile_next_search.argtypes = [P, P]
+    L.awq_profile_next_search.restype = None
+    L.awq_status_string.argtypes = [ctypes.c_int]
+    L.awq_status_string.restype = ctypes.c_char_p
+    for fn in ("awq_act_stats", "awq_alpha_scales", "awq_quant_dequant", "awq_search_layer", "awq_pack",
+               "awq_get_status"):
+        getattr(L, fn).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise AWQError(code, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _rowmajor(t: torch.Tensor, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with contiguous rows")
+
+
+def default_alphas(n: int = 20, device="cuda") -> torch.Tensor:
+    """The grid alpha_i = RN32(i / n), i = 0..n-1."""
+    return torch.tensor([i / n for i in range(n)], dtype=torch.float32, device=device)
+
+
+def _qcfg(bits, group):
+    return QCfg(int(bits), int(group), 1)
+
+
+def act_stats(X: torch.Tensor, stream=None) -> torch.Tensor:
+    """a_j = mean_t |X[t, j]| for fp16 X[T, K] (rows may be strided)."""
+    _rowmajor(X, "X")
+    T, K = X.shape
+    a = torch.empty(K, dtype=torch.float32, device=X.device)
+    _check(lib().awq_act_stats(_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(a, torch.float32, "a"),
+                               _stream(stream)), "awq_act_stats")
+    return a
+
+
+def alpha_scales(a: torch.Tensor, alphas: torch.Tensor, stream=None) -> torch.Tensor:
+    """s[i, j] = a_j ** alpha_i (binary64 pow rounded to binary32)."""
+    n = alphas.numel()
+    s = torch.empty((n, a.numel()), dtype=torch.float32, device=a.device)
+    _check(lib().awq_alpha_scales(_dev(a, torch.float32, "a"), a.numel(), _dev(alphas, torch.float32, "alphas"),
+                                  n, _dev(s, torch.float32, "s"), _stream(stream)), "awq_alpha_scales")
+    return s
+
+
+def quant_dequant(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128, stream=None):
+    """W_hat = Q(W diag(s)) diag(s)^-1 in fp16 (the per-element function of the search)."""
+    W = W.contiguous()
+    N, K = W.shape
+    out = torch.empty_like(W)
+    _check(lib().awq_quant_dequant(_dev(W, torch.float16, "W"), N, K, _dev(s, torch.float32, "s"),
+                                   _qcfg(bits, group), _dev(out, torch.float16, "W_hat"), _stream(stream)),
+           "awq_quant_dequant")
+    return out
+
+
+def search_workspace_bytes(N, K, T, bits=4, group=128, n_alpha=20) -> int:
+    return int(lib().awq_search_workspace_bytes(N, K, T, _qcfg(bits, group), n_alpha))
+
+
+def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, bits: int = 4,
+                 group: int = 128, workspace: torch.Tensor | None = None, row_losses: bool = False,
+                 losses_out: torch.Tensor | None = None, stream=None):
+    """Per-alpha MSE of the layer output, ||(W_hat_alpha - W) X^T||^2 / (N T).
+
+    Returns ``losses`` (float32 [n_alpha]) or ``(losses, row_losses)`` with
+    row_losses float32 [n_alpha, N] holding unnormalised per-row sums."""
+    _rowmajor(X, "X")
+    if not W.is_contiguous():
+        raise ValueError("W must be contiguous")
+    N, K = W.shape
+    T = X.shape[0]
+    n = alphas.numel()
+    need = search_workspace_bytes(N, K, T, bits, group, n)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    losses = losses_out if losses_out is not None else torch.empty(n, dtype=torch.float32, device=W.device)
+    rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
+    _check(lib().awq_search_layer(
+        _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X"), T, X.stride(0),
+        _dev(a, torch.float32, "a"), _qcfg(bits, group), _dev(alphas, torch.float32, "alphas"), n,
+        _dev(losses, torch.float32, "losses"),
+        _dev(rl, torch.float32, "row_losses") if rl is not None else None,
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)), "awq_search_layer")
+    return (losses, rl) if row_losses else losses
+
+
+def pack(W: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, losses: torch.Tensor, bits: int = 4,
+         group: int = 128, out: dict | None = None, stream=None) -> dict:
+    """Argmin over the grid, then packed codes, fp16 scales/zeros and s at the best alpha."""
+    N, K = W.shape
+    dev = W.device
+    per = 16 if bits == 2 else 8
+    o = out if out is not None else dict(
+        best_idx=torch.empty(1, dtype=torch.int32, device=dev),
+        s_best=torch.empty(K, dtype=torch.float32, device=dev),
+        codes=torch.empty((N, K // per), dtype=torch.int32, device=dev),
+        scales=torch.empty((N, K // group), dtype=torch.float16, device=dev),
+        zeros=torch.empty((N, K // group), dtype=torch.float16, device=dev))
+    _check(lib().awq_pack(
+        _dev(W, torch.float16, "W"), N, K, _dev(a, torch.float32, "a"), _qcfg(bits, group),
+        _dev(alphas, torch.float32, "alphas"), _dev(losses, torch.float32, "losses"), alphas.numel(),
+        _dev(o["best_idx"], torch.int32, "best_idx"), _dev(o["s_best"], torch.float32, "s_best"),
+        _dev(o["codes"], torch.int32, "codes"), _dev(o["scales"], torch.float16, "scales"),
+        _dev(o["zeros"], torch.float16, "zeros"), _stream(stream)), "awq_pack")
+    return o
+
+
+def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,
+                   group: int = 128, workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """The whole path for one layer: statistics, grid search, argmin, packing.
+
+    W and X may live in host memory (pinned for asynchronous copies); they are
+    then copied to the current device first and the results copied back."""
+    host = not W.is_cuda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Wd = W.to(dev, non_blocking=True) if host else W
+    Xd = X.to(dev, non_blocking=True) if host else X
+    al = default_alphas(device=dev) if alphas is None else alphas.to(dev)
+    a = act_stats(Xd, stream)
+    losses = search_layer(Wd, Xd, a, al, bits, group, workspace=workspace, stream=stream)
+    res = pack(Wd, a, al, losses, bits, group, stream=stream)
+    res["losses"] = losses
+    res["a"] = a
+    if host:
+        res = {k: v.to("cpu", non_blocking=True) for k, v in res.items()}
+        torch.cuda.current_stream().synchronize()
+    return res
+
+
+def get_status(stream=None) -> None:
+    """Synchronise and raise if a kernel reported an error on the device."""
+    _check(lib().awq_get_status(_stream(stream)), "awq_get_status")
+
+
+def set_wait_timeout_ms(ms: int) -> None:
+    lib().awq_set_wait_timeout_ms(int(ms))
+
+
+def profile_next_search(begin: torch.cuda.Event, end: torch.cuda.Event) -> None:
+    """Bracket the tensor-core kernel of the next search_layer call (this thread) with two events."""
+    lib().awq_profile_next_search(ctypes.c_void_p(begin.cuda_event), ctypes.c_void_p(end.cuda_event))

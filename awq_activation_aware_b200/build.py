@@ -1,0 +1,65 @@
+"""Builds libawq.so (the C-ABI library) in-tree for sm_100a.
+
+    python -m awq_activation_aware_b200.build [--verbose]
+
+nvcc cross-compiles without a GPU.  The CUDA runtime is linked statically so
+the library does not depend on which libcudart another package has loaded.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+from pathlib import Path
+
+PKG = Path(__file__).resolve().parent
+ROOT = PKG.parent
+CSRC = PKG / "csrc"
+LIB = PKG / "libawq.so"
+SOURCES = [CSRC / "awq_abi.cu"]
+DEPS = SOURCES + [CSRC / "awq_kernels.cuh", CSRC / "awq_device.cuh", ROOT / "include" / "awq.h"]
+
+NVCC_FLAGS = [
+    "-O3", "-std=c++17",
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-lineinfo",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    "-shared", "-cudart", "static",
+    "-Xptxas", "-v",
+]
+
+
+def nvcc() -> str:
+    cand = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    p = Path(cand) / "bin" / "nvcc"
+    return str(p) if p.exists() else "nvcc"
+
+
+def needs_build() -> bool:
+    if not LIB.exists():
+        return True
+    t = LIB.stat().st_mtime
+    return any(d.stat().st_mtime > t for d in DEPS)
+
+
+def build(force: bool = False, verbose: bool = False) -> Path:
+    if not force and not needs_build():
+        return LIB
+    tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", str(ROOT / "include"), "-I", str(CSRC),
+           "-o", str(tmp), *map(str, SOURCES)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    log = res.stdout + res.stderr
+    (PKG / "build.log").write_text(" ".join(cmd) + "\n" + log)
+    if res.returncode != 0:
+        sys.stderr.write(log)
+        raise RuntimeError(f"nvcc failed ({res.returncode}); see {PKG / 'build.log'}")
+    if verbose:
+        sys.stdout.write(log)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose="--verbose" in sys.argv)
+    print(LIB)

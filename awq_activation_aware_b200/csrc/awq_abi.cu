@@ -1,0 +1,325 @@
+// Host side of the C ABI declared in include/awq.h: argument validation,
+// workspace layout, TMA descriptor encoding and kernel launches.  Every step
+// of the search runs in the kernels of awq_kernels.cuh; nothing here computes
+// on the host beyond sizes and launch shapes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "awq.h"
+#include "awq_kernels.cuh"
+
+namespace {
+
+std::atomic<uint32_t> g_timeout_ms{4000};
+
+// One-shot, per-thread request to bracket the next search kernel with events.
+thread_local cudaEvent_t t_prof_begin = nullptr;
+thread_local cudaEvent_t t_prof_end = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_qcfg(const awq_qcfg &q) {
+    return (q.bits == 2 || q.bits == 3 || q.bits == 4) && (q.group_size == 64 || q.group_size == 128) &&
+           q.zero_point == 1;
+}
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+constexpr int kMaxAlpha = 64;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of awq_search_layer, carved in this order (each 256-byte aligned):
+//   s_tab   float [n_alpha][K]
+//   rs_tab  float [n_alpha][K]
+//   params  uint2 [n_alpha][K/g][N]
+//   partial float [n_alpha][ceil(T/512)][N]
+struct SearchWs {
+    size_t s_off, rs_off, prm_off, part_off, total;
+};
+SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alpha) {
+    SearchWs w{};
+    const int64_t n_tb = (T + awq::srch::BT - 1) / awq::srch::BT;
+    size_t off = 0;
+    w.s_off = off;    off = round_up(off + sizeof(float) * (size_t)n_alpha * K, 256);
+    w.rs_off = off;   off = round_up(off + sizeof(float) * (size_t)n_alpha * K, 256);
+    w.prm_off = off;  off = round_up(off + sizeof(uint2) * (size_t)n_alpha * (K / group) * N, 256);
+    w.part_off = off; off = round_up(off + sizeof(float) * (size_t)n_alpha * n_tb * N, 256);
+    w.total = off;
+    return w;
+}
+
+awq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
+
+awq_status last_launch() { return cuda_status(cudaGetLastError()); }
+
+// Per-device facts, queried once.
+struct DevInfo {
+    int sms = 0;
+    int cc_major = 0;
+    bool search_attr = false;
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+awq_status device_info(DevInfo &out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return AWQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            d.sms = 0;
+            return AWQ_ERR_CUDA;
+        }
+    }
+    if (d.cc_major != 10) return AWQ_ERR_UNSUPPORTED;
+    if (!d.search_attr) {
+        if (cudaFuncSetAttribute(awq::srch::search_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::srch::SMEM_BYTES) != cudaSuccess)
+            return AWQ_ERR_CUDA;
+        d.search_attr = true;
+    }
+    out = d;
+    return AWQ_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// X[T, ldx] fp16 as a 2-D tensor (inner dimension K), boxes of 64 x 256,
+// 128-byte swizzle; rows past T read as zeros.
+bool encode_x_map(CUtensorMap *m, const void *X, int64_t T, int64_t K, int64_t ldx) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    cuuint32_t box[2] = {(cuuint32_t)awq::srch::BK, (cuuint32_t)awq::srch::BN};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int blocks_for(int64_t threads_total, int block) {
+    int64_t b = (threads_total + block - 1) / block;
+    return (int)(b < 1 ? 1 : b);
+}
+
+awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, const float *s_tab,
+                               int n_alpha, float qmax, uint2 *params, cudaStream_t st) {
+    const int G = (int)(K / group);
+    const int tpg = group / 16;
+    const int grid = blocks_for(N * G * tpg, 256);
+    if (tpg == 8)
+        awq::group_params_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, s_tab, n_alpha, qmax, params);
+    else
+        awq::group_params_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, s_tab, n_alpha, qmax, params);
+    return last_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *awq_status_string(awq_status s) {
+    switch (s) {
+        case AWQ_OK: return "AWQ_OK";
+        case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG";
+        case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED";
+        case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
+        case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT";
+        case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE";
+    }
+    return "AWQ_ERR_UNKNOWN";
+}
+
+void awq_set_wait_timeout_ms(uint32_t ms) { g_timeout_ms.store(ms == 0 ? 1 : ms); }
+
+void awq_profile_next_search(void *ev_begin, void *ev_end) {
+    t_prof_begin = static_cast<cudaEvent_t>(ev_begin);
+    t_prof_end = static_cast<cudaEvent_t>(ev_end);
+}
+
+awq_status awq_act_stats(const void *X, int64_t T, int64_t K, int64_t ldx, float *a, void *stream) {
+    if (!X || !a || !aligned16(X) || !aligned16(a)) return AWQ_ERR_INVALID_ARG;
+    if (T < 1 || T > kMaxDim || K < 8 || K > kMaxDim || K % 8 || ldx < K || ldx % 8) return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    const int slabs = (int)((K + awq::kStatsCols - 1) / awq::kStatsCols);
+    awq::act_stats_kernel<<<slabs * awq::kStatsCluster, awq::kStatsThreads, 0, (cudaStream_t)stream>>>(
+        (const __half *)X, T, K, ldx, a);
+    return last_launch();
+}
+
+awq_status awq_alpha_scales(const float *a, int64_t K, const float *alphas, int32_t n_alpha, float *s,
+                            void *stream) {
+    if (!a || !alphas || !s || !aligned16(a) || !aligned16(s) || !aligned16(alphas)) return AWQ_ERR_INVALID_ARG;
+    if (K < 1 || K > kMaxDim || n_alpha < 1 || n_alpha > kMaxAlpha) return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    const int grid = blocks_for((int64_t)n_alpha * K, 256);
+    awq::alpha_scales_kernel<<<grid < 4 * d.sms ? grid : 4 * d.sms, 256, 0, (cudaStream_t)stream>>>(
+        a, K, alphas, n_alpha, s, nullptr);
+    return last_launch();
+}
+
+awq_status awq_quant_dequant(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, void *W_hat,
+                             void *stream) {
+    if (!W || !s || !W_hat || !aligned16(W) || !aligned16(s) || !aligned16(W_hat)) return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || K < q.group_size || K > kMaxDim || K % q.group_size)
+        return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    const int G = (int)(K / q.group_size);
+    const int tpg = q.group_size / 16;
+    const int grid = blocks_for(N * G * tpg, 256);
+    const float qmax = (float)((1 << q.bits) - 1);
+    if (tpg == 8)
+        awq::quant_dequant_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax,
+                                                                            (__half *)W_hat);
+    else
+        awq::quant_dequant_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax,
+                                                                            (__half *)W_hat);
+    return last_launch();
+}
+
+size_t awq_search_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q, int32_t n_alpha) {
+    if (!valid_qcfg(q) || N < 1 || K < 1 || T < 1 || n_alpha < 1 || K % q.group_size) return 0;
+    return search_ws_layout(N, K, T, q.group_size, n_alpha).total;
+}
+
+awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx,
+                            const float *a, awq_qcfg q, const float *alphas, int32_t n_alpha, float *losses,
+                            float *row_losses, void *ws, size_t ws_bytes, void *stream) {
+    if (!W || !X || !a || !alphas || !losses) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(X) || !aligned16(a) || !aligned16(alphas) || !aligned16(losses) ||
+        (row_losses && !aligned16(row_losses)))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || T < 1 || T > kMaxDim || K < 64 || K > kMaxDim || K % 64 ||
+        K % q.group_size || ldx < K || ldx % 8 || n_alpha < 1 || n_alpha > kMaxAlpha)
+        return AWQ_ERR_INVALID_ARG;
+    const SearchWs L = search_ws_layout(N, K, T, q.group_size, n_alpha);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *s_tab = reinterpret_cast<float *>(base + L.s_off);
+    float *rs_tab = reinterpret_cast<float *>(base + L.rs_off);
+    uint2 *params = reinterpret_cast<uint2 *>(base + L.prm_off);
+    float *partial = reinterpret_cast<float *>(base + L.part_off);
+    const float qmax = (float)((1 << q.bits) - 1);
+
+    // a2: s and 1/s for every alpha
+    {
+        const int grid = blocks_for((int64_t)n_alpha * K, 256);
+        awq::alpha_scales_kernel<<<grid < 4 * d.sms ? grid : 4 * d.sms, 256, 0, st>>>(a, K, alphas, n_alpha,
+                                                                                     s_tab, rs_tab);
+        if (awq_status e = last_launch()) return e;
+    }
+    // a3 (group parameters for every alpha)
+    if (awq_status e = launch_group_params(W, N, K, q.group_size, s_tab, n_alpha, qmax, params, st)) return e;
+
+    // a4-a6: the tensor-core search
+    CUtensorMap tmap;
+    if (!encode_x_map(&tmap, X, T, K, ldx)) return AWQ_ERR_CUDA;
+    awq::srch::Args A;
+    A.W = (const __half *)W;
+    A.params = params;
+    A.s_tab = s_tab;
+    A.rs_tab = rs_tab;
+    A.partial = partial;
+    A.N = N;
+    A.K = K;
+    A.T = T;
+    A.n_alpha = n_alpha;
+    A.G = (int)(K / q.group_size);
+    A.group = q.group_size;
+    A.n_nb = (int)((N + awq::srch::BM - 1) / awq::srch::BM);
+    A.n_tb = (int)((T + awq::srch::BT - 1) / awq::srch::BT);
+    A.n_kb = (int)(K / awq::srch::BK);
+    A.n_units = (int64_t)A.n_nb * A.n_tb * n_alpha;
+    A.qmax = qmax;
+    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+    const int grid = (int)(A.n_units < d.sms ? A.n_units : d.sms);
+    cudaEvent_t pb = t_prof_begin, pe = t_prof_end;
+    t_prof_begin = t_prof_end = nullptr;
+    if (pb && cudaEventRecord(pb, st) != cudaSuccess) return AWQ_ERR_CUDA;
+    awq::srch::search_kernel<<<grid, awq::srch::NUM_THREADS, awq::srch::SMEM_BYTES, st>>>(tmap, A);
+    if (awq_status e = last_launch()) return e;
+    if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
+
+    // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
+    awq::loss_reduce_kernel<<<n_alpha, 256, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
+    return last_launch();
+}
+
+awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcfg q, const float *alphas,
+                    const float *losses, int32_t n_alpha, int32_t *best_idx, float *s_best, uint32_t *codes,
+                    void *scales, void *zeros, void *stream) {
+    if (!W || !a || !alphas || !losses || !best_idx || !s_best || !codes || !scales || !zeros)
+        return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(a) || !aligned16(s_best) || !aligned16(codes) || !aligned16(scales) ||
+        !aligned16(zeros) || !aligned16(alphas) || !aligned16(losses) || !aligned16(best_idx))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || K < q.group_size || K > kMaxDim || K % q.group_size ||
+        n_alpha < 1 || n_alpha > kMaxAlpha)
+        return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    {
+        int grid = blocks_for(K, 256);
+        if (grid > 2 * d.sms) grid = 2 * d.sms;
+        awq::best_scale_kernel<<<grid, 256, 0, st>>>(a, K, alphas, losses, n_alpha, best_idx, s_best);
+        if (awq_status e = last_launch()) return e;
+    }
+    const int G = (int)(K / q.group_size);
+    const int tpg = q.group_size / 16;
+    const int grid = blocks_for(N * G * tpg, 256);
+    if (tpg == 8)
+        awq::pack_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
+                                                  (__half *)scales, (__half *)zeros);
+    else
+        awq::pack_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
+                                                  (__half *)scales, (__half *)zeros);
+    return last_launch();
+}
+
+awq_status awq_get_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return AWQ_ERR_CUDA;
+    unsigned flags = 0;
+    if (cudaMemcpyFromSymbol(&flags, awq::g_dev_error, sizeof(flags)) != cudaSuccess) return AWQ_ERR_CUDA;
+    if (flags) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(awq::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return AWQ_ERR_CUDA;
+        if (flags & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
+        if (flags & awq::kDevErrBadAlpha) return AWQ_ERR_INVALID_ARG;
+    }
+    return last_launch();
+}
+
+}  // extern "C"

@@ -1,0 +1,312 @@
+// Device-side building blocks of the AWQ search library (sm_100a only):
+//   * the quantizer arithmetic of the per-layer scale search, written once and
+//     used by every kernel that evaluates it (group parameters, the search
+//     producer, the standalone dequantizer and the packer), so that all of them
+//     produce bit-identical codes;
+//   * thin inline-PTX wrappers for mbarriers, TMA and the tcgen05 tensor core.
+//
+// Sources (web pages): [QAS-QA] "Как работает quantization-aware scaling в AWQ
+// для защиты важных весов?" §5, §9; [AWQ-note] "AWQ: Activation-Aware Weight
+// Quantization For On-Device LLM Compression AND Acceleration", "Measures";
+// [AWQ-wiki] "AWQ" (French), "Fondements techniques".
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+namespace awq {
+
+// ---------------------------------------------------------------------------
+// Device error word (read and cleared by awq_get_status on the host).  The
+// library is a single translation unit, so the definition lives here.
+// ---------------------------------------------------------------------------
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBadAlpha = 2u };
+__device__ unsigned g_dev_error = 0;
+
+// ---------------------------------------------------------------------------
+// Quantizer arithmetic.  Every binary32 step is an explicit round-to-nearest
+// intrinsic so the compiler cannot contract or reorder it.
+// ---------------------------------------------------------------------------
+
+// 1.5 * 2^23: for |x| <= 2^22, RN32(x + kMagic) = kMagic + rint(x) (ties to
+// even, because kMagic is even and the spacing of binary32 there is 1).
+constexpr float kMagic = 12582912.0f;
+constexpr float kMinScale = 5.9604644775390625e-8f;   // 2^-24, smallest fp16 subnormal
+constexpr float kMaxScale = 65504.0f;                  // largest finite fp16
+
+// Per-(row, group) quantizer parameters derived from the group's min and max of
+// w' = RN32(w*s) ([QAS-QA] §9: zero_point = True, q_group_size, w_bit):
+//   scale = RN32(RN32(mx - mn) / qmax), sh = RN16(clamp(scale, 2^-24, 65504)),
+//   r = RN32(1/sh), z = clamp(rint(RN32(-mn * r)), 0, qmax).
+struct QParams {
+    float r;     // reciprocal of the stored fp16 scale
+    float sh;    // the stored fp16 scale, as binary32
+    float z;     // zero point, an integer in [0, qmax]
+};
+
+__device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax) {
+    QParams p;
+    float range = __fsub_rn(mx, mn);
+    float scale = __fdiv_rn(range, qmax);
+    scale = fminf(fmaxf(scale, kMinScale), kMaxScale);
+    p.sh = __half2float(__float2half_rn(scale));
+    p.r = __frcp_rn(p.sh);
+    const float zr = rintf(__fmul_rn(-mn, p.r));
+    p.z = zr > 0.0f ? fminf(zr, qmax) : 0.0f;   // a code in [0, qmax]; never -0
+    return p;
+}
+
+// Compact 8-byte form kept in the search workspace: r as binary32, the fp16
+// scale bits and the zero point.
+__device__ __forceinline__ uint2 pack_qparams(const QParams &p) {
+    uint16_t shb = __half_as_ushort(__float2half_rn(p.sh));
+    return make_uint2(__float_as_uint(p.r), (uint32_t)shb | ((uint32_t)p.z << 16));
+}
+__device__ __forceinline__ QParams unpack_qparams(uint2 v) {
+    QParams p;
+    p.r = __uint_as_float(v.x);
+    p.sh = __half2float(__ushort_as_half((unsigned short)(v.y & 0xFFFFu)));
+    p.z = (float)(v.y >> 16);
+    return p;
+}
+
+// Element constants derived once per (row, group): clamp bounds of t = w'*r in
+// units of codes relative to the zero point, and -kMagic*sh (exact: kMagic has
+// two significant bits and sh eleven).
+struct QElem {
+    float r, lo, hi, sh, nmsh;
+};
+__device__ __forceinline__ QElem make_qelem(const QParams &p, float qmax) {
+    QElem e;
+    e.r = p.r;
+    e.lo = -p.z;
+    e.hi = __fsub_rn(qmax, p.z);
+    e.sh = p.sh;
+    e.nmsh = __fmul_rn(-kMagic, p.sh);
+    return e;
+}
+
+// RN32((q - z) * sh) with q = clamp(rint(RN32(w'*r)) + z, 0, qmax).
+// Because z is an integer, q - z = rint(clamp(RN32(w'*r), -z, qmax - z)); the
+// magic add rounds that value (|.| <= qmax) to an integer, and one FMA turns
+// (v - kMagic) * sh into a single rounding of the exact product (which is
+// itself exact: |q - z| <= 15 and sh has 11 significant bits).
+__device__ __forceinline__ float dequant_code_times_scale(float wp, const QElem &e) {
+    float t = __fmul_rn(wp, e.r);
+    t = fminf(fmaxf(t, e.lo), e.hi);
+    float v = __fadd_rn(t, kMagic);
+    return __fmaf_rn(v, e.sh, e.nmsh);
+}
+
+// The integer code q itself (used by the packer).
+__device__ __forceinline__ uint32_t quant_code(float wp, const QElem &e, float z) {
+    float t = __fmul_rn(wp, e.r);
+    t = fminf(fmaxf(t, e.lo), e.hi);
+    float d = __fsub_rn(__fadd_rn(t, kMagic), kMagic);   // rint(t), exact
+    return (uint32_t)__float2int_rn(__fadd_rn(d, z));
+}
+
+// w_hat = RN16(RN32(RN32((q - z) * sh) * rs)), rs = RN32(1/s)
+// ([AWQ-wiki] "Fondements techniques": the inverse scaling after dequantization).
+__device__ __forceinline__ __half dequant_unscale(float wp, const QElem &e, float rs) {
+    return __float2half_rn(__fmul_rn(dequant_code_times_scale(wp, e), rs));
+}
+
+// ---------------------------------------------------------------------------
+// Small PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// Streaming 16-byte load that does not allocate in L1 (read-once data).
+__device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// ----- mbarrier -------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: returns false (after raising the device timeout flag and the
+// CTA's abort flag) when the phase does not complete within `limit_ns`, or
+// when another role of the CTA has already aborted.  Never traps.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort_flag, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicOr(&g_dev_error, kDevErrTimeout);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
+                                               volatile int *abort_flag, uint64_t limit_ns) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, limit_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    return ok != 0;
+}
+
+// ----- TMA ------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, int32_t c0,
+                                            int32_t c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core reads operands through it).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ----- tcgen05 --------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, fp16 inputs, fp32 accumulation.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation issued so far by this
+// thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives lane
+// (warp quadrant base + i), columns col .. col+31.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand stored in the
+// 128-byte-swizzled canonical layout: rows of 64 fp16 (128 B), 8-row groups
+// 1024 B apart, 16-byte chunks XOR-permuted by (row mod 8).  The tile base
+// must be 1024-byte aligned; advancing `saddr` by 32 B steps through K = 16
+// slices inside the 128-byte row.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);   // start address / 16
+    d |= (uint64_t)1u << 16;                    // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(1024u >> 4) << 32;          // stride byte offset: 8 rows * 128 B
+    d |= (uint64_t)1u << 46;                    // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                    // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor of tcgen05.mma.kind::f16: fp32 accumulator, fp16 A
+// and B, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t mma_idesc_f16_f32(int M, int N) {
+    return (1u << 4)                          // D format: f32
+           | (0u << 7) | (0u << 10)           // A, B format: f16
+           | (0u << 15) | (0u << 16)          // A, B K-major
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
+// 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+}  // namespace awq

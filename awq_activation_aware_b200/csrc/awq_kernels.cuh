@@ -1,0 +1,656 @@
+// Kernels of the AWQ per-layer scale search on B200 (sm_100a).
+//
+//   act_stats_kernel      a_j = mean_t |X[t,j]|              (HBM-bound column reduction)
+//   alpha_scales_kernel   s = a^alpha, rs = RN32(1/s)        (tiny)
+//   group_params_kernel   per (alpha, row, group): sh, r, z  (one pass over W for all alphas)
+//   search_kernel         per alpha: sum ((W_hat - W) X^T)^2 (tcgen05 / TMEM / TMA)
+//   loss_reduce_kernel    per-alpha MSE and per-row sums     (deterministic, binary64)
+//   best_scale_kernel     argmin over the grid + s_best
+//   pack_kernel           codes / fp16 scales / fp16 zeros   (HBM-bound)
+//   quant_dequant_kernel  W_hat for one s (the a3/a4 step on its own)
+//
+// Sources (web pages): [AWQ-note] "AWQ: Activation-Aware Weight Quantization For
+// On-Device LLM Compression AND Acceleration", section "Measures"; [QAS-QA]
+// "Как работает quantization-aware scaling в AWQ для защиты важных весов?" §5, §6,
+// §9; [GPTQ-AWQ] "GPTQ与AWQ", section "量化方法"; [AWQ-wiki] "AWQ" (French),
+// "Fondements techniques".
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cfloat>
+#include <cstdint>
+
+#include "awq_device.cuh"
+
+namespace awq {
+
+namespace cg = cooperative_groups;
+
+// ===========================================================================
+// a1. Activation statistics: a_j = RN32(RN64(sum_t |X[t,j]|) / T)
+//     ([AWQ-note] "Measures"; [GPTQ-AWQ] "量化方法": X.abs().mean(dim=0)).
+//
+// A cluster of 8 CTAs owns a slab of 128 columns; each CTA reads every 8th
+// group of 16 rows with 16-byte loads (16 threads cover one 256-byte row
+// segment), accumulates |x| in binary64 -- exact, since every fp16 value is a
+// multiple of 2^-24 and the sums stay below 2^29 -- reduces its 16 row lanes
+// in shared memory, and CTA 0 of the cluster sums the 8 partial vectors
+// through distributed shared memory.  No workspace, one launch.
+// ===========================================================================
+constexpr int kStatsCols = 128;
+constexpr int kStatsTPR = 16;                      // threads per row segment
+constexpr int kStatsThreads = 256;
+constexpr int kStatsRowsPerCta = kStatsThreads / kStatsTPR;   // 16
+constexpr int kStatsCluster = 8;
+constexpr int kStatsUnroll = 8;
+
+__global__ void __cluster_dims__(kStatsCluster, 1, 1) __launch_bounds__(kStatsThreads)
+act_stats_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx,
+                 float *__restrict__ a) {
+    __shared__ double red[kStatsRowsPerCta][kStatsCols + 1];
+    __shared__ double part[kStatsCols];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int slab = blockIdx.x / kStatsCluster;
+    const int cc = threadIdx.x % kStatsTPR;
+    const int rl = threadIdx.x / kStatsTPR;
+    const int64_t col0 = (int64_t)slab * kStatsCols + cc * 8;
+    const bool active = col0 < K;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+
+    const int64_t rstride = (int64_t)kStatsRowsPerCta * kStatsCluster;   // 128 rows
+    int64_t t = (int64_t)rank * kStatsRowsPerCta + rl;
+    if (active) {
+        for (; t + (kStatsUnroll - 1) * rstride < T; t += kStatsUnroll * rstride) {
+            uint4 v[kStatsUnroll];
+#pragma unroll
+            for (int u = 0; u < kStatsUnroll; ++u)
+                v[u] = ldg_stream_v4(X + (t + u * rstride) * ldx + col0);
+#pragma unroll
+            for (int u = 0; u < kStatsUnroll; ++u) {
+                const __half2 *h = reinterpret_cast<const __half2 *>(&v[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = __half22float2(__habs2(h[e]));
+                    acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
+                    acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
+                }
+            }
+        }
+        for (; t < T; t += rstride) {
+            uint4 v = ldg_stream_v4(X + t * ldx + col0);
+            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float2 f = __half22float2(__habs2(h[e]));
+                acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
+                acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rl][cc * 8 + e] = acc[e];
+    __syncthreads();
+    if (threadIdx.x < kStatsCols) {
+        double s = 0.0;
+#pragma unroll
+        for (int r = 0; r < kStatsRowsPerCta; ++r) s = __dadd_rn(s, red[r][threadIdx.x]);
+        part[threadIdx.x] = s;
+    }
+    cluster.sync();
+    if (rank == 0 && threadIdx.x < kStatsCols) {
+        double s = 0.0;
+        for (int q = 0; q < kStatsCluster; ++q)
+            s = __dadd_rn(s, *cluster.map_shared_rank(&part[threadIdx.x], q));
+        const int64_t col = (int64_t)slab * kStatsCols + threadIdx.x;
+        if (col < K) a[col] = __double2float_rn(__ddiv_rn(s, (double)T));
+    }
+    cluster.sync();   // keep every CTA's shared memory alive until CTA 0 has read it
+}
+
+// ===========================================================================
+// a2. Search space: s[i,j] = RN32(pow(max(a_j, FLT_MIN), alpha_i)), evaluated in
+//     binary64 ([AWQ-note] "Measures": compute a^alpha for each candidate),
+//     and its reciprocal rs = RN32(1/s) used to undo the scaling.
+// ===========================================================================
+__global__ void alpha_scales_kernel(const float *__restrict__ a, int64_t K,
+                                    const float *__restrict__ alphas, int n_alpha,
+                                    float *__restrict__ s, float *__restrict__ rs) {
+    const int64_t total = (int64_t)n_alpha * K;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int ai = (int)(i / K);
+        const int64_t j = i - (int64_t)ai * K;
+        const float al = alphas[ai];
+        if (!(al >= 0.0f && al <= 1.0f)) atomicOr(&g_dev_error, kDevErrBadAlpha);
+        const float aj = fmaxf(a[j], FLT_MIN);
+        const float sv = __double2float_rn(pow((double)aj, (double)al));
+        s[i] = sv;
+        if (rs) rs[i] = __frcp_rn(sv);
+    }
+}
+
+// ===========================================================================
+// a3 (group half). For every (alpha, row, group): min/max of w' = RN32(w*s) and
+// the quantizer parameters ([QAS-QA] §5, §9).  W is read once: each thread
+// keeps 16 weights in registers and walks the alpha grid.  Layout of the
+// result: params[(alpha * G + group) * N + row] (rows contiguous, so the
+// search producer reads 8 bytes per row of its tile).
+// ===========================================================================
+template <int TPG>   // threads per group = group_size / 16
+__global__ void __launch_bounds__(256)
+group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
+                    const float *__restrict__ s_tab, int n_alpha, float qmax,
+                    uint2 *__restrict__ params) {
+    const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
+    const int sub = threadIdx.x % TPG;
+    const bool active = gid < N * (int64_t)G;
+    const int64_t n = active ? gid / G : 0;
+    const int grp = active ? (int)(gid - n * G) : 0;
+    const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
+    float w[16];
+    {
+        uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
+        uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
+        const __half2 *h0 = reinterpret_cast<const __half2 *>(&v0);
+        const __half2 *h1 = reinterpret_cast<const __half2 *>(&v1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f0 = __half22float2(h0[e]), f1 = __half22float2(h1[e]);
+            w[2 * e] = f0.x; w[2 * e + 1] = f0.y;
+            w[8 + 2 * e] = f1.x; w[8 + 2 * e + 1] = f1.y;
+        }
+    }
+    for (int ai = 0; ai < n_alpha; ++ai) {
+        const float4 *sp = reinterpret_cast<const float4 *>(s_tab + (int64_t)ai * K + k0);
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 sv = __ldg(sp + q);
+            const float p0 = __fmul_rn(w[4 * q + 0], sv.x), p1 = __fmul_rn(w[4 * q + 1], sv.y);
+            const float p2 = __fmul_rn(w[4 * q + 2], sv.z), p3 = __fmul_rn(w[4 * q + 3], sv.w);
+            mn = fminf(mn, fminf(fminf(p0, p1), fminf(p2, p3)));
+            mx = fmaxf(mx, fmaxf(fmaxf(p0, p1), fmaxf(p2, p3)));
+        }
+#pragma unroll
+        for (int off = 1; off < TPG; off <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        }
+        if (active && sub == 0) {
+            const QParams p = make_qparams(mn, mx, qmax);
+            params[((int64_t)ai * G + grp) * N + n] = pack_qparams(p);
+        }
+    }
+}
+
+// ===========================================================================
+// a3/a4 standalone: W_hat = RN16(RN32(RN32((q - z) sh) * RN32(1/s))) for one s.
+// ===========================================================================
+template <int TPG>
+__global__ void __launch_bounds__(256)
+quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
+                     const float *__restrict__ s, float qmax, __half *__restrict__ W_hat) {
+    const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
+    const int sub = threadIdx.x % TPG;
+    const bool active = gid < N * (int64_t)G;
+    const int64_t n = active ? gid / G : 0;
+    const int grp = active ? (int)(gid - n * G) : 0;
+    const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
+    float wp[16], rs[16];
+    {
+        uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
+        uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
+        const __half *h0 = reinterpret_cast<const __half *>(&v0);
+        const __half *h1 = reinterpret_cast<const __half *>(&v1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float sv = active ? __ldg(s + k0 + e) : 1.0f;
+            const float wv = __half2float(e < 8 ? h0[e] : h1[e - 8]);
+            wp[e] = __fmul_rn(wv, sv);
+            rs[e] = __frcp_rn(sv);
+        }
+    }
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) { mn = fminf(mn, wp[e]); mx = fmaxf(mx, wp[e]); }
+#pragma unroll
+    for (int off = 1; off < TPG; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    const QParams p = make_qparams(mn, mx, qmax);
+    const QElem qe = make_qelem(p, qmax);
+    if (!active) return;
+    __align__(16) __half out[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) out[e] = dequant_unscale(wp[e], qe, rs[e]);
+    *reinterpret_cast<uint4 *>(W_hat + n * K + k0) = *reinterpret_cast<const uint4 *>(&out[0]);
+    *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[8]);
+}
+
+// ===========================================================================
+// a5/a6. The search.  For every work unit (tile of 128 W rows x 512 tokens,
+// alpha) it accumulates E = (W_hat_alpha - W) X^T for the tile in tensor
+// memory over all of K, squares and sums E on chip, and writes one fp32
+// partial per (alpha, token block, row).  E is never written to memory.
+//
+// Roles (448 threads, one CTA per SM, persistent over work units):
+//   warps 0-3   epilogue: tcgen05.ld the 128 x 512 fp32 accumulator, sum squares
+//   warp 4      TMA producer for X tiles (64 k x 256 tokens, 128-byte swizzle);
+//               also allocates / frees tensor memory
+//   warp 5      MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128, N=256,
+//               two accumulators side by side (512 TMEM columns)
+//   warps 6-13  producer of the A operand: reads W (+ per-group parameters),
+//               applies s, rounds, dequantizes, unscales, subtracts W and stores
+//               Delta W = W_hat - W (fp16) straight into the swizzled shared
+//               memory tile the tensor core reads.  W_hat never reaches HBM.
+// ===========================================================================
+namespace srch {
+constexpr int BM = 128;                 // W rows per tile (MMA M)
+constexpr int BN = 256;                 // tokens per MMA (MMA N)
+constexpr int NJ = 2;                   // accumulators per tile
+constexpr int BT = BN * NJ;             // tokens per tile
+constexpr int BK = 64;                  // K per pipeline stage (one 128-byte row)
+constexpr int XS = 3;                   // X stages
+constexpr int AS = 2;                   // Delta W stages
+constexpr int X_HALF_BYTES = BN * BK * 2;          // 32 KiB
+constexpr int X_STAGE_BYTES = BT * BK * 2;         // 64 KiB
+constexpr int A_STAGE_BYTES = BM * BK * 2;         // 16 KiB
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int TMA_WARP = 4;
+constexpr int MMA_WARP = 5;
+constexpr int PROD_WARP0 = 6;
+constexpr int NUM_PROD_WARPS = 8;
+constexpr int NUM_THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;   // 448
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t IDESC = mma_idesc_f16_f32(BM, BN);
+
+struct Smem {
+    uint8_t x[XS][X_STAGE_BYTES];       // 1024-aligned (base aligned, sizes multiples of 1024)
+    uint8_t a[AS][A_STAGE_BYTES];
+    uint64_t x_full[XS], x_empty[XS];
+    uint64_t a_full[AS], a_empty[AS];
+    uint64_t acc_full, acc_empty, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + slack to align the base
+
+struct Args {
+    const __half *W;            // [N, K]
+    const uint2 *params;        // [n_alpha][G][N]
+    const float *s_tab;         // [n_alpha][K]
+    const float *rs_tab;        // [n_alpha][K]
+    float *partial;             // [n_alpha][n_tb][N]
+    int64_t N, K, T;
+    int n_alpha, G, group;
+    int n_nb, n_tb, n_kb;
+    int64_t n_units;
+    float qmax;                 // 2^bits - 1
+    uint64_t timeout_ns;
+};
+
+struct UnitIdx { int nb, tb, alpha; };
+__device__ __forceinline__ UnitIdx unit_index(int64_t u, const Args &A) {
+    UnitIdx r;
+    const int64_t tile = u / A.n_alpha;
+    r.alpha = (int)(u - tile * A.n_alpha);
+    r.nb = (int)(tile / A.n_tb);
+    r.tb = (int)(tile - (int64_t)r.nb * A.n_tb);
+    return r;
+}
+
+// Per-thread slice of one producer stage: 4 rows x 8 columns.
+struct ProdLoad {
+    uint4 w[4];
+    uint2 prm[4];
+    float4 s0, s1, r0, r1;
+};
+
+__device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, const UnitIdx &ui,
+                                                 int kb, int c, int rbase) {
+    const int64_t k = (int64_t)kb * BK + c * 8;
+    const float4 *sp = reinterpret_cast<const float4 *>(A.s_tab + (int64_t)ui.alpha * A.K + k);
+    const float4 *rp = reinterpret_cast<const float4 *>(A.rs_tab + (int64_t)ui.alpha * A.K + k);
+    L.s0 = __ldg(sp); L.s1 = __ldg(sp + 1);
+    L.r0 = __ldg(rp); L.r1 = __ldg(rp + 1);
+    const int grp = (int)(((int64_t)kb * BK) / A.group);
+    const uint2 *pp = A.params + ((int64_t)ui.alpha * A.G + grp) * A.N;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
+        if (n < A.N) {
+            L.w[i] = ldg_nc_v4(A.W + n * A.K + k);
+            L.prm[i] = __ldg(pp + n);
+        } else {
+            L.w[i] = make_uint4(0, 0, 0, 0);
+            L.prm[i] = make_uint2(0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ uint4 prod_compute_row(const uint4 wv, const uint2 prm, const float (&s)[8],
+                                                  const float (&rs)[8], float qmax, bool valid) {
+    if (!valid) return make_uint4(0, 0, 0, 0);
+    const QElem e = make_qelem(unpack_qparams(prm), qmax);
+    const __half2 *wh = reinterpret_cast<const __half2 *>(&wv);
+    uint4 out;
+    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 wf = __half22float2(wh[p]);
+        const __half h0 = dequant_unscale(__fmul_rn(wf.x, s[2 * p]), e, rs[2 * p]);
+        const __half h1 = dequant_unscale(__fmul_rn(wf.y, s[2 * p + 1]), e, rs[2 * p + 1]);
+        const __half2 d = __hsub2(__halves2half2(h0, h1), wh[p]);
+        o[p] = *reinterpret_cast<const uint32_t *>(&d);
+    }
+    return out;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < XS; ++i) { mbar_init(&S.x_full[i], 1); mbar_init(&S.x_empty[i], 1); }
+        for (int i = 0; i < AS; ++i) { mbar_init(&S.a_full[i], NUM_PROD_WARPS); mbar_init(&S.a_empty[i], 1); }
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.acc_empty, NUM_EPI_WARPS);
+        mbar_init(&S.drain, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == TMA_WARP) {
+        tmem_alloc(&S.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == TMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_x);
+            int xs = 0;
+            uint32_t xph = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < A.n_units && ok; u += gridDim.x) {
+                const UnitIdx ui = unit_index(u, A);
+                const int t0 = ui.tb * BT;
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.x_empty[xs], xph ^ 1u, abort_flag, A.timeout_ns)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S.x_full[xs], X_STAGE_BYTES);
+                    tma_load_2d(&S.x[xs][0], &tmap_x, kb * BK, t0, &S.x_full[xs]);
+                    tma_load_2d(&S.x[xs][X_HALF_BYTES], &tmap_x, kb * BK, t0 + BN, &S.x_full[xs]);
+                    if (++xs == XS) { xs = 0; xph ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // Let every load already issued land before the CTA can exit.
+                for (int i = 0; i < XS; ++i) {
+                    // Stage i was last filled in phase (xph ^ (i >= xs)); waiting on a
+                    // completed or never-started phase returns at once.
+                    const uint32_t ph = (i < xs) ? xph : (xph ^ 1u);
+                    mbar_wait_bounded(&S.x_full[i], ph, abort_flag, A.timeout_ns);
+                }
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0) {
+            int xs = 0, as = 0;
+            uint32_t xph = 0, aph = 0, accph = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < A.n_units && ok; u += gridDim.x) {
+                if (!mbar_wait_bounded(&S.acc_empty, accph ^ 1u, abort_flag, A.timeout_ns)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
+                        !mbar_wait_bounded(&S.x_full[xs], xph, abort_flag, A.timeout_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(&S.a[as][0]);
+                    const uint32_t x_base = smem_u32(&S.x[xs][0]);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j) {
+                            const uint64_t bdesc = sw128_kmajor_desc(x_base + j * X_HALF_BYTES + kk * 32);
+                            mma_f16_ss(tmem + j * BN, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&S.x_empty[xs]);
+                    mma_commit(&S.a_empty[as]);
+                    if (++xs == XS) { xs = 0; xph ^= 1u; }
+                    if (++as == AS) { as = 0; aph ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(&S.acc_full);
+                accph ^= 1u;
+            }
+            // Drain: every MMA issued by this thread completes before teardown.
+            mma_commit(&S.drain);
+            mbar_wait_bounded(&S.drain, 0, abort_flag, A.timeout_ns);
+        }
+    } else if (warp < NUM_EPI_WARPS) {
+        uint32_t accph = 0;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        for (int64_t u = blockIdx.x; u < A.n_units; u += gridDim.x) {
+            const UnitIdx ui = unit_index(u, A);
+            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns)) break;
+            tc_fence_after();
+            float sum = 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < TMEM_COLS / 32; c += 2) {
+                float v0[32], v1[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v0);
+                tmem_ld_32x32b_x32(tmem + lane_base + (c + 1) * 32, v1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sum = __fmaf_rn(v0[i], v0[i], sum);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sum = __fmaf_rn(v1[i], v1[i], sum);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty);
+            const int64_t n = (int64_t)ui.nb * BM + warp * 32 + lane;
+            if (n < A.N) A.partial[((int64_t)ui.alpha * A.n_tb + ui.tb) * A.N + n] = sum;
+            accph ^= 1u;
+        }
+    } else if (warp >= PROD_WARP0) {
+        const int p = threadIdx.x - PROD_WARP0 * 32;   // 0..255
+        const int c = p & 7;                            // 16-byte chunk of the 128-byte row
+        const int rbase = p >> 3;                       // rows rbase + 32 i
+        int as = 0;
+        uint32_t aph = 0;
+        int64_t u = blockIdx.x;
+        int kb = 0;
+        if (u < A.n_units) {
+            ProdLoad cur;
+            UnitIdx ui = unit_index(u, A);
+            prod_issue_loads(cur, A, ui, kb, c, rbase);
+            while (true) {
+                // Next (unit, kb) and its loads, issued before this stage's math.
+                int64_t un = u;
+                int kbn = kb + 1;
+                if (kbn == A.n_kb) { kbn = 0; un += gridDim.x; }
+                const bool has_next = un < A.n_units;
+                UnitIdx uin = ui;
+                ProdLoad nxt;
+                if (has_next) {
+                    if (un != u) uin = unit_index(un, A);
+                    prod_issue_loads(nxt, A, uin, kbn, c, rbase);
+                }
+                float s8[8] = {cur.s0.x, cur.s0.y, cur.s0.z, cur.s0.w, cur.s1.x, cur.s1.y, cur.s1.z, cur.s1.w};
+                float r8[8] = {cur.r0.x, cur.r0.y, cur.r0.z, cur.r0.w, cur.r1.x, cur.r1.y, cur.r1.z, cur.r1.w};
+                uint4 outv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
+                    outv[i] = prod_compute_row(cur.w[i], cur.prm[i], s8, r8, A.qmax, n < A.N);
+                }
+                if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) break;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t row = rbase + 32 * i;
+                    *reinterpret_cast<uint4 *>(&S.a[as][sw128_offset(row, c)]) = outv[i];
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.a_full[as]);
+                if (++as == AS) { as = 0; aph ^= 1u; }
+                if (!has_next) break;
+                u = un; kb = kbn; ui = uin; cur = nxt;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == TMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+}  // namespace srch
+
+// ===========================================================================
+// a6 (reduction). losses[i] = RN32(sum over token blocks and rows of the
+// partials, in binary64 and a fixed order, / (N T)); optional per-row sums.
+// One block per alpha.
+// ===========================================================================
+__global__ void __launch_bounds__(256)
+loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int n_tb,
+                   float *__restrict__ losses, float *__restrict__ row_losses) {
+    const int ai = blockIdx.x;
+    const float *p = partial + (int64_t)ai * n_tb * N;
+    double acc = 0.0;
+    for (int64_t n = threadIdx.x; n < N; n += blockDim.x) {
+        float rsum = 0.0f;
+        double dsum = 0.0;
+        for (int tb = 0; tb < n_tb; ++tb) {
+            const float v = p[(int64_t)tb * N + n];
+            rsum = __fadd_rn(rsum, v);
+            dsum = __dadd_rn(dsum, (double)v);
+        }
+        if (row_losses) row_losses[(int64_t)ai * N + n] = rsum;
+        acc = __dadd_rn(acc, dsum);
+    }
+    __shared__ double red[256];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int off = 128; off > 0; off >>= 1) {
+        if ((int)threadIdx.x < off) red[threadIdx.x] = __dadd_rn(red[threadIdx.x], red[threadIdx.x + off]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) losses[ai] = __double2float_rn(red[0] / ((double)N * (double)T));
+}
+
+// ===========================================================================
+// a7. Argmin over the grid (first index, NaN = +inf) and s at the best alpha.
+// Every block re-derives the argmin from the n_alpha losses (no host round trip).
+// ===========================================================================
+__device__ __forceinline__ int argmin_losses(const float *losses, int n) {
+    int best = 0;
+    float bv = INFINITY;
+    bool have = false;
+    for (int i = 0; i < n; ++i) {
+        float v = losses[i];
+        if (isnan(v)) v = INFINITY;
+        if (!have || v < bv) { bv = v; best = i; have = true; }
+    }
+    return best;
+}
+
+__global__ void best_scale_kernel(const float *__restrict__ a, int64_t K,
+                                  const float *__restrict__ alphas,
+                                  const float *__restrict__ losses, int n_alpha,
+                                  int32_t *__restrict__ best_idx, float *__restrict__ s_best) {
+    __shared__ int sb;
+    if (threadIdx.x == 0) {
+        sb = argmin_losses(losses, n_alpha);
+        if (blockIdx.x == 0) *best_idx = sb;
+    }
+    __syncthreads();
+    const float al = alphas[sb];
+    if (!(al >= 0.0f && al <= 1.0f) && threadIdx.x == 0) atomicOr(&g_dev_error, kDevErrBadAlpha);
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < K;
+         j += (int64_t)gridDim.x * blockDim.x) {
+        const float aj = fmaxf(a[j], FLT_MIN);
+        s_best[j] = __double2float_rn(pow((double)aj, (double)al));
+    }
+}
+
+// ===========================================================================
+// a8. Pack: per (row, group) recompute w' = RN32(w s_best), the group's
+// parameters and every code; store codes LSB-first, fp16 scale and zero
+// ([AWQ-note] "Measures": keep the quantized weights and their metadata).
+// Each thread owns 16 consecutive columns: two 32-bit words of 4-bit
+// containers (w_bit 3/4) or one word of 2-bit containers (w_bit 2).
+// ===========================================================================
+template <int TPG>
+__global__ void __launch_bounds__(256)
+pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
+            const float *__restrict__ s_best, uint32_t *__restrict__ codes,
+            __half *__restrict__ scales, __half *__restrict__ zeros) {
+    const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
+    const int sub = threadIdx.x % TPG;
+    const bool active = gid < N * (int64_t)G;
+    const int64_t n = active ? gid / G : 0;
+    const int grp = active ? (int)(gid - n * G) : 0;
+    const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
+    const float qmax = (float)((1 << bits) - 1);
+    float wp[16];
+    {
+        uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
+        uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
+        const __half *h0 = reinterpret_cast<const __half *>(&v0);
+        const __half *h1 = reinterpret_cast<const __half *>(&v1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float sv = active ? __ldg(s_best + k0 + e) : 1.0f;
+            wp[e] = __fmul_rn(__half2float(e < 8 ? h0[e] : h1[e - 8]), sv);
+        }
+    }
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) { mn = fminf(mn, wp[e]); mx = fmaxf(mx, wp[e]); }
+#pragma unroll
+    for (int off = 1; off < TPG; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    const QParams p = make_qparams(mn, mx, qmax);
+    const QElem qe = make_qelem(p, qmax);
+    if (!active) return;
+    if (bits == 2) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) word |= quant_code(wp[e], qe, p.z) << (2 * e);
+        codes[n * (K / 16) + k0 / 16] = word;
+    } else {
+        uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            w0 |= quant_code(wp[e], qe, p.z) << (4 * e);
+            w1 |= quant_code(wp[8 + e], qe, p.z) << (4 * e);
+        }
+        *reinterpret_cast<uint2 *>(codes + n * (K / 8) + k0 / 8) = make_uint2(w0, w1);
+    }
+    if (sub == 0) {
+        scales[n * G + grp] = __float2half_rn(p.sh);
+        zeros[n * G + grp] = __float2half_rn(p.z);
+    }
+}
+
+}  // namespace awq

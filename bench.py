@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the AWQ per-layer scale search on B200.
+
+One step = one pass of the whole path over one synthetic layer:
+activation statistics -> 20-alpha grid search (tensor cores) -> argmin + pack.
+
+    python bench.py [--gpus N --steps K --warmup W] [--config attn4096] [--impl reference]
+
+Prints ONE JSON line on rank 0.  ``value`` is useful search work
+(2 N K T |grid| flops per layer) divided by the device time of the whole step,
+summed over ranks (each rank quantizes its own layer: weak scaling, no
+collective on the data path).  Inputs live in HBM before the timed region and
+L2 is flushed between steps (the layer's W and X fit in the 126 MB L2).
+
+``--impl reference`` times the CPU oracle as it stands on this host's cores over
+a bounded row sample of the same layer (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "AWQ search TFLOP/s (20-α grid, 4096² layer, T=4096) & % of FP16 TC peak"
+UNIT = "TFLOP/s"
+LAUNCHES_PER_STEP = 7      # act_stats, alpha_scales, group_params, search, loss_reduce, best_scale, pack
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = ROOT / "profiles" / "search_kernel_traffic.json"
+KERNEL_SOURCES = [ROOT / "awq_activation_aware_b200" / "csrc" / f for f in
+                  ("awq_kernels.cuh", "awq_device.cuh", "awq_abi.cu")]
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["awq", "reference"], default="awq")
+    p.add_argument("--config", default="attn4096")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
+    p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(values, world, device):
+    """Element-wise max over ranks of a list of floats."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# host facts
+# ---------------------------------------------------------------------------
+def load_peaks():
+    f = ROOT / "MEASURED_PEAKS.json"
+    if f.exists():
+        d = json.loads(f.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="awq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in Path(self.path).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        loaded = [r for r in rows if (num(r[3]) or 0) > 0.5 * max(power or [0])] or rows
+        sm_loaded = [num(r[1]) for r in loaded if num(r[1]) is not None] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm_loaded) if sm_loaded else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def search_traffic(cfg_name):
+    """DRAM bytes per search launch from a committed ncu capture, or None if the
+    kernel sources changed since it was taken (or there is none)."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    d = json.loads(TRAFFIC_FILE.read_text())
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    e = d.get("per_launch_bytes", {}).get(cfg_name)
+    return None if e is None else float(e)
+
+
+# ---------------------------------------------------------------------------
+# oracle sample (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg, W, X, alphas, rows):
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    a = oracle.act_stats(X)
+    r = oracle.search(W, X, a, cfg.bits, cfg.group, alphas, rows=rows)
+    oracle.pack(W, a, cfg.bits, cfg.group, alphas, r["losses"], rows=rows)
+    return time.perf_counter() - t0
+
+
+def pick_rows(cfg, W, X, alphas, budget_s):
+    import oracle
+    oracle.build()
+    probe = np.arange(8)
+    t0 = time.perf_counter()
+    oracle.search(W, X, oracle.act_stats(X), cfg.bits, cfg.group, alphas[:2], rows=probe)
+    per_row_alpha = (time.perf_counter() - t0) / (8 * 2)
+    rows = int(budget_s / max(per_row_alpha * len(alphas), 1e-9))
+    return max(8, min(cfg.N, rows))
+
+
+def cpu_measure(cfg, W, X, alphas, args):
+    rows_n = args.cpu_rows or pick_rows(cfg, W, X, alphas, args.cpu_budget_s)
+    rows = np.linspace(0, cfg.N - 1, rows_n).astype(np.int64)
+    dt = oracle_sample(cfg, W, X, alphas, rows)
+    flops = 2.0 * rows_n * cfg.K * cfg.T * len(alphas)
+    return flops / dt / 1e12, dt, rows_n
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+def config_dict(cfg, n_alpha, extra=None):
+    d = {"workload": f"{cfg.name}, {n_alpha}-alpha grid", "N": cfg.N, "K": cfg.K, "T": cfg.T,
+         "bits": cfg.bits, "group_size": cfg.group, "n_alpha": n_alpha,
+         "inputs": "seeded synthetic: W ~ N(0, %g^2) fp16; X ~ N(0,1) fp16 with %d outlier channels x10-100"
+                   % (cfg.w_std, cfg.n_outliers),
+         "l2": "flushed between steps (256 MiB write)"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def run_reference(args):
+    from awq_activation_aware_b200 import synth
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[args.config]
+    W, X, _ = synth.generate(cfg)
+    alphas = synth.default_alphas()
+    per_step = max(2.0, args.cpu_budget_s * 6 / max(args.steps + args.warmup, 1))
+    rows_n = args.cpu_rows or pick_rows(cfg, W, X, alphas, per_step)
+    rows = np.linspace(0, cfg.N - 1, rows_n).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, W, X, alphas, rows)
+    times = [oracle_sample(cfg, W, X, alphas, rows) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    flops = 2.0 * rows_n * cfg.K * cfg.T * len(alphas)
+    value = flops / t / 1e12
+    sample = f"{rows_n} of {cfg.N} rows of W, all {cfg.K} columns, all {cfg.T} tokens, all {len(alphas)} alphas"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(cfg, len(alphas)),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_awq(args):
+    import torch
+
+    import awq_activation_aware_b200 as awq
+    from awq_activation_aware_b200 import synth
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    base = synth.CONFIGS[args.config]
+    # every rank quantizes its own layer of the same shape (independent problems)
+    cfg = synth.LayerConfig(**{**base.as_dict(), "seed": base.seed + 1000 * rank})
+    W, X, _ = synth.generate(cfg)
+    alphas_np = synth.default_alphas()
+    n_alpha = len(alphas_np)
+    flops = 2.0 * cfg.N * cfg.K * cfg.T * n_alpha
+
+    W_h = torch.from_numpy(W).pin_memory()
+    X_h = torch.from_numpy(X).pin_memory()
+    Wd = W_h.to(dev)
+    Xd = X_h.to(dev)
+    alphas = torch.from_numpy(alphas_np).to(dev)
+    ws = torch.empty(awq.search_workspace_bytes(cfg.N, cfg.K, cfg.T, cfg.bits, cfg.group, n_alpha),
+                     dtype=torch.uint8, device=dev)
+    losses = torch.empty(n_alpha, dtype=torch.float32, device=dev)
+    per = 16 if cfg.bits == 2 else 8
+    out = dict(best_idx=torch.empty(1, dtype=torch.int32, device=dev),
+               s_best=torch.empty(cfg.K, dtype=torch.float32, device=dev),
+               codes=torch.empty((cfg.N, cfg.K // per), dtype=torch.int32, device=dev),
+               scales=torch.empty((cfg.N, cfg.K // cfg.group), dtype=torch.float16, device=dev),
+               zeros=torch.empty((cfg.N, cfg.K // cfg.group), dtype=torch.float16, device=dev))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(prof=None):
+        a = awq.act_stats(Xd)
+        if prof is not None:
+            awq.profile_next_search(*prof)
+        awq.search_layer(Wd, Xd, a, alphas, cfg.bits, cfg.group, workspace=ws, losses_out=losses)
+        awq.pack(Wd, a, alphas, losses, cfg.bits, cfg.group, out=out)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    awq.get_status()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for b, e in sev:          # materialise the events before handing their handles to the library
+        b.record(stream)
+        e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier(world)
+    if sampler:
+        sampler.start()
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(prof=sev[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    awq.get_status()
+    step_ms = [b.elapsed_time(e) for b, e in ev]
+    search_ms = [b.elapsed_time(e) for b, e in sev]
+    total_ms, search_avg = reduce_max([sum(step_ms), sum(search_ms) / K], world, dev)
+    ms_per_step = total_ms / K
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    long_region = total_ms > 1000.0
+    peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+    achieved = flops / (search_avg * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": search_traffic(args.config),
+                "kernel": "search_kernel (tcgen05 f16 MMA + fused quantize producer + loss epilogue)",
+                "peak_source": f"{peak_src} {'sustained' if long_region else 'burst'} bf16 dense "
+                               f"(fp16 has the same nominal dense rate)",
+                "search_ms": search_avg}
+
+    # end to end through the public API with host buffers: H2D of W and X, the
+    # path, D2H of losses, best index, s_best, codes, scales and zeros
+    e2e = None
+    if not args.no_e2e:
+        d2h = (n_alpha * 4 + 4 + cfg.K * 4 + cfg.N * cfg.K // per * 4 + 2 * cfg.N * cfg.K // cfg.group * 2)
+        h2d = W_h.numel() * 2 + X_h.numel() * 2
+        res_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+        loss_h = torch.empty(n_alpha, dtype=torch.float32).pin_memory()
+        Wd2 = torch.empty_like(Wd)
+        Xd2 = torch.empty_like(Xd)
+
+        def e2e_step():
+            Wd2.copy_(W_h, non_blocking=True)
+            Xd2.copy_(X_h, non_blocking=True)
+            a = awq.act_stats(Xd2)
+            awq.search_layer(Wd2, Xd2, a, alphas, cfg.bits, cfg.group, workspace=ws, losses_out=losses)
+            awq.pack(Wd2, a, alphas, losses, cfg.bits, cfg.group, out=out)
+            loss_h.copy_(losses, non_blocking=True)
+            for k in out:
+                res_h[k].copy_(out[k], non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.e2e_steps)]
+        barrier(world)
+        for b, e in ee:
+            flush.zero_()
+            b.record(stream)
+            e2e_step()
+            e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max([sum(b.elapsed_time(e) for b, e in ee) / len(ee)], world, dev)[0]
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cv, dt, rows_n = cpu_measure(cfg, W, X, alphas_np, args)
+        cpu = {"value": cv, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+               "sample": f"{rows_n} of {cfg.N} rows of W x all {cfg.K} columns x all {cfg.T} tokens x "
+                         f"{n_alpha} alphas (+ statistics over all of X and packing of the sampled rows): "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+                "config": config_dict(cfg, n_alpha, {"parallelism": f"{world} independent layers"
+                                                     if world > 1 else "1 GPU"}),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": LAUNCHES_PER_STEP * K, "clocks": clocks,
+                "pct_of_peak": 100.0 * value / peak}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_awq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

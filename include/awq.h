@@ -1,0 +1,175 @@
+/*
+ * awq.h -- C ABI of the B200 (sm_100a) AWQ per-layer scale search.
+ *
+ * The operation: for one linear layer with fp16 weights W[N,K] and calibration
+ * activations X[T,K], take the per-input-channel activation magnitudes
+ * a_j = mean_t |X[t,j]|; for every alpha of a grid form s_j = a_j^alpha, quantize
+ * W*diag(s) group-wise along K with round-to-nearest, dequantize and divide by
+ * s, score the output error ||(W_hat - W) X^T||^2, keep the best alpha, and
+ * emit packed low-bit codes with fp16 scales and zero points.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [QAS-QA]   "Как работает quantization-aware scaling в AWQ для защиты важных
+ *              весов?" -- §5 mechanism, §6 objective (MSE), §9 quant_config
+ *              {zero_point, q_group_size, w_bit}
+ *   [AWQ-note] "AWQ: Activation-Aware Weight Quantization For On-Device LLM
+ *              Compression AND Acceleration" -- section "Measures"
+ *   [GPTQ-AWQ] "GPTQ与AWQ" -- section "量化方法" (W is (out_features,
+ *              in_features), X is (batch, in_features))
+ *   [AWQ-wiki] "AWQ" (French encyclopedia page) -- "Fondements techniques"
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers owned by the caller unless stated; the
+ *     library never allocates, frees or retains them.  fp16 data is IEEE
+ *     binary16 passed as `const void*`.  Every pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are stream-ordered and asynchronous; the returned status covers argument
+ *     validation and launch errors only.  Errors raised while kernels run
+ *     (a bounded wait that ran out) are reported by awq_get_status().
+ *   - Matrices are row-major.  W rows are contiguous (row stride K); X rows
+ *     have stride ldx >= K elements, ldx a multiple of 8.
+ *   - Sizes: 1 <= N, T <= 2^31 - 1; K a multiple of group_size.
+ *   - Invalid arguments return AWQ_ERR_INVALID_ARG before anything is launched.
+ *   - Calls are thread-safe and keep no state between calls, except the
+ *     device error word read and cleared by awq_get_status().
+ */
+#ifndef AWQ_B200_AWQ_H
+#define AWQ_B200_AWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AWQ_OK = 0,
+    AWQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or config        */
+    AWQ_ERR_UNSUPPORTED = 2,   /* no sm_100 device, or a config not implemented  */
+    AWQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed           */
+    AWQ_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (device flag)  */
+    AWQ_ERR_WORKSPACE = 5      /* workspace missing or smaller than required     */
+} awq_status;
+
+/* Quantizer configuration ([QAS-QA] §9 quant_config):
+ *   bits        w_bit, one of 2, 3, 4  (codes 0 .. 2^bits - 1)
+ *   group_size  q_group_size along K, one of 64, 128
+ *   zero_point  must be 1 (asymmetric quantization with a zero point)        */
+typedef struct {
+    int32_t bits;
+    int32_t group_size;
+    int32_t zero_point;
+} awq_qcfg;
+
+/* Step a1 -- activation statistics ([AWQ-note] "Measures": average absolute
+ * activation per input channel; [GPTQ-AWQ] "量化方法": X.abs().mean(dim=0)).
+ *   X   fp16 [T, ldx] (only the first K columns are read)
+ *   a   float [K] output: a_j = RN32(RN64(sum_t |X[t,j]|) / T).  The column
+ *       sum is accumulated exactly (binary64 holds every partial sum while
+ *       T * max|x| < 2^29), so the result is independent of summation order.
+ * Requires K % 8 == 0. */
+AWQ_API awq_status awq_act_stats(const void *X, int64_t T, int64_t K, int64_t ldx,
+                         float *a, void *stream);
+
+/* Step a2 -- the search space s = a^alpha ([AWQ-note] "Measures": for each
+ * candidate alpha compute a^alpha).
+ *   a       float [K]
+ *   alphas  float [n_alpha], every value in [0, 1]  (device pointer)
+ *   s       float [n_alpha, K] output: s[i,j] = RN32(pow(max(a_j, FLT_MIN), alpha_i))
+ *           evaluated in binary64 (alpha = 0 gives exactly 1).
+ * 1 <= n_alpha <= 64.  An alpha outside [0, 1] raises AWQ_ERR_INVALID_ARG
+ * through awq_get_status(). */
+AWQ_API awq_status awq_alpha_scales(const float *a, int64_t K, const float *alphas, int32_t n_alpha,
+                            float *s, void *stream);
+
+/* Steps a3/a4 standalone -- scale, group-wise asymmetric round-to-nearest,
+ * dequantize, unscale ([QAS-QA] §5; [AWQ-wiki] "Fondements techniques": the
+ * inverse scaling is applied after dequantization).  For one scale vector s:
+ *   per row n and group G of group_size columns:
+ *     w'    = RN32(w * s)
+ *     scale = RN32(RN32(max w' - min w') / qmax),  sh = RN16(clamp(scale, 2^-24, 65504))
+ *     r     = RN32(1 / sh),  z = clamp(rint(RN32(-min w' * r)), 0, qmax)
+ *     q     = clamp(rint(RN32(w' * r)) + z, 0, qmax)
+ *     w_hat = RN16(RN32(RN32((q - z) * sh) * RN32(1 / s)))
+ *   W      fp16 [N, K];  s  float [K];  W_hat  fp16 [N, K] output.
+ * This is the exact per-element function the search evaluates for every
+ * alpha; it never runs inside the search (the search keeps W_hat on chip). */
+AWQ_API awq_status awq_quant_dequant(const void *W, int64_t N, int64_t K, const float *s,
+                             awq_qcfg q, void *W_hat, void *stream);
+
+/* Bytes of device workspace awq_search_layer needs for these sizes. */
+AWQ_API size_t awq_search_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q,
+                                  int32_t n_alpha);
+
+/* Steps a2-a6 -- the grid search ([AWQ-note] "Measures": collect X, take
+ * a = mean|x|, compute a^alpha for each candidate alpha and measure the error;
+ * Δy = (W_hat - W) x; [QAS-QA] §6: minimise the MSE between the outputs of the
+ * original and the quantized layer on calibration data).
+ *   W           fp16 [N, K]
+ *   X           fp16 [T, ldx]
+ *   a           float [K]  (awq_act_stats output, or any positive statistics)
+ *   alphas      float [n_alpha] in [0, 1]
+ *   losses      float [n_alpha] output: MSE_i = ||(W_hat_i - W) X^T||_F^2 / (N T)
+ *   row_losses  float [n_alpha, N] output or NULL: per-row sums
+ *               sum_t ((W_hat_i - W) X^T)[n, t]^2 (unnormalised)
+ *   ws          device workspace of ws_bytes >= awq_search_workspace_bytes(...)
+ * Requires K % 64 == 0 and 1 <= n_alpha <= 64.  The error matrix is never
+ * written to memory: a tensor-core kernel forms (W_hat - W) X^T tile by tile in
+ * tensor memory and reduces its squares on chip. */
+AWQ_API awq_status awq_search_layer(const void *W, int64_t N, int64_t K,
+                            const void *X, int64_t T, int64_t ldx,
+                            const float *a, awq_qcfg q,
+                            const float *alphas, int32_t n_alpha,
+                            float *losses, float *row_losses,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* Steps a7-a8 -- argmin over the grid and packing ([AWQ-note] "Measures":
+ * scale by the best alpha's s, group-quantize, keep the quantized weights and
+ * the necessary metadata).
+ *   best_idx  int32 [1] output: first index of the smallest loss (NaN = +inf)
+ *   s_best    float [K] output: s at the best alpha
+ *   codes     uint32 [N, K*c/32] output, c = 4 for bits 3/4 (8 codes per word),
+ *             c = 2 for bits 2 (16 per word); code of column k at bit c*(k mod 32/c)
+ *             of word k/(32/c) (least significant first)
+ *   scales    fp16 [N, K/group_size] output: sh per group
+ *   zeros     fp16 [N, K/group_size] output: z per group (an integer code)
+ * The argmin runs on the device; nothing is read back to the host.
+ * Dequantization: w_hat = RN16(RN32(RN32((code - zero) * scale) * RN32(1/s_best))). */
+AWQ_API awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcfg q,
+                    const float *alphas, const float *losses, int32_t n_alpha,
+                    int32_t *best_idx, float *s_best, uint32_t *codes,
+                    void *scales, void *zeros, void *stream);
+
+/* Synchronises `stream`, then reports (and clears) errors raised on the device
+ * since the last call: AWQ_ERR_TIMEOUT if a kernel's bounded wait ran out,
+ * AWQ_ERR_INVALID_ARG if a kernel saw an alpha outside [0, 1], AWQ_ERR_CUDA for
+ * a pending CUDA error.  AWQ_OK otherwise. */
+AWQ_API awq_status awq_get_status(void *stream);
+
+/* Upper bound, in milliseconds, on any single wait inside the library's
+ * kernels (default 4000).  Applies to launches made after the call. */
+AWQ_API void awq_set_wait_timeout_ms(uint32_t ms);
+
+/* Profiling hook.  The next awq_search_layer call made by the calling thread
+ * records `ev_begin` immediately before and `ev_end` immediately after the
+ * launch of its tensor-core search kernel, on that call's stream, so a caller
+ * can time that kernel alone with cudaEventElapsedTime.  Both are cudaEvent_t
+ * created by the caller; NULL clears the request.  The request is consumed by
+ * that one call. */
+AWQ_API void awq_profile_next_search(void *ev_begin, void *ev_end);
+
+/* A static, human-readable name for a status code. */
+AWQ_API const char *awq_status_string(awq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_AWQ_H */

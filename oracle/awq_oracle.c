@@ -170,7 +170,7 @@ void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s
             double sh = awq_oracle_h2d(shb);
             float r = rn32(1.0 / sh);
             double z = nearbyint((double)rn32(-(double)mn * (double)r));
-            if (z < 0.0) z = 0.0;
+            if (!(z > 0.0)) z = 0.0;        /* a code in [0, qmax]: never -0 */
             if (z > qmax) z = qmax;
             if (sh_out) sh_out[n * G + gi] = shb;
             if (z_out) z_out[n * G + gi] = (float)z;

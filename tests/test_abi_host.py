@@ -1,0 +1,96 @@
+"""The C-ABI library on the host: it loads, exports every entry point that
+include/awq.h declares, sizes its workspace, and rejects bad arguments before
+touching the GPU (so these run without one)."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import awq_activation_aware_b200 as awq
+from awq_activation_aware_b200 import QCfg
+
+ROOT = Path(__file__).resolve().parents[1]
+
+BOGUS = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def declared_symbols():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        names |= set(re.findall(r"AWQ_API\s+[\w\s\*]+?\b(awq_\w+)\s*\(", h.read_text()))
+    return names
+
+
+def test_library_builds_and_loads():
+    from awq_activation_aware_b200 import build
+    build.build()
+    assert awq.LIB_PATH.exists()
+    assert awq.lib() is not None
+
+
+def test_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert names >= {"awq_act_stats", "awq_search_layer", "awq_pack"}
+    L = awq.lib()
+    for n in sorted(names):
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    L = awq.lib()
+    for code, name in awq.STATUS.items():
+        assert L.awq_status_string(code).decode() == name
+
+
+def test_workspace_size():
+    ws = awq.search_workspace_bytes(4096, 4096, 4096, 4, 128, 20)
+    # s and 1/s tables, 8-byte group parameters, fp32 partials per 512-token block
+    expect = 2 * 20 * 4096 * 4 + 20 * 32 * 4096 * 8 + 20 * 8 * 4096 * 4
+    assert expect <= ws <= expect + 4 * 256
+    assert awq.search_workspace_bytes(100, 100, 10, 4, 128, 20) == 0      # K not a multiple of g
+    assert awq.search_workspace_bytes(64, 128, 10, 5, 128, 20) == 0       # bits 5 unsupported
+
+
+def _search(**kw):
+    args = dict(W=BOGUS, N=256, K=512, X=BOGUS, T=512, ldx=512, a=BOGUS, q=QCfg(4, 128, 1), alphas=BOGUS,
+                n_alpha=20, losses=BOGUS, row_losses=None, ws=BOGUS, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return awq.lib().awq_search_layer(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(W=None), dict(X=None), dict(a=None), dict(alphas=None), dict(losses=None),
+    dict(W=MISALIGNED), dict(row_losses=MISALIGNED),
+    dict(N=0), dict(T=0), dict(K=100), dict(K=96), dict(ldx=500), dict(ldx=516),
+    dict(q=QCfg(5, 128, 1)), dict(q=QCfg(4, 32, 1)), dict(q=QCfg(4, 128, 0)), dict(q=QCfg(4, 128, 1), K=192),
+    dict(n_alpha=0), dict(n_alpha=65), dict(N=1 << 31),
+])
+def test_search_rejects_bad_arguments(bad):
+    assert _search(**bad) == 1   # AWQ_ERR_INVALID_ARG
+
+
+def test_search_rejects_small_workspace():
+    assert _search(ws_bytes=1024) == 5               # AWQ_ERR_WORKSPACE
+    assert _search(ws=None) == 5
+    assert _search(ws=ctypes.c_void_p(0x10010)) == 5  # not 256-byte aligned
+
+
+def test_other_entry_points_reject_bad_arguments():
+    L = awq.lib()
+    assert L.awq_act_stats(None, 16, 64, 64, BOGUS, None) == 1
+    assert L.awq_act_stats(BOGUS, 16, 60, 64, BOGUS, None) == 1      # K % 8
+    assert L.awq_act_stats(BOGUS, 0, 64, 64, BOGUS, None) == 1
+    assert L.awq_alpha_scales(BOGUS, 64, BOGUS, 0, BOGUS, None) == 1
+    assert L.awq_quant_dequant(BOGUS, 4, 100, BOGUS, QCfg(4, 128, 1), BOGUS, None) == 1
+    assert L.awq_pack(BOGUS, 4, 128, BOGUS, QCfg(3, 64, 1), BOGUS, BOGUS, 20, BOGUS, BOGUS, MISALIGNED,
+                      BOGUS, BOGUS, None) == 1
+    assert L.awq_pack(BOGUS, 4, 128, BOGUS, QCfg(3, 64, 1), BOGUS, BOGUS, 99, BOGUS, BOGUS, BOGUS,
+                      BOGUS, BOGUS, None) == 1
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        awq.act_stats(torch.zeros((4, 64), dtype=torch.float16))
