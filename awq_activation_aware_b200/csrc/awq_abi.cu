@@ -139,6 +139,27 @@ awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, c
     return last_launch();
 }
 
+// Scratch for awq_search_layer_noalloc: lives in the library's device image,
+// so no allocation happens at call time.  In host code `g_noalloc_scratch` is
+// only a stand-in symbol, never a device address: the address is looked up
+// once per device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[AWQ_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};
+
+awq_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return AWQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return AWQ_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return AWQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -274,6 +295,20 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
     // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
     awq::loss_reduce_kernel<<<n_alpha, 256, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
     return last_launch();
+}
+
+awq_status awq_search_layer_noalloc(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx,
+                                    const float *a, awq_qcfg q, const float *alphas, int32_t n_alpha,
+                                    float *losses, float *row_losses, void *stream) {
+    const size_t need = awq_search_workspace_bytes(N, K, T, q, n_alpha);
+    if (need == 0) return AWQ_ERR_INVALID_ARG;
+    if (need > AWQ_NOALLOC_SCRATCH_BYTES) return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    void *ws = nullptr;
+    if (awq_status e = noalloc_scratch(&ws)) return e;
+    return awq_search_layer(W, N, K, X, T, ldx, a, q, alphas, n_alpha, losses, row_losses, ws,
+                            AWQ_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcfg q, const float *alphas,

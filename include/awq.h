@@ -130,6 +130,43 @@ AWQ_API awq_status awq_search_layer(const void *W, int64_t N, int64_t K,
                             float *losses, float *row_losses,
                             void *ws, size_t ws_bytes, void *stream);
 
+/* Size of the scratch array built into the library for
+ * awq_search_layer_noalloc: 32 MiB of device memory. */
+#define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* awq_search_layer without a caller-provided workspace.  (The pages have no
+ * counterpart: this is a property of the library's interface, not of AWQ.)
+ *
+ * For callers that cannot allocate device memory when they call the search:
+ * plugin or callback code that runs inside another runtime's execution step
+ * (where allocating, and the device synchronisation cudaMalloc may imply, is
+ * not allowed), programs that reserved their whole device-memory budget at
+ * start-up, and latency-critical paths that must not wait on an allocator.
+ *
+ * Arguments and results are exactly those of awq_search_layer minus `ws` and
+ * `ws_bytes`; the caller still provides W, X, a, alphas, losses and
+ * row_losses.  The scratch is a file-scope device array of
+ * AWQ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library's kernels holds until the process exits.  This call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on that device.
+ *   - Layers whose awq_search_workspace_bytes(...) exceeds
+ *     AWQ_NOALLOC_SCRATCH_BYTES are rejected with AWQ_ERR_WORKSPACE before
+ *     anything is launched.  (The 4096 x 4096, T = 4096, 20-alpha layer needs
+ *     about 24 MiB.)
+ *   - Every call shares the one array and it keeps the last call's contents.
+ *     Nothing in it has to start at zero: each call writes every byte it later
+ *     reads.  Calls whose kernels overlap on the GPU (different streams, or
+ *     threads without ordering between their streams) race on the array and
+ *     corrupt each other's results: order them, e.g. on one stream. */
+AWQ_API awq_status awq_search_layer_noalloc(const void *W, int64_t N, int64_t K,
+                                            const void *X, int64_t T, int64_t ldx,
+                                            const float *a, awq_qcfg q,
+                                            const float *alphas, int32_t n_alpha,
+                                            float *losses, float *row_losses, void *stream);
+
 /* Steps a7-a8 -- argmin over the grid and packing ([AWQ-note] "Measures":
  * scale by the best alpha's s, group-quantize, keep the quantized weights and
  * the necessary metadata).
