@@ -23,6 +23,7 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo",
+    "-fmad=false",          # no implicit multiply-add contraction: every FMA in the code is explicit
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "-shared", "-cudart", "static",
     "-Xptxas", "-v",

@@ -112,6 +112,67 @@ __device__ __forceinline__ __half dequant_unscale(float wp, const QElem &e, floa
     return __float2half_rn(__fmul_rn(dequant_code_times_scale(wp, e), rs));
 }
 
+// Packed binary32 pair arithmetic (sm_100 FMUL2/FADD2/FFMA2).  Written as PTX
+// with an explicit .rn rounding modifier: such instructions are never
+// contracted into a fused multiply-add, so each one rounds exactly once, as
+// the quantizer's definition requires.  (A contracted w'*r + kMagic would
+// decide ties of rint from the unrounded product.)
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// The same quantize-dequantize-unscale for two neighbouring weights in packed
+// binary32 pairs, as the search producer evaluates it.  Per pair:
+// w' = RN32(w s), t = RN32(w' r) clamped to [-z, qmax - z], v = RN32(t + kMagic)
+// (= kMagic + rint(t), ties to even), (q - z) sh = fma(v, sh, -kMagic sh),
+// w_hat = RN16(RN32(((q - z) sh) rs)).  The clamp sits between the product and
+// the magic add on purpose: the two must never be fused into one FMA, which
+// would decide ties of rint from the unrounded product (the library is also
+// built with contraction off).
+struct QPair {
+    float2 r, magic, sh, nmsh;
+    float lo, hi;
+};
+__device__ __forceinline__ QPair make_qpair(const QParams &p, float qmax) {
+    QPair q;
+    q.r = make_float2(p.r, p.r);
+    q.magic = make_float2(kMagic, kMagic);
+    q.sh = make_float2(p.sh, p.sh);
+    const float nm = __fmul_rn(-kMagic, p.sh);
+    q.nmsh = make_float2(nm, nm);
+    q.lo = -p.z;
+    q.hi = __fsub_rn(qmax, p.z);
+    return q;
+}
+__device__ __forceinline__ __half2 dequant_unscale_pair(float2 w, float2 s, float2 rs, const QPair &q) {
+    float2 t = mul2_rn(mul2_rn(w, s), q.r);
+    t.x = fminf(fmaxf(t.x, q.lo), q.hi);
+    t.y = fminf(fmaxf(t.y, q.lo), q.hi);
+    const float2 v = add2_rn(t, q.magic);
+    return __float22half2_rn(mul2_rn(fma2_rn(v, q.sh, q.nmsh), rs));
+}
+
 // ---------------------------------------------------------------------------
 // Small PTX helpers
 // ---------------------------------------------------------------------------
@@ -169,15 +230,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` elapse, instead of spinning on the barrier.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: returns false (after raising the device timeout flag and the
 // CTA's abort flag) when the phase does not complete within `limit_ns`, or
-// when another role of the CTA has already aborted.  Never traps.
+// when another role of the CTA has already aborted.  Never traps.  Waiting
+// threads are suspended by the hardware between checks, so a long wait costs
+// almost no issue slots.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
@@ -207,6 +284,13 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, in
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// One 16-byte shared-memory store (a single 128-bit access per thread).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
@@ -256,26 +340,32 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
         : "memory");
 }
 
-// 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives lane
-// (warp quadrant base + i), columns col .. col+31.
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// 32 lanes x 64 consecutive fp32 columns: thread i of the warp receives lane
+// (warp quadrant base + i), columns col .. col+63.  The load and its
+// tcgen05.wait::ld sit in ONE asm statement: the destination registers of an
+// asynchronous tcgen05.ld are undefined until the wait, and separate
+// statements would let the compiler schedule their uses above the wait.
+__device__ __forceinline__ void tmem_ld_32x32b_x64_sync(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr));
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Shared-memory matrix descriptor for a K-major operand stored in the

@@ -201,7 +201,7 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
     const int64_t n = active ? gid / G : 0;
     const int grp = active ? (int)(gid - n * G) : 0;
     const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
-    float wp[16], rs[16];
+    float wv[16], sv[16], wp[16], rs[16];
     {
         uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
         uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
@@ -209,10 +209,10 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
         const __half *h1 = reinterpret_cast<const __half *>(&v1);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float sv = active ? __ldg(s + k0 + e) : 1.0f;
-            const float wv = __half2float(e < 8 ? h0[e] : h1[e - 8]);
-            wp[e] = __fmul_rn(wv, sv);
-            rs[e] = __frcp_rn(sv);
+            sv[e] = active ? __ldg(s + k0 + e) : 1.0f;
+            wv[e] = __half2float(e < 8 ? h0[e] : h1[e - 8]);
+            wp[e] = __fmul_rn(wv[e], sv[e]);
+            rs[e] = __frcp_rn(sv[e]);
         }
     }
     float mn = INFINITY, mx = -INFINITY;
@@ -223,14 +223,15 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
-    const QParams p = make_qparams(mn, mx, qmax);
-    const QElem qe = make_qelem(p, qmax);
+    const QPair qp = make_qpair(make_qparams(mn, mx, qmax), qmax);
     if (!active) return;
-    __align__(16) __half out[16];
+    __align__(16) __half2 out[8];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) out[e] = dequant_unscale(wp[e], qe, rs[e]);
+    for (int e = 0; e < 8; ++e)
+        out[e] = dequant_unscale_pair(make_float2(wv[2 * e], wv[2 * e + 1]), make_float2(sv[2 * e], sv[2 * e + 1]),
+                                      make_float2(rs[2 * e], rs[2 * e + 1]), qp);
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0) = *reinterpret_cast<const uint4 *>(&out[0]);
-    *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[8]);
+    *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[4]);
 }
 
 // ===========================================================================
@@ -334,19 +335,18 @@ __device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, con
     }
 }
 
-__device__ __forceinline__ uint4 prod_compute_row(const uint4 wv, const uint2 prm, const float (&s)[8],
-                                                  const float (&rs)[8], float qmax, bool valid) {
+// Delta W = W_hat - W (fp16) for 8 consecutive weights of one row, using the
+// packed quantizer of dequant_unscale_pair.
+__device__ __forceinline__ uint4 prod_compute_row(const uint4 wv, const uint2 prm, const float2 (&s)[4],
+                                                  const float2 (&rs)[4], float qmax, bool valid) {
     if (!valid) return make_uint4(0, 0, 0, 0);
-    const QElem e = make_qelem(unpack_qparams(prm), qmax);
+    const QPair q = make_qpair(unpack_qparams(prm), qmax);
     const __half2 *wh = reinterpret_cast<const __half2 *>(&wv);
     uint4 out;
     uint32_t *o = reinterpret_cast<uint32_t *>(&out);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        const float2 wf = __half22float2(wh[p]);
-        const __half h0 = dequant_unscale(__fmul_rn(wf.x, s[2 * p]), e, rs[2 * p]);
-        const __half h1 = dequant_unscale(__fmul_rn(wf.y, s[2 * p + 1]), e, rs[2 * p + 1]);
-        const __half2 d = __hsub2(__halves2half2(h0, h1), wh[p]);
+        const __half2 d = __hsub2(dequant_unscale_pair(__half22float2(wh[p]), s[p], rs[p], q), wh[p]);
         o[p] = *reinterpret_cast<const uint32_t *>(&d);
     }
     return out;
@@ -448,18 +448,18 @@ search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
             const UnitIdx ui = unit_index(u, A);
             if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns)) break;
             tc_fence_after();
-            float sum = 0.0f;
+            float2 sum2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-            for (int c = 0; c < TMEM_COLS / 32; c += 2) {
-                float v0[32], v1[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v0);
-                tmem_ld_32x32b_x32(tmem + lane_base + (c + 1) * 32, v1);
-                tmem_ld_wait();
+            for (int c = 0; c < TMEM_COLS; c += 64) {
+                float v[64];
+                tmem_ld_32x32b_x64_sync(tmem + lane_base + c, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sum = __fmaf_rn(v0[i], v0[i], sum);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sum = __fmaf_rn(v1[i], v1[i], sum);
+                for (int i = 0; i < 64; i += 2) {
+                    const float2 e = make_float2(v[i], v[i + 1]);
+                    sum2 = fma2_rn(e, e, sum2);
+                }
             }
+            const float sum = __fadd_rn(sum2.x, sum2.y);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.acc_empty);
@@ -491,20 +491,20 @@ search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
                     if (un != u) uin = unit_index(un, A);
                     prod_issue_loads(nxt, A, uin, kbn, c, rbase);
                 }
-                float s8[8] = {cur.s0.x, cur.s0.y, cur.s0.z, cur.s0.w, cur.s1.x, cur.s1.y, cur.s1.z, cur.s1.w};
-                float r8[8] = {cur.r0.x, cur.r0.y, cur.r0.z, cur.r0.w, cur.r1.x, cur.r1.y, cur.r1.z, cur.r1.w};
+                const float2 s4[4] = {make_float2(cur.s0.x, cur.s0.y), make_float2(cur.s0.z, cur.s0.w),
+                                      make_float2(cur.s1.x, cur.s1.y), make_float2(cur.s1.z, cur.s1.w)};
+                const float2 r4[4] = {make_float2(cur.r0.x, cur.r0.y), make_float2(cur.r0.z, cur.r0.w),
+                                      make_float2(cur.r1.x, cur.r1.y), make_float2(cur.r1.z, cur.r1.w)};
                 uint4 outv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
-                    outv[i] = prod_compute_row(cur.w[i], cur.prm[i], s8, r8, A.qmax, n < A.N);
+                    outv[i] = prod_compute_row(cur.w[i], cur.prm[i], s4, r4, A.qmax, n < A.N);
                 }
                 if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) break;
+                const uint32_t a_base = smem_u32(&S.a[as][0]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t row = rbase + 32 * i;
-                    *reinterpret_cast<uint4 *>(&S.a[as][sw128_offset(row, c)]) = outv[i];
-                }
+                for (int i = 0; i < 4; ++i) st_shared_v4(a_base + sw128_offset(rbase + 32 * i, c), outv[i]);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.a_full[as]);

@@ -132,6 +132,26 @@ def test_quant_dequant_bit_exact(awq, bits, group):
         assert np.array_equal(got.view(np.uint16), ref.view(np.uint16)), al
 
 
+def test_quant_dequant_every_alpha_large(awq):
+    """All 20 alphas on a 1024 x 1024 layer: about one element in four thousand
+    has w'*r exactly on a half-integer, where a fused multiply-add (or any
+    other rounding slip) would flip the code."""
+    W, X = gen(1024, 1024, 256, seed=77)
+    a = oracle.act_stats(X)
+    Wd = dev(W)
+    ties = 0
+    for al in synth.default_alphas():
+        s = oracle.scales(a, float(al))
+        got = host(awq.quant_dequant(Wd, dev(s), 4, 128))
+        ref = oracle.quantize(W, s, 4, 128)
+        assert np.array_equal(got.view(np.uint16), ref["what"].view(np.uint16)), float(al)
+        if float(al) == 0.0:
+            sh = np.repeat(ref["sh"].astype(np.float32), 128, axis=1)
+            t = (W.astype(np.float32) * (np.float32(1) / sh).astype(np.float32)).astype(np.float32)
+            ties = int(np.sum(t - np.floor(t) == 0.5))
+    assert ties > 0          # the case really exercises exact ties
+
+
 # ---------------------------------------------------------------------------
 # a2-a6: the search
 # ---------------------------------------------------------------------------
