@@ -37,86 +37,67 @@ constexpr float kMaxScale = 65504.0f;                  // largest finite fp16
 // Per-(row, group) quantizer parameters derived from the group's min and max of
 // w' = RN32(w*s) ([QAS-QA] §9: zero_point = True, q_group_size, w_bit):
 //   scale = RN32(RN32(mx - mn) / qmax), sh = RN16(clamp(scale, 2^-24, 65504)),
-//   r = RN32(1/sh), z = clamp(rint(RN32(-mn * r)), 0, qmax).
+//   r = RN32(1/sh), z = clamp(rint(-mn * r), 0, qmax),
+// where every product inside rint is exact (rint is the only rounding of
+// w'/scale).  RN32(x + kMagic) with x an exact product is kMagic + rint(x) for
+// |x| <= 2^22 and is monotone in x, so one FMA with kMagic evaluates rint of an
+// exact product, and clamping in that shifted domain clamps the code.
+// `clamp` records whether any code of the group needs clamping:
+// rint(mn r) + z < 0 or rint(mx r) + z > qmax.  The rounding is monotone in w',
+// so when neither end needs it no element of the group does.
 struct QParams {
     float r;     // reciprocal of the stored fp16 scale
     float sh;    // the stored fp16 scale, as binary32
-    float z;     // zero point, an integer in [0, qmax]
+    float z;     // zero point, an integer in [0, qmax] (never -0)
+    bool clamp;  // some code of the group leaves [0, qmax] before clamping
 };
 
 __device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax) {
     QParams p;
-    float range = __fsub_rn(mx, mn);
+    const float range = __fsub_rn(mx, mn);
     float scale = __fdiv_rn(range, qmax);
     scale = fminf(fmaxf(scale, kMinScale), kMaxScale);
     p.sh = __half2float(__float2half_rn(scale));
     p.r = __frcp_rn(p.sh);
-    const float zr = rintf(__fmul_rn(-mn, p.r));
-    p.z = zr > 0.0f ? fminf(zr, qmax) : 0.0f;   // a code in [0, qmax]; never -0
+    const float top = __fadd_rn(kMagic, qmax);
+    const float vz = __fmaf_rn(-mn, p.r, kMagic);
+    p.z = __fsub_rn(fminf(fmaxf(vz, kMagic), top), kMagic);
+    const float vmn = __fmaf_rn(mn, p.r, kMagic);
+    const float vmx = __fmaf_rn(mx, p.r, kMagic);
+    p.clamp = (vmn < __fsub_rn(kMagic, p.z)) || (vmx > __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));
     return p;
 }
 
-// Compact 8-byte form kept in the search workspace: r as binary32, the fp16
-// scale bits and the zero point.
+// Compact 8-byte form kept in the search workspace: r as binary32, then the
+// fp16 scale and the fp16 zero point whose sign bit carries the clamp flag
+// (so one half2 -> float2 conversion unpacks both).
 __device__ __forceinline__ uint2 pack_qparams(const QParams &p) {
-    uint16_t shb = __half_as_ushort(__float2half_rn(p.sh));
-    return make_uint2(__float_as_uint(p.r), (uint32_t)shb | ((uint32_t)p.z << 16));
+    const uint32_t shb = __half_as_ushort(__float2half_rn(p.sh));
+    const uint32_t zb = __half_as_ushort(__float2half_rn(p.z)) | (p.clamp ? 0x8000u : 0u);
+    return make_uint2(__float_as_uint(p.r), shb | (zb << 16));
 }
 __device__ __forceinline__ QParams unpack_qparams(uint2 v) {
     QParams p;
     p.r = __uint_as_float(v.x);
-    p.sh = __half2float(__ushort_as_half((unsigned short)(v.y & 0xFFFFu)));
-    p.z = (float)(v.y >> 16);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
+    p.sh = f.x;
+    p.z = fabsf(f.y);
+    p.clamp = (v.y >> 31) != 0;
     return p;
 }
 
-// Element constants derived once per (row, group): clamp bounds of t = w'*r in
-// units of codes relative to the zero point, and -kMagic*sh (exact: kMagic has
-// two significant bits and sh eleven).
-struct QElem {
-    float r, lo, hi, sh, nmsh;
-};
-__device__ __forceinline__ QElem make_qelem(const QParams &p, float qmax) {
-    QElem e;
-    e.r = p.r;
-    e.lo = -p.z;
-    e.hi = __fsub_rn(qmax, p.z);
-    e.sh = p.sh;
-    e.nmsh = __fmul_rn(-kMagic, p.sh);
-    return e;
+// The integer code q = clamp(rint(w' r) + z, 0, qmax) (used by the packer).
+__device__ __forceinline__ uint32_t quant_code(float wp, const QParams &p, float qmax) {
+    float v = __fmaf_rn(wp, p.r, kMagic);
+    v = fminf(fmaxf(v, __fsub_rn(kMagic, p.z)), __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));
+    return (uint32_t)__float2int_rn(__fadd_rn(__fsub_rn(v, kMagic), p.z));
 }
 
-// RN32((q - z) * sh) with q = clamp(rint(RN32(w'*r)) + z, 0, qmax).
-// Because z is an integer, q - z = rint(clamp(RN32(w'*r), -z, qmax - z)); the
-// magic add rounds that value (|.| <= qmax) to an integer, and one FMA turns
-// (v - kMagic) * sh into a single rounding of the exact product (which is
-// itself exact: |q - z| <= 15 and sh has 11 significant bits).
-__device__ __forceinline__ float dequant_code_times_scale(float wp, const QElem &e) {
-    float t = __fmul_rn(wp, e.r);
-    t = fminf(fmaxf(t, e.lo), e.hi);
-    float v = __fadd_rn(t, kMagic);
-    return __fmaf_rn(v, e.sh, e.nmsh);
-}
-
-// The integer code q itself (used by the packer).
-__device__ __forceinline__ uint32_t quant_code(float wp, const QElem &e, float z) {
-    float t = __fmul_rn(wp, e.r);
-    t = fminf(fmaxf(t, e.lo), e.hi);
-    float d = __fsub_rn(__fadd_rn(t, kMagic), kMagic);   // rint(t), exact
-    return (uint32_t)__float2int_rn(__fadd_rn(d, z));
-}
-
-// w_hat = RN16(RN32(RN32((q - z) * sh) * rs)), rs = RN32(1/s)
-// ([AWQ-wiki] "Fondements techniques": the inverse scaling after dequantization).
-__device__ __forceinline__ __half dequant_unscale(float wp, const QElem &e, float rs) {
-    return __float2half_rn(__fmul_rn(dequant_code_times_scale(wp, e), rs));
-}
-
-// Packed binary32 pair arithmetic (sm_100 FMUL2/FADD2/FFMA2).  Written as PTX
-// with an explicit .rn rounding modifier: such instructions are never
-// contracted into a fused multiply-add, so each one rounds exactly once, as
-// the quantizer's definition requires.  (A contracted w'*r + kMagic would
-// decide ties of rint from the unrounded product.)
+// Packed binary32 pair arithmetic (sm_100 FMUL2/FADD2/FFMA2), as PTX with an
+// explicit .rn rounding modifier.  Each multiply and add must round exactly
+// once where the quantizer's definition says so; the library is built with
+// -fmad=false so that no multiply-add pair is contracted behind our back, and
+// every intended fusion is written as fma2_rn / __fmaf_rn.
 __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -142,17 +123,18 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
     return d;
 }
 
-// The same quantize-dequantize-unscale for two neighbouring weights in packed
-// binary32 pairs, as the search producer evaluates it.  Per pair:
-// w' = RN32(w s), t = RN32(w' r) clamped to [-z, qmax - z], v = RN32(t + kMagic)
-// (= kMagic + rint(t), ties to even), (q - z) sh = fma(v, sh, -kMagic sh),
-// w_hat = RN16(RN32(((q - z) sh) rs)).  The clamp sits between the product and
-// the magic add on purpose: the two must never be fused into one FMA, which
-// would decide ties of rint from the unrounded product (the library is also
-// built with contraction off).
+// Quantize-dequantize-unscale of two neighbouring weights in packed binary32
+// pairs, as the search producer evaluates it:
+//   v = RN32(w' r + kMagic) = kMagic + rint(w' r)      (w' = RN32(w s), one FMA)
+//   v clamped to [kMagic - z, kMagic + qmax - z]        (only when `clamp`)
+//   (q - z) sh = RN32(v sh - kMagic sh)                  (exact, one FMA)
+//   w_hat = RN16(RN32(((q - z) sh) rs))
+// Clamping after the shifted rint equals clamping the code, because the
+// shifted rint is monotone in w'.  A caller may pass clamp = false only when
+// make_qparams found that no code of the group needs it.
 struct QPair {
     float2 r, magic, sh, nmsh;
-    float lo, hi;
+    float vlo, vhi;
 };
 __device__ __forceinline__ QPair make_qpair(const QParams &p, float qmax) {
     QPair q;
@@ -161,15 +143,17 @@ __device__ __forceinline__ QPair make_qpair(const QParams &p, float qmax) {
     q.sh = make_float2(p.sh, p.sh);
     const float nm = __fmul_rn(-kMagic, p.sh);
     q.nmsh = make_float2(nm, nm);
-    q.lo = -p.z;
-    q.hi = __fsub_rn(qmax, p.z);
+    q.vlo = __fsub_rn(kMagic, p.z);
+    q.vhi = __fadd_rn(kMagic, __fsub_rn(qmax, p.z));
     return q;
 }
+template <bool kClamp>
 __device__ __forceinline__ __half2 dequant_unscale_pair(float2 w, float2 s, float2 rs, const QPair &q) {
-    float2 t = mul2_rn(mul2_rn(w, s), q.r);
-    t.x = fminf(fmaxf(t.x, q.lo), q.hi);
-    t.y = fminf(fmaxf(t.y, q.lo), q.hi);
-    const float2 v = add2_rn(t, q.magic);
+    float2 v = fma2_rn(mul2_rn(w, s), q.r, q.magic);
+    if (kClamp) {
+        v.x = fminf(fmaxf(v.x, q.vlo), q.vhi);
+        v.y = fminf(fmaxf(v.y, q.vlo), q.vhi);
+    }
     return __float22half2_rn(mul2_rn(fma2_rn(v, q.sh, q.nmsh), rs));
 }
 
@@ -245,30 +229,37 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parit
 }
 
 // Bounded wait: returns false (after raising the device timeout flag and the
-// CTA's abort flag) when the phase does not complete within `limit_ns`, or
-// when another role of the CTA has already aborted.  Never traps.  Waiting
-// threads are suspended by the hardware between checks, so a long wait costs
-// almost no issue slots.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort_flag, uint64_t limit_ns) {
+// CTA's abort flag) when the phase does not complete within about `limit_ns`,
+// or when another role of the CTA has already aborted.  Never traps.  Waiting
+// threads are suspended by the hardware between polls (and may also sleep
+// `sleep_ns` between polls); the abort flag and the clock are checked only
+// every 16 polls to keep a long wait cheap in issue slots.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                  uint64_t limit_ns, uint32_t sleep_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
+    uint64_t t0 = 0;
+    for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            atomicOr(&g_dev_error, kDevErrTimeout);
-            return false;
+        if (sleep_ns) __nanosleep(sleep_ns);
+        if ((n & 15u) == 0) {
+            if (*abort_flag) return false;
+            const uint64_t now = global_timer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicOr(&g_dev_error, kDevErrTimeout);
+                return false;
+            }
         }
     }
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
-                                               volatile int *abort_flag, uint64_t limit_ns) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                               uint64_t limit_ns, uint32_t sleep_ns = 0) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, limit_ns) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, limit_ns, sleep_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     return ok != 0;
 }

@@ -223,13 +223,19 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
-    const QPair qp = make_qpair(make_qparams(mn, mx, qmax), qmax);
+    const QParams prm = make_qparams(mn, mx, qmax);
+    const QPair qp = make_qpair(prm, qmax);
     if (!active) return;
     __align__(16) __half2 out[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-        out[e] = dequant_unscale_pair(make_float2(wv[2 * e], wv[2 * e + 1]), make_float2(sv[2 * e], sv[2 * e + 1]),
-                                      make_float2(rs[2 * e], rs[2 * e + 1]), qp);
+        out[e] = prm.clamp
+                     ? dequant_unscale_pair<true>(make_float2(wv[2 * e], wv[2 * e + 1]),
+                                                  make_float2(sv[2 * e], sv[2 * e + 1]),
+                                                  make_float2(rs[2 * e], rs[2 * e + 1]), qp)
+                     : dequant_unscale_pair<false>(make_float2(wv[2 * e], wv[2 * e + 1]),
+                                                   make_float2(sv[2 * e], sv[2 * e + 1]),
+                                                   make_float2(rs[2 * e], rs[2 * e + 1]), qp);
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0) = *reinterpret_cast<const uint4 *>(&out[0]);
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[4]);
 }
@@ -335,21 +341,30 @@ __device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, con
     }
 }
 
-// Delta W = W_hat - W (fp16) for 8 consecutive weights of one row, using the
-// packed quantizer of dequant_unscale_pair.
-__device__ __forceinline__ uint4 prod_compute_row(const uint4 wv, const uint2 prm, const float2 (&s)[4],
-                                                  const float2 (&rs)[4], float qmax, bool valid) {
-    if (!valid) return make_uint4(0, 0, 0, 0);
-    const QPair q = make_qpair(unpack_qparams(prm), qmax);
-    const __half2 *wh = reinterpret_cast<const __half2 *>(&wv);
-    uint4 out;
-    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+// Delta W = W_hat - W (fp16) for this thread's slice of a stage: 4 rows x 8
+// consecutive weights, all 16 pairs in one unrolled block so their dependency
+// chains interleave.  kClamp selects the code-clamping variant; the warp takes
+// it only when one of its rows has a group that needs it (about 0.1% of groups
+// on LLM-like weights, so ~2% of stages).
+template <bool kClamp>
+__device__ __forceinline__ void prod_compute_stage(const ProdLoad &L, const QParams (&qp)[4], const bool (&valid)[4],
+                                                   float qmax, uint4 (&out)[4]) {
+    const float2 s4[4] = {make_float2(L.s0.x, L.s0.y), make_float2(L.s0.z, L.s0.w),
+                          make_float2(L.s1.x, L.s1.y), make_float2(L.s1.z, L.s1.w)};
+    const float2 r4[4] = {make_float2(L.r0.x, L.r0.y), make_float2(L.r0.z, L.r0.w),
+                          make_float2(L.r1.x, L.r1.y), make_float2(L.r1.z, L.r1.w)};
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const __half2 d = __hsub2(dequant_unscale_pair(__half22float2(wh[p]), s[p], rs[p], q), wh[p]);
-        o[p] = *reinterpret_cast<const uint32_t *>(&d);
+    for (int i = 0; i < 4; ++i) {
+        const QPair q = make_qpair(qp[i], qmax);
+        const __half2 *wh = reinterpret_cast<const __half2 *>(&L.w[i]);
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const __half2 d = __hsub2(dequant_unscale_pair<kClamp>(__half22float2(wh[p]), s4[p], r4[p], q), wh[p]);
+            o[p] = valid[i] ? *reinterpret_cast<const uint32_t *>(&d) : 0u;
+        }
+        out[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    return out;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -446,7 +461,7 @@ search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         for (int64_t u = blockIdx.x; u < A.n_units; u += gridDim.x) {
             const UnitIdx ui = unit_index(u, A);
-            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns)) break;
+            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns, 256)) break;
             tc_fence_after();
             float2 sum2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
@@ -491,16 +506,20 @@ search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
                     if (un != u) uin = unit_index(un, A);
                     prod_issue_loads(nxt, A, uin, kbn, c, rbase);
                 }
-                const float2 s4[4] = {make_float2(cur.s0.x, cur.s0.y), make_float2(cur.s0.z, cur.s0.w),
-                                      make_float2(cur.s1.x, cur.s1.y), make_float2(cur.s1.z, cur.s1.w)};
-                const float2 r4[4] = {make_float2(cur.r0.x, cur.r0.y), make_float2(cur.r0.z, cur.r0.w),
-                                      make_float2(cur.r1.x, cur.r1.y), make_float2(cur.r1.z, cur.r1.w)};
-                uint4 outv[4];
+                QParams qp[4];
+                bool valid[4];
+                bool need = false;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
-                    outv[i] = prod_compute_row(cur.w[i], cur.prm[i], s4, r4, A.qmax, n < A.N);
+                    qp[i] = unpack_qparams(cur.prm[i]);
+                    valid[i] = (int64_t)ui.nb * BM + rbase + 32 * i < A.N;
+                    need |= valid[i] && qp[i].clamp;
                 }
+                uint4 outv[4];
+                if (__any_sync(0xffffffffu, need))
+                    prod_compute_stage<true>(cur, qp, valid, A.qmax, outv);
+                else
+                    prod_compute_stage<false>(cur, qp, valid, A.qmax, outv);
                 if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) break;
                 const uint32_t a_base = smem_u32(&S.a[as][0]);
 #pragma unroll
@@ -631,19 +650,18 @@ pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
     const QParams p = make_qparams(mn, mx, qmax);
-    const QElem qe = make_qelem(p, qmax);
     if (!active) return;
     if (bits == 2) {
         uint32_t word = 0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) word |= quant_code(wp[e], qe, p.z) << (2 * e);
+        for (int e = 0; e < 16; ++e) word |= quant_code(wp[e], p, qmax) << (2 * e);
         codes[n * (K / 16) + k0 / 16] = word;
     } else {
         uint32_t w0 = 0, w1 = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            w0 |= quant_code(wp[e], qe, p.z) << (4 * e);
-            w1 |= quant_code(wp[8 + e], qe, p.z) << (4 * e);
+            w0 |= quant_code(wp[e], p, qmax) << (4 * e);
+            w1 |= quant_code(wp[8 + e], p, qmax) << (4 * e);
         }
         *reinterpret_cast<uint2 *>(codes + n * (K / 8) + k0 / 8) = make_uint2(w0, w1);
     }

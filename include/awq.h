@@ -95,9 +95,10 @@ AWQ_API awq_status awq_alpha_scales(const float *a, int64_t K, const float *alph
  *   per row n and group G of group_size columns:
  *     w'    = RN32(w * s)
  *     scale = RN32(RN32(max w' - min w') / qmax),  sh = RN16(clamp(scale, 2^-24, 65504))
- *     r     = RN32(1 / sh),  z = clamp(rint(RN32(-min w' * r)), 0, qmax)
- *     q     = clamp(rint(RN32(w' * r)) + z, 0, qmax)
+ *     r     = RN32(1 / sh),  z = clamp(rint(-min w' * r), 0, qmax)
+ *     q     = clamp(rint(w' * r) + z, 0, qmax)
  *     w_hat = RN16(RN32(RN32((q - z) * sh) * RN32(1 / s)))
+ *   (the products inside rint are exact: rint is their only rounding)
  *   W      fp16 [N, K];  s  float [K];  W_hat  fp16 [N, K] output.
  * This is the exact per-element function the search evaluates for every
  * alpha; it never runs inside the search (the search keeps W_hat on chip). */

@@ -133,8 +133,10 @@ void awq_oracle_scales(const float *a, int64_t K, float alpha, float *s)
 /*   scale  = RN32(RN32(mx - mn) / qmax)                               */
 /*   sh     = RN16(clamp(scale, 2^-24, 65504))  (stored fp16 scale)    */
 /*   r      = RN32(1 / sh)                                             */
-/*   z      = clamp(rint(RN32(-mn * r)), 0, qmax)   (zero point, a code)*/
-/*   q_k    = clamp(rint(RN32(w'_k * r)) + z, 0, qmax)                 */
+/*   z      = clamp(rint(-mn * r), 0, qmax)   (zero point, a code)     */
+/*   q_k    = clamp(rint(w'_k * r) + z, 0, qmax)                       */
+/* The products inside rint are exact (binary32 x binary32 fits in      */
+/* binary64): q = round(w'/scale) is rounded once, by rint itself.      */
 /*   what_k = RN16(RN32(RN32((q_k - z) * sh) * RN32(1 / s_k)))         */
 /* no_round != 0 replaces rint by the identity in q_k (and drops the   */
 /* clamp), which turns quantization into an exact identity up to       */
@@ -169,13 +171,13 @@ void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s
             uint16_t shb = awq_oracle_rn16(sc);
             double sh = awq_oracle_h2d(shb);
             float r = rn32(1.0 / sh);
-            double z = nearbyint((double)rn32(-(double)mn * (double)r));
+            double z = nearbyint(-(double)mn * (double)r);    /* exact product */
             if (!(z > 0.0)) z = 0.0;        /* a code in [0, qmax]: never -0 */
             if (z > qmax) z = qmax;
             if (sh_out) sh_out[n * G + gi] = shb;
             if (z_out) z_out[n * G + gi] = (float)z;
             for (int k = 0; k < g; ++k) {
-                double t = rn32((double)wp[k] * (double)r);
+                double t = (double)wp[k] * (double)r;          /* exact product */
                 double q;
                 if (no_round) {
                     q = t + z;

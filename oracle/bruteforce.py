@@ -52,11 +52,11 @@ def quantize_group(w, s, bits):
     scale = min(max(float(scale), 2.0 ** -24), 65504.0)
     sh = to_f16(scale)
     r = f32(f32(1.0) / f32(sh))
-    z = round(float(f32(-mn * r)))          # round(): ties to even
+    z = round(-float(mn) * float(r))        # exact product (24 x 24 bits); round(): ties to even
     z = min(max(z, 0), qmax)
     q, what = [], []
     for k in range(len(w)):
-        t = float(f32(wp[k] * r))
+        t = float(wp[k]) * float(r)         # exact product
         qk = min(max(round(t) + z, 0), qmax)
         rs = f32(f32(1.0) / s[k])
         deq = f32(f32(qk - z) * f32(sh))

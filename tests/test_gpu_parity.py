@@ -180,6 +180,25 @@ def test_search_losses(awq, N, K, T, bits, group, seed):
     assert_alpha_choice(oracle.argmin(losses.astype(np.float64)), ref["losses"])
 
 
+def test_search_degenerate_groups(awq):
+    """Rows whose groups need the code clamp (one-signed rows, a constant
+    group, a huge weight), so the producer's clamp path runs."""
+    W, X = gen(160, 512, 600, seed=12, outlier_frac=0.02)
+    W[0, :] = 0
+    W[1, :128] = np.float16(0.013)
+    W[2, :] = np.abs(W[2, :]) + np.float16(0.5)
+    W[3, :] = -np.abs(W[3, :]) - np.float16(0.5)
+    W[4, 5] = np.float16(60000.0)
+    W[130, :] = np.abs(W[130, :]) + np.float16(0.25)
+    alphas = synth.default_alphas()
+    a = oracle.act_stats(X)
+    losses, rows = awq.search_layer(dev(W), dev(X), dev(a), dev(alphas), 4, 128, row_losses=True)
+    awq.get_status()
+    ref = oracle.search(W, X, a, 4, 128, alphas)
+    np.testing.assert_allclose(host(losses), ref["losses"], rtol=LOSS_RTOL)
+    np.testing.assert_allclose(host(rows), ref["row_sums"], rtol=LOSS_RTOL, atol=1e-12)
+
+
 def test_search_with_strided_x_and_one_alpha(awq):
     W, X = gen(128, 256, 600, seed=9)
     Xpad = np.zeros((600, 264), dtype=np.float16)
