@@ -36,18 +36,19 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace of awq_search_layer, carved in this order (each 256-byte aligned):
 //   s_tab   float [n_alpha][K]
 //   rs_tab  float [n_alpha][K]
-//   params  uint2 [n_alpha][K/g][N]
+//   params  uint2 [n_alpha][K/g][N_pad]   (N_pad = N rounded up to 256; padded rows are zero)
 //   partial float [n_alpha][ceil(T/512)][N]
+int64_t padded_rows(int64_t N) { return (N + awq::srch2::PM - 1) / awq::srch2::PM * awq::srch2::PM; }
 struct SearchWs {
     size_t s_off, rs_off, prm_off, part_off, total;
 };
 SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alpha) {
     SearchWs w{};
-    const int64_t n_tb = (T + awq::srch::BT - 1) / awq::srch::BT;
+    const int64_t n_tb = (T + awq::srch2::BT - 1) / awq::srch2::BT;
     size_t off = 0;
     w.s_off = off;    off = round_up(off + sizeof(float) * (size_t)n_alpha * K, 256);
     w.rs_off = off;   off = round_up(off + sizeof(float) * (size_t)n_alpha * K, 256);
-    w.prm_off = off;  off = round_up(off + sizeof(uint2) * (size_t)n_alpha * (K / group) * N, 256);
+    w.prm_off = off;  off = round_up(off + sizeof(uint2) * (size_t)n_alpha * (K / group) * padded_rows(N), 256);
     w.part_off = off; off = round_up(off + sizeof(float) * (size_t)n_alpha * n_tb * N, 256);
     w.total = off;
     return w;
@@ -62,6 +63,7 @@ struct DevInfo {
     int sms = 0;
     int cc_major = 0;
     bool search_attr = false;
+    int max_pairs = 0;       // CTA pairs of the search kernel that fit on the device at once
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -80,9 +82,22 @@ awq_status device_info(DevInfo &out) {
     }
     if (d.cc_major != 10) return AWQ_ERR_UNSUPPORTED;
     if (!d.search_attr) {
-        if (cudaFuncSetAttribute(awq::srch::search_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::srch::SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(awq::srch2::search_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::srch2::SMEM_BYTES) != cudaSuccess)
             return AWQ_ERR_CUDA;
+        // A pair must sit in one GPC, so fewer than sms/2 pairs may fit at once;
+        // the persistent grid never exceeds what is co-resident.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (d.sms / 2), 1, 1);
+        cfg.blockDim = dim3(awq::srch2::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = awq::srch2::SMEM_BYTES;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, (void *)awq::srch2::search_pair_kernel, &cfg) != cudaSuccess ||
+            clusters <= 0) {
+            (void)cudaGetLastError();
+            clusters = d.sms / 2;
+        }
+        d.max_pairs = clusters < d.sms / 2 ? clusters : d.sms / 2;
         d.search_attr = true;
     }
     out = d;
@@ -107,16 +122,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// X[T, ldx] fp16 as a 2-D tensor (inner dimension K), boxes of 64 x 256,
-// 128-byte swizzle; rows past T read as zeros.
-bool encode_x_map(CUtensorMap *m, const void *X, int64_t T, int64_t K, int64_t ldx) {
+// A row-major fp16 matrix [rows, ld] as a 2-D tensor (inner dimension
+// `cols`), boxes of 64 columns x box_rows rows, 128-byte swizzle; rows past the
+// end read as zeros.
+bool encode_rows_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
-    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-    cuuint32_t box[2] = {(cuuint32_t)awq::srch::BK, (cuuint32_t)awq::srch::BN};
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)awq::srch2::BK, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), dims, strides, box, estr,
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -131,11 +147,14 @@ awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, c
                                int n_alpha, float qmax, uint2 *params, cudaStream_t st) {
     const int G = (int)(K / group);
     const int tpg = group / 16;
-    const int grid = blocks_for(N * G * tpg, 256);
+    const int64_t N_pad = padded_rows(N);
+    const int grid = blocks_for(N_pad * G * tpg, 256);
     if (tpg == 8)
-        awq::group_params_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, s_tab, n_alpha, qmax, params);
+        awq::group_params_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, N_pad, K, G, s_tab, n_alpha, qmax,
+                                                          params);
     else
-        awq::group_params_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, s_tab, n_alpha, qmax, params);
+        awq::group_params_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, N_pad, K, G, s_tab, n_alpha, qmax,
+                                                          params);
     return last_launch();
 }
 
@@ -263,11 +282,12 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
     // a3 (group parameters for every alpha)
     if (awq_status e = launch_group_params(W, N, K, q.group_size, s_tab, n_alpha, qmax, params, st)) return e;
 
-    // a4-a6: the tensor-core search
-    CUtensorMap tmap;
-    if (!encode_x_map(&tmap, X, T, K, ldx)) return AWQ_ERR_CUDA;
-    awq::srch::Args A;
-    A.W = (const __half *)W;
+    // a4-a6: the tensor-core search on CTA pairs
+    CUtensorMap tmap_x, tmap_w;
+    if (!encode_rows_map(&tmap_x, X, T, K, ldx, awq::srch2::HN) ||
+        !encode_rows_map(&tmap_w, W, N, K, K, awq::srch2::BM))
+        return AWQ_ERR_CUDA;
+    awq::srch2::Args A;
     A.params = params;
     A.s_tab = s_tab;
     A.rs_tab = rs_tab;
@@ -275,20 +295,21 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
     A.N = N;
     A.K = K;
     A.T = T;
+    A.N_pad = padded_rows(N);
     A.n_alpha = n_alpha;
     A.G = (int)(K / q.group_size);
     A.group = q.group_size;
-    A.n_nb = (int)((N + awq::srch::BM - 1) / awq::srch::BM);
-    A.n_tb = (int)((T + awq::srch::BT - 1) / awq::srch::BT);
-    A.n_kb = (int)(K / awq::srch::BK);
-    A.n_units = (int64_t)A.n_nb * A.n_tb * n_alpha;
+    A.n_tb = (int)((T + awq::srch2::BT - 1) / awq::srch2::BT);
+    A.n_kb = (int)(K / awq::srch2::BK);
+    A.n_units = (A.N_pad / awq::srch2::PM) * A.n_tb * n_alpha;
     A.qmax = qmax;
     A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
-    const int grid = (int)(A.n_units < d.sms ? A.n_units : d.sms);
+    const int64_t pairs = A.n_units < d.max_pairs ? A.n_units : d.max_pairs;
+    const int grid = (int)(2 * pairs);
     cudaEvent_t pb = t_prof_begin, pe = t_prof_end;
     t_prof_begin = t_prof_end = nullptr;
     if (pb && cudaEventRecord(pb, st) != cudaSuccess) return AWQ_ERR_CUDA;
-    awq::srch::search_kernel<<<grid, awq::srch::NUM_THREADS, awq::srch::SMEM_BYTES, st>>>(tmap, A);
+    awq::srch2::search_pair_kernel<<<grid, awq::srch2::NUM_THREADS, awq::srch2::SMEM_BYTES, st>>>(tmap_x, tmap_w, A);
     if (awq_status e = last_launch()) return e;
     if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
 

@@ -143,14 +143,15 @@ __global__ void alpha_scales_kernel(const float *__restrict__ a, int64_t K,
 // ===========================================================================
 template <int TPG>   // threads per group = group_size / 16
 __global__ void __launch_bounds__(256)
-group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
+group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int64_t K, int G,
                     const float *__restrict__ s_tab, int n_alpha, float qmax,
                     uint2 *__restrict__ params) {
     const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
     const int sub = threadIdx.x % TPG;
-    const bool active = gid < N * (int64_t)G;
-    const int64_t n = active ? gid / G : 0;
-    const int grp = active ? (int)(gid - n * G) : 0;
+    const bool in_pad = gid < N_pad * (int64_t)G;            // rows [N, N_pad) get zero parameters
+    const int64_t n = in_pad ? gid / G : 0;
+    const int grp = in_pad ? (int)(gid - n * G) : 0;
+    const bool active = in_pad && n < N;
     const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
     float w[16];
     {
@@ -181,9 +182,9 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
-        if (active && sub == 0) {
+        if (in_pad && sub == 0) {
             const QParams p = make_qparams(mn, mx, qmax);
-            params[((int64_t)ai * G + grp) * N + n] = pack_qparams(p);
+            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(p) : make_uint2(0, 0);
         }
     }
 }
@@ -324,8 +325,8 @@ __device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, con
     const int64_t k = (int64_t)kb * BK + c * 8;
     const float4 *sp = reinterpret_cast<const float4 *>(A.s_tab + (int64_t)ui.alpha * A.K + k);
     const float4 *rp = reinterpret_cast<const float4 *>(A.rs_tab + (int64_t)ui.alpha * A.K + k);
-    L.s0 = __ldg(sp); L.s1 = __ldg(sp + 1);
-    L.r0 = __ldg(rp); L.r1 = __ldg(rp + 1);
+    L.s0 = ldg_nc_f4(sp); L.s1 = ldg_nc_f4(sp + 1);
+    L.r0 = ldg_nc_f4(rp); L.r1 = ldg_nc_f4(rp + 1);
     const int grp = (int)(((int64_t)kb * BK) / A.group);
     const uint2 *pp = A.params + ((int64_t)ui.alpha * A.G + grp) * A.N;
 #pragma unroll
@@ -333,7 +334,7 @@ __device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, con
         const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
         if (n < A.N) {
             L.w[i] = ldg_nc_v4(A.W + n * A.K + k);
-            L.prm[i] = __ldg(pp + n);
+            L.prm[i] = ldg_nc_v2(pp + n);
         } else {
             L.w[i] = make_uint4(0, 0, 0, 0);
             L.prm[i] = make_uint2(0, 0);
@@ -542,6 +543,349 @@ search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
     }
 }
 }  // namespace srch
+
+// ===========================================================================
+// a4-a6 on a CTA pair.  Two CTAs of a cluster share one tcgen05 cta_group::2
+// MMA of M = 256 (each CTA owns 128 W rows of the unit) by N = 256 tokens
+// (each CTA holds 128 of them), two accumulators side by side: a work unit is
+// 256 W rows x 512 tokens for one alpha.  Per CTA and 64-column k-step:
+//   * the X warp TMA-loads this CTA's two 128-token halves (32 KiB) and counts
+//     their bytes on the leader's full barrier;
+//   * the W warp TMA-loads the CTA's W tile (128 x 64, 128-byte swizzle), its
+//     1 KiB of group parameters and 64 s and 1/s values into a 4-deep ring, so
+//     the producer reads everything from shared memory;
+//   * 8 producer warps build Delta W = W_hat - W in the A tile and arrive on
+//     their own CTA's A barrier; in the peer one thread forwards a single
+//     cluster-scope arrive per stage to the leader (9 arrivals per stage);
+//   * the leader's MMA thread issues the pair MMAs and releases both CTAs'
+//     stages with one multicast commit; the epilogue of each CTA drains its
+//     own 128 TMEM lanes and tells the leader (8 arrivals per unit).
+// Halving the X tile per SM (against one CTA doing M = 128) is what frees the
+// shared memory for the W ring.
+// ===========================================================================
+namespace srch2 {
+constexpr int BM = 128;                 // W rows per CTA
+constexpr int PM = 2 * BM;              // W rows per unit (MMA M)
+constexpr int BN = 256;                 // tokens per MMA (MMA N, 128 per CTA)
+constexpr int HN = BN / 2;
+constexpr int NJ = 2;                   // accumulators per unit
+constexpr int BT = BN * NJ;             // tokens per unit
+constexpr int BK = 64;                  // K per stage (one 128-byte swizzled row)
+constexpr int XS = 3, AS = 3, WS = 4;   // ring depths
+constexpr int X_J_BYTES = HN * BK * 2;               // 16 KiB
+constexpr int X_STAGE_BYTES = NJ * X_J_BYTES;        // 32 KiB per CTA
+constexpr int A_STAGE_BYTES = BM * BK * 2;           // 16 KiB
+constexpr int W_TILE_BYTES = BM * BK * 2;            // 16 KiB
+constexpr int PRM_BYTES = BM * 8;                    // 1 KiB
+constexpr int SV_BYTES = BK * 4;                     // 256 B
+constexpr int W_TX_BYTES = W_TILE_BYTES + PRM_BYTES + 2 * SV_BYTES;
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int XTMA_WARP = 4;
+constexpr int MMA_WARP = 5;
+constexpr int WTMA_WARP = 6;
+constexpr int PROD_WARP0 = 8;
+constexpr int NUM_PROD_WARPS = 8;
+constexpr int NUM_THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;   // 512
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t IDESC = mma_idesc_f16_f32(PM, BN);
+constexpr uint16_t PAIR_MASK = 0x3;
+
+struct Smem {
+    uint8_t x[XS][X_STAGE_BYTES];       // every tile 1024-byte aligned
+    uint8_t a[AS][A_STAGE_BYTES];
+    uint8_t w[WS][W_TILE_BYTES];
+    uint2 prm[WS][BM];
+    float sv[WS][BK];
+    float rsv[WS][BK];
+    uint64_t x_full[XS], x_empty[XS];
+    uint64_t a_full[AS], a_empty[AS];
+    uint64_t w_full[WS], w_empty[WS];
+    uint64_t acc_full, acc_empty, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+
+struct Args {
+    const uint2 *params;        // [n_alpha][G][N_pad]
+    const float *s_tab;         // [n_alpha][K]
+    const float *rs_tab;        // [n_alpha][K]
+    float *partial;             // [n_alpha][n_tb][N]
+    int64_t N, K, T, N_pad;
+    int n_alpha, G, group;
+    int n_tb, n_kb;
+    int64_t n_units;
+    float qmax;
+    uint64_t timeout_ns;
+};
+
+struct UnitIdx { int nb, tb, alpha; };
+__device__ __forceinline__ UnitIdx unit_index(int64_t u, const Args &A) {
+    UnitIdx r;
+    const int64_t tile = u / A.n_alpha;
+    r.alpha = (int)(u - tile * A.n_alpha);
+    r.nb = (int)(tile / A.n_tb);
+    r.tb = (int)(tile - (int64_t)r.nb * A.n_tb);
+    return r;
+}
+
+// Delta W for this thread's 4 rows x 8 columns of a stage (see srch::prod_compute_stage).
+template <bool kClamp>
+__device__ __forceinline__ void compute_stage(const uint4 (&w)[4], const QParams (&qp)[4], const float4 (&sv)[2],
+                                              const float4 (&rv)[2], float qmax, uint4 (&out)[4]) {
+    const float2 s4[4] = {make_float2(sv[0].x, sv[0].y), make_float2(sv[0].z, sv[0].w),
+                          make_float2(sv[1].x, sv[1].y), make_float2(sv[1].z, sv[1].w)};
+    const float2 r4[4] = {make_float2(rv[0].x, rv[0].y), make_float2(rv[0].z, rv[0].w),
+                          make_float2(rv[1].x, rv[1].y), make_float2(rv[1].z, rv[1].w)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const QPair q = make_qpair(qp[i], qmax);
+        const __half2 *wh = reinterpret_cast<const __half2 *>(&w[i]);
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const __half2 d = __hsub2(dequant_unscale_pair<kClamp>(__half22float2(wh[p]), s4[p], r4[p], q), wh[p]);
+            o[p] = *reinterpret_cast<const uint32_t *>(&d);
+        }
+        out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const Args A) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1;
+    const int64_t npairs = gridDim.x >> 1;
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < XS; ++i) { mbar_init(&S.x_full[i], 1); mbar_init(&S.x_empty[i], 1); }
+        // leader: its 8 producer warps + one forwarded arrival from the peer; peer: its 8 producer warps
+        for (int i = 0; i < AS; ++i) {
+            mbar_init(&S.a_full[i], leader ? NUM_PROD_WARPS + 1 : NUM_PROD_WARPS);
+            mbar_init(&S.a_empty[i], 1);
+        }
+        for (int i = 0; i < WS; ++i) { mbar_init(&S.w_full[i], 1); mbar_init(&S.w_empty[i], NUM_PROD_WARPS); }
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.acc_empty, 2 * NUM_EPI_WARPS);
+        mbar_init(&S.drain, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == XTMA_WARP) {
+        tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
+        tc_fence_before();
+    }
+    __syncthreads();
+    cluster_sync_all();      // both CTAs' barriers exist before anyone signals across the pair
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    bool aborted = false;
+
+    if (warp == XTMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_x);
+            int xs = 0;
+            uint32_t xph = 0;
+            for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
+                const UnitIdx ui = unit_index(u, A);
+                const int t0 = ui.tb * BT + (int)rank * HN;
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.x_empty[xs], xph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    if (leader) mbar_arrive_expect_tx(&S.x_full[xs], 2 * X_STAGE_BYTES);
+                    const uint32_t full_l = mapa_shared(smem_u32(&S.x_full[xs]), 0);
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j)
+                        tma_load_2d_pair(&S.x[xs][j * X_J_BYTES], &tmap_x, kb * BK, t0 + j * BN, full_l);
+                    if (++xs == XS) { xs = 0; xph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == WTMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_w);
+            int ws = 0;
+            uint32_t wph = 0;
+            for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
+                const UnitIdx ui = unit_index(u, A);
+                const int n0 = ui.nb * PM + (int)rank * BM;
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.w_empty[ws], wph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    mbar_arrive_expect_tx(&S.w_full[ws], W_TX_BYTES);
+                    tma_load_2d(&S.w[ws][0], &tmap_w, kb * BK, n0, &S.w_full[ws]);
+                    const int grp = (int)(((int64_t)kb * BK) / A.group);
+                    bulk_load(&S.prm[ws][0], A.params + ((int64_t)ui.alpha * A.G + grp) * A.N_pad + n0, PRM_BYTES,
+                              &S.w_full[ws]);
+                    bulk_load(&S.sv[ws][0], A.s_tab + (int64_t)ui.alpha * A.K + (int64_t)kb * BK, SV_BYTES,
+                              &S.w_full[ws]);
+                    bulk_load(&S.rsv[ws][0], A.rs_tab + (int64_t)ui.alpha * A.K + (int64_t)kb * BK, SV_BYTES,
+                              &S.w_full[ws]);
+                    if (++ws == WS) { ws = 0; wph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == MMA_WARP && !leader) {
+        // Peer: forward "my half of A stage `as` is written" to the leader with a
+        // single cluster-scope arrive per stage (the producers arrive locally,
+        // with cheap CTA-scope release; release is cumulative, so this arrive
+        // also orders their writes for the leader's MMA).
+        if (lane == 0) {
+            int as = 0;
+            uint32_t aph = 0;
+            for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&S.a_full[as]), 0));
+                    if (++as == AS) { as = 0; aph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0) {
+            int xs = 0, as = 0;
+            uint32_t xph = 0, aph = 0, accph = 0;
+            for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
+                if (!mbar_wait_bounded(&S.acc_empty, accph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < A.n_kb; ++kb) {
+                    if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
+                        !mbar_wait_bounded(&S.x_full[xs], xph, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(&S.a[as][0]);
+                    const uint32_t x_base = smem_u32(&S.x[xs][0]);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j) {
+                            const uint64_t bdesc = sw128_kmajor_desc(x_base + j * X_J_BYTES + kk * 32);
+                            mma_f16_ss_pair(tmem + j * BN, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit_pair_mc(&S.x_empty[xs], PAIR_MASK);
+                    mma_commit_pair_mc(&S.a_empty[as], PAIR_MASK);
+                    if (++xs == XS) { xs = 0; xph ^= 1u; }
+                    if (++as == AS) { as = 0; aph ^= 1u; }
+                }
+                if (aborted) break;
+                mma_commit_pair_mc(&S.acc_full, PAIR_MASK);
+                accph ^= 1u;
+            }
+            mma_commit_pair(&S.drain);                  // every pair MMA of this thread done before teardown
+            mbar_wait_bounded(&S.drain, 0, abort_flag, A.timeout_ns);
+        }
+    } else if (warp < NUM_EPI_WARPS) {
+        uint32_t accph = 0;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t acc_empty_l = mapa_shared(smem_u32(&S.acc_empty), 0);
+        for (int64_t u = pair; u < A.n_units; u += npairs) {
+            const UnitIdx ui = unit_index(u, A);
+            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns, 256)) { aborted = true; break; }
+            tc_fence_after();
+            float2 sum2 = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+            for (int c = 0; c < TMEM_COLS; c += 64) {
+                float v[64];
+                tmem_ld_32x32b_x64_sync(tmem + lane_base + c, v);
+#pragma unroll
+                for (int i = 0; i < 64; i += 2) {
+                    const float2 e = make_float2(v[i], v[i + 1]);
+                    sum2 = fma2_rn(e, e, sum2);
+                }
+            }
+            const float sum = __fadd_rn(sum2.x, sum2.y);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(&S.acc_empty);
+                else mbar_arrive_cluster(acc_empty_l);
+            }
+            const int64_t n = (int64_t)ui.nb * PM + rank * BM + warp * 32 + lane;
+            if (n < A.N) A.partial[((int64_t)ui.alpha * A.n_tb + ui.tb) * A.N + n] = sum;
+            accph ^= 1u;
+        }
+    } else if (warp >= PROD_WARP0) {
+        const int p = threadIdx.x - PROD_WARP0 * 32;   // 0..255
+        const int c = p & 7;                            // 16-byte chunk of the 128-byte row
+        const int rbase = p >> 3;                       // rows rbase + 32 i
+        int ws = 0, as = 0;
+        uint32_t wph = 0, aph = 0;
+        for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
+            for (int kb = 0; kb < A.n_kb; ++kb) {
+                if (!mbar_wait_warp(&S.w_full[ws], wph, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                const uint32_t wb = smem_u32(&S.w[ws][0]);
+                uint4 w[4];
+                QParams qp[4];
+                bool need = false;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    w[i] = lds_v4(wb + sw128_offset(rbase + 32 * i, c));
+                    qp[i] = unpack_qparams(lds_v2(smem_u32(&S.prm[ws][rbase + 32 * i])));
+                    need |= qp[i].clamp;
+                }
+                float4 sv[2], rv[2];
+                sv[0] = lds_f4(smem_u32(&S.sv[ws][c * 8]));
+                sv[1] = lds_f4(smem_u32(&S.sv[ws][c * 8 + 4]));
+                rv[0] = lds_f4(smem_u32(&S.rsv[ws][c * 8]));
+                rv[1] = lds_f4(smem_u32(&S.rsv[ws][c * 8 + 4]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.w_empty[ws]);   // the stage's reads are done
+                if (++ws == WS) { ws = 0; wph ^= 1u; }
+                uint4 outv[4];
+                if (__any_sync(0xffffffffu, need))
+                    compute_stage<true>(w, qp, sv, rv, A.qmax, outv);
+                else
+                    compute_stage<false>(w, qp, sv, rv, A.qmax, outv);
+                if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                const uint32_t a_base = smem_u32(&S.a[as][0]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) st_shared_v4(a_base + sw128_offset(rbase + 32 * i, c), outv[i]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.a_full[as]);      // local; the peer's is forwarded
+                if (++as == AS) { as = 0; aph ^= 1u; }
+            }
+        }
+    }
+
+    // On an abort, give copies already in flight time to land before the CTA
+    // can leave (bounded: about 200 microseconds).
+    if (aborted || *abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();      // neither CTA leaves while its pair may still signal it or read its tiles
+    if (warp == XTMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+}  // namespace srch2
 
 // ===========================================================================
 // a6 (reduction). losses[i] = RN32(sum over token blocks and rows of the
