@@ -3,7 +3,7 @@
 //   act_stats_kernel      a_j = mean_t |X[t,j]|              (HBM-bound column reduction)
 //   alpha_scales_kernel   s = a^alpha, rs = RN32(1/s)        (tiny)
 //   group_params_kernel   per (alpha, row, group): sh, r, z  (one pass over W for all alphas)
-//   search_kernel         per alpha: sum ((W_hat - W) X^T)^2 (tcgen05 / TMEM / TMA)
+//   search_pair_kernel    per alpha: sum ((W_hat - W) X^T)^2 (tcgen05 cta_group::2 / TMEM / TMA)
 //   loss_reduce_kernel    per-alpha MSE and per-row sums     (deterministic, binary64)
 //   best_scale_kernel     argmin over the grid + s_best
 //   pack_kernel           codes / fp16 scales / fp16 zeros   (HBM-bound)
@@ -242,309 +242,6 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
 }
 
 // ===========================================================================
-// a5/a6. The search.  For every work unit (tile of 128 W rows x 512 tokens,
-// alpha) it accumulates E = (W_hat_alpha - W) X^T for the tile in tensor
-// memory over all of K, squares and sums E on chip, and writes one fp32
-// partial per (alpha, token block, row).  E is never written to memory.
-//
-// Roles (448 threads, one CTA per SM, persistent over work units):
-//   warps 0-3   epilogue: tcgen05.ld the 128 x 512 fp32 accumulator, sum squares
-//   warp 4      TMA producer for X tiles (64 k x 256 tokens, 128-byte swizzle);
-//               also allocates / frees tensor memory
-//   warp 5      MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128, N=256,
-//               two accumulators side by side (512 TMEM columns)
-//   warps 6-13  producer of the A operand: reads W (+ per-group parameters),
-//               applies s, rounds, dequantizes, unscales, subtracts W and stores
-//               Delta W = W_hat - W (fp16) straight into the swizzled shared
-//               memory tile the tensor core reads.  W_hat never reaches HBM.
-// ===========================================================================
-namespace srch {
-constexpr int BM = 128;                 // W rows per tile (MMA M)
-constexpr int BN = 256;                 // tokens per MMA (MMA N)
-constexpr int NJ = 2;                   // accumulators per tile
-constexpr int BT = BN * NJ;             // tokens per tile
-constexpr int BK = 64;                  // K per pipeline stage (one 128-byte row)
-constexpr int XS = 3;                   // X stages
-constexpr int AS = 2;                   // Delta W stages
-constexpr int X_HALF_BYTES = BN * BK * 2;          // 32 KiB
-constexpr int X_STAGE_BYTES = BT * BK * 2;         // 64 KiB
-constexpr int A_STAGE_BYTES = BM * BK * 2;         // 16 KiB
-constexpr int NUM_EPI_WARPS = 4;
-constexpr int TMA_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int PROD_WARP0 = 6;
-constexpr int NUM_PROD_WARPS = 8;
-constexpr int NUM_THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;   // 448
-constexpr int TMEM_COLS = 512;
-constexpr uint32_t IDESC = mma_idesc_f16_f32(BM, BN);
-
-struct Smem {
-    uint8_t x[XS][X_STAGE_BYTES];       // 1024-aligned (base aligned, sizes multiples of 1024)
-    uint8_t a[AS][A_STAGE_BYTES];
-    uint64_t x_full[XS], x_empty[XS];
-    uint64_t a_full[AS], a_empty[AS];
-    uint64_t acc_full, acc_empty, drain;
-    uint32_t tmem_base;
-    int abort_flag;
-};
-constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + slack to align the base
-
-struct Args {
-    const __half *W;            // [N, K]
-    const uint2 *params;        // [n_alpha][G][N]
-    const float *s_tab;         // [n_alpha][K]
-    const float *rs_tab;        // [n_alpha][K]
-    float *partial;             // [n_alpha][n_tb][N]
-    int64_t N, K, T;
-    int n_alpha, G, group;
-    int n_nb, n_tb, n_kb;
-    int64_t n_units;
-    float qmax;                 // 2^bits - 1
-    uint64_t timeout_ns;
-};
-
-struct UnitIdx { int nb, tb, alpha; };
-__device__ __forceinline__ UnitIdx unit_index(int64_t u, const Args &A) {
-    UnitIdx r;
-    const int64_t tile = u / A.n_alpha;
-    r.alpha = (int)(u - tile * A.n_alpha);
-    r.nb = (int)(tile / A.n_tb);
-    r.tb = (int)(tile - (int64_t)r.nb * A.n_tb);
-    return r;
-}
-
-// Per-thread slice of one producer stage: 4 rows x 8 columns.
-struct ProdLoad {
-    uint4 w[4];
-    uint2 prm[4];
-    float4 s0, s1, r0, r1;
-};
-
-__device__ __forceinline__ void prod_issue_loads(ProdLoad &L, const Args &A, const UnitIdx &ui,
-                                                 int kb, int c, int rbase) {
-    const int64_t k = (int64_t)kb * BK + c * 8;
-    const float4 *sp = reinterpret_cast<const float4 *>(A.s_tab + (int64_t)ui.alpha * A.K + k);
-    const float4 *rp = reinterpret_cast<const float4 *>(A.rs_tab + (int64_t)ui.alpha * A.K + k);
-    L.s0 = ldg_nc_f4(sp); L.s1 = ldg_nc_f4(sp + 1);
-    L.r0 = ldg_nc_f4(rp); L.r1 = ldg_nc_f4(rp + 1);
-    const int grp = (int)(((int64_t)kb * BK) / A.group);
-    const uint2 *pp = A.params + ((int64_t)ui.alpha * A.G + grp) * A.N;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t n = (int64_t)ui.nb * BM + rbase + 32 * i;
-        if (n < A.N) {
-            L.w[i] = ldg_nc_v4(A.W + n * A.K + k);
-            L.prm[i] = ldg_nc_v2(pp + n);
-        } else {
-            L.w[i] = make_uint4(0, 0, 0, 0);
-            L.prm[i] = make_uint2(0, 0);
-        }
-    }
-}
-
-// Delta W = W_hat - W (fp16) for this thread's slice of a stage: 4 rows x 8
-// consecutive weights, all 16 pairs in one unrolled block so their dependency
-// chains interleave.  kClamp selects the code-clamping variant; the warp takes
-// it only when one of its rows has a group that needs it (about 0.1% of groups
-// on LLM-like weights, so ~2% of stages).
-template <bool kClamp>
-__device__ __forceinline__ void prod_compute_stage(const ProdLoad &L, const QParams (&qp)[4], const bool (&valid)[4],
-                                                   float qmax, uint4 (&out)[4]) {
-    const float2 s4[4] = {make_float2(L.s0.x, L.s0.y), make_float2(L.s0.z, L.s0.w),
-                          make_float2(L.s1.x, L.s1.y), make_float2(L.s1.z, L.s1.w)};
-    const float2 r4[4] = {make_float2(L.r0.x, L.r0.y), make_float2(L.r0.z, L.r0.w),
-                          make_float2(L.r1.x, L.r1.y), make_float2(L.r1.z, L.r1.w)};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const QPair q = make_qpair(qp[i], qmax);
-        const __half2 *wh = reinterpret_cast<const __half2 *>(&L.w[i]);
-        uint32_t o[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const __half2 d = __hsub2(dequant_unscale_pair<kClamp>(__half22float2(wh[p]), s4[p], r4[p], q), wh[p]);
-            o[p] = valid[i] ? *reinterpret_cast<const uint32_t *>(&d) : 0u;
-        }
-        out[i] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-}
-
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-search_kernel(const __grid_constant__ CUtensorMap tmap_x, const Args A) {
-    extern __shared__ uint8_t smem_raw[];
-    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    volatile int *abort_flag = &S.abort_flag;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < XS; ++i) { mbar_init(&S.x_full[i], 1); mbar_init(&S.x_empty[i], 1); }
-        for (int i = 0; i < AS; ++i) { mbar_init(&S.a_full[i], NUM_PROD_WARPS); mbar_init(&S.a_empty[i], 1); }
-        mbar_init(&S.acc_full, 1);
-        mbar_init(&S.acc_empty, NUM_EPI_WARPS);
-        mbar_init(&S.drain, 1);
-        S.abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == TMA_WARP) {
-        tmem_alloc(&S.tmem_base, TMEM_COLS);
-        tmem_relinquish();
-        tc_fence_before();
-    }
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = S.tmem_base;
-
-    if (warp == TMA_WARP) {
-        if (lane == 0) {
-            tma_prefetch_desc(&tmap_x);
-            int xs = 0;
-            uint32_t xph = 0;
-            bool ok = true;
-            for (int64_t u = blockIdx.x; u < A.n_units && ok; u += gridDim.x) {
-                const UnitIdx ui = unit_index(u, A);
-                const int t0 = ui.tb * BT;
-                for (int kb = 0; kb < A.n_kb; ++kb) {
-                    if (!mbar_wait_bounded(&S.x_empty[xs], xph ^ 1u, abort_flag, A.timeout_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S.x_full[xs], X_STAGE_BYTES);
-                    tma_load_2d(&S.x[xs][0], &tmap_x, kb * BK, t0, &S.x_full[xs]);
-                    tma_load_2d(&S.x[xs][X_HALF_BYTES], &tmap_x, kb * BK, t0 + BN, &S.x_full[xs]);
-                    if (++xs == XS) { xs = 0; xph ^= 1u; }
-                }
-            }
-            if (!ok) {
-                // Let every load already issued land before the CTA can exit.
-                for (int i = 0; i < XS; ++i) {
-                    // Stage i was last filled in phase (xph ^ (i >= xs)); waiting on a
-                    // completed or never-started phase returns at once.
-                    const uint32_t ph = (i < xs) ? xph : (xph ^ 1u);
-                    mbar_wait_bounded(&S.x_full[i], ph, abort_flag, A.timeout_ns);
-                }
-            }
-        }
-    } else if (warp == MMA_WARP) {
-        if (lane == 0) {
-            int xs = 0, as = 0;
-            uint32_t xph = 0, aph = 0, accph = 0;
-            bool ok = true;
-            for (int64_t u = blockIdx.x; u < A.n_units && ok; u += gridDim.x) {
-                if (!mbar_wait_bounded(&S.acc_empty, accph ^ 1u, abort_flag, A.timeout_ns)) { ok = false; break; }
-                tc_fence_after();
-                for (int kb = 0; kb < A.n_kb; ++kb) {
-                    if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
-                        !mbar_wait_bounded(&S.x_full[xs], xph, abort_flag, A.timeout_ns)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a_base = smem_u32(&S.a[as][0]);
-                    const uint32_t x_base = smem_u32(&S.x[xs][0]);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
-#pragma unroll
-                        for (int j = 0; j < NJ; ++j) {
-                            const uint64_t bdesc = sw128_kmajor_desc(x_base + j * X_HALF_BYTES + kk * 32);
-                            mma_f16_ss(tmem + j * BN, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
-                        }
-                    }
-                    mma_commit(&S.x_empty[xs]);
-                    mma_commit(&S.a_empty[as]);
-                    if (++xs == XS) { xs = 0; xph ^= 1u; }
-                    if (++as == AS) { as = 0; aph ^= 1u; }
-                }
-                if (!ok) break;
-                mma_commit(&S.acc_full);
-                accph ^= 1u;
-            }
-            // Drain: every MMA issued by this thread completes before teardown.
-            mma_commit(&S.drain);
-            mbar_wait_bounded(&S.drain, 0, abort_flag, A.timeout_ns);
-        }
-    } else if (warp < NUM_EPI_WARPS) {
-        uint32_t accph = 0;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        for (int64_t u = blockIdx.x; u < A.n_units; u += gridDim.x) {
-            const UnitIdx ui = unit_index(u, A);
-            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns, 256)) break;
-            tc_fence_after();
-            float2 sum2 = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-            for (int c = 0; c < TMEM_COLS; c += 64) {
-                float v[64];
-                tmem_ld_32x32b_x64_sync(tmem + lane_base + c, v);
-#pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    const float2 e = make_float2(v[i], v[i + 1]);
-                    sum2 = fma2_rn(e, e, sum2);
-                }
-            }
-            const float sum = __fadd_rn(sum2.x, sum2.y);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.acc_empty);
-            const int64_t n = (int64_t)ui.nb * BM + warp * 32 + lane;
-            if (n < A.N) A.partial[((int64_t)ui.alpha * A.n_tb + ui.tb) * A.N + n] = sum;
-            accph ^= 1u;
-        }
-    } else if (warp >= PROD_WARP0) {
-        const int p = threadIdx.x - PROD_WARP0 * 32;   // 0..255
-        const int c = p & 7;                            // 16-byte chunk of the 128-byte row
-        const int rbase = p >> 3;                       // rows rbase + 32 i
-        int as = 0;
-        uint32_t aph = 0;
-        int64_t u = blockIdx.x;
-        int kb = 0;
-        if (u < A.n_units) {
-            ProdLoad cur;
-            UnitIdx ui = unit_index(u, A);
-            prod_issue_loads(cur, A, ui, kb, c, rbase);
-            while (true) {
-                // Next (unit, kb) and its loads, issued before this stage's math.
-                int64_t un = u;
-                int kbn = kb + 1;
-                if (kbn == A.n_kb) { kbn = 0; un += gridDim.x; }
-                const bool has_next = un < A.n_units;
-                UnitIdx uin = ui;
-                ProdLoad nxt;
-                if (has_next) {
-                    if (un != u) uin = unit_index(un, A);
-                    prod_issue_loads(nxt, A, uin, kbn, c, rbase);
-                }
-                QParams qp[4];
-                bool valid[4];
-                bool need = false;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    qp[i] = unpack_qparams(cur.prm[i]);
-                    valid[i] = (int64_t)ui.nb * BM + rbase + 32 * i < A.N;
-                    need |= valid[i] && qp[i].clamp;
-                }
-                uint4 outv[4];
-                if (__any_sync(0xffffffffu, need))
-                    prod_compute_stage<true>(cur, qp, valid, A.qmax, outv);
-                else
-                    prod_compute_stage<false>(cur, qp, valid, A.qmax, outv);
-                if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) break;
-                const uint32_t a_base = smem_u32(&S.a[as][0]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) st_shared_v4(a_base + sw128_offset(rbase + 32 * i, c), outv[i]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.a_full[as]);
-                if (++as == AS) { as = 0; aph ^= 1u; }
-                if (!has_next) break;
-                u = un; kb = kbn; ui = uin; cur = nxt;
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == TMA_WARP) {
-        tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
-    }
-}
-}  // namespace srch
-
-// ===========================================================================
 // a4-a6 on a CTA pair.  Two CTAs of a cluster share one tcgen05 cta_group::2
 // MMA of M = 256 (each CTA owns 128 W rows of the unit) by N = 256 tokens
 // (each CTA holds 128 of them), two accumulators side by side: a work unit is
@@ -629,7 +326,11 @@ __device__ __forceinline__ UnitIdx unit_index(int64_t u, const Args &A) {
     return r;
 }
 
-// Delta W for this thread's 4 rows x 8 columns of a stage (see srch::prod_compute_stage).
+// Delta W = W_hat - W (fp16) for this thread's slice of a stage: 4 rows x 8
+// consecutive weights, all 16 pairs in one unrolled block so their dependency
+// chains interleave.  kClamp selects the code-clamping variant; the warp takes
+// it only when one of its rows has a group that needs it (about 0.1% of groups
+// on LLM-like weights, so ~2% of stages).
 template <bool kClamp>
 __device__ __forceinline__ void compute_stage(const uint4 (&w)[4], const QParams (&qp)[4], const float4 (&sv)[2],
                                               const float4 (&rv)[2], float qmax, uint4 (&out)[4]) {

@@ -38,9 +38,8 @@ METRIC = "AWQ search TFLOP/s (20-α grid, 4096² layer, T=4096) & % of FP16 TC p
 UNIT = "TFLOP/s"
 LAUNCHES_PER_STEP = 7      # act_stats, alpha_scales, group_params, search, loss_reduce, best_scale, pack
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-TRAFFIC_FILE = ROOT / "profiles" / "search_kernel_traffic.json"
-KERNEL_SOURCES = [ROOT / "awq_activation_aware_b200" / "csrc" / f for f in
-                  ("awq_kernels.cuh", "awq_device.cuh", "awq_abi.cu")]
+TRAFFIC_FILE = ROOT / "profiles" / "search_pair_kernel_traffic.json"
+CSRC = ROOT / "awq_activation_aware_b200" / "csrc"
 
 
 def parse_args():
@@ -172,9 +171,15 @@ class ClockSampler:
 
 
 def kernel_source_hash():
+    """Hash of the search kernel's source: its namespace block plus the device
+    helpers it is built from.  A traffic figure taken from an older build of
+    the kernel no longer applies once this changes."""
+    kern = (CSRC / "awq_kernels.cuh").read_text()
+    a = kern.index("namespace srch2 {")
+    b = kern.index("}  // namespace srch2")
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        h.update(f.read_bytes())
+    h.update(kern[a:b].encode())
+    h.update((CSRC / "awq_device.cuh").read_bytes())
     return h.hexdigest()[:16]
 
 
@@ -204,14 +209,20 @@ def oracle_sample(cfg, W, X, alphas, rows):
 
 
 def pick_rows(cfg, W, X, alphas, budget_s):
+    """Rows of W for an oracle sample of about budget_s seconds: time two row
+    counts over the full grid and fit time = fixed + rows * per_row."""
     import oracle
     oracle.build()
-    probe = np.arange(8)
-    t0 = time.perf_counter()
-    oracle.search(W, X, oracle.act_stats(X), cfg.bits, cfg.group, alphas[:2], rows=probe)
-    per_row_alpha = (time.perf_counter() - t0) / (8 * 2)
-    rows = int(budget_s / max(per_row_alpha * len(alphas), 1e-9))
-    return max(8, min(cfg.N, rows))
+    a = oracle.act_stats(X)
+    times = {}
+    for r in (16, 64):
+        t0 = time.perf_counter()
+        oracle.search(W, X, a, cfg.bits, cfg.group, alphas, rows=np.arange(min(r, cfg.N)))
+        times[r] = time.perf_counter() - t0
+    per_row = max((times[64] - times[16]) / 48.0, 1e-6)
+    fixed = max(times[16] - 16 * per_row, 0.0)
+    rows = int((budget_s - fixed) / per_row)
+    return max(16, min(cfg.N, rows))
 
 
 def cpu_measure(cfg, W, X, alphas, args):
@@ -346,7 +357,8 @@ def run_awq(args):
     achieved = flops / (search_avg * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": search_traffic(args.config),
-                "kernel": "search_kernel (tcgen05 f16 MMA + fused quantize producer + loss epilogue)",
+                "kernel": "search_pair_kernel (tcgen05 cta_group::2 f16 MMA, fused quantize producer, "
+                          "on-chip squared-error epilogue)",
                 "peak_source": f"{peak_src} {'sustained' if long_region else 'burst'} bf16 dense "
                                f"(fp16 has the same nominal dense rate)",
                 "search_ms": search_avg}
