@@ -146,15 +146,18 @@ int blocks_for(int64_t threads_total, int block) {
 awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, const float *s_tab,
                                int n_alpha, float qmax, uint2 *params, cudaStream_t st) {
     const int G = (int)(K / group);
-    const int tpg = group / 16;
+    const int lpr = group / awq::kGpCols;
     const int64_t N_pad = padded_rows(N);
-    const int grid = blocks_for(N_pad * G * tpg, 256);
-    if (tpg == 8)
-        awq::group_params_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, N_pad, K, G, s_tab, n_alpha, qmax,
-                                                          params);
+    const int64_t rows_per_block = awq::kGpThreads / lpr;
+    const int64_t row_blocks = (N_pad + rows_per_block - 1) / rows_per_block;
+    const size_t smem = sizeof(float) * (size_t)n_alpha * lpr * (awq::kGpCols + 4);
+    const unsigned grid = (unsigned)(row_blocks * G);
+    if (lpr == 2)
+        awq::group_params_kernel<2><<<grid, awq::kGpThreads, smem, st>>>((const __half *)W, N, N_pad, K, G, s_tab,
+                                                                        n_alpha, qmax, params);
     else
-        awq::group_params_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, N_pad, K, G, s_tab, n_alpha, qmax,
-                                                          params);
+        awq::group_params_kernel<1><<<grid, awq::kGpThreads, smem, st>>>((const __half *)W, N, N_pad, K, G, s_tab,
+                                                                        n_alpha, qmax, params);
     return last_launch();
 }
 
@@ -314,7 +317,7 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
     if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
 
     // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
-    awq::loss_reduce_kernel<<<n_alpha, 256, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
+    awq::loss_reduce_kernel<<<n_alpha, awq::kLossThreads, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
     return last_launch();
 }
 
@@ -353,14 +356,15 @@ awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcf
         if (awq_status e = last_launch()) return e;
     }
     const int G = (int)(K / q.group_size);
-    const int tpg = q.group_size / 16;
-    const int grid = blocks_for(N * G * tpg, 256);
-    if (tpg == 8)
-        awq::pack_kernel<8><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
-                                                  (__half *)scales, (__half *)zeros);
+    const int lpr = q.group_size / awq::kGpCols;
+    const int64_t rows_per_block = awq::kGpThreads / lpr;
+    const unsigned grid = (unsigned)(((N + rows_per_block - 1) / rows_per_block) * G);
+    if (lpr == 2)
+        awq::pack_kernel<2><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
+                                                             (__half *)scales, (__half *)zeros);
     else
-        awq::pack_kernel<4><<<grid, 256, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
-                                                  (__half *)scales, (__half *)zeros);
+        awq::pack_kernel<1><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
+                                                             (__half *)scales, (__half *)zeros);
     return last_launch();
 }
 

@@ -87,10 +87,26 @@ __device__ __forceinline__ QParams unpack_qparams(uint2 v) {
 }
 
 // The integer code q = clamp(rint(w' r) + z, 0, qmax) (used by the packer).
-__device__ __forceinline__ uint32_t quant_code(float wp, const QParams &p, float qmax) {
+// v = RN32(w' r + kMagic) = kMagic + (q - z) once clamped; in [2^23, 2^24) the
+// spacing of binary32 is 1, so the bit pattern of v minus that of kMagic is
+// q - z exactly, and q = bits(v) - (bits(kMagic) - z).  `clamp` may be false
+// only when make_qparams found the group needs no clamping.
+__device__ __forceinline__ uint32_t quant_code(float wp, const QParams &p, float qmax, bool clamp) {
     float v = __fmaf_rn(wp, p.r, kMagic);
-    v = fminf(fmaxf(v, __fsub_rn(kMagic, p.z)), __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));
-    return (uint32_t)__float2int_rn(__fadd_rn(__fsub_rn(v, kMagic), p.z));
+    if (clamp) v = fminf(fmaxf(v, __fsub_rn(kMagic, p.z)), __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));
+    return (uint32_t)(__float_as_int(v) - (__float_as_int(kMagic) - (int)p.z));
+}
+
+// Three-input minimum / maximum (sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // Packed binary32 pair arithmetic (sm_100 FMUL2/FADD2/FFMA2), as PTX with an

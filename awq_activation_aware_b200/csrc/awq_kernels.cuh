@@ -32,17 +32,17 @@ namespace cg = cooperative_groups;
 // a1. Activation statistics: a_j = RN32(RN64(sum_t |X[t,j]|) / T)
 //     ([AWQ-note] "Measures"; [GPTQ-AWQ] "量化方法": X.abs().mean(dim=0)).
 //
-// A cluster of 8 CTAs owns a slab of 128 columns; each CTA reads every 8th
-// group of 16 rows with 16-byte loads (16 threads cover one 256-byte row
+// A cluster of 8 CTAs owns a slab of 64 columns; each CTA reads every 8th
+// group of 32 rows with 16-byte loads (8 threads cover one 128-byte row
 // segment), accumulates |x| in binary64 -- exact, since every fp16 value is a
 // multiple of 2^-24 and the sums stay below 2^29 -- reduces its 16 row lanes
 // in shared memory, and CTA 0 of the cluster sums the 8 partial vectors
 // through distributed shared memory.  No workspace, one launch.
 // ===========================================================================
-constexpr int kStatsCols = 128;
-constexpr int kStatsTPR = 16;                      // threads per row segment
+constexpr int kStatsCols = 64;
+constexpr int kStatsTPR = 8;                       // threads per row segment (128 bytes)
 constexpr int kStatsThreads = 256;
-constexpr int kStatsRowsPerCta = kStatsThreads / kStatsTPR;   // 16
+constexpr int kStatsRowsPerCta = kStatsThreads / kStatsTPR;   // 32
 constexpr int kStatsCluster = 8;
 constexpr int kStatsUnroll = 8;
 
@@ -62,7 +62,7 @@ act_stats_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 
-    const int64_t rstride = (int64_t)kStatsRowsPerCta * kStatsCluster;   // 128 rows
+    const int64_t rstride = (int64_t)kStatsRowsPerCta * kStatsCluster;   // 256 rows
     int64_t t = (int64_t)rank * kStatsRowsPerCta + rl;
     if (active) {
         for (; t + (kStatsUnroll - 1) * rstride < T; t += kStatsUnroll * rstride) {
@@ -136,56 +136,81 @@ __global__ void alpha_scales_kernel(const float *__restrict__ a, int64_t K,
 
 // ===========================================================================
 // a3 (group half). For every (alpha, row, group): min/max of w' = RN32(w*s) and
-// the quantizer parameters ([QAS-QA] §5, §9).  W is read once: each thread
-// keeps 16 weights in registers and walks the alpha grid.  Layout of the
-// result: params[(alpha * G + group) * N + row] (rows contiguous, so the
-// search producer reads 8 bytes per row of its tile).
+// the quantizer parameters ([QAS-QA] §5, §9).  A block owns one column group
+// and 128 / LPR rows; each lane holds 64 consecutive weights of one row as
+// binary32 in registers (LPR = group/64 lanes per row) and walks the whole
+// alpha grid, reading the group's s values -- staged once per block in shared
+// memory, where all lanes of a warp read the same address -- so W is read once
+// and s is not re-fetched per row.  Layout of the result:
+// params[(alpha * G + group) * N_pad + row]; rows [N, N_pad) get zeros.
 // ===========================================================================
-template <int TPG>   // threads per group = group_size / 16
-__global__ void __launch_bounds__(256)
-group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int64_t K, int G,
-                    const float *__restrict__ s_tab, int n_alpha, float qmax,
-                    uint2 *__restrict__ params) {
-    const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
-    const int sub = threadIdx.x % TPG;
-    const bool in_pad = gid < N_pad * (int64_t)G;            // rows [N, N_pad) get zero parameters
-    const int64_t n = in_pad ? gid / G : 0;
-    const int grp = in_pad ? (int)(gid - n * G) : 0;
-    const bool active = in_pad && n < N;
-    const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
-    float w[16];
-    {
-        uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
-        uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
-        const __half2 *h0 = reinterpret_cast<const __half2 *>(&v0);
-        const __half2 *h1 = reinterpret_cast<const __half2 *>(&v1);
+constexpr int kGpThreads = 128;
+constexpr int kGpCols = 64;              // columns per lane
+
+__device__ __forceinline__ void load_row64(const __half *src, float (&w)[kGpCols]) {
+#pragma unroll
+    for (int q = 0; q < kGpCols / 8; ++q) {
+        const uint4 v = ldg_stream_v4(src + 8 * q);
+        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            float2 f0 = __half22float2(h0[e]), f1 = __half22float2(h1[e]);
-            w[2 * e] = f0.x; w[2 * e + 1] = f0.y;
-            w[8 + 2 * e] = f1.x; w[8 + 2 * e + 1] = f1.y;
+            const float2 f = __half22float2(h[e]);
+            w[8 * q + 2 * e] = f.x;
+            w[8 * q + 2 * e + 1] = f.y;
         }
     }
+}
+
+// min and max of w[k] * s[k] over the lane's 64 columns (s in shared memory).
+__device__ __forceinline__ void minmax64(const float (&w)[kGpCols], const float *s_sm, float &mn, float &mx) {
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kGpCols / 4; ++q) {
+        const float4 sv = *reinterpret_cast<const float4 *>(s_sm + 4 * q);
+        const float2 p0 = mul2_rn(make_float2(w[4 * q], w[4 * q + 1]), make_float2(sv.x, sv.y));
+        const float2 p1 = mul2_rn(make_float2(w[4 * q + 2], w[4 * q + 3]), make_float2(sv.z, sv.w));
+        lo = fmin3(lo, fminf(p0.x, p0.y), fminf(p1.x, p1.y));
+        hi = fmax3(hi, fmaxf(p0.x, p0.y), fmaxf(p1.x, p1.y));
+    }
+    mn = lo;
+    mx = hi;
+}
+
+template <int LPR>   // lanes per row = group_size / 64
+__global__ void __launch_bounds__(kGpThreads)
+group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int64_t K, int G,
+                    const float *__restrict__ s_tab, int n_alpha, float qmax, uint2 *__restrict__ params) {
+    extern __shared__ float s_sm[];                 // [n_alpha][LPR][kGpCols + 4] (+4: the halves sit in other banks)
+    constexpr int kRowsPerBlock = kGpThreads / LPR;
+    constexpr int kStride = kGpCols + 4;
+    const int grp = blockIdx.x % G;
+    const int64_t n0 = (int64_t)(blockIdx.x / G) * kRowsPerBlock;
+    const int64_t k0 = (int64_t)grp * (kGpCols * LPR);
+    for (int i = threadIdx.x; i < n_alpha * LPR * kGpCols; i += kGpThreads) {
+        const int ai = i / (LPR * kGpCols), rem = i % (LPR * kGpCols);
+        s_sm[(ai * LPR + rem / kGpCols) * kStride + rem % kGpCols] = __ldg(s_tab + (int64_t)ai * K + k0 + rem);
+    }
+    __syncthreads();
+    const int half = threadIdx.x % LPR;
+    const int64_t n = n0 + threadIdx.x / LPR;
+    const bool active = n < N;
+    float w[kGpCols];
+    if (active) {
+        load_row64(W + n * K + k0 + half * kGpCols, w);
+    } else {
+#pragma unroll
+        for (int e = 0; e < kGpCols; ++e) w[e] = 0.0f;
+    }
     for (int ai = 0; ai < n_alpha; ++ai) {
-        const float4 *sp = reinterpret_cast<const float4 *>(s_tab + (int64_t)ai * K + k0);
-        float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 sv = __ldg(sp + q);
-            const float p0 = __fmul_rn(w[4 * q + 0], sv.x), p1 = __fmul_rn(w[4 * q + 1], sv.y);
-            const float p2 = __fmul_rn(w[4 * q + 2], sv.z), p3 = __fmul_rn(w[4 * q + 3], sv.w);
-            mn = fminf(mn, fminf(fminf(p0, p1), fminf(p2, p3)));
-            mx = fmaxf(mx, fmaxf(fmaxf(p0, p1), fmaxf(p2, p3)));
+        float mn, mx;
+        minmax64(w, s_sm + (ai * LPR + half) * kStride, mn, mx);
+        if (LPR == 2) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         }
-#pragma unroll
-        for (int off = 1; off < TPG; off <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        }
-        if (in_pad && sub == 0) {
-            const QParams p = make_qparams(mn, mx, qmax);
-            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(p) : make_uint2(0, 0);
-        }
+        if (half == 0 && n < N_pad)
+            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(make_qparams(mn, mx, qmax))
+                                                                 : make_uint2(0, 0);
     }
 }
 
@@ -593,27 +618,33 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 // partials, in binary64 and a fixed order, / (N T)); optional per-row sums.
 // One block per alpha.
 // ===========================================================================
-__global__ void __launch_bounds__(256)
+constexpr int kLossThreads = 1024;
+__global__ void __launch_bounds__(kLossThreads)
 loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int n_tb,
                    float *__restrict__ losses, float *__restrict__ row_losses) {
     const int ai = blockIdx.x;
     const float *p = partial + (int64_t)ai * n_tb * N;
     double acc = 0.0;
-    for (int64_t n = threadIdx.x; n < N; n += blockDim.x) {
+    for (int64_t n = threadIdx.x; n < N; n += kLossThreads) {
         float rsum = 0.0f;
         double dsum = 0.0;
-        for (int tb = 0; tb < n_tb; ++tb) {
-            const float v = p[(int64_t)tb * N + n];
-            rsum = __fadd_rn(rsum, v);
-            dsum = __dadd_rn(dsum, (double)v);
+        for (int tb0 = 0; tb0 < n_tb; tb0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = tb0 + j < n_tb ? __ldg(p + (int64_t)(tb0 + j) * N + n) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                rsum = __fadd_rn(rsum, v[j]);
+                dsum = __dadd_rn(dsum, (double)v[j]);
+            }
         }
         if (row_losses) row_losses[(int64_t)ai * N + n] = rsum;
         acc = __dadd_rn(acc, dsum);
     }
-    __shared__ double red[256];
+    __shared__ double red[kLossThreads];
     red[threadIdx.x] = acc;
     __syncthreads();
-    for (int off = 128; off > 0; off >>= 1) {
+    for (int off = kLossThreads / 2; off > 0; off >>= 1) {
         if ((int)threadIdx.x < off) red[threadIdx.x] = __dadd_rn(red[threadIdx.x], red[threadIdx.x + off]);
         __syncthreads();
     }
@@ -657,60 +688,83 @@ __global__ void best_scale_kernel(const float *__restrict__ a, int64_t K,
 
 // ===========================================================================
 // a8. Pack: per (row, group) recompute w' = RN32(w s_best), the group's
-// parameters and every code; store codes LSB-first, fp16 scale and zero
+// parameters and every code; store codes LSB-first, the fp16 scale and zero
 // ([AWQ-note] "Measures": keep the quantized weights and their metadata).
-// Each thread owns 16 consecutive columns: two 32-bit words of 4-bit
-// containers (w_bit 3/4) or one word of 2-bit containers (w_bit 2).
+// Same layout as group_params_kernel: a block owns one column group and
+// 128 / LPR rows, a lane holds 64 consecutive weights, s_best is staged in
+// shared memory.  A lane's 64 codes are 8 words of 4-bit containers
+// (w_bit 3/4) or 4 words of 2-bit containers (w_bit 2).
 // ===========================================================================
-template <int TPG>
-__global__ void __launch_bounds__(256)
+template <int LPR>
+__global__ void __launch_bounds__(kGpThreads)
 pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
             const float *__restrict__ s_best, uint32_t *__restrict__ codes,
             __half *__restrict__ scales, __half *__restrict__ zeros) {
-    const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
-    const int sub = threadIdx.x % TPG;
-    const bool active = gid < N * (int64_t)G;
-    const int64_t n = active ? gid / G : 0;
-    const int grp = active ? (int)(gid - n * G) : 0;
-    const int64_t k0 = (int64_t)grp * (TPG * 16) + sub * 16;
+    __shared__ __align__(16) float s_sm[LPR * (kGpCols + 4)];
+    constexpr int kRowsPerBlock = kGpThreads / LPR;
+    constexpr int kStride = kGpCols + 4;
+    const int grp = blockIdx.x % G;
+    const int64_t n0 = (int64_t)(blockIdx.x / G) * kRowsPerBlock;
+    const int64_t k0 = (int64_t)grp * (kGpCols * LPR);
+    for (int i = threadIdx.x; i < LPR * kGpCols; i += kGpThreads)
+        s_sm[(i / kGpCols) * kStride + i % kGpCols] = __ldg(s_best + k0 + i);
+    __syncthreads();
+    const int half = threadIdx.x % LPR;
+    const int64_t n = n0 + threadIdx.x / LPR;
+    const bool active = n < N;
     const float qmax = (float)((1 << bits) - 1);
-    float wp[16];
-    {
-        uint4 v0 = active ? ldg_stream_v4(W + n * K + k0) : make_uint4(0, 0, 0, 0);
-        uint4 v1 = active ? ldg_stream_v4(W + n * K + k0 + 8) : make_uint4(0, 0, 0, 0);
-        const __half *h0 = reinterpret_cast<const __half *>(&v0);
-        const __half *h1 = reinterpret_cast<const __half *>(&v1);
+    float w[kGpCols];
+    if (active) {
+        load_row64(W + n * K + k0 + half * kGpCols, w);
+    } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const float sv = active ? __ldg(s_best + k0 + e) : 1.0f;
-            wp[e] = __fmul_rn(__half2float(e < 8 ? h0[e] : h1[e - 8]), sv);
-        }
+        for (int e = 0; e < kGpCols; ++e) w[e] = 0.0f;
+    }
+    const float *sp = s_sm + half * kStride;
+#pragma unroll
+    for (int q = 0; q < kGpCols / 4; ++q) {
+        const float4 sv = *reinterpret_cast<const float4 *>(sp + 4 * q);
+        const float2 p0 = mul2_rn(make_float2(w[4 * q], w[4 * q + 1]), make_float2(sv.x, sv.y));
+        const float2 p1 = mul2_rn(make_float2(w[4 * q + 2], w[4 * q + 3]), make_float2(sv.z, sv.w));
+        w[4 * q] = p0.x; w[4 * q + 1] = p0.y; w[4 * q + 2] = p1.x; w[4 * q + 3] = p1.y;   // now w'
     }
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) { mn = fminf(mn, wp[e]); mx = fmaxf(mx, wp[e]); }
-#pragma unroll
-    for (int off = 1; off < TPG; off <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    for (int e = 0; e < kGpCols; e += 2) {
+        mn = fmin3(mn, w[e], w[e + 1]);
+        mx = fmax3(mx, w[e], w[e + 1]);
+    }
+    if (LPR == 2) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     }
     const QParams p = make_qparams(mn, mx, qmax);
     if (!active) return;
+    const int64_t col = k0 + half * kGpCols;
     if (bits == 2) {
-        uint32_t word = 0;
+        uint32_t word[4];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) word |= quant_code(wp[e], p, qmax) << (2 * e);
-        codes[n * (K / 16) + k0 / 16] = word;
-    } else {
-        uint32_t w0 = 0, w1 = 0;
+        for (int j = 0; j < 4; ++j) {
+            uint32_t v = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            w0 |= quant_code(wp[e], p, qmax) << (4 * e);
-            w1 |= quant_code(wp[8 + e], p, qmax) << (4 * e);
+            for (int e = 0; e < 16; ++e) v |= quant_code(w[16 * j + e], p, qmax, p.clamp) << (2 * e);
+            word[j] = v;
         }
-        *reinterpret_cast<uint2 *>(codes + n * (K / 8) + k0 / 8) = make_uint2(w0, w1);
+        *reinterpret_cast<uint4 *>(codes + n * (K / 16) + col / 16) = make_uint4(word[0], word[1], word[2], word[3]);
+    } else {
+        uint32_t word[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v |= quant_code(w[8 * j + e], p, qmax, p.clamp) << (4 * e);
+            word[j] = v;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(codes + n * (K / 8) + col / 8);
+        dst[0] = make_uint4(word[0], word[1], word[2], word[3]);
+        dst[1] = make_uint4(word[4], word[5], word[6], word[7]);
     }
-    if (sub == 0) {
+    if (half == 0) {
         scales[n * G + grp] = __float2half_rn(p.sh);
         zeros[n * G + grp] = __float2half_rn(p.z);
     }
