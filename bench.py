@@ -276,6 +276,13 @@ def run_reference(args):
     return 0
 
 
+def rank_layer_config(base, rank):
+    """Each rank quantizes its own layer of the base shape (independent problems):
+    the same recipe with seed + 1000 * rank."""
+    from awq_activation_aware_b200 import synth
+    return synth.LayerConfig(**{**base.as_dict(), "seed": base.seed + 1000 * rank})
+
+
 def run_awq(args):
     import torch
 
@@ -286,9 +293,7 @@ def run_awq(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist_init(world, "nccl")
-    base = synth.CONFIGS[args.config]
-    # every rank quantizes its own layer of the same shape (independent problems)
-    cfg = synth.LayerConfig(**{**base.as_dict(), "seed": base.seed + 1000 * rank})
+    cfg = rank_layer_config(synth.CONFIGS[args.config], rank)
     W, X, _ = synth.generate(cfg)
     alphas_np = synth.default_alphas()
     n_alpha = len(alphas_np)
