@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "AWQError", "lib", "act_stats", "alpha_scales", "quant_dequant", "search_workspace_bytes",
     "search_layer", "pack", "quantize_layer", "get_status", "set_wait_timeout_ms", "default_alphas",
-    "profile_next_search",
+    "profile_next_search", "quantize_shared_input", "selftest_bounded_wait",
     "LIB_PATH",
 ]
 
@@ -60,6 +60,8 @@ def lib():
     L.awq_get_status.argtypes = [P]
     L.awq_set_wait_timeout_ms.argtypes = [ctypes.c_uint32]
     L.awq_set_wait_timeout_ms.restype = None
+    L.awq_selftest_bounded_wait.argtypes = [P]
+    L.awq_selftest_bounded_wait.restype = ctypes.c_int
     L.awq_profile_next_search.argtypes = [P, P]
     L.awq_profile_next_search.restype = None
     L.awq_status_string.argtypes = [ctypes.c_int]
@@ -207,9 +209,36 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None
     return res
 
 
+def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,
+                          group: int = 128, stream=None) -> list:
+    """Layers that read the same input (an MLP's gate and up projections, an
+    attention block's Q/K/V) must share one s, because 1/s is folded into that
+    one input.  Their weights are stacked row-wise and searched as one layer,
+    so the loss is the sum of their output errors and one alpha is chosen for
+    all of them; the packed output is split back per layer.
+
+    Returns one dict per layer (codes, scales, zeros) plus the shared
+    best_idx, s_best, losses and a."""
+    rows = [w.shape[0] for w in Ws]
+    W = torch.cat([w.contiguous() for w in Ws], dim=0)
+    res = quantize_layer(W, X, alphas, bits, group, stream=stream)
+    out, r0 = [], 0
+    for n in rows:
+        d = {k: res[k][r0:r0 + n] for k in ("codes", "scales", "zeros")}
+        d.update({k: res[k] for k in ("best_idx", "s_best", "losses", "a")})
+        out.append(d)
+        r0 += n
+    return out
+
+
 def get_status(stream=None) -> None:
     """Synchronise and raise if a kernel reported an error on the device."""
     _check(lib().awq_get_status(_stream(stream)), "awq_get_status")
+
+
+def selftest_bounded_wait(stream=None) -> None:
+    """Launch the bounded-wait self-test (see include/awq.h); the next get_status raises AWQError(TIMEOUT)."""
+    _check(lib().awq_selftest_bounded_wait(_stream(stream)), "awq_selftest_bounded_wait")
 
 
 def set_wait_timeout_ms(ms: int) -> None:

@@ -368,6 +368,13 @@ awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcf
     return last_launch();
 }
 
+awq_status awq_selftest_bounded_wait(void *stream) {
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    awq::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)g_timeout_ms.load() * 1000000ull);
+    return last_launch();
+}
+
 awq_status awq_get_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return AWQ_ERR_CUDA;

@@ -770,4 +770,24 @@ pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
     }
 }
 
+// ===========================================================================
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// ever arrives on.  The wait gives up after the library's limit, raises the
+// device timeout flag and returns -- the path every role of the search kernel
+// takes when a pipeline stalls.  (Library infrastructure; the pages have no
+// counterpart.)
+// ===========================================================================
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, timeout_ns);
+    __syncthreads();
+}
+
 }  // namespace awq

@@ -52,6 +52,8 @@ CONFIGS = {
                             4096, 4096, 4096, 0.02, 41, 10.0, 100.0, 4, 128, 1),
     "mlp_gate11008": LayerConfig("LLaMA-7B MLP gate/up 11008x4096, T=4096, INT4 g128",
                                  11008, 4096, 4096, 0.02, 41, 10.0, 100.0, 4, 128, 2),
+    "mlp_gateup22016": LayerConfig("LLaMA-7B MLP gate+up stacked 22016x4096 (one shared X), T=4096, INT4 g128",
+                                   22016, 4096, 4096, 0.02, 41, 10.0, 100.0, 4, 128, 2),
     "mlp_down4096": LayerConfig("LLaMA-7B MLP down 4096x11008, T=4096, INT4 g128",
                                 4096, 11008, 4096, 0.02, 110, 10.0, 100.0, 4, 128, 2),
     "attn4096_int3": LayerConfig("4096x4096, T=4096, INT3 g128", 4096, 4096, 4096,

@@ -191,6 +191,15 @@ AWQ_API awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a,
  * a pending CUDA error.  AWQ_OK otherwise. */
 AWQ_API awq_status awq_get_status(void *stream);
 
+/* Self-test of device-side failure detection (no counterpart on the pages: it
+ * checks the library, not the method).  Launches one warp that waits on a
+ * barrier nothing ever completes, with the same bounded wait every role of the
+ * search kernel uses.  Expected: the launch returns AWQ_OK, the kernel ends by
+ * itself after the wait limit (awq_set_wait_timeout_ms), and the next
+ * awq_get_status(stream) reports AWQ_ERR_TIMEOUT and clears it; the context
+ * stays usable.  Never traps, never faults. */
+AWQ_API awq_status awq_selftest_bounded_wait(void *stream);
+
 /* Upper bound, in milliseconds, on any single wait inside the library's
  * kernels (default 4000).  Applies to launches made after the call. */
 AWQ_API void awq_set_wait_timeout_ms(uint32_t ms);

@@ -48,7 +48,7 @@ def unpack_codes(codes, bits):
 
 
 @pytest.mark.parametrize("name", ["attn4096", "attn4096_int3", "attn4096_int2", "mlp_gate11008",
-                                  "mlp_down4096", "mlp_up28672"])
+                                  "mlp_gateup22016", "mlp_down4096", "mlp_up28672"])
 def test_fullsize_layer(awq, name):
     cfg = synth.CONFIGS[name]
     W, X, _ = synth.generate(cfg)

@@ -112,6 +112,27 @@ def test_bad_alpha_reported(awq):
     awq.get_status()                             # the flag is cleared
 
 
+def test_bounded_wait_reports_timeout_and_context_survives(awq):
+    """A wait that can never complete ends by itself, is reported as
+    AWQ_ERR_TIMEOUT, and the context still runs the search correctly."""
+    awq.get_status()
+    awq.set_wait_timeout_ms(100)
+    try:
+        awq.selftest_bounded_wait()
+        with pytest.raises(awq.AWQError) as e:
+            awq.get_status()
+        assert e.value.code == 4                 # AWQ_ERR_TIMEOUT
+        awq.get_status()                         # cleared
+    finally:
+        awq.set_wait_timeout_ms(2000)
+    W, X = gen(128, 256, 300, seed=41)
+    a = oracle.act_stats(X)
+    alphas = synth.default_alphas()
+    got = host(awq.search_layer(dev(W), dev(X), dev(a), dev(alphas), 4, 128))
+    awq.get_status()
+    np.testing.assert_allclose(got, oracle.search(W, X, a, 4, 128, alphas)["losses"], rtol=LOSS_RTOL)
+
+
 # ---------------------------------------------------------------------------
 # a3/a4: W_hat bit-exact for every alpha, and on degenerate groups
 # ---------------------------------------------------------------------------
@@ -270,3 +291,33 @@ def test_whole_path_layer512(awq):
     err = oracle.output_error_sum(W, what, X).sum() / (cfg.N * cfg.T)
     assert err == pytest.approx(ref["losses"][best], rel=LOSS_RTOL)
     assert ref["losses"][best] < ref["losses"][0]          # better than plain RTN
+
+
+# ---------------------------------------------------------------------------
+# Layers sharing one input: one s for all, loss = sum of their output errors
+# ---------------------------------------------------------------------------
+def test_shared_input_joint_search(awq):
+    K, T = 256, 600
+    W1, X = gen(200, K, T, seed=51, outlier_frac=0.03)
+    W2, _ = gen(136, K, T, seed=52, outlier_frac=0.03)
+    alphas = synth.default_alphas()
+    res = awq.quantize_shared_input([dev(W1), dev(W2)], dev(X), dev(alphas), 4, 128)
+    awq.get_status()
+    a = oracle.act_stats(X)
+    Wst = np.concatenate([W1, W2], axis=0)
+    ref = oracle.search(Wst, X, a, 4, 128, alphas)
+    joint = host(res[0]["losses"]).astype(np.float64)
+    np.testing.assert_allclose(joint, ref["losses"], rtol=LOSS_RTOL)
+    # the joint loss is the row-weighted mean of the layers' own losses
+    l1 = oracle.search(W1, X, a, 4, 128, alphas)["losses"]
+    l2 = oracle.search(W2, X, a, 4, 128, alphas)["losses"]
+    np.testing.assert_allclose(ref["losses"], (200 * l1 + 136 * l2) / 336, rtol=1e-12)
+    best = int(host(res[0]["best_idx"])[0])
+    assert_alpha_choice(best, ref["losses"])
+    pk = oracle.pack(Wst, a, 4, 128, alphas, joint)
+    assert pk["best"] == best
+    codes = np.concatenate([host(r["codes"]) for r in res]).view(np.uint32)
+    assert np.array_equal(codes, pk["codes"])
+    assert np.array_equal(np.concatenate([host(r["scales"]) for r in res]).view(np.uint16),
+                          pk["scales"].view(np.uint16))
+    assert np.array_equal(host(res[1]["zeros"]).view(np.uint16), pk["zeros"][200:].view(np.uint16))
