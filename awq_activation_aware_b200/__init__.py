@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "AWQError", "lib", "act_stats", "alpha_scales", "quant_dequant", "search_workspace_bytes",
     "search_layer", "pack", "quantize_layer", "get_status", "set_wait_timeout_ms", "default_alphas",
-    "profile_next_search", "quantize_shared_input", "selftest_bounded_wait",
+    "profile_next_search", "quantize_shared_input", "selftest_bounded_wait", "qlinear",
     "LIB_PATH",
 ]
 
@@ -60,6 +60,10 @@ def lib():
     L.awq_get_status.argtypes = [P]
     L.awq_set_wait_timeout_ms.argtypes = [ctypes.c_uint32]
     L.awq_set_wait_timeout_ms.restype = None
+    L.awq_qlinear_workspace_bytes.argtypes = [i64, i64, i64]
+    L.awq_qlinear_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_qlinear.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
+    L.awq_qlinear.restype = ctypes.c_int
     L.awq_selftest_bounded_wait.argtypes = [P]
     L.awq_selftest_bounded_wait.restype = ctypes.c_int
     L.awq_profile_next_search.argtypes = [P, P]
@@ -207,6 +211,25 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None
         res = {k: v.to("cpu", non_blocking=True) for k, v in res.items()}
         torch.cuda.current_stream().synchronize()
     return res
+
+
+def qlinear(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, s_best: torch.Tensor,
+            X: torch.Tensor, bits: int = 4, group: int = 128, workspace: torch.Tensor | None = None,
+            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X W_hat^T straight from the packed codes (the layer's input X is fp16 [T, K];
+    1/s_best is folded into it).  Returns float32 [T, N]."""
+    _rowmajor(X, "X")
+    N = codes.shape[0]
+    T, K = X.shape
+    need = int(lib().awq_qlinear_workspace_bytes(T, K, N))
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
+    Y = out if out is not None else torch.empty((T, N), dtype=torch.float32, device=X.device)
+    _check(lib().awq_qlinear(_dev(codes, torch.int32, "codes"), _dev(scales, torch.float16, "scales"),
+                             _dev(zeros, torch.float16, "zeros"), _dev(s_best, torch.float32, "s_best"), N, K,
+                             _qcfg(bits, group), _dev(X, torch.float16, "X"), T, X.stride(0),
+                             _dev(Y, torch.float32, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                             _stream(stream)), "awq_qlinear")
+    return Y
 
 
 def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,

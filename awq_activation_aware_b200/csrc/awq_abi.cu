@@ -98,6 +98,15 @@ awq_status device_info(DevInfo &out) {
             clusters = d.sms / 2;
         }
         d.max_pairs = clusters < d.sms / 2 ? clusters : d.sms / 2;
+        if (cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess)
+            return AWQ_ERR_CUDA;
         d.search_attr = true;
     }
     out = d;
@@ -135,6 +144,22 @@ bool encode_rows_map(CUtensorMap *m, const void *base, int64_t rows, int64_t col
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Packed codes [rows][words] (uint32) as a 2-D tensor, boxes of
+// qlv::WORDS words x qlv::ROWS rows, no swizzle; rows and words past the end
+// read as zeros.
+bool encode_codes_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64_t words) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)words * 4};
+    cuuint32_t box[2] = {(cuuint32_t)awq::qlv::WORDS, (cuuint32_t)awq::qlv::ROWS};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(codes), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -180,6 +205,25 @@ awq_status noalloc_scratch(void **out) {
     }
     *out = g_noalloc_ptr[dev];
     return AWQ_OK;
+}
+
+// Workspace of awq_qlinear: x' = x / s as binary32 [T_pad][Kp] in the decode
+// kernel's stage order (T rounded up to the tokens of one pass, K to the
+// widest stage), the partial sums of row blocks split across blocks, and the
+// per row block arrival counters.
+constexpr int64_t kQlMaxGrid = 1024;
+int64_t ql_rows_pad(int64_t T) { return (T + awq::qlv::TOKENS - 1) / awq::qlv::TOKENS * awq::qlv::TOKENS; }
+int64_t ql_cols_pad(int64_t K, int64_t sc) { return (K + sc - 1) / sc * sc; }
+size_t ql_xs_bytes(int64_t T, int64_t K) {
+    return round_up(sizeof(float) * (size_t)ql_rows_pad(T) * ql_cols_pad(K, awq::qlv::MAX_STAGE_COLS), 256);
+}
+int64_t ql_row_blocks(int64_t N) { return (N + awq::qlv::ROWS - 1) / awq::qlv::ROWS; }
+size_t ql_part_bytes(int64_t N) {
+    return round_up(sizeof(float) * (size_t)(ql_row_blocks(N) + kQlMaxGrid) * awq::qlv::SLOT_FLOATS, 256);
+}
+size_t qlinear_ws(int64_t T, int64_t K, int64_t N) {
+    return ql_xs_bytes(T, K) + ql_part_bytes(N) +
+           round_up(sizeof(unsigned) * (size_t)ql_row_blocks(N) * awq::qlv::RGROUPS, 256);
 }
 
 }  // namespace
@@ -366,6 +410,80 @@ awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcf
         awq::pack_kernel<1><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
                                                              (__half *)scales, (__half *)zeros);
     return last_launch();
+}
+
+size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+    if (T < 1 || K < 1 || N < 1) return 0;
+    return qlinear_ws(T, K, N);
+}
+
+awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
+                                  int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
+                                  void *ws, size_t ws_bytes, void *stream) {
+    if (!codes || !scales || !zeros || !s_best || !X || !Y) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(s_best) || !aligned16(X) ||
+        !aligned16(Y))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || T < 1 || T > kMaxDim || K < 64 || K > kMaxDim || K % 64 ||
+        K % q.group_size || ldx < K || ldx % 8)
+        return AWQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qlinear_ws(T, K, N) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool c2 = q.bits == 2;
+    const int64_t cpw = c2 ? 16 : 8;                       // codes per 32-bit word
+    const int64_t sc = awq::qlv::WORDS * cpw;              // columns per stage
+    const int64_t Kp = ql_cols_pad(K, sc), T_pad = ql_rows_pad(T);
+    const int64_t row_blocks = ql_row_blocks(N);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    float *xs = reinterpret_cast<float *>(w8);
+    float *part = reinterpret_cast<float *>(w8 + ql_xs_bytes(T, K));
+    unsigned *cnt = reinterpret_cast<unsigned *>(w8 + ql_xs_bytes(T, K) + ql_part_bytes(N));
+    {
+        int grid = blocks_for(T_pad * Kp / 4, 256);
+        if (grid > 4 * d.sms) grid = 4 * d.sms;
+        awq::qlinear_prep_kernel<<<grid, 256, 0, st>>>((const __half *)X, T, T_pad, K, Kp, ldx, (int)cpw, s_best,
+                                                       xs, cnt, row_blocks * awq::qlv::RGROUPS);
+        if (awq_status e = last_launch()) return e;
+    }
+    CUtensorMap tmap;
+    if (!encode_codes_map(&tmap, codes, N, K / cpw)) return AWQ_ERR_CUDA;
+    awq::qlv::Args A;
+    A.Kp = Kp;
+    A.scales = (const __half *)scales;
+    A.zeros = (const __half *)zeros;
+    A.N = N;
+    A.K = K;
+    A.G = (int)(K / q.group_size);
+    A.group = q.group_size;
+    A.n_steps = Kp / sc;
+    A.units = row_blocks * A.n_steps;
+    A.gps = (int)(sc / q.group_size);
+    A.sz_mode = A.G % 8 == 0 ? 16 : (A.G % 2 == 0 ? 4 : 2);
+    const int tt = T == 1 ? 1 : 2;
+    A.n_stages = awq::qlv::ring_stages((int)sc, tt, A.gps);
+    const size_t smem = (size_t)A.n_stages * awq::qlv::stage_bytes((int)sc, tt, A.gps) + awq::qlv::fixed_smem();
+    A.part = part;
+    A.cnt = cnt;
+    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+    // one block per SM, each streaming an equal share of the units
+    int64_t grid = d.sms < kQlMaxGrid ? d.sms : kQlMaxGrid;
+    if (grid > A.units) grid = A.units;
+    for (int64_t t0 = 0; t0 < T; t0 += awq::qlv::TOKENS) {
+        A.xs = xs + t0 * Kp;
+        A.Y = Y + t0 * N;
+        A.T = (int)(T - t0 < awq::qlv::TOKENS ? T - t0 : awq::qlv::TOKENS);
+        // one token alone takes the single-token kernel; an odd last token of a
+        // longer batch reads the zero row that pads x'
+#define AWQ_QL_LAUNCH(CB, TT) \
+    awq::qlinear_gemv_kernel<CB, TT><<<(unsigned)grid, awq::qlv::THREADS, smem, st>>>(tmap, A)
+        if (T == 1) { if (c2) AWQ_QL_LAUNCH(2, 1); else AWQ_QL_LAUNCH(4, 1); }
+        else { if (c2) AWQ_QL_LAUNCH(2, 2); else AWQ_QL_LAUNCH(4, 2); }
+#undef AWQ_QL_LAUNCH
+        if (awq_status e = last_launch()) return e;
+    }
+    return AWQ_OK;
 }
 
 awq_status awq_selftest_bounded_wait(void *stream) {

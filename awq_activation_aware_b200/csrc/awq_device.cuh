@@ -109,27 +109,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// Packed binary32 pair arithmetic (sm_100 FMUL2/FADD2/FFMA2), as PTX with an
-// explicit .rn rounding modifier.  Each multiply and add must round exactly
+// Packed binary32 pair arithmetic (sm_100 FMUL2/FFMA2) through the CUDA
+// builtins with round-to-nearest-even per component.  Each multiply and add must round exactly
 // once where the quantizer's definition says so; the library is built with
 // -fmad=false so that no multiply-add pair is contracted behind our back, and
 // every intended fusion is written as fma2_rn / __fmaf_rn.
-__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // Quantize-dequantize-unscale of two neighbouring weights in packed binary32
 // pairs, as the search producer evaluates it:
@@ -232,15 +218,17 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parit
 // Bounded wait: returns false (after raising the device timeout flag and the
 // CTA's abort flag) when the phase does not complete within about `limit_ns`,
 // or when another role of the CTA has already aborted.  Never traps.  Waiting
-// threads are suspended by the hardware between polls (and may also sleep
-// `sleep_ns` between polls); the abort flag and the clock are checked only
-// every 16 polls to keep a long wait cheap in issue slots.
+// threads are suspended by the hardware between polls (kSuspend; otherwise
+// they poll) and may also sleep `sleep_ns` between polls; the abort flag and
+// the clock are checked only every 16 polls to keep a long wait cheap in
+// issue slots.
+template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                   uint64_t limit_ns, uint32_t sleep_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = 0;
     for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if (kSuspend ? mbar_try_wait_hint(bar, parity, 20000u) : mbar_try_wait(bar, parity)) return true;
         if (sleep_ns) __nanosleep(sleep_ns);
         if ((n & 15u) == 0) {
             if (*abort_flag) return false;
@@ -257,10 +245,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                uint64_t limit_ns, uint32_t sleep_ns = 0) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, limit_ns, sleep_ns) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded<kSuspend>(bar, parity, abort_flag, limit_ns, sleep_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     return ok != 0;
 }
@@ -315,6 +304,18 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
             smem_u32(smem_dst)),
         "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+// Asynchronous global -> shared copies of 16 (L2 only) or 4 bytes, and the
+// arrive that fires on `bar` once all of this thread's earlier ones landed
+// (.noinc: the barrier's expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -771,6 +771,363 @@ pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
 }
 
 // ===========================================================================
+// Consumer of the packed format: the quantized linear layer Y = X W_hat^T for
+// a few tokens (decode), read straight from codes, fp16 scales and zeros
+// ([AWQ-note] "Tiny Chat": dequantize inside the kernel, never writing fp16
+// weights to DRAM).  Definition (fp32 accumulation, order unspecified):
+//   Y[t, n] = sum_k x'[t, k] (q[n, k] - z[n, G]) sh[n, G],
+//   x'[t, k] = RN32(x[t, k] RN32(1 / s_k))      (1/s folded into the input)
+// The work is HBM-bound on the codes (K/2 bytes per row at 4 bits), so the
+// kernel is SIMT: codes stream through a TMA ring in shared memory, (q - z) is
+// dequantized exactly by byte permutes, and the products are packed fp32
+// multiply-adds.
+// ===========================================================================
+namespace qlv {
+constexpr int ROWS = 64;                 // W rows per row block
+constexpr int RGROUPS = 8;               // row groups of RPW rows
+constexpr int RPW = ROWS / RGROUPS;
+constexpr int CWARPS = 2 * RGROUPS;      // consumer warps: a row group x a column half
+constexpr int THREADS = (CWARPS + 1) * 32;
+constexpr int MAX_STAGES = 4;
+constexpr int TOKENS = 2;                // tokens per pass (activations stay in registers)
+constexpr int WORDS = 128;               // code words per row per stage (512 B)
+constexpr int CODE_BYTES = ROWS * WORDS * 4;                 // 32 KiB
+constexpr int MAX_STAGE_COLS = WORDS * 16;                   // columns per stage at 2 bits
+constexpr int SLOT_FLOATS = RGROUPS * 32;                    // one partial-sum slot (a row block segment)
+constexpr int PAIR_FLOATS = RGROUPS * 2 * 32;                // column-half exchange, 2 slots per row group
+constexpr int SMEM_LIMIT = 226 * 1024;         // dynamic shared memory per block (static use stays below 1 KiB)
+// One ring stage: codes [ROWS][WORDS] (TMA tile), x' [TT][SC] floats, then
+// the fp16 scales and zeros of the stage's gps groups, [2][ROWS][gps].
+__host__ __device__ constexpr int stage_bytes(int sc, int tt, int gps) {
+    return (CODE_BYTES + tt * sc * 4 + 4 * ROWS * gps + 127) / 128 * 128;
+}
+__host__ __device__ constexpr int fixed_smem() {
+    return PAIR_FLOATS * 4 + (2 * MAX_STAGES + 4 * RGROUPS) * 8 + 128;
+}
+inline int ring_stages(int sc, int tt, int gps) {
+    const int n = (SMEM_LIMIT - fixed_smem()) / stage_bytes(sc, tt, gps);
+    return n < MAX_STAGES ? n : MAX_STAGES;
+}
+
+struct Args {
+    const float *xs;          // x' of this pass's tokens, stage-permuted rows of Kp floats
+    int64_t Kp;
+    const __half *scales, *zeros;
+    int64_t N, K;
+    int G, group, T;          // T: tokens of this pass (<= TT)
+    int gps;                  // groups per stage
+    int n_stages;             // ring depth
+    int sz_mode;              // scale/zero copies: 16 = 16-byte, 4 = 4-byte, 2 = plain loads
+    int64_t n_steps, units;   // stages per row block; row blocks x n_steps
+    float *Y;                 // this pass's output rows, [T][N]
+    float *part;              // partial sums of split row blocks, slot rb + b (see the kernel)
+    unsigned *cnt;            // [row blocks][RGROUPS] arrival counters, zero between launches
+    uint64_t timeout_ns;
+};
+
+// The block whose unit range [units*b/grid, units*(b+1)/grid) holds unit u.
+__device__ __forceinline__ int64_t block_of(int64_t u, int64_t units, int64_t grid) {
+    return ((u + 1) * grid - 1) / units;
+}
+}  // namespace qlv
+
+// x'[t, k] = RN32(x[t, k] RN32(1 / s_k)) for t < T_pad, stored in the order the
+// decode kernel reads a stage of SC = 128 CPW columns: the stage's columns
+// split into two halves, each lane owning 2 consecutive code words (2 CPW
+// columns) of a half; the 4-column chunk q of word i of lane l in half h sits
+// at float4 slot ((2h + i) CPW/4 + q) * 32 + l, so a warp's 16-byte reads of
+// one chunk cover 512 contiguous bytes.  Rows t >= T and columns k >= K are
+// zero.  Also clears the decode kernel's arrival counters.
+__global__ void qlinear_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t T_pad, int64_t K,
+                                    int64_t Kp, int64_t ldx, int CPW, const float *__restrict__ s,
+                                    float *__restrict__ xs, unsigned *__restrict__ cnt, int64_t n_cnt) {
+    const int SC = qlv::WORDS * CPW;
+    const int64_t chunks = Kp / 4, total = T_pad * chunks;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (int64_t i = i0; i < n_cnt; i += stride) cnt[i] = 0u;
+    for (int64_t i = i0; i < total; i += stride) {
+        const int64_t t = i / chunks, d = i - t * chunks;
+        const int64_t j = d / (SC / 4);
+        const int slot = (int)(d - j * (SC / 4));
+        const int l = slot % 32, rest = slot / 32;
+        const int q = rest % (CPW / 4), wi = (rest / (CPW / 4)) % 2, h = rest / (CPW / 2);
+        const int64_t c0 = j * SC + h * (SC / 2) + l * 2 * CPW + wi * CPW + 4 * q;
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (t < T && c0 < K) {
+            const uint2 hx = *reinterpret_cast<const uint2 *>(X + t * ldx + c0);
+            const float4 sv = *reinterpret_cast<const float4 *>(s + c0);
+            const float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&hx.x));
+            const float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&hx.y));
+            v = make_float4(__fmul_rn(x01.x, __frcp_rn(sv.x)), __fmul_rn(x01.y, __frcp_rn(sv.y)),
+                            __fmul_rn(x23.x, __frcp_rn(sv.z)), __fmul_rn(x23.y, __frcp_rn(sv.w)));
+        }
+        reinterpret_cast<float4 *>(xs)[i] = v;
+    }
+}
+
+// (q - z) of the 32/CB codes in one 32-bit word as exact binary32 values: each
+// code c becomes the float 2^23 + c by placing its byte under the exponent bits
+// of 2^23 (one byte permute), and one packed subtraction of 2^23 + z leaves
+// q - z.
+template <int CB>
+__device__ __forceinline__ void dequant_word(uint32_t w, float zsub, float *d) {
+    const float2 off = make_float2(-zsub, -zsub);
+    const float2 one = make_float2(1.0f, 1.0f);
+    if (CB == 4) {
+        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;   // codes 2b / 2b+1 in byte b
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const float2 f = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | b)),
+                                         __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | b)));
+            const float2 r = fma2_rn(f, one, off);
+            d[2 * b] = r.x;
+            d[2 * b + 1] = r.y;
+        }
+    } else {
+        uint32_t m[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m[j] = (w >> (2 * j)) & 0x03030303u;     // code 4b + j in byte b of m[j]
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                const float2 f = make_float2(__uint_as_float(__byte_perm(m[j], 0x4B000000u, 0x7440u | b)),
+                                             __uint_as_float(__byte_perm(m[j + 1], 0x4B000000u, 0x7440u | b)));
+                const float2 r = fma2_rn(f, one, off);
+                d[4 * b + j] = r.x;
+                d[4 * b + j + 1] = r.y;
+            }
+    }
+}
+
+// Reduce V values spread over the 32 lanes of a warp so that lane l ends with
+// the warp-wide sum of value (l % V) -- a reduce-scatter butterfly.
+template <int V>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[V]) {
+#pragma unroll
+    for (int width = V; width > 1; width >>= 1) {
+        const int half = width >> 1;
+        const bool upper = (threadIdx.x & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    float x = v[0];
+#pragma unroll
+    for (int off = V; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// Persistent decode kernel, one block per SM.  The work is a list of units
+// (row block of 64 W rows, stage of 1024 columns at 4 bits / 2048 at 2 bits),
+// row block major; block b takes the contiguous range
+// [units*b/grid, units*(b+1)/grid), so every SM streams the same number of
+// code bytes.  Warp 16 feeds a shared-memory ring (up to 4 stages): lane 0
+// issues the unit's codes (one 2-D TMA tile, 64 rows x 128 words = 32 KiB)
+// and the stage's x' of each token (one bulk copy per token); all 32 lanes
+// copy the fp16 scales and zeros of the unit's rows and groups (cp.async,
+// counted on the same barrier).  Warps 0-15 each own 8 rows (row group
+// warp % 8) and one half of the stage's columns (warp / 8); a lane takes 2
+// code words of each row and the matching x' (16-byte, conflict-free
+// shared-memory reads in the permuted order).  When a row block's segment
+// ends, the column-half warp hands its sums to its row group's other warp
+// through a 2-slot shared-memory exchange.  A row block finished inside one
+// block is written to Y directly; one split across blocks leaves a partial
+// sum per block, and the last block to arrive (counted per row block and row
+// group) adds the partials in block order, so Y does not depend on timing.
+// Partial slot of (row block rb, block b): rb + b, unique because both grow
+// along the unit list.
+template <int CB, int TT>
+__global__ void __launch_bounds__(qlv::THREADS, 1)
+qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::Args A) {
+    using namespace qlv;
+    constexpr int CPW = 32 / CB;                 // columns per word
+    constexpr int SC = WORDS * CPW;              // columns per stage
+    constexpr int V = RPW * TT;
+    constexpr uint32_t TX_BYTES = CODE_BYTES + TT * SC * 4;
+    const int gps = A.gps;
+    const uint32_t STAGE_BYTES = stage_bytes(SC, TT, gps);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float *pair_buf = reinterpret_cast<float *>(base + A.n_stages * STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(pair_buf + PAIR_FLOATS);
+    uint64_t *empty = full + MAX_STAGES;
+    uint64_t *pair_full = empty + MAX_STAGES;    // [RGROUPS][2]
+    uint64_t *pair_empty = pair_full + 2 * RGROUPS;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t grid = gridDim.x;
+    const int64_t u_begin = A.units * blockIdx.x / grid, u_end = A.units * (blockIdx.x + 1) / grid;
+    if (threadIdx.x == 0) {
+        // full: the producer's expect-tx arrive plus one cp.async arrive per lane
+        for (int i = 0; i < A.n_stages; ++i) { mbar_init(&full[i], 33); mbar_init(&empty[i], CWARPS); }
+        for (int i = 0; i < 2 * RGROUPS; ++i) { mbar_init(&pair_full[i], 1); mbar_init(&pair_empty[i], 1); }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == CWARPS) {                        // producer
+        if (lane == 0) tma_prefetch_desc(&tmap_codes);
+        int st = 0;
+        uint32_t ph = 0;
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+        const int per = A.sz_mode / 2;                   // groups per copy (16- or 4-byte modes)
+        const int lcpr = __ffs(A.gps / per) - 1;          // log2(copies per row); gps and per are powers of 2
+        static_assert(ROWS == 64, "copy indexing takes 6 bits for the row");
+        for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0, ++rb) : 0)) {
+            if (!mbar_wait_warp(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
+            uint8_t *stage = base + st * STAGE_BYTES;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[st], TX_BYTES);
+                tma_load_2d(stage, &tmap_codes, (int32_t)(j * WORDS), (int32_t)(rb * ROWS), &full[st]);
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    bulk_load(stage + CODE_BYTES + t * SC * 4, A.xs + t * A.Kp + j * SC, SC * 4, &full[st]);
+            }
+            // scales then zeros of rows rb*64.. and groups j*gps.. (groups past G
+            // belong to lanes past K, which never read them; rows past N repeat row N-1)
+            __half *sz = reinterpret_cast<__half *>(stage + TX_BYTES);
+            const int64_t g0 = j * gps;
+            if (A.sz_mode == 2) {
+                for (int e = lane; e < 2 * ROWS * gps; e += 32) {
+                    const int arr = e / (ROWS * gps), rem = e % (ROWS * gps), r = rem / gps, g = rem % gps;
+                    int64_t n = rb * ROWS + r;
+                    n = n < A.N ? n : A.N - 1;
+                    if (g0 + g < A.G) sz[e] = (arr ? A.zeros : A.scales)[n * A.G + g0 + g];
+                }
+                mbar_arrive(&full[st]);
+            } else {
+                for (int e = lane; e < (2 * ROWS) << lcpr; e += 32) {
+                    const int arr = e >> (6 + lcpr), r = (e >> lcpr) & (ROWS - 1), c = e & ((1 << lcpr) - 1);
+                    int64_t n = rb * ROWS + r;
+                    n = n < A.N ? n : A.N - 1;
+                    if (g0 + c * per >= A.G) continue;
+                    const __half *src = (arr ? A.zeros : A.scales) + n * A.G + g0 + c * per;
+                    __half *dst = sz + (arr * ROWS + r) * gps + c * per;
+                    if (A.sz_mode == 16) cp_async_16(dst, src); else cp_async_4(dst, src);
+                }
+                cp_async_arrive_noinc(&full[st]);
+            }
+            if (++st == A.n_stages) { st = 0; ph ^= 1u; }
+        }
+    } else {                                     // consumers
+        const int rg = warp % RGROUPS, hh = warp / RGROUPS;
+        const int lane_col = hh * (SC / 2) + lane * 2 * CPW;     // first column of the lane in a stage
+        const int gl = lane_col / A.group;                        // the lane's group within a stage
+        float acc[RPW][TT];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int t = 0; t < TT; ++t) acc[r][t] = 0.0f;
+        int st = 0, ps = 0;
+        uint32_t ph = 0, pph = 0;
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps - 1;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            if (++j == A.n_steps) { j = 0; ++rb; }
+            if (!mbar_wait_warp(&full[st], ph, &abort_flag, A.timeout_ns)) break;
+            const uint8_t *stage = base + st * STAGE_BYTES;
+            if (j * SC + lane_col < A.K) {                       // lanes past K hold zero fill
+                const __half *sz = reinterpret_cast<const __half *>(stage + TX_BYTES);
+                uint2 w[RPW];
+                float zs[RPW], sh[RPW];
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    w[r] = *reinterpret_cast<const uint2 *>(stage + ((rg * RPW + r) * WORDS + hh * 64 + 2 * lane) * 4);
+                    sh[r] = __half2float(sz[(rg * RPW + r) * gps + gl]);
+                    zs[r] = __fadd_rn(8388608.0f, __half2float(sz[(ROWS + rg * RPW + r) * gps + gl]));
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float x[TT][CPW];
+#pragma unroll
+                    for (int t = 0; t < TT; ++t)
+#pragma unroll
+                        for (int q = 0; q < CPW / 4; ++q) {
+                            const float4 v = *reinterpret_cast<const float4 *>(
+                                stage + CODE_BYTES + (t * SC + (((hh * 2 + i) * (CPW / 4) + q) * 32 + lane) * 4) * 4);
+                            x[t][4 * q] = v.x; x[t][4 * q + 1] = v.y; x[t][4 * q + 2] = v.z; x[t][4 * q + 3] = v.w;
+                        }
+#pragma unroll
+                    for (int r = 0; r < RPW; ++r) {
+                        float d[CPW];
+                        dequant_word<CB>(i == 0 ? w[r].x : w[r].y, zs[r], d);
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) {
+                            float2 s2 = mul2_rn(make_float2(x[t][0], x[t][1]), make_float2(d[0], d[1]));
+#pragma unroll
+                            for (int e = 2; e < CPW; e += 2)
+                                s2 = fma2_rn(make_float2(x[t][e], x[t][e + 1]), make_float2(d[e], d[e + 1]), s2);
+                            acc[r][t] = __fmaf_rn(sh[r], __fadd_rn(s2.x, s2.y), acc[r][t]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);       // this warp is done with the stage
+            if (++st == A.n_stages) { st = 0; ph ^= 1u; }
+            if (j != A.n_steps - 1 && u != u_end - 1) continue;
+            // ---- row block rb ends here (or this block's range does): flush ----
+            float v[V];
+#pragma unroll
+            for (int r = 0; r < RPW; ++r)
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+                    v[r * TT + t] = acc[r][t];
+                    acc[r][t] = 0.0f;
+                }
+            float mine = warp_reduce_scatter<V>(v);
+            // the two column halves of the row group meet in shared memory
+            float *slot = pair_buf + (rg * 2 + ps) * 32;
+            if (hh == 1) {
+                if (!mbar_wait_warp(&pair_empty[rg * 2 + ps], pph ^ 1u, &abort_flag, A.timeout_ns)) break;
+                slot[lane] = mine;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pair_full[rg * 2 + ps]);
+                if (++ps == 2) { ps = 0; pph ^= 1u; }
+                continue;
+            }
+            if (!mbar_wait_warp(&pair_full[rg * 2 + ps], pph, &abort_flag, A.timeout_ns)) break;
+            mine = __fadd_rn(mine, slot[lane]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pair_empty[rg * 2 + ps]);
+            if (++ps == 2) { ps = 0; pph ^= 1u; }
+            const int r = (lane % V) / TT, t = lane % TT;
+            const int64_t n = rb * ROWS + rg * RPW + r;
+            const bool writer = lane < V && n < A.N && t < A.T;
+            const int64_t rb_u0 = rb * A.n_steps, rb_u1 = rb_u0 + A.n_steps;
+            if (u_begin <= rb_u0 && u_end >= rb_u1) {       // whole row block in this block
+                if (writer) A.Y[t * A.N + n] = mine;
+                continue;
+            }
+            A.part[(rb + blockIdx.x) * SLOT_FLOATS + rg * 32 + lane] = mine;
+            __threadfence();
+            __syncwarp();
+            const int64_t b0 = block_of(rb_u0, A.units, grid), b1 = block_of(rb_u1 - 1, A.units, grid);
+            unsigned old = 0;
+            if (lane == 0) old = atomicAdd(&A.cnt[rb * RGROUPS + rg], 1u);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old != (unsigned)(b1 - b0)) continue;
+            __threadfence();                              // last to arrive: sum the partials in block order
+            float y = 0.0f;
+            for (int64_t b = b0; b <= b1; ++b) y = __fadd_rn(y, __ldcg(&A.part[(rb + b) * SLOT_FLOATS + rg * 32 + lane]));
+            if (writer) A.Y[t * A.N + n] = y;
+            if (lane == 0) A.cnt[rb * RGROUPS + rg] = 0u;    // ready for the next launch
+        }
+    }
+    // copies issued by the producer land before the block can leave
+    if (abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+}
+
+// ===========================================================================
 // Self-test of the bounded wait: one thread waits on an mbarrier that nothing
 // ever arrives on.  The wait gives up after the library's limit, raises the
 // device timeout flag and returns -- the path every role of the search kernel

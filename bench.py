@@ -54,6 +54,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    p.add_argument("--op", choices=["search", "qlinear"], default="search",
+                   help="search: the AWQ scale-search path (the benchmark); qlinear: the quantized "
+                        "linear layer on the packed output vs the fp16 GEMM")
+    p.add_argument("--tokens", default="1,4,16", help="token counts for --op qlinear")
     return p.parse_args()
 
 
@@ -428,10 +432,94 @@ def run_awq(args):
     return 0
 
 
+def run_qlinear(args):
+    """The packed layer as a linear layer at decode token counts: awq_qlinear
+    (codes streamed from HBM) against the fp16 GEMM (cuBLAS) on the dequantized
+    weights.  Each arm runs a sequence of distinct copies of the layer, as
+    the layers of a model run one after another, together more than 4x the L2,
+    so every call reads its weights from HBM; the sequence is captured in one
+    CUDA graph, so host launch cost is not counted.  One JSON line per token
+    count, with the time per call."""
+    import torch
+
+    import awq_activation_aware_b200 as awq
+    from awq_activation_aware_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    cfg = synth.CONFIGS[args.config]
+    W, X, _ = synth.generate(cfg)
+    Wd = torch.from_numpy(W).to(dev)
+    Xd = torch.from_numpy(X).to(dev)
+    al = awq.default_alphas(device=dev)
+    a = awq.act_stats(Xd)
+    losses = awq.search_layer(Wd, Xd, a, al, cfg.bits, cfg.group)
+    pk = awq.pack(Wd, a, al, losses, cfg.bits, cfg.group)
+    W_hat = awq.quant_dequant(Wd, pk["s_best"], cfg.bits, cfg.group)      # fp16 weights for the cuBLAS arm
+    awq.get_status()
+    del Wd
+    peaks, src = load_peaks()
+    hbm = peaks.get("hbm_gbs")
+    reps = max(args.steps, 3)
+    per = 16 if cfg.bits == 2 else 8
+    layer_bytes = (pk["codes"].numel() * pk["codes"].element_size() + pk["scales"].numel() * 2
+                   + pk["zeros"].numel() * 2)
+    total = 512 << 20                                    # > 4x the 126 MB L2
+    n_awq = max(2, -(-total // layer_bytes))
+    n_ref = max(2, -(-total // (W_hat.numel() * 2)))
+    copies = [{k: pk[k].clone() for k in ("codes", "scales", "zeros", "s_best")} for _ in range(n_awq)]
+    refs = [W_hat.clone() for _ in range(n_ref)]
+    del W_hat
+
+    def per_call_us(calls):
+        for fn in calls:                                 # warm-up, outside capture
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for fn in calls:
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(1_000_000)
+            b.record()
+            g.replay()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(b.elapsed_time(e) * 1e3 / len(calls))
+        del g
+        return statistics.median(ts)
+
+    for T in [int(t) for t in args.tokens.split(",")]:
+        Xt = Xd[:T].contiguous()
+        ws = torch.empty(int(awq.lib().awq_qlinear_workspace_bytes(T, cfg.K, cfg.N)), dtype=torch.uint8, device=dev)
+        Y = torch.empty((T, cfg.N), dtype=torch.float32, device=dev)
+        Yh = torch.empty((T, cfg.N), dtype=torch.float16, device=dev)
+        t_awq = per_call_us([
+            (lambda c=c: awq.qlinear(c["codes"], c["scales"], c["zeros"], c["s_best"], Xt, cfg.bits, cfg.group,
+                                     workspace=ws, out=Y)) for c in copies])
+        awq.get_status()
+        t_ref = per_call_us([(lambda w=w: torch.matmul(Xt, w.t(), out=Yh)) for w in refs])
+        nbytes = (cfg.N * cfg.K // per * 4 + 2 * 2 * cfg.N * cfg.K // cfg.group + cfg.K * 4 + T * cfg.K * 2
+                  + T * cfg.N * 4)
+        gbs = nbytes / (t_awq * 1e-6) / 1e9
+        print(json.dumps({"op": "qlinear", "config": cfg.name, "tokens": T, "awq_us": t_awq,
+                          "fp16_gemm_us": t_ref, "speedup_vs_fp16": t_ref / t_awq,
+                          "awq_bytes": nbytes, "awq_GBps": gbs, "hbm_frac": gbs / hbm if hbm else None,
+                          "hbm_peak_source": src, "layer_copies": [n_awq, n_ref],
+                          "launches": 1 + (T + 1) // 2}), flush=True)
+    awq.get_status()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "qlinear":
+        return run_qlinear(args)
     return run_awq(args)
 
 

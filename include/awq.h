@@ -191,6 +191,30 @@ AWQ_API awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a,
  * a pending CUDA error.  AWQ_OK otherwise. */
 AWQ_API awq_status awq_get_status(void *stream);
 
+/* Consumer of the packed format: the quantized linear layer for a few tokens
+ * (decode), computed straight from the codes ([AWQ-note] "Tiny Chat": the
+ * weights are dequantized inside the kernel and never written back as fp16;
+ * [QAS-QA] §5: the layer's input is divided by s).
+ *   Y[t, n] = sum_k x'[t, k] * (q[n, k] - z[n, k/g]) * sh[n, k/g],
+ *   x'[t, k] = RN32(x[t, k] * RN32(1 / s_best[k])),
+ * accumulated in binary32 (summation order unspecified).
+ *   codes, scales, zeros, s_best  awq_pack's outputs for W [N, K]
+ *   X   fp16 [T, ldx] (the layer's input, not yet divided by s)
+ *   Y   float [T, N] output, row-major
+ *   ws  device workspace of ws_bytes >= awq_qlinear_workspace_bytes(T, K, N),
+ *       256-byte aligned (x' as binary32, partial sums of row blocks split
+ *       across thread blocks, arrival counters); overwritten by every call
+ * Requires K % 64 == 0.  Built for small T (decode), where streaming the
+ * packed codes from HBM is the cost: tokens are processed two at a time, each
+ * pass re-reading the codes.  The summation order depends on the device's SM
+ * count, not on timing: repeated calls on one device give identical Y.
+ * Calls that share a workspace must be ordered (one stream). */
+AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
+AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
+                               const float *s_best, int64_t N, int64_t K, awq_qcfg q,
+                               const void *X, int64_t T, int64_t ldx, float *Y,
+                               void *ws, size_t ws_bytes, void *stream);
+
 /* Self-test of device-side failure detection (no counterpart on the pages: it
  * checks the library, not the method).  Launches one warp that waits on a
  * barrier nothing ever completes, with the same bounded wait every role of the

@@ -232,3 +232,35 @@ def round_to_step(w: float, step: float) -> float:
 def absmax_step(w, bits: int) -> float:
     w = np.ascontiguousarray(w, dtype=np.float64)
     return float(_load().awq_oracle_absmax_step(_ptr(w), w.size, int(bits)))
+
+
+# --------------------------------------------------------------------------
+# Consumer of the packed format: the quantized linear layer
+# ([AWQ-note] "Tiny Chat": dequantize inside the kernel, never writing fp16
+# weights back; [QAS-QA] §5: the activation is divided by s).
+# --------------------------------------------------------------------------
+
+def unpack_codes(codes: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Codes [N, K] from the packed words (least-significant first)."""
+    c = 2 if bits == 2 else 4
+    per = 32 // c
+    words = np.ascontiguousarray(codes).view(np.uint32).astype(np.uint64)
+    q = np.empty((words.shape[0], K), dtype=np.int64)
+    for i in range(per):
+        q[:, i::per] = (words >> np.uint64(c * i)) & np.uint64((1 << c) - 1)
+    return q
+
+
+def qlinear(codes, scales, zeros, s_best, X, bits: int, group: int) -> np.ndarray:
+    """Y[t, n] = sum_k x'[t, k] * (q[n, k] - z[n, k/g]) * sh[n, k/g] in binary64, where
+    x'[t, k] = RN32(x[t, k] * RN32(1 / s_k)) is the input divided by s (folded into
+    the input, as the layer's 1/s is in a deployed model)."""
+    X = np.asarray(X)
+    K = X.shape[1]
+    q = unpack_codes(codes, K, bits).astype(np.float64)
+    sh = np.repeat(np.asarray(scales).astype(np.float64), group, axis=1)
+    z = np.repeat(np.asarray(zeros).astype(np.float64), group, axis=1)
+    Wq = (q - z) * sh                                            # exact
+    rs = (np.float32(1.0) / np.asarray(s_best, dtype=np.float32)).astype(np.float32)
+    xs = (X.astype(np.float32) * rs[None, :]).astype(np.float32)  # one binary32 rounding
+    return xs.astype(np.float64) @ Wq.T

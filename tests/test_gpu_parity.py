@@ -321,3 +321,34 @@ def test_shared_input_joint_search(awq):
     assert np.array_equal(np.concatenate([host(r["scales"]) for r in res]).view(np.uint16),
                           pk["scales"].view(np.uint16))
     assert np.array_equal(host(res[1]["zeros"]).view(np.uint16), pk["zeros"][200:].view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# The quantized linear layer (consumer of the packed format)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,T,bits,group", [(1000, 1024, 1, 4, 128), (256, 512, 3, 3, 128),
+                                              (300, 512, 4, 2, 64), (64, 4096, 7, 4, 128),
+                                              (136, 640, 2, 2, 128), (520, 256, 9, 4, 64),
+                                              (4096, 3072, 1, 4, 128), (2048, 8192, 2, 4, 128),
+                                              (1000, 4096, 3, 2, 64)])
+def test_qlinear(awq, N, K, T, bits, group):
+    W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
+    a = oracle.act_stats(X)
+    alphas = synth.default_alphas()
+    losses = np.linspace(1.0, 0.5, 20).astype(np.float32)      # chooses alpha = 0.95
+    pk = oracle.pack(W, a, bits, group, alphas, losses.astype(np.float64))
+    Y = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]), dev(pk["s_best"]),
+                         dev(X), bits, group))
+    awq.get_status()
+    ref = oracle.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, bits, group)
+    # binary32 accumulation: bound by the sum of |terms|
+    q = oracle.unpack_codes(pk["codes"], K, bits).astype(np.float64)
+    Gi = np.arange(K) // group
+    wq = np.abs((q - pk["zeros"].astype(np.float64)[:, Gi]) * pk["scales"].astype(np.float64)[:, Gi])
+    xs = np.abs(X.astype(np.float32) * (np.float32(1) / pk["s_best"]).astype(np.float32)).astype(np.float64)
+    bound = xs @ wq.T
+    assert np.all(np.abs(Y - ref) <= 2e-6 * bound + 1e-30)
+    # row blocks split across thread blocks are summed in a fixed order
+    Y2 = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]),
+                          dev(pk["s_best"]), dev(X), bits, group))
+    assert np.array_equal(Y, Y2)

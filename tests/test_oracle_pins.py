@@ -307,3 +307,33 @@ def test_premise_activation_aware_beats_rtn(oracle_mod):
     L = r["losses"]
     assert r["best"] > 0 and L[r["best"]] < L[0]
     assert not np.all(np.diff(L) >= 0)
+
+
+# ---------------------------------------------------------------------------
+# The consumer of the packed format (quantized linear layer)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (2, 64)])
+def test_qlinear_identity_input_gives_dequantized_weights(oracle_mod, bits, group):
+    """x = e_t (T = K) and s = 1: Y[t, n] = (q[n, t] - z) sh exactly, read back
+    from the packed words."""
+    W, X, _ = synth.generate(synth.make_config(12, 128, 8, bits=bits, group=group, seed=61))
+    s = np.ones(128, dtype=np.float32)
+    r = oracle_mod.quantize(W, s, bits, group)
+    codes = oracle_mod.pack_codes(r["q"], bits)
+    Y = oracle_mod.qlinear(codes, r["sh"], r["z"].astype(np.float16), s, np.eye(128, dtype=np.float16),
+                           bits, group)
+    G = np.arange(128) // group
+    expect = (r["q"].astype(np.float64) - r["z"][:, G]) * r["sh"].astype(np.float64)[:, G]
+    assert np.array_equal(Y, expect.T)
+
+
+def test_qlinear_matches_dequantized_matmul(oracle_mod):
+    """With s folded into the input, Y equals X W_hat^T up to W_hat's fp16 rounding."""
+    W, X, _ = synth.generate(synth.make_config(48, 256, 16, seed=62))
+    a = oracle_mod.act_stats(X)
+    al = synth.default_alphas()
+    pk = oracle_mod.pack(W, a, 4, 128, al, oracle_mod.search(W, X, a, 4, 128, al)["losses"])
+    Y = oracle_mod.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, 4, 128)
+    Yh = X.astype(np.float64) @ pk["what"].astype(np.float64).T
+    assert np.linalg.norm(Y - Yh) / np.linalg.norm(Yh) < 2.0 ** -11
