@@ -63,8 +63,9 @@ def _load():
     lib.awq_oracle_rn16.argtypes = [ctypes.c_double]
     lib.awq_oracle_act_stats.argtypes = [P, i64, i64, i64, P]
     lib.awq_oracle_scales.argtypes = [P, i64, ctypes.c_float, P]
-    lib.awq_oracle_quantize.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int,
+    lib.awq_oracle_quantize.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
                                         ctypes.c_int, P, P, P, P]
+    lib.awq_oracle_topk.argtypes = [P, i64, i64, P]
     lib.awq_oracle_pack_codes.argtypes = [P, i64, i64, ctypes.c_int, P]
     lib.awq_oracle_argmin.restype = ctypes.c_int
     lib.awq_oracle_argmin.argtypes = [P, ctypes.c_int]
@@ -129,8 +130,13 @@ def scales(a: np.ndarray, alpha: float) -> np.ndarray:
 # Steps a3/a4 -- [QAS-QA] §5, §9; [AWQ-wiki] "Fondements techniques"
 # --------------------------------------------------------------------------
 
-def quantize(W: np.ndarray, s: np.ndarray, bits: int, group: int, no_round: bool = False):
-    """Group-wise asymmetric RTN of W*diag(s), dequantized and divided by s.
+def quantize(W: np.ndarray, s: np.ndarray, bits: int, group: int, no_round: bool = False,
+             zero_point: bool = True, mask=None):
+    """Group-wise RTN of W*diag(s), dequantized and divided by s.
+
+    zero_point=True: asymmetric (min/max, a zero-point code); False: symmetric
+    absmax with the zero fixed at the middle code 2^(bits-1).  mask: channels
+    kept in fp16 (excluded from their group's range, W_hat = W there).
 
     Returns dict(q=[N,K] uint8 codes, sh=[N,K/g] fp16 scales, z=[N,K/g] float32
     zero points, what=[N,K] fp16 dequantized-and-unscaled weights)."""
@@ -139,12 +145,15 @@ def quantize(W: np.ndarray, s: np.ndarray, bits: int, group: int, no_round: bool
     assert K % group == 0 and group <= 256
     s = np.ascontiguousarray(s, dtype=np.float32)
     assert s.shape == (K,)
+    m = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    assert m is None or m.shape == (K,)
     G = K // group
     q = np.empty((N, K), dtype=np.uint8)
     sh = np.empty((N, G), dtype=np.uint16)
     z = np.empty((N, G), dtype=np.float32)
     what = np.empty((N, K), dtype=np.uint16)
     _load().awq_oracle_quantize(_ptr(W.view(np.uint16)), N, K, _ptr(s), int(bits), int(group),
+                                int(bool(zero_point)), None if m is None else _ptr(m),
                                 int(bool(no_round)), _ptr(q), _ptr(sh), _ptr(z), _ptr(what))
     return dict(q=q, sh=sh.view(np.float16), z=z, what=what.view(np.float16))
 
@@ -162,7 +171,7 @@ def output_error_sum(W: np.ndarray, What: np.ndarray, X: np.ndarray) -> np.ndarr
 
 
 def search(W: np.ndarray, X: np.ndarray, a: np.ndarray, bits: int, group: int,
-           alphas=DEFAULT_ALPHAS, rows=None, no_round: bool = False):
+           alphas=DEFAULT_ALPHAS, rows=None, no_round: bool = False, zero_point: bool = True):
     """The per-layer grid search.
 
     For each alpha_i: s = a^alpha_i, Ŵ = Q(W diag(s)) diag(s)^-1, and the loss
@@ -173,22 +182,39 @@ def search(W: np.ndarray, X: np.ndarray, a: np.ndarray, bits: int, group: int,
 
     Returns dict(losses=[n_alpha] float64 MSE over the scored rows,
                  row_sums=[n_alpha, len(rows)] float64, best=int)."""
+    s_table = np.stack([scales(a, float(al)) for al in alphas])
+    return search_scales(W, X, s_table, bits, group, rows=rows, no_round=no_round, zero_point=zero_point)
+
+
+def search_scales(W: np.ndarray, X: np.ndarray, s_table, bits: int, group: int, rows=None,
+                  no_round: bool = False, zero_point: bool = True, mask=None):
+    """The same loss for caller-given scale vectors s_table[i] (the baselines:
+    s = 1 is plain RTN, s = 2 on the salient channels the fixed-scale variant)
+    and, with ``mask``, the channels kept in fp16 contribute no error."""
     W = _as_f16(W)
     X = _as_f16(X)
-    N, K = W.shape
     T = X.shape[0]
+    s_table = np.atleast_2d(np.asarray(s_table, dtype=np.float32))
     Ws = W if rows is None else np.ascontiguousarray(W[np.asarray(rows)])
     nr = Ws.shape[0]
-    losses = np.empty(len(alphas), dtype=np.float64)
-    row_sums = np.empty((len(alphas), nr), dtype=np.float64)
-    for i, al in enumerate(alphas):
-        s = scales(a, float(al))
-        what = quantize(Ws, s, bits, group, no_round=no_round)["what"]
+    losses = np.empty(len(s_table), dtype=np.float64)
+    row_sums = np.empty((len(s_table), nr), dtype=np.float64)
+    for i, s in enumerate(s_table):
+        what = quantize(Ws, s, bits, group, no_round=no_round, zero_point=zero_point, mask=mask)["what"]
         rs = output_error_sum(Ws, what, X)
         row_sums[i] = rs
         losses[i] = rs.sum() / (nr * T)
     best = argmin(losses)
     return dict(losses=losses, row_sums=row_sums, best=best)
+
+
+def topk_mask(stat, k: int) -> np.ndarray:
+    """mask[j] = 1 for the k channels with the largest statistic (ties: lower
+    index first; NaN ranks last)."""
+    v = np.ascontiguousarray(stat, dtype=np.float32)
+    m = np.empty(v.size, dtype=np.uint8)
+    _load().awq_oracle_topk(_ptr(v), v.size, int(k), _ptr(m))
+    return m
 
 
 def argmin(losses) -> int:
@@ -210,14 +236,22 @@ def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
     return codes
 
 
-def pack(W: np.ndarray, a: np.ndarray, bits: int, group: int, alphas, losses, rows=None):
+def pack(W: np.ndarray, a: np.ndarray, bits: int, group: int, alphas, losses, rows=None,
+         zero_point: bool = True):
     """Argmin over the grid, then codes / fp16 scales / fp16 zeros / s_best."""
-    W = _as_f16(W)
     best = argmin(losses)
-    s = scales(a, float(alphas[best]))
+    out = pack_scales(W, scales(a, float(alphas[best])), bits, group, rows=rows, zero_point=zero_point)
+    out["best"] = best
+    return out
+
+
+def pack_scales(W: np.ndarray, s, bits: int, group: int, rows=None, zero_point: bool = True):
+    """Codes / fp16 scales / fp16 zeros of W quantized with a given s."""
+    W = _as_f16(W)
+    s = np.ascontiguousarray(s, dtype=np.float32)
     Ws = W if rows is None else np.ascontiguousarray(W[np.asarray(rows)])
-    qz = quantize(Ws, s, bits, group)
-    return dict(best=best, s_best=s, codes=pack_codes(qz["q"], bits), q=qz["q"],
+    qz = quantize(Ws, s, bits, group, zero_point=zero_point)
+    return dict(s_best=s, codes=pack_codes(qz["q"], bits), q=qz["q"],
                 scales=qz["sh"], zeros=qz["z"].astype(np.float16), what=qz["what"])
 
 

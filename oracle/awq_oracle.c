@@ -119,8 +119,7 @@ void awq_oracle_scales(const float *a, int64_t K, float alpha, float *s)
 }
 
 /* ------------------------------------------------------------------ */
-/* Steps a3/a4: scale, group-wise asymmetric round-to-nearest, dequant, */
-/* unscale.                                                            */
+/* Steps a3/a4: scale, group-wise round-to-nearest, dequant, unscale.  */
 /*   [QAS-QA] §5: multiply the channel's weights by s, divide the      */
 /*   activation by s, quantize with group-wise round-to-nearest; §9:   */
 /*   quant_config zero_point=True, q_group_size=128, w_bit=4.           */
@@ -130,27 +129,37 @@ void awq_oracle_scales(const float *a, int64_t K, float alpha, float *s)
 /* Per row n and group G of g consecutive columns:                     */
 /*   w'_k   = RN32(w_k * s_k)                                          */
 /*   mn,mx  = min, max of w'_k over the group                          */
+/* asymmetric (zero_point = 1):                                         */
 /*   scale  = RN32(RN32(mx - mn) / qmax)                               */
+/*   z      = clamp(rint(-mn * r), 0, qmax)   (zero point, a code)     */
+/* symmetric (zero_point = 0; [AWQ-note] "Measures": the INT3 grid of  */
+/* step max|w| / (2^(b-1) - 1)):                                        */
+/*   scale  = RN32(max(-mn, mx) / (2^(b-1) - 1)),  z = 2^(b-1)          */
+/* both:                                                               */
 /*   sh     = RN16(clamp(scale, 2^-24, 65504))  (stored fp16 scale)    */
 /*   r      = RN32(1 / sh)                                             */
-/*   z      = clamp(rint(-mn * r), 0, qmax)   (zero point, a code)     */
 /*   q_k    = clamp(rint(w'_k * r) + z, 0, qmax)                       */
 /* The products inside rint are exact (binary32 x binary32 fits in      */
 /* binary64): q = round(w'/scale) is rounded once, by rint itself.      */
 /*   what_k = RN16(RN32(RN32((q_k - z) * sh) * RN32(1 / s_k)))         */
+/* mask (may be NULL): channels k with mask[k] != 0 stay in fp16        */
+/* ([AWQ-note] "Measures": keeping 1% of the channels in FP16): they    */
+/* take no part in their group's min and max and what_k = w_k; a group  */
+/* with every channel masked has mn = mx = 0.                           */
 /* no_round != 0 replaces rint by the identity in q_k (and drops the   */
 /* clamp), which turns quantization into an exact identity up to       */
 /* binary32/binary16 rounding (a test hook).                           */
 /* ------------------------------------------------------------------ */
 
 void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s,
-                         int bits, int g, int no_round,
+                         int bits, int g, int zero_point, const uint8_t *mask, int no_round,
                          uint8_t *q_out,        /* [N,K]  codes (may be NULL)        */
                          uint16_t *sh_out,      /* [N,K/g] fp16 bits (may be NULL)   */
                          float *z_out,          /* [N,K/g] zero points (may be NULL) */
                          uint16_t *what_out)    /* [N,K]  fp16 bits of W-hat         */
 {
     const double qmax = (double)((1 << bits) - 1);
+    const double qsym = (double)((1 << (bits - 1)) - 1);
     const int64_t G = K / g;
     #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
@@ -160,20 +169,33 @@ void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s
             float mn = INFINITY, mx = -INFINITY;
             for (int k = 0; k < g; ++k) {
                 wp[k] = rn32(awq_oracle_h2d(W[n * K + k0 + k]) * (double)s[k0 + k]);
+                if (mask && mask[k0 + k]) continue;
                 if (wp[k] < mn) mn = wp[k];
                 if (wp[k] > mx) mx = wp[k];
             }
-            float range = rn32((double)mx - (double)mn);
-            float scale = rn32((double)range / qmax);
+            if (mn > mx) { mn = 0.0f; mx = 0.0f; }      /* every channel kept in fp16 */
+            float scale;
+            if (zero_point) {
+                float range = rn32((double)mx - (double)mn);
+                scale = rn32((double)range / qmax);
+            } else {
+                double amax = -(double)mn > (double)mx ? -(double)mn : (double)mx;
+                scale = rn32(amax / qsym);
+            }
             double sc = scale;
             if (sc < ldexp(1.0, -24)) sc = ldexp(1.0, -24);
             if (sc > 65504.0) sc = 65504.0;
             uint16_t shb = awq_oracle_rn16(sc);
             double sh = awq_oracle_h2d(shb);
             float r = rn32(1.0 / sh);
-            double z = nearbyint(-(double)mn * (double)r);    /* exact product */
-            if (!(z > 0.0)) z = 0.0;        /* a code in [0, qmax]: never -0 */
-            if (z > qmax) z = qmax;
+            double z;
+            if (zero_point) {
+                z = nearbyint(-(double)mn * (double)r);    /* exact product */
+                if (!(z > 0.0)) z = 0.0;        /* a code in [0, qmax]: never -0 */
+                if (z > qmax) z = qmax;
+            } else {
+                z = qsym + 1.0;                 /* 2^(b-1): the middle code */
+            }
             if (sh_out) sh_out[n * G + gi] = shb;
             if (z_out) z_out[n * G + gi] = (float)z;
             for (int k = 0; k < g; ++k) {
@@ -189,10 +211,36 @@ void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s
                 float rs = rn32(1.0 / (double)s[k0 + k]);
                 float deq = rn32((q - z) * sh);
                 float un = rn32((double)deq * (double)rs);
-                what_out[n * K + k0 + k] = awq_oracle_rn16(un);
+                what_out[n * K + k0 + k] = (mask && mask[k0 + k]) ? W[n * K + k0 + k] : awq_oracle_rn16(un);
                 if (q_out) q_out[n * K + k0 + k] = (uint8_t)q;
             }
         }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Channel selection for the FP16-protection baselines ([AWQ-note]     */
+/* "Measures": keep the 1% most important channels, judged by the      */
+/* activation, or -- the weaker choice -- by the weights).             */
+/* mask[j] = 1 for the k channels of largest stat (ties: lower index    */
+/* first; NaN ranks below every number), 0 elsewhere.  Plain O(K^2).    */
+/* ------------------------------------------------------------------ */
+
+void awq_oracle_topk(const float *stat, int64_t K, int64_t k, uint8_t *mask)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < K; ++j) {
+        int64_t above = 0;
+        const int nj = isnan(stat[j]);
+        for (int64_t i = 0; i < K; ++i) {
+            if (i == j) continue;
+            const int ni = isnan(stat[i]);
+            int before;
+            if (ni || nj) before = (!ni && nj) || (ni && nj && i < j);
+            else before = stat[i] > stat[j] || (stat[i] == stat[j] && i < j);
+            above += before;
+        }
+        mask[j] = above < k ? 1 : 0;
     }
 }
 

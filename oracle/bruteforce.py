@@ -42,30 +42,43 @@ def mean_abs(column) -> np.float32:
     return f32(float(tot) / len(column))
 
 
-def quantize_group(w, s, bits):
-    """One group: w (binary16 values as floats), s (float32).  Returns q, sh, z, what."""
+def quantize_group(w, s, bits, sym=False, keep=None):
+    """One group: w (binary16 values as floats), s (float32).  Returns q, sh, z, what.
+
+    sym: the symmetric absmax quantizer (step max|w'| / (2^(bits-1) - 1), zero
+    at the middle code 2^(bits-1)).  keep: per-column flags of channels held
+    in fp16 -- left out of the range, returned unchanged."""
     qmax = (1 << bits) - 1
+    keep = [False] * len(w) if keep is None else [bool(v) for v in keep]
     wp = [f32(f32(w[k]) * s[k]) for k in range(len(w))]
-    mn = min(wp)
-    mx = max(wp)
-    scale = f32(f32(mx - mn) / f32(qmax))
+    ranged = [wp[k] for k in range(len(w)) if not keep[k]] or [f32(0.0)]
+    mn = min(ranged)
+    mx = max(ranged)
+    if sym:
+        half = (1 << (bits - 1)) - 1
+        scale = f32(max(-mn, mx) / f32(half))
+    else:
+        scale = f32(f32(mx - mn) / f32(qmax))
     scale = min(max(float(scale), 2.0 ** -24), 65504.0)
     sh = to_f16(scale)
     r = f32(f32(1.0) / f32(sh))
-    z = round(-float(mn) * float(r))        # exact product (24 x 24 bits); round(): ties to even
-    z = min(max(z, 0), qmax)
+    if sym:
+        z = 1 << (bits - 1)
+    else:
+        z = round(-float(mn) * float(r))    # exact product (24 x 24 bits); round(): ties to even
+        z = min(max(z, 0), qmax)
     q, what = [], []
     for k in range(len(w)):
         t = float(wp[k]) * float(r)         # exact product
         qk = min(max(round(t) + z, 0), qmax)
         rs = f32(f32(1.0) / s[k])
         deq = f32(f32(qk - z) * f32(sh))
-        what.append(to_f16(float(f32(deq * rs))))
+        what.append(float(w[k]) if keep[k] else to_f16(float(f32(deq * rs))))
         q.append(qk)
     return q, sh, z, what
 
 
-def quantize(W, s, bits, group):
+def quantize(W, s, bits, group, sym=False, keep=None):
     N, K = len(W), len(W[0])
     Q = [[0] * K for _ in range(N)]
     WH = [[0.0] * K for _ in range(N)]
@@ -74,7 +87,8 @@ def quantize(W, s, bits, group):
     for n in range(N):
         for gi in range(K // group):
             sl = slice(gi * group, (gi + 1) * group)
-            q, sh, z, what = quantize_group(W[n][sl], s[sl], bits)
+            q, sh, z, what = quantize_group(W[n][sl], s[sl], bits, sym,
+                                            None if keep is None else keep[sl])
             Q[n][sl] = q
             WH[n][sl] = what
             SH[n][gi] = sh
@@ -96,7 +110,7 @@ def exact_loss(W, WH, X):
     return tot
 
 
-def search(W16: np.ndarray, X16: np.ndarray, bits: int, group: int, alphas):
+def search(W16: np.ndarray, X16: np.ndarray, bits: int, group: int, alphas, sym=False):
     """Enumerate every alpha independently.  Returns dict(a, losses, best, q, sh, z)."""
     W = [[float(v) for v in row] for row in W16.astype(np.float64)]
     X = [[float(v) for v in row] for row in X16.astype(np.float64)]
@@ -106,9 +120,18 @@ def search(W16: np.ndarray, X16: np.ndarray, bits: int, group: int, alphas):
     per_alpha = []
     for al in alphas:
         s = [f32(math.pow(max(float(aj), 2.0 ** -126), float(f32(al)))) for aj in a]
-        Q, SH, Z, WH = quantize(W, s, bits, group)
+        Q, SH, Z, WH = quantize(W, s, bits, group, sym)
         losses.append(exact_loss(W, WH, X) / (N * T))
         per_alpha.append((Q, SH, Z, WH, s))
     best = min(range(len(losses)), key=lambda i: (losses[i], i))
     return dict(a=np.array(a, dtype=np.float32), losses=[float(v) for v in losses],
                 exact_losses=losses, best=best, per_alpha=per_alpha)
+
+
+def masked_loss(W16: np.ndarray, X16: np.ndarray, s, bits: int, group: int, keep, sym=False):
+    """Exact MSE of the layer with the channels flagged in `keep` held in fp16."""
+    W = [[float(v) for v in row] for row in W16.astype(np.float64)]
+    X = [[float(v) for v in row] for row in X16.astype(np.float64)]
+    s = [f32(v) for v in s]
+    _, _, _, WH = quantize(W, s, bits, group, sym, list(keep))
+    return float(exact_loss(W, WH, X) / (len(W) * len(X))), WH

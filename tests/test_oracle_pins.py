@@ -337,3 +337,133 @@ def test_qlinear_matches_dequantized_matmul(oracle_mod):
     Y = oracle_mod.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, 4, 128)
     Yh = X.astype(np.float64) @ pk["what"].astype(np.float64).T
     assert np.linalg.norm(Y - Yh) / np.linalg.norm(Yh) < 2.0 ** -11
+
+
+# ---------------------------------------------------------------------------
+# Quantizer variants and baselines: the symmetric absmax quantizer, channels
+# held in fp16, caller-given scale vectors, top-k channel selection
+# ---------------------------------------------------------------------------
+
+def test_awq_note_example_through_symmetric_quantizer(oracle_mod):
+    """[AWQ-note] "Measures": the INT3 grid of step max|w| / (2^(b-1) - 1) is the
+    symmetric quantizer at w_bit = 3.  Group [1.0, 0.2, 0, 0]: step 1/3 (fp16),
+    middle code 4, W_hat[1] x 10 = 3.333; s = 2 on that channel keeps the group
+    maximum and gives 1.667; scaling it to 2.0 makes the step 2/3."""
+    g = _gold("awq_note_int3_example.json")
+    W = np.array([[1.0, 0.2, 0.0, 0.0]], dtype=np.float16)
+    def tol(v):
+        return 0.5 * 10.0 ** -g["printed_decimals"] + abs(v) * 2 * 2.0 ** -11
+    r0 = oracle_mod.quantize(W, np.ones(4, dtype=np.float32), bits=g["bits"], group=4, zero_point=False)
+    assert float(r0["sh"][0, 0]) == pytest.approx(g["step"], rel=2 ** -11)
+    assert float(r0["z"][0, 0]) == 4.0
+    assert list(r0["q"][0]) == [7, 5, 4, 4]
+    assert float(r0["what"][0, 1]) * g["activation_second"] == pytest.approx(g["rtn_output"], abs=tol(g["rtn_output"]))
+    s = np.array([1.0, g["s"], 1.0, 1.0], dtype=np.float32)
+    r1 = oracle_mod.quantize(W, s, bits=g["bits"], group=4, zero_point=False)
+    assert float(r1["sh"][0, 0]) == float(r0["sh"][0, 0])
+    assert float(r1["what"][0, 1]) * g["activation_second"] == pytest.approx(g["scaled_output"], abs=tol(g["scaled_output"]))
+    s2 = np.array([1.0, g["overscaled_W"][1] / float(W[0, 1]), 1.0, 1.0], dtype=np.float32)
+    r2 = oracle_mod.quantize(W, s2, bits=g["bits"], group=4, zero_point=False)
+    assert float(r2["sh"][0, 0]) == pytest.approx(g["overscaled_step"], rel=2 ** -10)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_symmetric_quantizer_is_odd(oracle_mod, bits):
+    """Q(-W) = -Q(W) (rint ties to even is odd), zero at 2^(bits-1), codes in
+    [1, 2^bits - 1] whenever the fp16 scale is not clamped."""
+    W, X, _ = synth.generate(synth.make_config(16, 256, 4, bits=bits, seed=71))
+    a = oracle_mod.act_stats(X)
+    s = oracle_mod.scales(a, 0.5)
+    r = oracle_mod.quantize(W, s, bits, 128, zero_point=False)
+    rn = oracle_mod.quantize(-W, s, bits, 128, zero_point=False)
+    assert np.array_equal(rn["what"], -r["what"])          # as values: a zero level is +0 on both sides
+    assert np.all(r["z"] == 2 ** (bits - 1))
+    assert r["q"].min() >= 1 and r["q"].max() <= 2 ** bits - 1
+
+
+@pytest.mark.parametrize("bits,group,sym", [(4, 16, False), (4, 16, True), (3, 8, True), (2, 8, False)])
+def test_variants_against_bruteforce(oracle_mod, bits, group, sym):
+    """The C oracle's symmetric quantizer and fp16-kept channels against the
+    independent binary32-scalar restatement, codes / scales / zeros / W_hat bit
+    for bit and the loss exactly (rational arithmetic)."""
+    from oracle import bruteforce as bf
+    rng = np.random.default_rng(bits * 100 + group)
+    W = (rng.standard_normal((5, 32)) * 0.05).astype(np.float16)
+    X = rng.standard_normal((6, 32)).astype(np.float16)
+    X[:, [3, 17]] *= np.float16(30)
+    s = (rng.random(32) * 3 + 0.25).astype(np.float32)
+    keep = np.zeros(32, dtype=np.uint8)
+    keep[[3, 9, 17]] = 1
+    keep[group:2 * group] = 1                       # a whole group held in fp16
+    r = oracle_mod.quantize(W, s, bits, group, zero_point=not sym, mask=keep)
+    Q, SH, Z, WH = bf.quantize([[float(v) for v in row] for row in W.astype(np.float64)],
+                               [np.float32(v) for v in s], bits, group, sym, list(keep))
+    assert np.array_equal(r["q"], np.array(Q, dtype=np.uint8))
+    assert np.array_equal(r["sh"].astype(np.float64), np.array(SH))
+    assert np.array_equal(r["z"].astype(np.float64), np.array(Z, dtype=np.float64))
+    assert np.array_equal(r["what"].astype(np.float64), np.array(WH))
+    assert np.array_equal(r["what"][:, keep == 1], W[:, keep == 1])
+    exact, _ = bf.masked_loss(W, X, s, bits, group, keep, sym)
+    got = oracle_mod.search_scales(W, X, s[None], bits, group, zero_point=not sym, mask=keep)["losses"][0]
+    assert got == pytest.approx(exact, rel=1e-12)
+
+
+def test_mask_extremes(oracle_mod):
+    """Every channel held in fp16: W_hat = W and zero loss.  No channel held:
+    the plain quantizer."""
+    W, X, _ = synth.generate(synth.make_config(8, 256, 16, seed=72))
+    s = np.ones(256, dtype=np.float32)
+    r = oracle_mod.quantize(W, s, 4, 128, mask=np.ones(256, dtype=np.uint8))
+    assert np.array_equal(r["what"].view(np.uint16), W.view(np.uint16))
+    assert oracle_mod.search_scales(W, X, s[None], 4, 128, mask=np.ones(256, np.uint8))["losses"][0] == 0.0
+    r0 = oracle_mod.quantize(W, s, 4, 128, mask=np.zeros(256, dtype=np.uint8))
+    r1 = oracle_mod.quantize(W, s, 4, 128)
+    assert np.array_equal(r0["what"].view(np.uint16), r1["what"].view(np.uint16))
+
+
+def test_topk_matches_sorted_order(oracle_mod):
+    """Top-k by value, ties to the lower index, NaN last -- against Python's sort."""
+    rng = np.random.default_rng(73)
+    v = rng.integers(0, 20, 300).astype(np.float32)       # many ties
+    v[[5, 50, 299]] = np.nan
+    for k in [0, 1, 3, 17, 150, 297, 298, 300]:
+        order = sorted(range(v.size), key=lambda j: (bool(np.isnan(v[j])), -(0 if np.isnan(v[j]) else v[j]), j))
+        expect = np.zeros(v.size, dtype=np.uint8)
+        expect[order[:k]] = 1
+        assert np.array_equal(oracle_mod.topk_mask(v, k), expect), k
+
+
+def test_given_scales_reduce_to_the_grid(oracle_mod):
+    """s = 1 is plain RTN, the alpha = 0 point of the grid; the grid's s
+    vectors passed as a table give the grid's losses."""
+    W, X, _ = synth.generate(synth.make_config(16, 256, 32, seed=74))
+    a = oracle_mod.act_stats(X)
+    al = np.array([0.0, 0.25, 0.5], dtype=np.float32)
+    grid = oracle_mod.search(W, X, a, 4, 128, al)["losses"]
+    table = np.stack([oracle_mod.scales(a, float(x)) for x in al])
+    assert np.array_equal(oracle_mod.search_scales(W, X, table, 4, 128)["losses"], grid)
+    assert oracle_mod.search_scales(W, X, np.ones((1, 256), np.float32), 4, 128)["losses"][0] == grid[0]
+
+
+def test_baselines_premise(oracle_mod):
+    """[AWQ-note] "Measures": keeping the 1% of channels with the largest
+    activations in fp16 helps far more than choosing them by weight magnitude;
+    scaling those channels by a fixed 2 helps, and the searched s helps more.
+    On a synthetic layer with 1% outlier input channels:"""
+    cfg = synth.make_config(256, 512, 256, seed=5)
+    W, X, idx = synth.generate(cfg)
+    a = oracle_mod.act_stats(X)
+    k = round(cfg.K / 100)
+    m_act = oracle_mod.topk_mask(a, k)
+    m_w = oracle_mod.topk_mask(oracle_mod.act_stats(W), k)       # mean |w| per input channel
+    assert np.all(m_act[idx] == 1)                                  # the outliers are found
+    one = np.ones((1, cfg.K), np.float32)
+    rtn = oracle_mod.search_scales(W, X, one, 4, 128)["losses"][0]
+    fp16_act = oracle_mod.search_scales(W, X, one, 4, 128, mask=m_act)["losses"][0]
+    fp16_w = oracle_mod.search_scales(W, X, one, 4, 128, mask=m_w)["losses"][0]
+    s2 = np.where(m_act == 1, 2.0, 1.0).astype(np.float32)[None]
+    fixed2 = oracle_mod.search_scales(W, X, s2, 4, 128)["losses"][0]
+    awq = oracle_mod.search(W, X, a, 4, 128, synth.default_alphas())["losses"].min()
+    assert fp16_act < 0.1 * rtn
+    assert fp16_w > 0.9 * rtn
+    assert awq < fixed2 < 0.5 * rtn
