@@ -18,7 +18,7 @@ __all__ = [
     "AWQError", "lib", "act_stats", "alpha_scales", "quant_dequant", "search_workspace_bytes",
     "search_layer", "pack", "quantize_layer", "get_status", "set_wait_timeout_ms", "default_alphas",
     "profile_next_search", "quantize_shared_input", "selftest_bounded_wait", "qlinear",
-    "LIB_PATH",
+    "search_scales", "channel_topk", "pack_scales", "salient_scales", "baselines", "LIB_PATH",
 ]
 
 _PKG = Path(__file__).resolve().parent
@@ -53,6 +53,13 @@ def lib():
     L.awq_act_stats.argtypes = [P, i64, i64, i64, P, P]
     L.awq_alpha_scales.argtypes = [P, i64, P, i32, P, P]
     L.awq_quant_dequant.argtypes = [P, i64, i64, P, QCfg, P, P]
+    L.awq_quant_dequant_masked.argtypes = [P, i64, i64, P, QCfg, P, P, P]
+    L.awq_search_scales_workspace_bytes.argtypes = [i64, i64, i64, QCfg, i32, i32]
+    L.awq_search_scales_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_search_scales.argtypes = [P, i64, i64, P, i64, i64, QCfg, P, i32, P, P, P, P, ctypes.c_size_t, P]
+    L.awq_channel_topk.argtypes = [P, i64, i64, P, P]
+    L.awq_pack_scales.argtypes = [P, i64, i64, P, QCfg, P, P, P, P]
+    L.awq_salient_scales.argtypes = [P, i64, ctypes.c_float, P, P]
     L.awq_search_workspace_bytes.argtypes = [i64, i64, i64, QCfg, i32]
     L.awq_search_workspace_bytes.restype = ctypes.c_size_t
     L.awq_search_layer.argtypes = [P, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P, ctypes.c_size_t, P]
@@ -71,7 +78,8 @@ def lib():
     L.awq_status_string.argtypes = [ctypes.c_int]
     L.awq_status_string.restype = ctypes.c_char_p
     for fn in ("awq_act_stats", "awq_alpha_scales", "awq_quant_dequant", "awq_search_layer", "awq_pack",
-               "awq_get_status"):
+               "awq_get_status", "awq_quant_dequant_masked", "awq_search_scales", "awq_channel_topk",
+               "awq_pack_scales", "awq_salient_scales"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -105,8 +113,8 @@ def default_alphas(n: int = 20, device="cuda") -> torch.Tensor:
     return torch.tensor([i / n for i in range(n)], dtype=torch.float32, device=device)
 
 
-def _qcfg(bits, group):
-    return QCfg(int(bits), int(group), 1)
+def _qcfg(bits, group, zero_point=True):
+    return QCfg(int(bits), int(group), 1 if zero_point else 0)
 
 
 def act_stats(X: torch.Tensor, stream=None) -> torch.Tensor:
@@ -128,24 +136,32 @@ def alpha_scales(a: torch.Tensor, alphas: torch.Tensor, stream=None) -> torch.Te
     return s
 
 
-def quant_dequant(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128, stream=None):
-    """W_hat = Q(W diag(s)) diag(s)^-1 in fp16 (the per-element function of the search)."""
+def quant_dequant(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128, stream=None,
+                  zero_point: bool = True, mask: torch.Tensor | None = None):
+    """W_hat = Q(W diag(s)) diag(s)^-1 in fp16 (the per-element function of the search).
+
+    mask (uint8 [K]): channels kept in fp16 (out of their group's range, W_hat = W)."""
     W = W.contiguous()
     N, K = W.shape
     out = torch.empty_like(W)
-    _check(lib().awq_quant_dequant(_dev(W, torch.float16, "W"), N, K, _dev(s, torch.float32, "s"),
-                                   _qcfg(bits, group), _dev(out, torch.float16, "W_hat"), _stream(stream)),
-           "awq_quant_dequant")
+    args = (_dev(W, torch.float16, "W"), N, K, _dev(s, torch.float32, "s"), _qcfg(bits, group, zero_point))
+    if mask is None:
+        _check(lib().awq_quant_dequant(*args, _dev(out, torch.float16, "W_hat"), _stream(stream)),
+               "awq_quant_dequant")
+    else:
+        _check(lib().awq_quant_dequant_masked(*args, _dev(mask, torch.uint8, "mask"),
+                                              _dev(out, torch.float16, "W_hat"), _stream(stream)),
+               "awq_quant_dequant_masked")
     return out
 
 
-def search_workspace_bytes(N, K, T, bits=4, group=128, n_alpha=20) -> int:
-    return int(lib().awq_search_workspace_bytes(N, K, T, _qcfg(bits, group), n_alpha))
+def search_workspace_bytes(N, K, T, bits=4, group=128, n_alpha=20, zero_point=True) -> int:
+    return int(lib().awq_search_workspace_bytes(N, K, T, _qcfg(bits, group, zero_point), n_alpha))
 
 
 def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, bits: int = 4,
                  group: int = 128, workspace: torch.Tensor | None = None, row_losses: bool = False,
-                 losses_out: torch.Tensor | None = None, stream=None):
+                 losses_out: torch.Tensor | None = None, stream=None, zero_point: bool = True):
     """Per-alpha MSE of the layer output, ||(W_hat_alpha - W) X^T||^2 / (N T).
 
     Returns ``losses`` (float32 [n_alpha]) or ``(losses, row_losses)`` with
@@ -156,14 +172,14 @@ def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torc
     N, K = W.shape
     T = X.shape[0]
     n = alphas.numel()
-    need = search_workspace_bytes(N, K, T, bits, group, n)
+    need = search_workspace_bytes(N, K, T, bits, group, n, zero_point)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     losses = losses_out if losses_out is not None else torch.empty(n, dtype=torch.float32, device=W.device)
     rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
     _check(lib().awq_search_layer(
         _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X"), T, X.stride(0),
-        _dev(a, torch.float32, "a"), _qcfg(bits, group), _dev(alphas, torch.float32, "alphas"), n,
+        _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point), _dev(alphas, torch.float32, "alphas"), n,
         _dev(losses, torch.float32, "losses"),
         _dev(rl, torch.float32, "row_losses") if rl is not None else None,
         ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)), "awq_search_layer")
@@ -171,7 +187,7 @@ def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torc
 
 
 def pack(W: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, losses: torch.Tensor, bits: int = 4,
-         group: int = 128, out: dict | None = None, stream=None) -> dict:
+         group: int = 128, out: dict | None = None, stream=None, zero_point: bool = True) -> dict:
     """Argmin over the grid, then packed codes, fp16 scales/zeros and s at the best alpha."""
     N, K = W.shape
     dev = W.device
@@ -183,7 +199,7 @@ def pack(W: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, losses: torch.T
         scales=torch.empty((N, K // group), dtype=torch.float16, device=dev),
         zeros=torch.empty((N, K // group), dtype=torch.float16, device=dev))
     _check(lib().awq_pack(
-        _dev(W, torch.float16, "W"), N, K, _dev(a, torch.float32, "a"), _qcfg(bits, group),
+        _dev(W, torch.float16, "W"), N, K, _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point),
         _dev(alphas, torch.float32, "alphas"), _dev(losses, torch.float32, "losses"), alphas.numel(),
         _dev(o["best_idx"], torch.int32, "best_idx"), _dev(o["s_best"], torch.float32, "s_best"),
         _dev(o["codes"], torch.int32, "codes"), _dev(o["scales"], torch.float16, "scales"),
@@ -192,7 +208,8 @@ def pack(W: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, losses: torch.T
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,
-                   group: int = 128, workspace: torch.Tensor | None = None, stream=None) -> dict:
+                   group: int = 128, workspace: torch.Tensor | None = None, stream=None,
+                   zero_point: bool = True) -> dict:
     """The whole path for one layer: statistics, grid search, argmin, packing.
 
     W and X may live in host memory (pinned for asynchronous copies); they are
@@ -203,8 +220,8 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None
     Xd = X.to(dev, non_blocking=True) if host else X
     al = default_alphas(device=dev) if alphas is None else alphas.to(dev)
     a = act_stats(Xd, stream)
-    losses = search_layer(Wd, Xd, a, al, bits, group, workspace=workspace, stream=stream)
-    res = pack(Wd, a, al, losses, bits, group, stream=stream)
+    losses = search_layer(Wd, Xd, a, al, bits, group, workspace=workspace, stream=stream, zero_point=zero_point)
+    res = pack(Wd, a, al, losses, bits, group, stream=stream, zero_point=zero_point)
     res["losses"] = losses
     res["a"] = a
     if host:
@@ -233,7 +250,7 @@ def qlinear(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, s_be
 
 
 def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,
-                          group: int = 128, stream=None) -> list:
+                          group: int = 128, stream=None, zero_point: bool = True) -> list:
     """Layers that read the same input (an MLP's gate and up projections, an
     attention block's Q/K/V) must share one s, because 1/s is folded into that
     one input.  Their weights are stacked row-wise and searched as one layer,
@@ -244,7 +261,7 @@ def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = Non
     best_idx, s_best, losses and a."""
     rows = [w.shape[0] for w in Ws]
     W = torch.cat([w.contiguous() for w in Ws], dim=0)
-    res = quantize_layer(W, X, alphas, bits, group, stream=stream)
+    res = quantize_layer(W, X, alphas, bits, group, stream=stream, zero_point=zero_point)
     out, r0 = [], 0
     for n in rows:
         d = {k: res[k][r0:r0 + n] for k in ("codes", "scales", "zeros")}
@@ -252,6 +269,88 @@ def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = Non
         out.append(d)
         r0 += n
     return out
+
+
+def search_scales(W: torch.Tensor, X: torch.Tensor, s_table: torch.Tensor, bits: int = 4, group: int = 128,
+                  zero_point: bool = True, mask: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  row_losses: bool = False, stream=None):
+    """MSE of the layer output for caller-given scale vectors s_table [n, K]
+    (float32, positive), with the channels in ``mask`` (uint8 [K]) held in fp16."""
+    _rowmajor(X, "X")
+    if not W.is_contiguous() or not s_table.is_contiguous():
+        raise ValueError("W and s_table must be contiguous")
+    N, K = W.shape
+    T = X.shape[0]
+    st = s_table.reshape(-1, K)
+    n = st.shape[0]
+    q = _qcfg(bits, group, zero_point)
+    need = int(lib().awq_search_scales_workspace_bytes(N, K, T, q, n, 0 if mask is None else 1))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    losses = torch.empty(n, dtype=torch.float32, device=W.device)
+    rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
+    _check(lib().awq_search_scales(
+        _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X"), T, X.stride(0), q,
+        _dev(st, torch.float32, "s_table"), n, None if mask is None else _dev(mask, torch.uint8, "mask"),
+        _dev(losses, torch.float32, "losses"), _dev(rl, torch.float32, "row_losses") if rl is not None else None,
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)), "awq_search_scales")
+    return (losses, rl) if row_losses else losses
+
+
+def channel_topk(stat: torch.Tensor, k: int, stream=None) -> torch.Tensor:
+    """uint8 [K] mask of the k channels with the largest statistic (ties: lower index)."""
+    K = stat.numel()
+    m = torch.empty(K, dtype=torch.uint8, device=stat.device)
+    _check(lib().awq_channel_topk(_dev(stat, torch.float32, "stat"), K, int(k), _dev(m, torch.uint8, "mask"),
+                                  _stream(stream)), "awq_channel_topk")
+    return m
+
+
+def salient_scales(mask: torch.Tensor, factor: float, stream=None) -> torch.Tensor:
+    """s[k] = factor where mask[k] != 0, else 1 (the fixed-scale variant; factor 1 gives RTN)."""
+    K = mask.numel()
+    s = torch.empty(K, dtype=torch.float32, device=mask.device)
+    _check(lib().awq_salient_scales(_dev(mask, torch.uint8, "mask"), K, float(factor), _dev(s, torch.float32, "s"),
+                                    _stream(stream)), "awq_salient_scales")
+    return s
+
+
+def pack_scales(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128, zero_point: bool = True,
+                stream=None) -> dict:
+    """Codes, fp16 scales and zeros of W quantized with a given s."""
+    N, K = W.shape
+    dev = W.device
+    per = 16 if bits == 2 else 8
+    o = dict(codes=torch.empty((N, K // per), dtype=torch.int32, device=dev),
+             scales=torch.empty((N, K // group), dtype=torch.float16, device=dev),
+             zeros=torch.empty((N, K // group), dtype=torch.float16, device=dev), s_best=s)
+    _check(lib().awq_pack_scales(_dev(W, torch.float16, "W"), N, K, _dev(s, torch.float32, "s"),
+                                 _qcfg(bits, group, zero_point), _dev(o["codes"], torch.int32, "codes"),
+                                 _dev(o["scales"], torch.float16, "scales"), _dev(o["zeros"], torch.float16, "zeros"),
+                                 _stream(stream)), "awq_pack_scales")
+    return o
+
+
+def baselines(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group: int = 128, alphas: torch.Tensor | None = None,
+              frac: float = 0.01, zero_point: bool = True, stream=None) -> dict:
+    """The comparisons of the AWQ pages on one layer, as output-error losses
+    (float32 device scalars): plain RTN, the fixed 2x scale on the salient
+    channels, fp16 protection of those channels chosen by activation and by
+    weight magnitude, and the AWQ grid search.  k = round(frac K) channels."""
+    K = W.shape[1]
+    k = max(1, int(round(frac * K)))
+    al = default_alphas(device=W.device) if alphas is None else alphas
+    a = act_stats(X, stream)
+    m_act = channel_topk(a, k, stream)
+    m_w = channel_topk(act_stats(W, stream), k, stream)          # mean |w| per input channel
+    table = torch.stack([salient_scales(m_act, 1.0, stream), salient_scales(m_act, 2.0, stream)])
+    fixed = search_scales(W, X, table, bits, group, zero_point, stream=stream)
+    ones = table[0:1].contiguous()
+    fp16_act = search_scales(W, X, ones, bits, group, zero_point, mask=m_act, stream=stream)
+    fp16_w = search_scales(W, X, ones, bits, group, zero_point, mask=m_w, stream=stream)
+    grid = search_layer(W, X, a, al, bits, group, stream=stream, zero_point=zero_point)
+    return dict(rtn=fixed[0], fixed_2x=fixed[1], fp16_act=fp16_act[0], fp16_weight=fp16_w[0], awq_grid=grid,
+                mask_act=m_act, mask_weight=m_w, k=k)
 
 
 def get_status(stream=None) -> None:

@@ -25,7 +25,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool valid_qcfg(const awq_qcfg &q) {
     return (q.bits == 2 || q.bits == 3 || q.bits == 4) && (q.group_size == 64 || q.group_size == 128) &&
-           q.zero_point == 1;
+           (q.zero_point == 0 || q.zero_point == 1);
 }
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
@@ -40,9 +40,10 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 //   partial float [n_alpha][ceil(T/512)][N]
 int64_t padded_rows(int64_t N) { return (N + awq::srch2::PM - 1) / awq::srch2::PM * awq::srch2::PM; }
 struct SearchWs {
-    size_t s_off, rs_off, prm_off, part_off, total;
+    size_t s_off, rs_off, prm_off, part_off, xm_off, total;
 };
-SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alpha) {
+// masked: room for X with the fp16-kept channels zeroed, [T][K] fp16.
+SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alpha, bool masked = false) {
     SearchWs w{};
     const int64_t n_tb = (T + awq::srch2::BT - 1) / awq::srch2::BT;
     size_t off = 0;
@@ -50,6 +51,7 @@ SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alph
     w.rs_off = off;   off = round_up(off + sizeof(float) * (size_t)n_alpha * K, 256);
     w.prm_off = off;  off = round_up(off + sizeof(uint2) * (size_t)n_alpha * (K / group) * padded_rows(N), 256);
     w.part_off = off; off = round_up(off + sizeof(float) * (size_t)n_alpha * n_tb * N, 256);
+    w.xm_off = off;   if (masked) off = round_up(off + 2 * (size_t)T * K, 256);
     w.total = off;
     return w;
 }
@@ -168,8 +170,11 @@ int blocks_for(int64_t threads_total, int block) {
     return (int)(b < 1 ? 1 : b);
 }
 
-awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, const float *s_tab,
-                               int n_alpha, float qmax, uint2 *params, cudaStream_t st) {
+awq_status launch_group_params(const void *W, int64_t N, int64_t K, awq_qcfg q, const float *s_tab,
+                               int n_alpha, const uint8_t *mask, uint2 *params, cudaStream_t st) {
+    const int group = q.group_size;
+    const float qmax = (float)((1 << q.bits) - 1);
+    const int sym = q.zero_point ? 0 : 1;
     const int G = (int)(K / group);
     const int lpr = group / awq::kGpCols;
     const int64_t N_pad = padded_rows(N);
@@ -179,10 +184,10 @@ awq_status launch_group_params(const void *W, int64_t N, int64_t K, int group, c
     const unsigned grid = (unsigned)(row_blocks * G);
     if (lpr == 2)
         awq::group_params_kernel<2><<<grid, awq::kGpThreads, smem, st>>>((const __half *)W, N, N_pad, K, G, s_tab,
-                                                                        n_alpha, qmax, params);
+                                                                        n_alpha, qmax, sym, mask, params);
     else
         awq::group_params_kernel<1><<<grid, awq::kGpThreads, smem, st>>>((const __half *)W, N, N_pad, K, G, s_tab,
-                                                                        n_alpha, qmax, params);
+                                                                        n_alpha, qmax, sym, mask, params);
     return last_launch();
 }
 
@@ -224,6 +229,68 @@ size_t ql_part_bytes(int64_t N) {
 size_t qlinear_ws(int64_t T, int64_t K, int64_t N) {
     return ql_xs_bytes(T, K) + ql_part_bytes(N) +
            round_up(sizeof(unsigned) * (size_t)ql_row_blocks(N) * awq::qlv::RGROUPS, 256);
+}
+
+// a8 for a given s: codes, fp16 scales and zeros.
+awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, uint32_t *codes,
+                       void *scales, void *zeros, cudaStream_t st) {
+    const int G = (int)(K / q.group_size);
+    const int lpr = q.group_size / awq::kGpCols;
+    const int sym = q.zero_point ? 0 : 1;
+    const int64_t rows_per_block = awq::kGpThreads / lpr;
+    const unsigned grid = (unsigned)(((N + rows_per_block - 1) / rows_per_block) * G);
+    if (lpr == 2)
+        awq::pack_kernel<2><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s, codes,
+                                                             (__half *)scales, (__half *)zeros);
+    else
+        awq::pack_kernel<1><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s, codes,
+                                                             (__half *)scales, (__half *)zeros);
+    return last_launch();
+}
+
+// a3-a6 on tables of n scale vectors already in the workspace: group
+// parameters, the tensor-core search against X, the loss reduction.
+awq_status search_core(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, awq_qcfg q,
+                       const float *s_tab, const float *rs_tab, int n_alpha, const uint8_t *mask, uint2 *params,
+                       float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st) {
+    const float qmax = (float)((1 << q.bits) - 1);
+    // a3 (group parameters for every alpha)
+    if (awq_status e = launch_group_params(W, N, K, q, s_tab, n_alpha, mask, params, st)) return e;
+
+    // a4-a6: the tensor-core search on CTA pairs
+    CUtensorMap tmap_x, tmap_w;
+    if (!encode_rows_map(&tmap_x, X, T, K, ldx, awq::srch2::HN) ||
+        !encode_rows_map(&tmap_w, W, N, K, K, awq::srch2::BM))
+        return AWQ_ERR_CUDA;
+    awq::srch2::Args A;
+    A.params = params;
+    A.s_tab = s_tab;
+    A.rs_tab = rs_tab;
+    A.partial = partial;
+    A.N = N;
+    A.K = K;
+    A.T = T;
+    A.N_pad = padded_rows(N);
+    A.n_alpha = n_alpha;
+    A.G = (int)(K / q.group_size);
+    A.group = q.group_size;
+    A.n_tb = (int)((T + awq::srch2::BT - 1) / awq::srch2::BT);
+    A.n_kb = (int)(K / awq::srch2::BK);
+    A.n_units = (A.N_pad / awq::srch2::PM) * A.n_tb * n_alpha;
+    A.qmax = qmax;
+    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+    const int64_t pairs = A.n_units < d.max_pairs ? A.n_units : d.max_pairs;
+    const int grid = (int)(2 * pairs);
+    cudaEvent_t pb = t_prof_begin, pe = t_prof_end;
+    t_prof_begin = t_prof_end = nullptr;
+    if (pb && cudaEventRecord(pb, st) != cudaSuccess) return AWQ_ERR_CUDA;
+    awq::srch2::search_pair_kernel<<<grid, awq::srch2::NUM_THREADS, awq::srch2::SMEM_BYTES, st>>>(tmap_x, tmap_w, A);
+    if (awq_status e = last_launch()) return e;
+    if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
+
+    // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
+    awq::loss_reduce_kernel<<<n_alpha, awq::kLossThreads, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
+    return last_launch();
 }
 
 }  // namespace
@@ -274,6 +341,11 @@ awq_status awq_alpha_scales(const float *a, int64_t K, const float *alphas, int3
 
 awq_status awq_quant_dequant(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, void *W_hat,
                              void *stream) {
+    return awq_quant_dequant_masked(W, N, K, s, q, nullptr, W_hat, stream);
+}
+
+awq_status awq_quant_dequant_masked(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q,
+                                    const uint8_t *mask, void *W_hat, void *stream) {
     if (!W || !s || !W_hat || !aligned16(W) || !aligned16(s) || !aligned16(W_hat)) return AWQ_ERR_INVALID_ARG;
     if (!valid_qcfg(q) || N < 1 || N > kMaxDim || K < q.group_size || K > kMaxDim || K % q.group_size)
         return AWQ_ERR_INVALID_ARG;
@@ -283,12 +355,13 @@ awq_status awq_quant_dequant(const void *W, int64_t N, int64_t K, const float *s
     const int tpg = q.group_size / 16;
     const int grid = blocks_for(N * G * tpg, 256);
     const float qmax = (float)((1 << q.bits) - 1);
+    const int sym = q.zero_point ? 0 : 1;
     if (tpg == 8)
-        awq::quant_dequant_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax,
-                                                                            (__half *)W_hat);
+        awq::quant_dequant_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax, sym,
+                                                                            mask, (__half *)W_hat);
     else
-        awq::quant_dequant_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax,
-                                                                            (__half *)W_hat);
+        awq::quant_dequant_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>((const __half *)W, N, K, G, s, qmax, sym,
+                                                                            mask, (__half *)W_hat);
     return last_launch();
 }
 
@@ -317,7 +390,6 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
     float *rs_tab = reinterpret_cast<float *>(base + L.rs_off);
     uint2 *params = reinterpret_cast<uint2 *>(base + L.prm_off);
     float *partial = reinterpret_cast<float *>(base + L.part_off);
-    const float qmax = (float)((1 << q.bits) - 1);
 
     // a2: s and 1/s for every alpha
     {
@@ -326,44 +398,10 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
                                                                                      s_tab, rs_tab);
         if (awq_status e = last_launch()) return e;
     }
-    // a3 (group parameters for every alpha)
-    if (awq_status e = launch_group_params(W, N, K, q.group_size, s_tab, n_alpha, qmax, params, st)) return e;
-
-    // a4-a6: the tensor-core search on CTA pairs
-    CUtensorMap tmap_x, tmap_w;
-    if (!encode_rows_map(&tmap_x, X, T, K, ldx, awq::srch2::HN) ||
-        !encode_rows_map(&tmap_w, W, N, K, K, awq::srch2::BM))
-        return AWQ_ERR_CUDA;
-    awq::srch2::Args A;
-    A.params = params;
-    A.s_tab = s_tab;
-    A.rs_tab = rs_tab;
-    A.partial = partial;
-    A.N = N;
-    A.K = K;
-    A.T = T;
-    A.N_pad = padded_rows(N);
-    A.n_alpha = n_alpha;
-    A.G = (int)(K / q.group_size);
-    A.group = q.group_size;
-    A.n_tb = (int)((T + awq::srch2::BT - 1) / awq::srch2::BT);
-    A.n_kb = (int)(K / awq::srch2::BK);
-    A.n_units = (A.N_pad / awq::srch2::PM) * A.n_tb * n_alpha;
-    A.qmax = qmax;
-    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
-    const int64_t pairs = A.n_units < d.max_pairs ? A.n_units : d.max_pairs;
-    const int grid = (int)(2 * pairs);
-    cudaEvent_t pb = t_prof_begin, pe = t_prof_end;
-    t_prof_begin = t_prof_end = nullptr;
-    if (pb && cudaEventRecord(pb, st) != cudaSuccess) return AWQ_ERR_CUDA;
-    awq::srch2::search_pair_kernel<<<grid, awq::srch2::NUM_THREADS, awq::srch2::SMEM_BYTES, st>>>(tmap_x, tmap_w, A);
-    if (awq_status e = last_launch()) return e;
-    if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
-
-    // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
-    awq::loss_reduce_kernel<<<n_alpha, awq::kLossThreads, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
-    return last_launch();
+    return search_core(W, N, K, X, T, ldx, q, s_tab, rs_tab, n_alpha, nullptr, params, partial, losses, row_losses,
+                       d, st);
 }
+
 
 awq_status awq_search_layer_noalloc(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx,
                                     const float *a, awq_qcfg q, const float *alphas, int32_t n_alpha,
@@ -377,6 +415,70 @@ awq_status awq_search_layer_noalloc(const void *W, int64_t N, int64_t K, const v
     if (awq_status e = noalloc_scratch(&ws)) return e;
     return awq_search_layer(W, N, K, X, T, ldx, a, q, alphas, n_alpha, losses, row_losses, ws,
                             AWQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t awq_search_scales_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q, int32_t n_s, int32_t masked) {
+    if (!valid_qcfg(q) || N < 1 || K < 1 || T < 1 || n_s < 1 || K % q.group_size) return 0;
+    return search_ws_layout(N, K, T, q.group_size, n_s, masked != 0).total;
+}
+
+awq_status awq_search_scales(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx,
+                             awq_qcfg q, const float *s_table, int32_t n_s, const uint8_t *mask, float *losses,
+                             float *row_losses, void *ws, size_t ws_bytes, void *stream) {
+    if (!W || !X || !s_table || !losses) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(X) || !aligned16(s_table) || !aligned16(losses) ||
+        (row_losses && !aligned16(row_losses)) || (mask && !aligned16(mask)))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || T < 1 || T > kMaxDim || K < 64 || K > kMaxDim || K % 64 ||
+        K % q.group_size || ldx < K || ldx % 8 || n_s < 1 || n_s > kMaxAlpha)
+        return AWQ_ERR_INVALID_ARG;
+    const SearchWs L = search_ws_layout(N, K, T, q.group_size, n_s, mask != nullptr);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *s_tab = reinterpret_cast<float *>(base + L.s_off);
+    float *rs_tab = reinterpret_cast<float *>(base + L.rs_off);
+    uint2 *params = reinterpret_cast<uint2 *>(base + L.prm_off);
+    float *partial = reinterpret_cast<float *>(base + L.part_off);
+    {
+        int grid = blocks_for((int64_t)n_s * K, 256);
+        if (grid > 4 * d.sms) grid = 4 * d.sms;
+        awq::scale_table_kernel<<<grid, 256, 0, st>>>(s_table, (int64_t)n_s * K, s_tab, rs_tab);
+        if (awq_status e = last_launch()) return e;
+    }
+    const void *Xs = X;
+    int64_t ld = ldx;
+    if (mask) {                        // the fp16-kept channels take no part in the loss
+        __half *Xm = reinterpret_cast<__half *>(base + L.xm_off);
+        int grid = blocks_for(T * (K / 8), 256);
+        if (grid > 8 * d.sms) grid = 8 * d.sms;
+        awq::mask_columns_kernel<<<grid, 256, 0, st>>>((const __half *)X, T, K, ldx, mask, Xm);
+        if (awq_status e = last_launch()) return e;
+        Xs = Xm;
+        ld = K;
+    }
+    return search_core(W, N, K, Xs, T, ld, q, s_tab, rs_tab, n_s, mask, params, partial, losses, row_losses, d, st);
+}
+
+awq_status awq_salient_scales(const uint8_t *mask, int64_t K, float factor, float *s, void *stream) {
+    if (!mask || !s || K < 1 || K > kMaxDim || !(factor > 0.0f && factor <= FLT_MAX)) return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    int grid = blocks_for(K, 256);
+    if (grid > 2 * d.sms) grid = 2 * d.sms;
+    awq::salient_scales_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(mask, K, factor, s);
+    return last_launch();
+}
+
+awq_status awq_channel_topk(const float *stat, int64_t K, int64_t k, uint8_t *mask, void *stream) {
+    if (!stat || !mask || K < 1 || K > kMaxDim || k < 0 || k > K) return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    const int grid = blocks_for(K, awq::kTopkThreads);
+    awq::topk_kernel<<<grid, awq::kTopkThreads, 0, (cudaStream_t)stream>>>(stat, K, k, mask);
+    return last_launch();
 }
 
 awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcfg q, const float *alphas,
@@ -399,17 +501,19 @@ awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcf
         awq::best_scale_kernel<<<grid, 256, 0, st>>>(a, K, alphas, losses, n_alpha, best_idx, s_best);
         if (awq_status e = last_launch()) return e;
     }
-    const int G = (int)(K / q.group_size);
-    const int lpr = q.group_size / awq::kGpCols;
-    const int64_t rows_per_block = awq::kGpThreads / lpr;
-    const unsigned grid = (unsigned)(((N + rows_per_block - 1) / rows_per_block) * G);
-    if (lpr == 2)
-        awq::pack_kernel<2><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
-                                                             (__half *)scales, (__half *)zeros);
-    else
-        awq::pack_kernel<1><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, s_best, codes,
-                                                             (__half *)scales, (__half *)zeros);
-    return last_launch();
+    return launch_pack(W, N, K, s_best, q, codes, scales, zeros, st);
+}
+
+awq_status awq_pack_scales(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, uint32_t *codes,
+                           void *scales, void *zeros, void *stream) {
+    if (!W || !s || !codes || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(s) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || K < q.group_size || K > kMaxDim || K % q.group_size)
+        return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    return launch_pack(W, N, K, s, q, codes, scales, zeros, (cudaStream_t)stream);
 }
 
 size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N) {
@@ -502,7 +606,7 @@ awq_status awq_get_status(void *stream) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(awq::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return AWQ_ERR_CUDA;
         if (flags & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
-        if (flags & awq::kDevErrBadAlpha) return AWQ_ERR_INVALID_ARG;
+        if (flags & (awq::kDevErrBadAlpha | awq::kDevErrBadScale)) return AWQ_ERR_INVALID_ARG;
     }
     return last_launch();
 }

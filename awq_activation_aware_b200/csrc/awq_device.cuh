@@ -20,7 +20,7 @@ namespace awq {
 // Device error word (read and cleared by awq_get_status on the host).  The
 // library is a single translation unit, so the definition lives here.
 // ---------------------------------------------------------------------------
-enum : unsigned { kDevErrTimeout = 1u, kDevErrBadAlpha = 2u };
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBadAlpha = 2u, kDevErrBadScale = 4u };
 __device__ unsigned g_dev_error = 0;
 
 // ---------------------------------------------------------------------------
@@ -52,16 +52,25 @@ struct QParams {
     bool clamp;  // some code of the group leaves [0, qmax] before clamping
 };
 
-__device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax) {
+// Group parameters from the group's range [mn, mx] of w' = RN32(w s).
+//   asymmetric: scale = RN32(RN32(mx - mn) / qmax), z = clamp(rint(-mn r), 0, qmax)
+//   symmetric (sym): scale = RN32(max(-mn, mx) / (2^(b-1) - 1)), z = 2^(b-1)
+//     with qmax = 2^b - 1, so 2^(b-1) = (qmax + 1) / 2
+// then sh = RN16(clamp(scale)), r = RN32(1 / sh).
+__device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax, bool sym = false) {
     QParams p;
-    const float range = __fsub_rn(mx, mn);
-    float scale = __fdiv_rn(range, qmax);
+    const float mid = __fmul_rn(0.5f, __fadd_rn(qmax, 1.0f));
+    float scale = sym ? __fdiv_rn(fmaxf(-mn, mx), __fsub_rn(mid, 1.0f)) : __fdiv_rn(__fsub_rn(mx, mn), qmax);
     scale = fminf(fmaxf(scale, kMinScale), kMaxScale);
     p.sh = __half2float(__float2half_rn(scale));
     p.r = __frcp_rn(p.sh);
     const float top = __fadd_rn(kMagic, qmax);
-    const float vz = __fmaf_rn(-mn, p.r, kMagic);
-    p.z = __fsub_rn(fminf(fmaxf(vz, kMagic), top), kMagic);
+    if (sym) {
+        p.z = mid;
+    } else {
+        const float vz = __fmaf_rn(-mn, p.r, kMagic);
+        p.z = __fsub_rn(fminf(fmaxf(vz, kMagic), top), kMagic);
+    }
     const float vmn = __fmaf_rn(mn, p.r, kMagic);
     const float vmx = __fmaf_rn(mx, p.r, kMagic);
     p.clamp = (vmn < __fsub_rn(kMagic, p.z)) || (vmx > __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));

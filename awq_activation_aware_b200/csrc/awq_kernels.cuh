@@ -8,6 +8,9 @@
 //   best_scale_kernel     argmin over the grid + s_best
 //   pack_kernel           codes / fp16 scales / fp16 zeros   (HBM-bound)
 //   quant_dequant_kernel  W_hat for one s (the a3/a4 step on its own)
+//   scale_table_kernel    a caller's s table checked, with RN32(1/s)  (tiny)
+//   mask_columns_kernel   X with the fp16-kept channels zeroed       (HBM-bound)
+//   topk_kernel           the k channels of largest statistic        (tiny)
 //
 // Sources (web pages): [AWQ-note] "AWQ: Activation-Aware Weight Quantization For
 // On-Device LLM Compression AND Acceleration", section "Measures"; [QAS-QA]
@@ -176,10 +179,27 @@ __device__ __forceinline__ void minmax64(const float (&w)[kGpCols], const float 
     mx = hi;
 }
 
+// The same over the channels not held in fp16 (keep: one flag byte per column
+// in shared memory); a lane whose columns are all kept returns +inf / -inf.
+__device__ __forceinline__ void minmax64_kept(const float (&w)[kGpCols], const float *s_sm, const uint8_t *keep,
+                                              float &mn, float &mx) {
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kGpCols; ++k) {
+        const float p = __fmul_rn(w[k], s_sm[k]);
+        lo = keep[k] ? lo : fminf(lo, p);
+        hi = keep[k] ? hi : fmaxf(hi, p);
+    }
+    mn = lo;
+    mx = hi;
+}
+
 template <int LPR>   // lanes per row = group_size / 64
 __global__ void __launch_bounds__(kGpThreads)
 group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int64_t K, int G,
-                    const float *__restrict__ s_tab, int n_alpha, float qmax, uint2 *__restrict__ params) {
+                    const float *__restrict__ s_tab, int n_alpha, float qmax, int sym,
+                    const uint8_t *__restrict__ mask, uint2 *__restrict__ params) {
+    __shared__ uint8_t keep_sm[LPR * kGpCols];
     extern __shared__ float s_sm[];                 // [n_alpha][LPR][kGpCols + 4] (+4: the halves sit in other banks)
     constexpr int kRowsPerBlock = kGpThreads / LPR;
     constexpr int kStride = kGpCols + 4;
@@ -190,6 +210,8 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int6
         const int ai = i / (LPR * kGpCols), rem = i % (LPR * kGpCols);
         s_sm[(ai * LPR + rem / kGpCols) * kStride + rem % kGpCols] = __ldg(s_tab + (int64_t)ai * K + k0 + rem);
     }
+    if (mask)
+        for (int i = threadIdx.x; i < LPR * kGpCols; i += kGpThreads) keep_sm[i] = __ldg(mask + k0 + i);
     __syncthreads();
     const int half = threadIdx.x % LPR;
     const int64_t n = n0 + threadIdx.x / LPR;
@@ -203,13 +225,17 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int6
     }
     for (int ai = 0; ai < n_alpha; ++ai) {
         float mn, mx;
-        minmax64(w, s_sm + (ai * LPR + half) * kStride, mn, mx);
+        if (mask)
+            minmax64_kept(w, s_sm + (ai * LPR + half) * kStride, keep_sm + half * kGpCols, mn, mx);
+        else
+            minmax64(w, s_sm + (ai * LPR + half) * kStride, mn, mx);
         if (LPR == 2) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         }
+        if (mn > mx) { mn = 0.0f; mx = 0.0f; }          // every channel of the group kept in fp16
         if (half == 0 && n < N_pad)
-            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(make_qparams(mn, mx, qmax))
+            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(make_qparams(mn, mx, qmax, sym != 0))
                                                                  : make_uint2(0, 0);
     }
 }
@@ -220,7 +246,8 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int6
 template <int TPG>
 __global__ void __launch_bounds__(256)
 quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
-                     const float *__restrict__ s, float qmax, __half *__restrict__ W_hat) {
+                     const float *__restrict__ s, float qmax, int sym, const uint8_t *__restrict__ mask,
+                     __half *__restrict__ W_hat) {
     const int64_t gid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / TPG;
     const int sub = threadIdx.x % TPG;
     const bool active = gid < N * (int64_t)G;
@@ -241,15 +268,22 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
             rs[e] = __frcp_rn(sv[e]);
         }
     }
+    bool kept[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) kept[e] = mask && active && __ldg(mask + k0 + e) != 0;
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) { mn = fminf(mn, wp[e]); mx = fmaxf(mx, wp[e]); }
+    for (int e = 0; e < 16; ++e) {
+        mn = kept[e] ? mn : fminf(mn, wp[e]);
+        mx = kept[e] ? mx : fmaxf(mx, wp[e]);
+    }
 #pragma unroll
     for (int off = 1; off < TPG; off <<= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
-    const QParams prm = make_qparams(mn, mx, qmax);
+    if (mn > mx) { mn = 0.0f; mx = 0.0f; }              // every channel of the group kept in fp16
+    const QParams prm = make_qparams(mn, mx, qmax, sym != 0);
     const QPair qp = make_qpair(prm, qmax);
     if (!active) return;
     __align__(16) __half2 out[8];
@@ -262,8 +296,90 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
                      : dequant_unscale_pair<false>(make_float2(wv[2 * e], wv[2 * e + 1]),
                                                    make_float2(sv[2 * e], sv[2 * e + 1]),
                                                    make_float2(rs[2 * e], rs[2 * e + 1]), qp);
+    if (mask) {                                      // channels kept in fp16 pass through
+        __half *o = reinterpret_cast<__half *>(out);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (kept[e]) o[e] = __float2half_rn(wv[e]);
+    }
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0) = *reinterpret_cast<const uint4 *>(&out[0]);
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[4]);
+}
+
+// ===========================================================================
+// Quantizer variants and baselines ([AWQ-note] "Measures": RTN, a fixed scale
+// of 2 on the salient channels, and keeping 1% of the channels in FP16,
+// chosen by activation or by weight magnitude).
+// ===========================================================================
+
+// A caller's scale table s[i][k] (scales given instead of a^alpha): copied
+// into the workspace with rs = RN32(1/s); a scale that is not a positive
+// finite number raises the bad-scale flag (the search would be meaningless).
+__global__ void scale_table_kernel(const float *__restrict__ s_in, int64_t total, float *__restrict__ s_tab,
+                                   float *__restrict__ rs_tab) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = s_in[i];
+        if (!(v > 0.0f && v <= FLT_MAX)) atomicOr(&g_dev_error, kDevErrBadScale);
+        s_tab[i] = v;
+        rs_tab[i] = __frcp_rn(v);
+    }
+}
+
+// Xm = X with the columns of the channels kept in fp16 set to +0: their
+// error is zero, so they must not reach the loss (the search contracts
+// W_hat - W against Xm).  8 columns per thread, 16-byte accesses.
+__global__ void mask_columns_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx,
+                                    const uint8_t *__restrict__ mask, __half *__restrict__ Xm) {
+    const int64_t per_row = K / 8, total = T * per_row;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_row, c = (i - t * per_row) * 8;
+        uint4 v = ldg_stream_v4(X + t * ldx + c);
+        const uint2 m = *reinterpret_cast<const uint2 *>(mask + c);
+        uint16_t *h = reinterpret_cast<uint16_t *>(&v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if ((e < 4 ? (m.x >> (8 * e)) : (m.y >> (8 * (e - 4)))) & 0xFFu) h[e] = 0;
+        *reinterpret_cast<uint4 *>(Xm + t * K + c) = v;
+    }
+}
+
+// s[k] = factor for the channels in the mask, 1 elsewhere: the variant that
+// scales only the salient channels by a fixed factor ([AWQ-note] "Measures":
+// scaling them by 2 instead of keeping them in FP16).
+__global__ void salient_scales_kernel(const uint8_t *__restrict__ mask, int64_t K, float factor,
+                                      float *__restrict__ s) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < K; i += (int64_t)gridDim.x * blockDim.x)
+        s[i] = mask[i] ? factor : 1.0f;
+}
+
+// mask[j] = 1 for the k channels of largest stat[j] (ties: lower index first;
+// NaN ranks below every number), by counting, for each j, the channels that
+// come before it.  A block stages a tile of the statistic in shared memory;
+// K^2 comparisons, microseconds for the layers here.
+constexpr int kTopkThreads = 256;
+__global__ void __launch_bounds__(kTopkThreads)
+topk_kernel(const float *__restrict__ stat, int64_t K, int64_t k, uint8_t *__restrict__ mask) {
+    __shared__ float tile[kTopkThreads];
+    const int64_t j = blockIdx.x * (int64_t)kTopkThreads + threadIdx.x;
+    const float vj = j < K ? stat[j] : 0.0f;
+    const bool nj = isnan(vj);
+    int64_t before = 0;
+    for (int64_t i0 = 0; i0 < K; i0 += kTopkThreads) {
+        __syncthreads();
+        tile[threadIdx.x] = i0 + threadIdx.x < K ? stat[i0 + threadIdx.x] : 0.0f;
+        __syncthreads();
+        const int lim = (int)(K - i0 < kTopkThreads ? K - i0 : kTopkThreads);
+        for (int q = 0; q < lim; ++q) {
+            const int64_t i = i0 + q;
+            const float vi = tile[q];
+            const bool ni = isnan(vi);
+            bool b;
+            if (ni || nj) b = (!ni && nj) || (ni && nj && i < j);
+            else b = vi > vj || (vi == vj && i < j);
+            before += (i != j && b) ? 1 : 0;
+        }
+    }
+    if (j < K) mask[j] = before < k ? 1 : 0;
 }
 
 // ===========================================================================
@@ -697,7 +813,7 @@ __global__ void best_scale_kernel(const float *__restrict__ a, int64_t K,
 // ===========================================================================
 template <int LPR>
 __global__ void __launch_bounds__(kGpThreads)
-pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
+pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits, int sym,
             const float *__restrict__ s_best, uint32_t *__restrict__ codes,
             __half *__restrict__ scales, __half *__restrict__ zeros) {
     __shared__ __align__(16) float s_sm[LPR * (kGpCols + 4)];
@@ -738,7 +854,7 @@ pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     }
-    const QParams p = make_qparams(mn, mx, qmax);
+    const QParams p = make_qparams(mn, mx, qmax, sym != 0);
     if (!active) return;
     const int64_t col = k0 + half * kGpCols;
     if (bits == 2) {
@@ -868,19 +984,17 @@ __global__ void qlinear_prep_kernel(const __half *__restrict__ X, int64_t T, int
 
 // (q - z) of the 32/CB codes in one 32-bit word as exact binary32 values: each
 // code c becomes the float 2^23 + c by placing its byte under the exponent bits
-// of 2^23 (one byte permute), and one packed subtraction of 2^23 + z leaves
-// q - z.
+// of 2^23 (one byte permute), and one packed addition of
+// noff = (-(2^23 + z), -(2^23 + z)) leaves q - z.
 template <int CB>
-__device__ __forceinline__ void dequant_word(uint32_t w, float zsub, float *d) {
-    const float2 off = make_float2(-zsub, -zsub);
-    const float2 one = make_float2(1.0f, 1.0f);
+__device__ __forceinline__ void dequant_word(uint32_t w, float2 noff, float *d) {
     if (CB == 4) {
         const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;   // codes 2b / 2b+1 in byte b
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             const float2 f = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | b)),
                                          __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | b)));
-            const float2 r = fma2_rn(f, one, off);
+            const float2 r = __fadd2_rn(f, noff);
             d[2 * b] = r.x;
             d[2 * b + 1] = r.y;
         }
@@ -894,7 +1008,7 @@ __device__ __forceinline__ void dequant_word(uint32_t w, float zsub, float *d) {
             for (int j = 0; j < 4; j += 2) {
                 const float2 f = make_float2(__uint_as_float(__byte_perm(m[j], 0x4B000000u, 0x7440u | b)),
                                              __uint_as_float(__byte_perm(m[j + 1], 0x4B000000u, 0x7440u | b)));
-                const float2 r = fma2_rn(f, one, off);
+                const float2 r = __fadd2_rn(f, noff);
                 d[4 * b + j] = r.x;
                 d[4 * b + j + 1] = r.y;
             }
@@ -1034,12 +1148,14 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
             if (j * SC + lane_col < A.K) {                       // lanes past K hold zero fill
                 const __half *sz = reinterpret_cast<const __half *>(stage + TX_BYTES);
                 uint2 w[RPW];
-                float zs[RPW], sh[RPW];
+                float sh[RPW];
+                float2 noff[RPW];                                // -(2^23 + z), twice
 #pragma unroll
                 for (int r = 0; r < RPW; ++r) {
                     w[r] = *reinterpret_cast<const uint2 *>(stage + ((rg * RPW + r) * WORDS + hh * 64 + 2 * lane) * 4);
                     sh[r] = __half2float(sz[(rg * RPW + r) * gps + gl]);
-                    zs[r] = __fadd_rn(8388608.0f, __half2float(sz[(ROWS + rg * RPW + r) * gps + gl]));
+                    const float nz = -__fadd_rn(8388608.0f, __half2float(sz[(ROWS + rg * RPW + r) * gps + gl]));
+                    noff[r] = make_float2(nz, nz);
                 }
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -1055,7 +1171,7 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
 #pragma unroll
                     for (int r = 0; r < RPW; ++r) {
                         float d[CPW];
-                        dequant_word<CB>(i == 0 ? w[r].x : w[r].y, zs[r], d);
+                        dequant_word<CB>(i == 0 ? w[r].x : w[r].y, noff[r], d);
 #pragma unroll
                         for (int t = 0; t < TT; ++t) {
                             float2 s2 = mul2_rn(make_float2(x[t][0], x[t][1]), make_float2(d[0], d[1]));

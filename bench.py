@@ -54,9 +54,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
-    p.add_argument("--op", choices=["search", "qlinear"], default="search",
+    p.add_argument("--op", choices=["search", "qlinear", "baselines"], default="search",
                    help="search: the AWQ scale-search path (the benchmark); qlinear: the quantized "
-                        "linear layer on the packed output vs the fp16 GEMM")
+                        "linear layer on the packed output vs the fp16 GEMM; baselines: the pages' "
+                        "comparisons (RTN, fixed 2x, fp16 1%%, symmetric) on one layer")
     p.add_argument("--tokens", default="1,4,16", help="token counts for --op qlinear")
     return p.parse_args()
 
@@ -514,12 +515,75 @@ def run_qlinear(args):
     return 0
 
 
+def run_baselines(args):
+    """The comparisons of the AWQ pages on one layer (RTN, the fixed 2x scale on
+    the salient 1%, fp16 protection of 1% chosen by activation and by weight
+    magnitude, the asymmetric and the symmetric grid search), each timed on
+    the device with CUDA events after warm-up.  One JSON line with the losses
+    and the time of each; value = the searched layer-scale evaluations per
+    second of the whole set."""
+    import torch
+
+    import awq_activation_aware_b200 as awq
+    from awq_activation_aware_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    cfg = synth.CONFIGS[args.config]
+    W, X, _ = synth.generate(cfg)
+    Wd = torch.from_numpy(W).to(dev)
+    Xd = torch.from_numpy(X).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 3)
+
+    def timed(fn):
+        for _ in range(3):
+            flush.zero_()
+            out = fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b.record()
+            out = fn()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(b.elapsed_time(e))
+        return out, statistics.median(ts)
+
+    r, t_all = timed(lambda: awq.baselines(Wd, Xd, cfg.bits, cfg.group))
+    a = awq.act_stats(Xd)
+    al = awq.default_alphas(device=dev)
+    sym, t_sym = timed(lambda: awq.search_layer(Wd, Xd, a, al, cfg.bits, cfg.group, zero_point=False))
+    table = torch.stack([awq.salient_scales(r["mask_act"], 1.0), awq.salient_scales(r["mask_act"], 2.0)])
+    _, t_two = timed(lambda: awq.search_scales(Wd, Xd, table, cfg.bits, cfg.group))
+    _, t_masked = timed(lambda: awq.search_scales(Wd, Xd, table[:1].contiguous(), cfg.bits, cfg.group,
+                                                  mask=r["mask_act"]))
+    awq.get_status()
+    evals = 2 + 1 + 1 + 20                              # scale vectors searched by baselines()
+    flops = 2.0 * cfg.N * cfg.K * cfg.T
+    print(json.dumps({
+        "op": "baselines", "config": cfg.name, "k_channels": int(r["k"]),
+        "losses": {"rtn": float(r["rtn"]), "fixed_2x": float(r["fixed_2x"]), "fp16_act": float(r["fp16_act"]),
+                   "fp16_weight": float(r["fp16_weight"]), "awq_grid_best": float(r["awq_grid"].min()),
+                   "awq_grid_best_symmetric": float(sym.min())},
+        "ms": {"baselines_all": t_all, "grid_symmetric_20": t_sym, "given_scales_2": t_two,
+               "given_scales_1_masked": t_masked},
+        "tflops": {"baselines_all": evals * flops / (t_all * 1e-3) / 1e12,
+                   "grid_symmetric_20": 20 * flops / (t_sym * 1e-3) / 1e12,
+                   "given_scales_2": 2 * flops / (t_two * 1e-3) / 1e12,
+                   "given_scales_1_masked": flops / (t_masked * 1e-3) / 1e12},
+        "l2": "flushed (256 MiB write) before every timed call"}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "qlinear":
         return run_qlinear(args)
+    if args.op == "baselines":
+        return run_baselines(args)
     return run_awq(args)
 
 

@@ -61,7 +61,13 @@ typedef enum {
 /* Quantizer configuration ([QAS-QA] §9 quant_config):
  *   bits        w_bit, one of 2, 3, 4  (codes 0 .. 2^bits - 1)
  *   group_size  q_group_size along K, one of 64, 128
- *   zero_point  must be 1 (asymmetric quantization with a zero point)        */
+ *   zero_point  1: asymmetric groups with a zero-point code
+ *                  (scale = (max w' - min w') / qmax, z = clamp(rint(-min w' / scale)))
+ *               0: symmetric absmax groups ([AWQ-note] "Measures": the INT3
+ *                  grid of step max|w| / (2^(b-1) - 1)): scale = max|w'| / (2^(bits-1) - 1)
+ *                  and the zero fixed at the middle code 2^(bits-1), stored in
+ *                  `zeros` like any zero point, so every consumer of the packed
+ *                  format treats both alike.                                    */
 typedef struct {
     int32_t bits;
     int32_t group_size;
@@ -89,7 +95,7 @@ AWQ_API awq_status awq_act_stats(const void *X, int64_t T, int64_t K, int64_t ld
 AWQ_API awq_status awq_alpha_scales(const float *a, int64_t K, const float *alphas, int32_t n_alpha,
                             float *s, void *stream);
 
-/* Steps a3/a4 standalone -- scale, group-wise asymmetric round-to-nearest,
+/* Steps a3/a4 standalone -- scale, group-wise round-to-nearest,
  * dequantize, unscale ([QAS-QA] §5; [AWQ-wiki] "Fondements techniques": the
  * inverse scaling is applied after dequantization).  For one scale vector s:
  *   per row n and group G of group_size columns:
@@ -99,11 +105,22 @@ AWQ_API awq_status awq_alpha_scales(const float *a, int64_t K, const float *alph
  *     q     = clamp(rint(w' * r) + z, 0, qmax)
  *     w_hat = RN16(RN32(RN32((q - z) * sh) * RN32(1 / s)))
  *   (the products inside rint are exact: rint is their only rounding)
+ *   (zero_point = 0: scale = RN32(max(-min w', max w') / (2^(bits-1) - 1)), z = 2^(bits-1))
  *   W      fp16 [N, K];  s  float [K];  W_hat  fp16 [N, K] output.
  * This is the exact per-element function the search evaluates for every
  * alpha; it never runs inside the search (the search keeps W_hat on chip). */
 AWQ_API awq_status awq_quant_dequant(const void *W, int64_t N, int64_t K, const float *s,
                              awq_qcfg q, void *W_hat, void *stream);
+
+/* The same with channels held in fp16 ([AWQ-note] "Measures": keeping 1% of
+ * the input channels in FP16 is the experiment that motivates the method).
+ *   mask  uint8 [K] (device) or NULL: mask[k] != 0 keeps channel k in fp16 --
+ *         it takes no part in its group's min and max, and W_hat[:, k] = W[:, k].
+ *         A group whose channels are all kept has min = max = 0.
+ * Mixed fp16/low-bit storage is not a packed format of this library: the
+ * mask serves the baselines' loss (awq_search_scales) and this W_hat. */
+AWQ_API awq_status awq_quant_dequant_masked(const void *W, int64_t N, int64_t K, const float *s,
+                                            awq_qcfg q, const uint8_t *mask, void *W_hat, void *stream);
 
 /* Bytes of device workspace awq_search_layer needs for these sizes. */
 AWQ_API size_t awq_search_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q,
@@ -168,6 +185,41 @@ AWQ_API awq_status awq_search_layer_noalloc(const void *W, int64_t N, int64_t K,
                                             const float *alphas, int32_t n_alpha,
                                             float *losses, float *row_losses, void *stream);
 
+/* Search over caller-given scale vectors instead of a^alpha: the baselines
+ * and variants the pages measure against AWQ ([AWQ-note] "Measures": plain
+ * RTN is s = 1; scaling only the salient 1% of channels by a fixed 2; keeping
+ * 1% of the channels in FP16, chosen by activation or by weight magnitude).
+ *   s_table  float [n_s, K] (device), every value positive and finite
+ *            (otherwise awq_get_status reports AWQ_ERR_INVALID_ARG)
+ *   mask     uint8 [K] (device) or NULL: channels held in fp16, as in
+ *            awq_quant_dequant_masked; they contribute no output error
+ *   losses, row_losses, ws: as awq_search_layer, one entry per scale vector;
+ *            ws >= awq_search_scales_workspace_bytes(N, K, T, q, n_s, mask != NULL)
+ * 1 <= n_s <= 64.  Everything else as awq_search_layer: with the table's rows
+ * equal to a^alpha_i the losses are awq_search_layer's. */
+AWQ_API size_t awq_search_scales_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q,
+                                                 int32_t n_s, int32_t masked);
+AWQ_API awq_status awq_search_scales(const void *W, int64_t N, int64_t K, const void *X, int64_t T,
+                                     int64_t ldx, awq_qcfg q, const float *s_table, int32_t n_s,
+                                     const uint8_t *mask, float *losses, float *row_losses,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* Channel selection for the FP16-protection baselines: mask[j] = 1 for the k
+ * channels with the largest stat[j], 0 for the rest; ties go to the lower
+ * index and NaN ranks below every number.  stat is a statistic per input
+ * channel: awq_act_stats of X (activation magnitude) or of W read as [N, K]
+ * rows (mean |w| per input channel, the weight-magnitude criterion).
+ *   stat  float [K] (device);  mask  uint8 [K] output (device);  0 <= k <= K. */
+AWQ_API awq_status awq_channel_topk(const float *stat, int64_t K, int64_t k, uint8_t *mask,
+                                    void *stream);
+
+/* s[k] = factor where mask[k] != 0, else 1: the scale vector of the variant
+ * that scales only the salient channels by a fixed factor ([AWQ-note]
+ * "Measures": scaling the 1% salient channels by 2); factor 1 gives plain RTN.
+ *   mask  uint8 [K] (device);  s  float [K] output (device);  factor > 0, finite. */
+AWQ_API awq_status awq_salient_scales(const uint8_t *mask, int64_t K, float factor, float *s,
+                                      void *stream);
+
 /* Steps a7-a8 -- argmin over the grid and packing ([AWQ-note] "Measures":
  * scale by the best alpha's s, group-quantize, keep the quantized weights and
  * the necessary metadata).
@@ -185,9 +237,16 @@ AWQ_API awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a,
                     int32_t *best_idx, float *s_best, uint32_t *codes,
                     void *scales, void *zeros, void *stream);
 
+/* Step a8 alone for a given scale vector s (float [K], device): the codes,
+ * scales and zeros of W diag(s) with the layout of awq_pack (a baseline's
+ * packed layer, or a scale chosen elsewhere). */
+AWQ_API awq_status awq_pack_scales(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q,
+                                   uint32_t *codes, void *scales, void *zeros, void *stream);
+
 /* Synchronises `stream`, then reports (and clears) errors raised on the device
  * since the last call: AWQ_ERR_TIMEOUT if a kernel's bounded wait ran out,
- * AWQ_ERR_INVALID_ARG if a kernel saw an alpha outside [0, 1], AWQ_ERR_CUDA for
+ * AWQ_ERR_INVALID_ARG if a kernel saw an alpha outside [0, 1] or a given scale
+ * that is not positive and finite, AWQ_ERR_CUDA for
  * a pending CUDA error.  AWQ_OK otherwise. */
 AWQ_API awq_status awq_get_status(void *stream);
 

@@ -64,7 +64,7 @@ def _search(**kw):
     dict(W=None), dict(X=None), dict(a=None), dict(alphas=None), dict(losses=None),
     dict(W=MISALIGNED), dict(row_losses=MISALIGNED),
     dict(N=0), dict(T=0), dict(K=100), dict(K=96), dict(ldx=500), dict(ldx=516),
-    dict(q=QCfg(5, 128, 1)), dict(q=QCfg(4, 32, 1)), dict(q=QCfg(4, 128, 0)), dict(q=QCfg(4, 128, 1), K=192),
+    dict(q=QCfg(5, 128, 1)), dict(q=QCfg(4, 32, 1)), dict(q=QCfg(4, 128, 2)), dict(q=QCfg(4, 128, 1), K=192),
     dict(n_alpha=0), dict(n_alpha=65), dict(N=1 << 31),
 ])
 def test_search_rejects_bad_arguments(bad):
@@ -94,3 +94,43 @@ def test_binding_requires_cuda_tensors():
     import torch
     with pytest.raises(TypeError):
         awq.act_stats(torch.zeros((4, 64), dtype=torch.float16))
+
+
+def _search_scales(**kw):
+    args = dict(W=BOGUS, N=256, K=512, X=BOGUS, T=512, ldx=512, q=QCfg(4, 128, 0), s_table=BOGUS, n_s=2,
+                mask=None, losses=BOGUS, row_losses=None, ws=BOGUS, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return awq.lib().awq_search_scales(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(W=None), dict(X=None), dict(s_table=None), dict(losses=None), dict(s_table=MISALIGNED),
+    dict(mask=MISALIGNED), dict(n_s=0), dict(n_s=65), dict(K=96), dict(ldx=500), dict(q=QCfg(4, 128, 3)),
+    dict(T=0),
+])
+def test_search_scales_rejects_bad_arguments(bad):
+    assert _search_scales(**bad) == 1
+
+
+def test_search_scales_workspace():
+    L = awq.lib()
+    q = QCfg(4, 128, 1)
+    plain = L.awq_search_scales_workspace_bytes(4096, 4096, 4096, q, 3, 0)
+    masked = L.awq_search_scales_workspace_bytes(4096, 4096, 4096, q, 3, 1)
+    assert plain == L.awq_search_workspace_bytes(4096, 4096, 4096, q, 3)
+    assert masked - plain == 2 * 4096 * 4096                # X with the kept channels zeroed
+    small = L.awq_search_scales_workspace_bytes(256, 512, 512, QCfg(4, 128, 0), 2, 0)
+    assert _search_scales(ws_bytes=small, mask=BOGUS) == 5  # a mask needs the larger workspace
+
+
+def test_variant_entry_points_reject_bad_arguments():
+    L = awq.lib()
+    assert L.awq_quant_dequant_masked(BOGUS, 4, 128, BOGUS, QCfg(4, 128, 5), BOGUS, BOGUS, None) == 1
+    assert L.awq_quant_dequant_masked(None, 4, 128, BOGUS, QCfg(4, 128, 0), BOGUS, BOGUS, None) == 1
+    assert L.awq_channel_topk(BOGUS, 64, 65, BOGUS, None) == 1          # k > K
+    assert L.awq_channel_topk(BOGUS, 64, -1, BOGUS, None) == 1
+    assert L.awq_channel_topk(None, 64, 1, BOGUS, None) == 1
+    assert L.awq_salient_scales(BOGUS, 64, ctypes.c_float(0.0), BOGUS, None) == 1
+    assert L.awq_salient_scales(BOGUS, 64, ctypes.c_float(float("inf")), BOGUS, None) == 1
+    assert L.awq_pack_scales(BOGUS, 4, 100, BOGUS, QCfg(4, 128, 0), BOGUS, BOGUS, BOGUS, None) == 1
+    assert L.awq_pack_scales(BOGUS, 4, 128, BOGUS, QCfg(4, 128, 0), MISALIGNED, BOGUS, BOGUS, None) == 1

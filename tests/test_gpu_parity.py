@@ -352,3 +352,161 @@ def test_qlinear(awq, N, K, T, bits, group):
     Y2 = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]),
                           dev(pk["s_best"]), dev(X), bits, group))
     assert np.array_equal(Y, Y2)
+
+
+# ---------------------------------------------------------------------------
+# Quantizer variants and baselines: symmetric groups, channels held in fp16,
+# caller-given scale vectors, top-k channel selection
+# ---------------------------------------------------------------------------
+def _mask(K, seed, group):
+    rng = np.random.default_rng(seed)
+    m = np.zeros(K, dtype=np.uint8)
+    m[rng.choice(K, max(1, K // 60), replace=False)] = 1
+    m[group:2 * group] = 1                            # one whole group held in fp16
+    return m
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (2, 64), (4, 64)])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("masked", [False, True])
+def test_quant_dequant_variants_bitexact(awq, bits, group, sym, masked):
+    W, X = gen(300, 1024, 64, bits=bits, group=group, seed=81 + bits)
+    a = oracle.act_stats(X)
+    s = oracle.scales(a, 0.45)
+    m = _mask(1024, bits, group) if masked else None
+    ref = oracle.quantize(W, s, bits, group, zero_point=not sym, mask=m)["what"]
+    got = host(awq.quant_dequant(dev(W), dev(s), bits, group, zero_point=not sym,
+                                 mask=None if m is None else dev(m)))
+    awq.get_status()
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("N,K,T,bits,group,sym,masked", [
+    (300, 1024, 700, 4, 128, False, True), (256, 512, 512, 4, 128, True, False),
+    (520, 768, 300, 3, 64, True, True), (136, 640, 1030, 2, 128, False, False),
+])
+def test_search_scales_matches_oracle(awq, N, K, T, bits, group, sym, masked):
+    W, X = gen(N, K, T, bits=bits, group=group, seed=N + K)
+    a = oracle.act_stats(X)
+    k = max(1, round(K / 100))
+    m_act = oracle.topk_mask(a, k)
+    table = np.stack([np.ones(K, np.float32), np.where(m_act == 1, 2.0, 1.0).astype(np.float32),
+                      oracle.scales(a, 0.5)])
+    m = _mask(K, N, group) if masked else None
+    ref = oracle.search_scales(W, X, table, bits, group, zero_point=not sym, mask=m)
+    losses, rows = awq.search_scales(dev(W), dev(X), dev(table), bits, group, zero_point=not sym,
+                                     mask=None if m is None else dev(m), row_losses=True)
+    awq.get_status()
+    np.testing.assert_allclose(host(losses).astype(np.float64), ref["losses"], rtol=LOSS_RTOL)
+    np.testing.assert_allclose(host(rows).astype(np.float64), ref["row_sums"], rtol=LOSS_RTOL, atol=1e-30)
+
+
+def test_search_scales_equals_grid_search(awq):
+    """The grid's own s vectors, passed as a table, give the grid's losses bit for bit."""
+    W, X = gen(256, 512, 512, seed=91)
+    Wd, Xd = dev(W), dev(X)
+    a = awq.act_stats(Xd)
+    al = awq.default_alphas()
+    grid = awq.search_layer(Wd, Xd, a, al)
+    table = awq.alpha_scales(a, al)
+    given = awq.search_scales(Wd, Xd, table)
+    awq.get_status()
+    assert torch.equal(grid, given)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 64), (2, 64)])
+def test_symmetric_whole_path(awq, bits, group):
+    """Grid search and packing with the symmetric quantizer against the oracle."""
+    W, X = gen(320, 512, 600, bits=bits, group=group, seed=92 + bits)
+    alphas = synth.default_alphas()
+    res = awq.quantize_layer(dev(W), dev(X), bits=bits, group=group, zero_point=False)
+    awq.get_status()
+    a = oracle.act_stats(X)
+    ref = oracle.search(W, X, a, bits, group, alphas, zero_point=False)
+    np.testing.assert_allclose(host(res["losses"]).astype(np.float64), ref["losses"], rtol=LOSS_RTOL)
+    best = int(host(res["best_idx"])[0])
+    assert_alpha_choice(best, ref["losses"])
+    losses_used = ref["losses"].copy()
+    losses_used[best] = -1.0                           # pack what the GPU chose
+    pk = oracle.pack(W, a, bits, group, alphas, losses_used, zero_point=False)
+    assert np.array_equal(host(res["codes"]).view(np.uint32), pk["codes"])
+    assert np.array_equal(host(res["scales"]).view(np.uint16), pk["scales"].view(np.uint16))
+    assert np.all(host(res["zeros"]) == 2 ** (bits - 1))
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_pack_scales_bitexact(awq, sym):
+    W, X = gen(200, 768, 8, bits=3, group=128, seed=93)
+    s = np.where(oracle.topk_mask(oracle.act_stats(X), 8) == 1, 2.0, 1.0).astype(np.float32)
+    out = awq.pack_scales(dev(W), dev(s), 3, 128, zero_point=not sym)
+    awq.get_status()
+    pk = oracle.pack_scales(W, s, 3, 128, zero_point=not sym)
+    assert np.array_equal(host(out["codes"]).view(np.uint32), pk["codes"])
+    assert np.array_equal(host(out["scales"]).view(np.uint16), pk["scales"].view(np.uint16))
+    assert np.array_equal(host(out["zeros"]).view(np.uint16), pk["zeros"].view(np.uint16))
+
+
+@pytest.mark.parametrize("K,k", [(1, 1), (300, 0), (300, 3), (4096, 41), (11008, 110), (5000, 5000)])
+def test_channel_topk_bitexact(awq, K, k):
+    rng = np.random.default_rng(K + k)
+    v = rng.integers(0, 50, K).astype(np.float32)          # many ties
+    if K > 10:
+        v[[1, K // 2, K - 1]] = np.nan
+    got = host(awq.channel_topk(dev(v), k))
+    awq.get_status()
+    assert np.array_equal(got, oracle.topk_mask(v, k))
+    assert int(got.sum()) == k
+
+
+def test_salient_scales(awq):
+    m = (np.arange(1000) % 7 == 0).astype(np.uint8)
+    s = host(awq.salient_scales(dev(m), 2.0))
+    assert np.array_equal(s, np.where(m == 1, 2.0, 1.0).astype(np.float32))
+
+
+def test_bad_given_scale_is_reported(awq):
+    W, X = gen(256, 256, 64, seed=94)
+    table = np.ones((2, 256), np.float32)
+    table[1, 17] = 0.0
+    awq.search_scales(dev(W), dev(X), dev(table))
+    with pytest.raises(awq.AWQError):
+        awq.get_status()
+    awq.get_status()                                   # the flag is cleared
+
+
+def test_baselines_match_oracle_and_premise(awq):
+    """The pages' comparisons on a synthetic layer with 1% outlier channels:
+    fp16 protection by activation << RTN, by weight magnitude ~ RTN, and
+    AWQ's searched s better than the fixed 2x; each loss against the oracle."""
+    cfg = synth.make_config(512, 1024, 1024, seed=95)
+    W, X, idx = synth.generate(cfg)
+    r = awq.baselines(dev(W), dev(X), 4, 128)
+    awq.get_status()
+    a = oracle.act_stats(X)
+    m_act = oracle.topk_mask(a, r["k"])
+    m_w = oracle.topk_mask(oracle.act_stats(W), r["k"])
+    assert np.array_equal(host(r["mask_act"]), m_act) and np.array_equal(host(r["mask_weight"]), m_w)
+    one = np.ones((1, cfg.K), np.float32)
+    ref = dict(rtn=oracle.search_scales(W, X, one, 4, 128)["losses"][0],
+               fixed_2x=oracle.search_scales(W, X, np.where(m_act == 1, 2.0, 1.0)[None].astype(np.float32),
+                                             4, 128)["losses"][0],
+               fp16_act=oracle.search_scales(W, X, one, 4, 128, mask=m_act)["losses"][0],
+               fp16_weight=oracle.search_scales(W, X, one, 4, 128, mask=m_w)["losses"][0])
+    for key, v in ref.items():
+        assert float(host(r[key])) == pytest.approx(v, rel=LOSS_RTOL), key
+    awq_best = float(host(r["awq_grid"]).min())
+    assert ref["fp16_act"] < 0.1 * ref["rtn"]
+    assert ref["fp16_weight"] > 0.9 * ref["rtn"]
+    assert awq_best < ref["fixed_2x"] < 0.5 * ref["rtn"]
+
+
+def test_qlinear_on_symmetric_pack(awq):
+    """The decode path reads symmetric packs unchanged (the zero is stored)."""
+    W, X = gen(700, 1024, 3, bits=4, group=128, seed=96, outlier_frac=0.02)
+    a = oracle.act_stats(X)
+    pk = oracle.pack(W, a, 4, 128, synth.default_alphas(), np.linspace(1.0, 0.5, 20), zero_point=False)
+    Y = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]),
+                         dev(pk["s_best"]), dev(X), 4, 128))
+    awq.get_status()
+    ref = oracle.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, 4, 128)
+    np.testing.assert_allclose(Y, ref, rtol=1e-4, atol=1e-4 * np.abs(ref).max())
