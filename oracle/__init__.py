@@ -66,6 +66,8 @@ def _load():
     lib.awq_oracle_quantize.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
                                         ctypes.c_int, P, P, P, P]
     lib.awq_oracle_topk.argtypes = [P, i64, i64, P]
+    lib.awq_oracle_gptq.argtypes = [P, i64, i64, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_double, i64, P, P, P, P, P]
     lib.awq_oracle_pack_codes.argtypes = [P, i64, i64, ctypes.c_int, P]
     lib.awq_oracle_argmin.restype = ctypes.c_int
     lib.awq_oracle_argmin.argtypes = [P, ctypes.c_int]
@@ -298,3 +300,62 @@ def qlinear(codes, scales, zeros, s_best, X, bits: int, group: int) -> np.ndarra
     rs = (np.float32(1.0) / np.asarray(s_best, dtype=np.float32)).astype(np.float32)
     xs = (X.astype(np.float32) * rs[None, :]).astype(np.float32)  # one binary32 rounding
     return xs.astype(np.float64) @ Wq.T
+
+
+# --------------------------------------------------------------------------
+# AWQ followed by GPTQ error compensation -- [AWQ-note] "Measures" (AWQ+GPTQ
+# at INT2); [Notes-52] §4 (round a column, push its error into the columns not
+# yet quantized, using second-order statistics of the real input);
+# [GPTQ-AWQ] "GPTQ" (column-wise sweep, Cholesky factor prepared once).
+# --------------------------------------------------------------------------
+
+def gptq_hessian(X: np.ndarray, s=None) -> np.ndarray:
+    """H = 2 X'^T X' in binary64 (one library matrix product), with the input
+    divided by s as the layer sees it after scaling: x' = RN32(x RN32(1/s))."""
+    X = _as_f16(X)
+    K = X.shape[1]
+    s = np.ones(K, np.float32) if s is None else np.ascontiguousarray(s, dtype=np.float32)
+    rs = (np.float32(1.0) / s).astype(np.float32)
+    Xs = (X.astype(np.float32) * rs[None, :]).astype(np.float32).astype(np.float64)
+    return 2.0 * (Xs.T @ Xs)
+
+
+def gptq_factor(H: np.ndarray, damp: float = 0.01) -> np.ndarray:
+    """U, the upper Cholesky factor of the damped inverse Hessian:
+    Hd = H + damp * mean(diag H) * I,  Hd^-1 = U^T U  (library inverse and
+    Cholesky, binary64)."""
+    H = np.asarray(H, dtype=np.float64)
+    Hd = H + damp * np.mean(np.diag(H)) * np.eye(H.shape[0])
+    return np.linalg.cholesky(np.linalg.inv(Hd)).T
+
+
+def gptq(W: np.ndarray, s, U, bits: int, group: int, zero_point: bool = True, rows=None,
+         fixed_step: float = 0.0, stop_after: int = -1):
+    """The GPTQ sweep over the scaled rows RN32(W s) with the binary32 factor U
+    (see awq_oracle_gptq).  Returns dict(q, sh, z, what, w) like quantize(),
+    w being the final scaled binary32 weights (dequantized values for the
+    columns done)."""
+    W = _as_f16(W)
+    Ws = W if rows is None else np.ascontiguousarray(W[np.asarray(rows)])
+    N, K = Ws.shape
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
+    assert U32.shape == (K, K)
+    G = K // group
+    q = np.zeros((N, K), dtype=np.uint8)
+    sh = np.zeros((N, G), dtype=np.uint16)
+    z = np.zeros((N, G), dtype=np.float32)
+    what = np.zeros((N, K), dtype=np.uint16)
+    w = np.empty((N, K), dtype=np.float32)
+    _load().awq_oracle_gptq(_ptr(Ws.view(np.uint16)), N, K, _ptr(s), _ptr(U32), int(bits), int(group),
+                            int(bool(zero_point)), float(fixed_step), int(stop_after), _ptr(q), _ptr(sh),
+                            _ptr(z), _ptr(what), _ptr(w))
+    return dict(q=q, sh=sh.view(np.float16), z=z, what=what.view(np.float16), w=w)
+
+
+def output_error(W: np.ndarray, What: np.ndarray, X: np.ndarray, rows=None) -> dict:
+    """MSE of the layer output for a given W_hat (any quantizer's), binary64."""
+    W = _as_f16(W)
+    Ws = W if rows is None else np.ascontiguousarray(W[np.asarray(rows)])
+    rs = output_error_sum(Ws, What, _as_f16(X))
+    return dict(loss=rs.sum() / (Ws.shape[0] * X.shape[0]), row_sums=rs)

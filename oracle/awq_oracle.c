@@ -245,6 +245,87 @@ void awq_oracle_topk(const float *stat, int64_t K, int64_t k, uint8_t *mask)
 }
 
 /* ------------------------------------------------------------------ */
+/* AWQ followed by GPTQ error compensation ([AWQ-note] "Measures": the  */
+/* two are complementary, AWQ+GPTQ at INT2; [Notes-52] §4: round one    */
+/* column at a time and push its error into the weights not yet         */
+/* quantized, weighted by second-order statistics of the real input;    */
+/* [GPTQ-AWQ] "GPTQ": column-wise, with a Cholesky factor prepared      */
+/* once).  The sweep below takes U, the upper Cholesky factor of the    */
+/* damped inverse Hessian (H^-1 = U^T U), as given, and works on the    */
+/* scaled weights w = RN32(W s) of one row, in binary32:                 */
+/*   for k = 0 .. K-1:                                                  */
+/*     at the first column of a group: the group's parameters from the  */
+/*       group's current weights (the quantizer above, w' = w);         */
+/*     q_k  = clamp(rint(w_k r) + z, 0, qmax)     (exact product)       */
+/*     wq_k = RN32((q_k - z) sh)                                        */
+/*     e    = RN32(RN32(w_k - wq_k) / U_kk)                             */
+/*     w_j  = fmaf(-e, U_kj, w_j)   for j = k+1 .. K-1, in order         */
+/*   what_k = RN16(RN32(wq_k RN32(1 / s_k)))                            */
+/* fixed_step > 0 replaces the group parameters by a fixed grid of that */
+/* step (q = rint(w / step), no clamp; a test hook for the pages' toy   */
+/* example).  stop_after >= 0 stops after that many columns and leaves  */
+/* the current weights in w_out (a test hook for one update step).      */
+/* ------------------------------------------------------------------ */
+
+void awq_oracle_gptq(const uint16_t *W, int64_t N, int64_t K, const float *s, const float *U,
+                     int bits, int g, int zero_point, double fixed_step, int64_t stop_after,
+                     uint8_t *q_out, uint16_t *sh_out, float *z_out, uint16_t *what_out, float *w_out)
+{
+    const double qmax = (double)((1 << bits) - 1);
+    const double qsym = (double)((1 << (bits - 1)) - 1);
+    const int64_t G = K / g;
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < N; ++n) {
+        float *w = w_out + n * K;
+        for (int64_t k = 0; k < K; ++k) w[k] = rn32(awq_oracle_h2d(W[n * K + k]) * (double)s[k]);
+        double sh = 1.0, r = 1.0, z = 0.0;
+        const int64_t last = stop_after >= 0 && stop_after < K ? stop_after : K;
+        for (int64_t k = 0; k < last; ++k) {
+            if (fixed_step <= 0.0 && k % g == 0) {
+                float mn = INFINITY, mx = -INFINITY;
+                for (int64_t j = k; j < k + g; ++j) {
+                    if (w[j] < mn) mn = w[j];
+                    if (w[j] > mx) mx = w[j];
+                }
+                float scale;
+                if (zero_point) scale = rn32((double)rn32((double)mx - (double)mn) / qmax);
+                else scale = rn32((-(double)mn > (double)mx ? -(double)mn : (double)mx) / qsym);
+                double sc = scale;
+                if (sc < ldexp(1.0, -24)) sc = ldexp(1.0, -24);
+                if (sc > 65504.0) sc = 65504.0;
+                uint16_t shb = awq_oracle_rn16(sc);
+                sh = awq_oracle_h2d(shb);
+                r = rn32(1.0 / sh);
+                if (zero_point) {
+                    z = nearbyint(-(double)mn * r);
+                    if (!(z > 0.0)) z = 0.0;
+                    if (z > qmax) z = qmax;
+                } else {
+                    z = qsym + 1.0;
+                }
+                if (sh_out) sh_out[n * G + k / g] = shb;
+                if (z_out) z_out[n * G + k / g] = (float)z;
+            }
+            double q, wq;
+            if (fixed_step > 0.0) {
+                q = nearbyint((double)w[k] / fixed_step);
+                wq = rn32(q * fixed_step);
+            } else {
+                q = nearbyint((double)w[k] * r) + z;
+                if (q < 0.0) q = 0.0;
+                if (q > qmax) q = qmax;
+                wq = rn32((q - z) * sh);
+            }
+            const float e = rn32((double)rn32((double)w[k] - wq) / (double)U[k * K + k]);
+            for (int64_t j = k + 1; j < K; ++j) w[j] = fmaf(-e, U[k * K + j], w[j]);
+            if (q_out) q_out[n * K + k] = (uint8_t)(q < 0 ? 0 : q);
+            if (what_out) what_out[n * K + k] = awq_oracle_rn16(rn32(wq * (double)rn32(1.0 / (double)s[k])));
+            w[k] = (float)wq;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Step a8: pack codes, LSB first.  The container is 4 bits for w_bit  */
 /* 3 and 4 (8 codes per 32-bit word) and 2 bits for w_bit 2 (16 per    */
 /* word): code of column k sits at bits c*(k mod 32/c) of word         */

@@ -467,3 +467,126 @@ def test_baselines_premise(oracle_mod):
     assert fp16_act < 0.1 * rtn
     assert fp16_w > 0.9 * rtn
     assert awq < fixed2 < 0.5 * rtn
+
+
+# ---------------------------------------------------------------------------
+# AWQ followed by GPTQ error compensation
+# ---------------------------------------------------------------------------
+
+def test_notes52_gptq_toy(oracle_mod):
+    """"52 · AWQ, GPTQ và SmoothQuant" §4: rounding 0.34, 0.33, 0.33 to step
+    0.25 gives 0.75; rounding column by column and pushing each error into the
+    rest gives exactly 1.00 (input 1 on each weight)."""
+    g = _gold("notes52_gptq_toy.json")
+    W = np.array([g["W"]], dtype=np.float16)
+    X = np.array([g["inputs"]], dtype=np.float16)
+    one = np.ones(3, np.float32)
+    rtn = np.round(W.astype(np.float64) / g["step"]) * g["step"]
+    assert float((rtn * X).sum()) == g["rtn_output"]
+    U = oracle_mod.gptq_factor(oracle_mod.gptq_hessian(X, one))
+    r = oracle_mod.gptq(W, one, U, 4, 3, fixed_step=g["step"])
+    assert float((r["w"].astype(np.float64) * X).sum()) == g["error_feedback_output"]
+    assert np.all(np.isin(r["w"], [0.0, 0.25, 0.5]))           # every weight on the grid
+
+
+def test_gptq_with_uncorrelated_inputs_is_rtn(oracle_mod):
+    """With orthogonal input channels H is diagonal, so U is and no error moves:
+    the sweep reproduces the plain quantizer bit for bit."""
+    rng = np.random.default_rng(101)
+    W = (rng.standard_normal((6, 128)) * 0.05).astype(np.float16)
+    X = np.zeros((128, 128), np.float16)
+    X[np.arange(128), np.arange(128)] = rng.uniform(0.5, 4.0, 128).astype(np.float16)
+    s = rng.uniform(0.5, 2.0, 128).astype(np.float32)
+    U = oracle_mod.gptq_factor(oracle_mod.gptq_hessian(X, s))
+    assert np.count_nonzero(np.triu(U, 1)) == 0
+    for zp in (True, False):
+        r = oracle_mod.gptq(W, s, U, 4, 64, zero_point=zp)
+        ref = oracle_mod.quantize(W, s, 4, 64, zero_point=zp)
+        assert np.array_equal(r["q"], ref["q"])
+        assert np.array_equal(r["what"].view(np.uint16), ref["what"].view(np.uint16))
+
+
+def test_gptq_step_is_the_least_squares_correction(oracle_mod):
+    """After the first column is rounded, the change the sweep makes to the
+    remaining weights is the one that minimises the (damped) output error with
+    that column fixed: dw_rest = -Hd_rr^-1 Hd_r0 dw_0 (normal equations, solved
+    by the library)."""
+    rng = np.random.default_rng(102)
+    K = 16
+    W = (rng.standard_normal((3, K)) * 0.1).astype(np.float16)
+    X = (rng.standard_normal((40, K)) + rng.standard_normal((40, 1))).astype(np.float16)   # correlated
+    one = np.ones(K, np.float32)
+    H = oracle_mod.gptq_hessian(X, one)
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    U = oracle_mod.gptq_factor(H)
+    r = oracle_mod.gptq(W, one, U, 4, 16, stop_after=1)
+    w0 = W.astype(np.float64)
+    d0 = r["w"][:, 0].astype(np.float64) - w0[:, 0]
+    expect = w0[:, 1:] - np.outer(d0, np.linalg.solve(Hd[1:, 1:], Hd[1:, 0]))
+    np.testing.assert_allclose(r["w"][:, 1:], expect, rtol=1e-5, atol=1e-6)
+
+
+def _rn32_exact(x):
+    """Nearest binary32 (ties to even) of an exact rational, without double rounding."""
+    from fractions import Fraction
+    f = np.float32(float(x))
+    lo, hi = (f, np.nextafter(f, np.float32(np.inf))) if Fraction(float(f)) <= x else \
+             (np.nextafter(f, np.float32(-np.inf)), f)
+    dl, dh = x - Fraction(float(lo)), Fraction(float(hi)) - x
+    if dl < dh or (dl == dh and (lo.view(np.uint32) & 1) == 0):
+        return lo
+    return hi
+
+
+def test_gptq_sweep_against_scalar_restatement(oracle_mod):
+    """The C sweep against a scalar restatement with exact rational FMAs
+    (asymmetric groups, 2 groups of 8, 3 rows)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(103)
+    K, g, bits = 16, 8, 3
+    qmax = (1 << bits) - 1
+    W = (rng.standard_normal((3, K)) * 0.1).astype(np.float16)
+    X = (rng.standard_normal((30, K)) + 0.5 * rng.standard_normal((30, 1))).astype(np.float16)
+    s = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    U = oracle_mod.gptq_factor(oracle_mod.gptq_hessian(X, s)).astype(np.float32)
+    got = oracle_mod.gptq(W, s, U, bits, g)
+    from oracle import bruteforce as bf
+    for n in range(3):
+        w = [np.float32(np.float32(W[n, k]) * s[k]) for k in range(K)]
+        for k in range(K):
+            if k % g == 0:
+                mn, mx = min(w[k:k + g]), max(w[k:k + g])
+                scale = np.float32(np.float32(mx - mn) / np.float32(qmax))
+                sh = bf.to_f16(min(max(float(scale), 2.0 ** -24), 65504.0))
+                r = np.float32(np.float32(1.0) / np.float32(sh))
+                z = min(max(round(-float(mn) * float(r)), 0), qmax)
+            qk = min(max(round(float(w[k]) * float(r)) + z, 0), qmax)
+            wq = np.float32(np.float32(qk - z) * np.float32(sh))
+            e = np.float32(np.float32(w[k] - wq) / U[k, k])
+            for j in range(k + 1, K):
+                w[j] = _rn32_exact(Fraction(float(w[j])) - Fraction(float(e)) * Fraction(float(U[k, j])))
+            assert got["q"][n, k] == qk, (n, k)
+            w[k] = wq
+        assert np.array_equal(got["w"][n], np.array(w, np.float32))
+
+
+@pytest.mark.parametrize("bits,group", [(2, 64), (3, 128), (4, 128)])
+def test_awq_gptq_premise(oracle_mod, bits, group):
+    """[AWQ-note] "Measures": AWQ's scaling and GPTQ's error compensation are
+    complementary -- AWQ+GPTQ below either alone (a synthetic layer with 1%
+    outlier channels; at INT2 plain GPTQ can do worse than RTN there)."""
+    cfg = synth.make_config(256, 512, 512, bits=bits, group=group, seed=11)
+    W, X, _ = synth.generate(cfg)
+    a = oracle_mod.act_stats(X)
+    al = synth.default_alphas()
+    res = oracle_mod.search(W, X, a, bits, group, al)
+    s_best = oracle_mod.scales(a, float(al[res["best"]]))
+    one = np.ones(cfg.K, np.float32)
+    gptq = oracle_mod.gptq(W, one, oracle_mod.gptq_factor(oracle_mod.gptq_hessian(X, one)), bits, group)
+    both = oracle_mod.gptq(W, s_best, oracle_mod.gptq_factor(oracle_mod.gptq_hessian(X, s_best)), bits, group)
+    l_gptq = oracle_mod.output_error(W, gptq["what"], X)["loss"]
+    l_both = oracle_mod.output_error(W, both["what"], X)["loss"]
+    assert l_both < res["losses"].min()
+    assert l_both < l_gptq
+    if bits > 2:
+        assert l_gptq < res["losses"][0]
