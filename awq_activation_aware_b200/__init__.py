@@ -18,7 +18,8 @@ __all__ = [
     "AWQError", "lib", "act_stats", "alpha_scales", "quant_dequant", "search_workspace_bytes",
     "search_layer", "pack", "quantize_layer", "get_status", "set_wait_timeout_ms", "default_alphas",
     "profile_next_search", "quantize_shared_input", "selftest_bounded_wait", "qlinear",
-    "search_scales", "channel_topk", "pack_scales", "salient_scales", "baselines", "LIB_PATH",
+    "search_scales", "channel_topk", "pack_scales", "salient_scales", "baselines", "output_error",
+    "gptq_hessian", "gptq_factor", "gptq_quantize", "gptq_layer", "awq_gptq", "LIB_PATH",
 ]
 
 _PKG = Path(__file__).resolve().parent
@@ -60,6 +61,14 @@ def lib():
     L.awq_channel_topk.argtypes = [P, i64, i64, P, P]
     L.awq_pack_scales.argtypes = [P, i64, i64, P, QCfg, P, P, P, P]
     L.awq_salient_scales.argtypes = [P, i64, ctypes.c_float, P, P]
+    L.awq_output_error_workspace_bytes.argtypes = [i64, i64, i64]
+    L.awq_output_error_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_output_error.argtypes = [P, P, i64, i64, P, i64, i64, P, P, P, ctypes.c_size_t, P]
+    L.awq_gptq_hessian.argtypes = [P, i64, i64, i64, P, P, P]
+    L.awq_gptq_factor_workspace_bytes.argtypes = [i64]
+    L.awq_gptq_factor_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_gptq_factor.argtypes = [P, i64, ctypes.c_float, P, P, ctypes.c_size_t, P]
+    L.awq_gptq_quantize.argtypes = [P, i64, i64, P, P, QCfg, P, P, P, P, P]
     L.awq_search_workspace_bytes.argtypes = [i64, i64, i64, QCfg, i32]
     L.awq_search_workspace_bytes.restype = ctypes.c_size_t
     L.awq_search_layer.argtypes = [P, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P, ctypes.c_size_t, P]
@@ -79,7 +88,8 @@ def lib():
     L.awq_status_string.restype = ctypes.c_char_p
     for fn in ("awq_act_stats", "awq_alpha_scales", "awq_quant_dequant", "awq_search_layer", "awq_pack",
                "awq_get_status", "awq_quant_dequant_masked", "awq_search_scales", "awq_channel_topk",
-               "awq_pack_scales", "awq_salient_scales"):
+               "awq_pack_scales", "awq_salient_scales", "awq_output_error", "awq_gptq_hessian", "awq_gptq_factor",
+               "awq_gptq_quantize"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -351,6 +361,87 @@ def baselines(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group: int = 128,
     grid = search_layer(W, X, a, al, bits, group, stream=stream, zero_point=zero_point)
     return dict(rtn=fixed[0], fixed_2x=fixed[1], fp16_act=fp16_act[0], fp16_weight=fp16_w[0], awq_grid=grid,
                 mask_act=m_act, mask_weight=m_w, k=k)
+
+
+def output_error(W: torch.Tensor, W_hat: torch.Tensor, X: torch.Tensor, row_losses: bool = False, stream=None):
+    """||(W_hat - W) X^T||^2 / (N T) for any quantized weights W_hat (fp16 [N, K])."""
+    _rowmajor(X, "X")
+    N, K = W.shape
+    T = X.shape[0]
+    ws = torch.empty(int(lib().awq_output_error_workspace_bytes(N, K, T)), dtype=torch.uint8, device=W.device)
+    loss = torch.empty(1, dtype=torch.float32, device=W.device)
+    rl = torch.empty((1, N), dtype=torch.float32, device=W.device) if row_losses else None
+    _check(lib().awq_output_error(_dev(W.contiguous(), torch.float16, "W"), _dev(W_hat.contiguous(), torch.float16, "W_hat"),
+                                  N, K, _dev(X, torch.float16, "X"), T, X.stride(0), _dev(loss, torch.float32, "loss"),
+                                  _dev(rl, torch.float32, "row_losses") if rl is not None else None,
+                                  ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)), "awq_output_error")
+    return (loss[0], rl[0]) if row_losses else loss[0]
+
+
+def gptq_hessian(X: torch.Tensor, s: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = 2 X'^T X' (float32 [K, K]) of the input divided by s."""
+    _rowmajor(X, "X")
+    T, K = X.shape
+    s = torch.ones(K, dtype=torch.float32, device=X.device) if s is None else s
+    H = torch.empty((K, K), dtype=torch.float32, device=X.device)
+    _check(lib().awq_gptq_hessian(_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(s, torch.float32, "s"),
+                                  _dev(H, torch.float32, "H"), _stream(stream)), "awq_gptq_hessian")
+    return H
+
+
+def gptq_factor(H: torch.Tensor, damp: float = 0.01, stream=None) -> torch.Tensor:
+    """U, upper, with (H + damp mean(diag H) I)^-1 = U^T U (float32 [K, K])."""
+    K = H.shape[0]
+    H = H.contiguous()
+    U = torch.empty_like(H)
+    ws = torch.empty(int(lib().awq_gptq_factor_workspace_bytes(K)), dtype=torch.uint8, device=H.device)
+    _check(lib().awq_gptq_factor(_dev(H, torch.float32, "H"), K, float(damp), _dev(U, torch.float32, "U"),
+                                 ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)), "awq_gptq_factor")
+    return U
+
+
+def gptq_quantize(W: torch.Tensor, s: torch.Tensor, U: torch.Tensor, bits: int = 4, group: int = 128,
+                  zero_point: bool = True, stream=None) -> dict:
+    """The GPTQ column sweep over RN32(W s) with factor U: packed codes, fp16
+    scales and zeros (awq_pack's layout) and the fp16 W_hat."""
+    W = W.contiguous()
+    N, K = W.shape
+    dev = W.device
+    per = 16 if bits == 2 else 8
+    o = dict(codes=torch.empty((N, K // per), dtype=torch.int32, device=dev),
+             scales=torch.empty((N, K // group), dtype=torch.float16, device=dev),
+             zeros=torch.empty((N, K // group), dtype=torch.float16, device=dev),
+             W_hat=torch.empty_like(W), s_best=s)
+    _check(lib().awq_gptq_quantize(_dev(W, torch.float16, "W"), N, K, _dev(s, torch.float32, "s"),
+                                   _dev(U.contiguous(), torch.float32, "U"), _qcfg(bits, group, zero_point),
+                                   _dev(o["codes"], torch.int32, "codes"), _dev(o["scales"], torch.float16, "scales"),
+                                   _dev(o["zeros"], torch.float16, "zeros"), _dev(o["W_hat"], torch.float16, "W_hat"),
+                                   _stream(stream)), "awq_gptq_quantize")
+    return o
+
+
+def gptq_layer(W: torch.Tensor, X: torch.Tensor, s: torch.Tensor | None = None, bits: int = 4, group: int = 128,
+               zero_point: bool = True, damp: float = 0.01, stream=None) -> dict:
+    """GPTQ on the layer scaled by s (s = 1: GPTQ alone): Hessian, factor, sweep,
+    and the output error of the result."""
+    K = W.shape[1]
+    s = torch.ones(K, dtype=torch.float32, device=W.device) if s is None else s
+    U = gptq_factor(gptq_hessian(X, s, stream), damp, stream)
+    o = gptq_quantize(W, s, U, bits, group, zero_point, stream)
+    o["loss"] = output_error(W, o["W_hat"], X, stream=stream)
+    return o
+
+
+def awq_gptq(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group: int = 128, alphas: torch.Tensor | None = None,
+             zero_point: bool = True, damp: float = 0.01, stream=None) -> dict:
+    """AWQ's scale search, then GPTQ on the layer scaled by the chosen s.
+    Returns the GPTQ result (codes, scales, zeros, W_hat, loss, s_best) plus the
+    AWQ grid's losses and best index."""
+    res = quantize_layer(W, X, alphas, bits, group, stream=stream, zero_point=zero_point)
+    o = gptq_layer(W, X, res["s_best"], bits, group, zero_point, damp, stream)
+    o["awq_losses"] = res["losses"]
+    o["best_idx"] = res["best_idx"]
+    return o
 
 
 def get_status(stream=None) -> None:

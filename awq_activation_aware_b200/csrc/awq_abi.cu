@@ -30,6 +30,7 @@ bool valid_qcfg(const awq_qcfg &q) {
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 constexpr int kMaxAlpha = 64;
+constexpr int64_t kMaxGptqK = 8192;      // the GPTQ sweep keeps its rows and a ring of U rows on chip
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -107,6 +108,8 @@ awq_status device_info(DevInfo &out) {
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess)
             return AWQ_ERR_CUDA;
         d.search_attr = true;
@@ -250,13 +253,23 @@ awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_
 
 // a3-a6 on tables of n scale vectors already in the workspace: group
 // parameters, the tensor-core search against X, the loss reduction.
+awq_status run_search(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, int group,
+                      float qmax, const float *s_tab, const float *rs_tab, int n_alpha, const uint2 *params,
+                      float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st);
+
 awq_status search_core(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, awq_qcfg q,
                        const float *s_tab, const float *rs_tab, int n_alpha, const uint8_t *mask, uint2 *params,
                        float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st) {
-    const float qmax = (float)((1 << q.bits) - 1);
     // a3 (group parameters for every alpha)
     if (awq_status e = launch_group_params(W, N, K, q, s_tab, n_alpha, mask, params, st)) return e;
+    return run_search(W, N, K, X, T, ldx, q.group_size, (float)((1 << q.bits) - 1), s_tab, rs_tab, n_alpha, params,
+                      partial, losses, row_losses, d, st);
+}
 
+// a4-a6 with the group parameters already in the workspace.
+awq_status run_search(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, int group,
+                      float qmax, const float *s_tab, const float *rs_tab, int n_alpha, const uint2 *params,
+                      float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st) {
     // a4-a6: the tensor-core search on CTA pairs
     CUtensorMap tmap_x, tmap_w;
     if (!encode_rows_map(&tmap_x, X, T, K, ldx, awq::srch2::HN) ||
@@ -272,8 +285,8 @@ awq_status search_core(const void *W, int64_t N, int64_t K, const void *X, int64
     A.T = T;
     A.N_pad = padded_rows(N);
     A.n_alpha = n_alpha;
-    A.G = (int)(K / q.group_size);
-    A.group = q.group_size;
+    A.G = (int)(K / group);
+    A.group = group;
     A.n_tb = (int)((T + awq::srch2::BT - 1) / awq::srch2::BT);
     A.n_kb = (int)(K / awq::srch2::BK);
     A.n_units = (A.N_pad / awq::srch2::PM) * A.n_tb * n_alpha;
@@ -472,6 +485,131 @@ awq_status awq_salient_scales(const uint8_t *mask, int64_t K, float factor, floa
     return last_launch();
 }
 
+size_t awq_output_error_workspace_bytes(int64_t N, int64_t K, int64_t T) {
+    if (N < 1 || K < 64 || T < 1 || K % 64) return 0;
+    return search_ws_layout(N, K, T, 64, 1).total + round_up(2 * (size_t)N * K, 256);
+}
+
+awq_status awq_output_error(const void *W, const void *W_hat, int64_t N, int64_t K, const void *X, int64_t T,
+                            int64_t ldx, float *loss, float *row_losses, void *ws, size_t ws_bytes, void *stream) {
+    if (!W || !W_hat || !X || !loss) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(W_hat) || !aligned16(X) || !aligned16(loss) ||
+        (row_losses && !aligned16(row_losses)))
+        return AWQ_ERR_INVALID_ARG;
+    if (N < 1 || N > kMaxDim || T < 1 || T > kMaxDim || K < 64 || K > kMaxDim || K % 64 || ldx < K || ldx % 8)
+        return AWQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < awq_output_error_workspace_bytes(N, K, T) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    const SearchWs L = search_ws_layout(N, K, T, 64, 1);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *s_tab = reinterpret_cast<float *>(base + L.s_off);
+    float *rs_tab = reinterpret_cast<float *>(base + L.rs_off);
+    uint2 *params = reinterpret_cast<uint2 *>(base + L.prm_off);
+    float *partial = reinterpret_cast<float *>(base + L.part_off);
+    __half *dW = reinterpret_cast<__half *>(base + L.total);
+    int grid = blocks_for(N * K, 256);
+    if (grid > 8 * d.sms) grid = 8 * d.sms;
+    awq::weight_diff_kernel<<<grid, 256, 0, st>>>((const __half *)W, (const __half *)W_hat, N * K, dW);
+    if (awq_status e = last_launch()) return e;
+    const int64_t n_prm = (K / 64) * padded_rows(N);
+    awq::zero_code_params_kernel<<<blocks_for(n_prm, 256) < 4 * d.sms ? blocks_for(n_prm, 256) : 4 * d.sms, 256, 0,
+                                   st>>>(params, n_prm);
+    if (awq_status e = last_launch()) return e;
+    awq::fill_kernel<<<blocks_for(K, 256), 256, 0, st>>>(s_tab, K, 1.0f);
+    awq::fill_kernel<<<blocks_for(K, 256), 256, 0, st>>>(rs_tab, K, 1.0f);
+    if (awq_status e = last_launch()) return e;
+    return run_search(dW, N, K, X, T, ldx, 64, 0.0f, s_tab, rs_tab, 1, params, partial, loss, row_losses, d, st);
+}
+
+awq_status awq_gptq_hessian(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s, float *H, void *stream) {
+    if (!X || !s || !H || !aligned16(X) || !aligned16(s) || !aligned16(H)) return AWQ_ERR_INVALID_ARG;
+    if (T < 1 || T > kMaxDim || K < 64 || K > kMaxGptqK || K % 64 || ldx < K || ldx % 8) return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    const int nb = (int)(K / awq::kGb);
+    awq::gptq_hessian_kernel<<<nb * (nb + 1) / 2, 256, 0, (cudaStream_t)stream>>>((const __half *)X, T, K, ldx, s, H);
+    return last_launch();
+}
+
+size_t awq_gptq_factor_workspace_bytes(int64_t K) {
+    if (K < 64 || K % 64 || K > kMaxGptqK) return 0;
+    return round_up(4 * (size_t)K * K, 256) + 256;
+}
+
+awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void *ws, size_t ws_bytes, void *stream) {
+    if (!H || !U || !aligned16(H) || !aligned16(U)) return AWQ_ERR_INVALID_ARG;
+    if (K < 64 || K % 64 || K > kMaxGptqK || !(damp >= 0.0f && damp <= 1e6f)) return AWQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < awq_gptq_factor_workspace_bytes(K) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    float *A = static_cast<float *>(ws);
+    float *add = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + round_up(4 * (size_t)K * K, 256));
+    awq::gptq_damp_kernel<<<1, 256, 0, st>>>(H, K, damp, add);
+    int grid = blocks_for(K * K, 256);
+    if (grid > 8 * d.sms) grid = 8 * d.sms;
+    awq::gptq_reverse_kernel<<<grid, 256, 0, st>>>(H, K, add, A);
+    if (awq_status e = last_launch()) return e;
+    const int nb = (int)(K / awq::kGb);
+    for (int p = 0; p < nb; ++p) {          // blocked Cholesky of the reversed, damped Hessian
+        awq::chol_diag_kernel<<<1, 256, 0, st>>>(A, K, p);
+        const int m = nb - p - 1;
+        if (m > 0) {
+            awq::chol_panel_kernel<<<m, awq::kGb, 0, st>>>(A, K, p);
+            awq::chol_update_kernel<<<m * (m + 1) / 2, 256, 0, st>>>(A, K, p);
+        }
+        if (awq_status e = last_launch()) return e;
+    }
+    awq::trinv_diag_kernel<<<nb, awq::kGb, 0, st>>>(A, K, U);           // M = L^-1 into U's storage
+    for (int dd = 1; dd < nb; ++dd) awq::trinv_offdiag_kernel<<<nb - dd, 256, 0, st>>>(A, K, dd, U);
+    if (awq_status e = last_launch()) return e;
+    grid = blocks_for((K * K + 1) / 2, 256);
+    if (grid > 8 * d.sms) grid = 8 * d.sms;
+    awq::gptq_rotate_kernel<<<grid, 256, 0, st>>>(U, K);                 // U = P M P, upper part
+    return last_launch();
+}
+
+awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const float *s, const float *U, awq_qcfg q,
+                             uint32_t *codes, void *scales, void *zeros, void *W_hat, void *stream) {
+    if (!W || !s || !U || !codes || !scales || !zeros || !W_hat) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(s) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) ||
+        !aligned16(zeros) || !aligned16(W_hat))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || K < 64 || K % 64 || K > kMaxGptqK || K % q.group_size)
+        return AWQ_ERR_INVALID_ARG;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    awq::gsw::Args A;
+    A.W = (const __half *)W;
+    A.N = N;
+    A.K = K;
+    A.s = s;
+    A.U = U;
+    A.group = q.group_size;
+    A.G = (int)(K / q.group_size);
+    A.bits = q.bits;
+    A.sym = q.zero_point ? 0 : 1;
+    A.qmax = (float)((1 << q.bits) - 1);
+    A.codes = codes;
+    A.scales = (__half *)scales;
+    A.zeros = (__half *)zeros;
+    A.W_hat = (__half *)W_hat;
+    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+    // as many rows per block as shared memory holds, next to a ring of U rows
+    A.ring = K <= 4096 ? 3 : 2;
+    A.rows = awq::gsw::MAX_ROWS;
+    while (A.rows > 1 && awq::gsw::smem_bytes(K, A.rows, A.ring) > (size_t)awq::qlv::SMEM_LIMIT) --A.rows;
+    const size_t smem = awq::gsw::smem_bytes(K, A.rows, A.ring);
+    if (smem > (size_t)awq::qlv::SMEM_LIMIT) return AWQ_ERR_UNSUPPORTED;
+    const unsigned grid = (unsigned)((N + A.rows - 1) / A.rows);
+    awq::gptq_sweep_kernel<<<grid, (awq::gsw::MAX_ROWS + 1) * 32, smem, (cudaStream_t)stream>>>(A);
+    return last_launch();
+}
+
 awq_status awq_channel_topk(const float *stat, int64_t K, int64_t k, uint8_t *mask, void *stream) {
     if (!stat || !mask || K < 1 || K > kMaxDim || k < 0 || k > K) return AWQ_ERR_INVALID_ARG;
     DevInfo d;
@@ -606,7 +744,7 @@ awq_status awq_get_status(void *stream) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(awq::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return AWQ_ERR_CUDA;
         if (flags & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
-        if (flags & (awq::kDevErrBadAlpha | awq::kDevErrBadScale)) return AWQ_ERR_INVALID_ARG;
+        if (flags & (awq::kDevErrBadAlpha | awq::kDevErrBadScale | awq::kDevErrNotPD)) return AWQ_ERR_INVALID_ARG;
     }
     return last_launch();
 }

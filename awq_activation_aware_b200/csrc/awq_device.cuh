@@ -20,7 +20,7 @@ namespace awq {
 // Device error word (read and cleared by awq_get_status on the host).  The
 // library is a single translation unit, so the definition lives here.
 // ---------------------------------------------------------------------------
-enum : unsigned { kDevErrTimeout = 1u, kDevErrBadAlpha = 2u, kDevErrBadScale = 4u };
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBadAlpha = 2u, kDevErrBadScale = 4u, kDevErrNotPD = 8u };
 __device__ unsigned g_dev_error = 0;
 
 // ---------------------------------------------------------------------------

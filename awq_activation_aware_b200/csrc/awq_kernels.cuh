@@ -1244,6 +1244,452 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
 }
 
 // ===========================================================================
+// AWQ followed by GPTQ error compensation ([AWQ-note] "Measures": AWQ+GPTQ;
+// [Notes-52] §4: round a column, push its error into the columns not yet
+// quantized, weighted by second-order statistics of the real input;
+// [GPTQ-AWQ] "GPTQ": a column sweep with a Cholesky factor prepared once).
+//   H  = 2 X'^T X',  x' = RN32(x RN32(1/s))                 (gptq_hessian_kernel)
+//   Hd = H + damp mean(diag H) I;  U upper with Hd^-1 = U^T U (gptq_* factor kernels)
+//   per row, in binary32: the column sweep                   (gptq_sweep_kernel)
+// All in binary32.  The factor: with P the order-reversing permutation,
+// A = P Hd P = L L^T (lower Cholesky), so Hd = R R^T with R = P L P upper and
+// Hd^-1 = (R^-1)^T R^-1: U = R^-1 = P L^-1 P, the 180-degree rotation of L^-1.
+// ===========================================================================
+constexpr int kGb = 64;                  // block size of the factor kernels and the Hessian tile
+
+// Index (bi, bj), bi >= bj, of the t-th block of a lower block triangle, rows first.
+__device__ __forceinline__ void lower_block(int t, int &bi, int &bj) {
+    int i = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+    while ((i + 1) * (i + 2) / 2 <= t) ++i;
+    while (i * (i + 1) / 2 > t) --i;
+    bi = i;
+    bj = t - i * (i + 1) / 2;
+}
+
+// H tile (bi, bj), bi >= bj, of 64 x 64: each thread a 4 x 4 patch, the
+// tokens in order (binary32 FMA), 16 tokens per shared-memory stage; the
+// tile and its mirror are written.
+__global__ void __launch_bounds__(256)
+gptq_hessian_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx, const float *__restrict__ s,
+                    float *__restrict__ H) {
+    __shared__ __align__(16) float xi[16][kGb + 4];
+    __shared__ __align__(16) float xj[16][kGb + 4];
+    int bi, bj;
+    lower_block(blockIdx.x, bi, bj);
+    const int64_t i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    const int lr = threadIdx.x / 16, lc = (threadIdx.x % 16) * 4;   // loader: token row, 4 columns
+    float rsi[4], rsj[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        rsi[e] = __frcp_rn(s[i0 + lc + e]);
+        rsj[e] = __frcp_rn(s[j0 + lc + e]);
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+    for (int64_t t0 = 0; t0 < T; t0 += 16) {
+        const int64_t t = t0 + lr;
+        float vi[4] = {0.0f, 0.0f, 0.0f, 0.0f}, vj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (t < T) {
+            const uint2 hi = *reinterpret_cast<const uint2 *>(X + t * ldx + i0 + lc);
+            const uint2 hj = *reinterpret_cast<const uint2 *>(X + t * ldx + j0 + lc);
+            const __half *pi = reinterpret_cast<const __half *>(&hi);
+            const __half *pj = reinterpret_cast<const __half *>(&hj);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                vi[e] = __fmul_rn(__half2float(pi[e]), rsi[e]);
+                vj[e] = __fmul_rn(__half2float(pj[e]), rsj[e]);
+            }
+        }
+        __syncthreads();
+        *reinterpret_cast<float4 *>(&xi[lr][lc]) = make_float4(vi[0], vi[1], vi[2], vi[3]);
+        *reinterpret_cast<float4 *>(&xj[lr][lc]) = make_float4(vj[0], vj[1], vj[2], vj[3]);
+        __syncthreads();
+#pragma unroll
+        for (int tt = 0; tt < 16; ++tt) {
+            const float4 a = *reinterpret_cast<const float4 *>(&xi[tt][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4 *>(&xj[tt][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[p][q] = __fmaf_rn(av[p], bv[q], acc[p][q]);
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t i = i0 + ty * 4 + p, j = j0 + tx * 4 + q;
+            const float v = __fmul_rn(2.0f, acc[p][q]);
+            H[i * K + j] = v;
+            if (bi != bj) H[j * K + i] = v;
+        }
+}
+
+// damp * mean(diag H), the damping term: one block, the diagonal summed in
+// index order in binary64 (the result does not depend on the launch).
+__global__ void __launch_bounds__(256)
+gptq_damp_kernel(const float *__restrict__ H, int64_t K, float damp, float *__restrict__ add) {
+    __shared__ double part[256];
+    double sum = 0.0;
+    for (int64_t i = threadIdx.x; i < K; i += 256) sum += (double)H[i * K + i];
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double tot = 0.0;
+        for (int i = 0; i < 256; ++i) tot += part[i];
+        *add = __fmul_rn(damp, (float)(tot / (double)K));
+    }
+}
+
+// A = P (H + add I) P: the damped Hessian with the order of rows and columns
+// reversed.
+__global__ void gptq_reverse_kernel(const float *__restrict__ H, int64_t K, const float *__restrict__ add,
+                                    float *__restrict__ A) {
+    const float ad = *add;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < K * K; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / K, j = e - i * K;
+        const float v = H[(K - 1 - i) * K + (K - 1 - j)];
+        A[e] = i == j ? __fadd_rn(v, ad) : v;
+    }
+}
+
+// Cholesky, step p of the blocked right-looking form on A (lower, row-major):
+// the diagonal block in shared memory, column by column.  A pivot that is not
+// positive raises the not-positive-definite flag (and is replaced by 1 so the
+// rest stays finite).
+__global__ void __launch_bounds__(256) chol_diag_kernel(float *__restrict__ A, int64_t K, int p) {
+    __shared__ float L[kGb][kGb + 1];
+    const int64_t o = (int64_t)p * kGb;
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) L[e / kGb][e % kGb] = A[(o + e / kGb) * K + o + e % kGb];
+    __syncthreads();
+    for (int c = 0; c < kGb; ++c) {
+        if (threadIdx.x == 0) {
+            float d = L[c][c];
+            if (!(d > 0.0f)) { atomicOr(&g_dev_error, kDevErrNotPD); d = 1.0f; }
+            L[c][c] = __fsqrt_rn(d);
+        }
+        __syncthreads();
+        for (int r = c + 1 + threadIdx.x; r < kGb; r += 256) L[r][c] = __fdiv_rn(L[r][c], L[c][c]);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+            const int r = e / kGb, q = e % kGb;
+            if (r > c && q > c && q <= r) L[r][q] = __fmaf_rn(-L[r][c], L[q][c], L[r][q]);
+        }
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+        const int r = e / kGb, q = e % kGb;
+        if (q <= r) A[(o + r) * K + o + q] = L[r][q];
+    }
+}
+
+// Cholesky step p: the panel below the diagonal block, A[i][p] <- A[i][p] L_pp^-T,
+// one block row per CTA, one row per thread (forward substitution).
+__global__ void __launch_bounds__(kGb) chol_panel_kernel(float *__restrict__ A, int64_t K, int p) {
+    __shared__ float L[kGb][kGb + 1];
+    const int64_t o = (int64_t)p * kGb;
+    const int64_t r0 = o + kGb + (int64_t)blockIdx.x * kGb;
+    for (int e = threadIdx.x; e < kGb * kGb; e += kGb) L[e / kGb][e % kGb] = A[(o + e / kGb) * K + o + e % kGb];
+    __syncthreads();
+    float x[kGb];
+    const int64_t row = r0 + threadIdx.x;
+#pragma unroll
+    for (int c = 0; c < kGb; ++c) x[c] = A[row * K + o + c];
+#pragma unroll
+    for (int c = 0; c < kGb; ++c) {
+        float v = x[c];
+#pragma unroll
+        for (int m = 0; m < c; ++m) v = __fmaf_rn(-x[m], L[c][m], v);
+        x[c] = __fdiv_rn(v, L[c][c]);
+    }
+#pragma unroll
+    for (int c = 0; c < kGb; ++c) A[row * K + o + c] = x[c];
+}
+
+// 64 x 64 x 64 block product on shared-memory tiles: acc[a][b] += sum_m P[r][m] Q[c][m]
+// for this thread's 4 x 4 patch (rows ty*4+a of P, rows tx*4+b of Q), m in order.
+__device__ __forceinline__ void block_mm_nt(const float (*P)[kGb + 4], const float (*Q)[kGb + 4], int ty, int tx,
+                                            float (&acc)[4][4]) {
+#pragma unroll 8
+    for (int m = 0; m < kGb; ++m) {
+        float pv[4], qv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) { pv[a] = P[ty * 4 + a][m]; qv[a] = Q[tx * 4 + a][m]; }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a], qv[b], acc[a][b]);
+    }
+}
+
+// Cholesky step p: trailing update A[i][j] -= L[i][p] L[j][p]^T for the lower
+// blocks p < j <= i, one block per CTA.
+__global__ void __launch_bounds__(256) chol_update_kernel(float *__restrict__ A, int64_t K, int p) {
+    __shared__ float Pi[kGb][kGb + 4], Pj[kGb][kGb + 4];
+    int bi, bj;
+    lower_block(blockIdx.x, bi, bj);
+    bi += p + 1;
+    bj += p + 1;
+    const int64_t o = (int64_t)p * kGb, i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb;
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+        Pi[e / kGb][e % kGb] = A[(i0 + e / kGb) * K + o + e % kGb];
+        Pj[e / kGb][e % kGb] = A[(j0 + e / kGb) * K + o + e % kGb];
+    }
+    __syncthreads();
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+    block_mm_nt(Pi, Pj, ty, tx, acc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float *d = &A[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b];
+            *d = __fsub_rn(*d, acc[a][b]);
+        }
+}
+
+// Inverse of the lower factor, M = L^-1, diagonal blocks: thread c solves
+// L_pp x = e_c by forward substitution.
+__global__ void __launch_bounds__(kGb) trinv_diag_kernel(const float *__restrict__ L, int64_t K,
+                                                         float *__restrict__ M) {
+    __shared__ float Lp[kGb][kGb + 1];
+    const int64_t o = (int64_t)blockIdx.x * kGb;
+    for (int e = threadIdx.x; e < kGb * kGb; e += kGb) Lp[e / kGb][e % kGb] = L[(o + e / kGb) * K + o + e % kGb];
+    __syncthreads();
+    const int c = threadIdx.x;
+    float x[kGb];
+#pragma unroll
+    for (int r = 0; r < kGb; ++r) {
+        float v = r == c ? 1.0f : 0.0f;
+#pragma unroll
+        for (int m = 0; m < r; ++m) v = __fmaf_rn(-Lp[r][m], x[m], v);
+        x[r] = r < c ? 0.0f : __fdiv_rn(v, Lp[r][r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kGb; ++r) M[(o + r) * K + o + c] = x[r];
+}
+
+// Off-diagonal blocks at block distance d (i = j + d):
+//   M[i][j] = -M[i][i] (sum_{k=j}^{i-1} L[i][k] M[k][j]),  k in order.
+__global__ void __launch_bounds__(256) trinv_offdiag_kernel(const float *__restrict__ L, int64_t K, int d,
+                                                            float *__restrict__ M) {
+    __shared__ float Pa[kGb][kGb + 4], Qb[kGb][kGb + 4];
+    const int bj = blockIdx.x, bi = bj + d;
+    const int64_t i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+    for (int bk = bj; bk < bi; ++bk) {
+        const int64_t k0 = (int64_t)bk * kGb;
+        __syncthreads();
+        for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+            Pa[e / kGb][e % kGb] = L[(i0 + e / kGb) * K + k0 + e % kGb];      // L[i][k] rows, k columns
+            Qb[e % kGb][e / kGb] = M[(k0 + e / kGb) * K + j0 + e % kGb];      // M[k][j] transposed: [j][k]
+        }
+        __syncthreads();
+        block_mm_nt(Pa, Qb, ty, tx, acc);
+    }
+    // S = acc (64 x 64); M[i][j] = -M_ii S
+    __syncthreads();
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) Pa[e / kGb][e % kGb] = M[(i0 + e / kGb) * K + i0 + e % kGb];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) Qb[tx * 4 + b][ty * 4 + a] = acc[a][b];      // S transposed: [col][row]
+    __syncthreads();
+    float out[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) out[a][b] = 0.0f;
+    block_mm_nt(Pa, Qb, ty, tx, out);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b] = -out[a][b];
+}
+
+// U = P M P restricted to the upper triangle, in place: element (a, b) and
+// (K-1-a, K-1-b) trade places; everything below the diagonal becomes 0.
+__global__ void gptq_rotate_kernel(float *__restrict__ M, int64_t K) {
+    const int64_t half = (K * K + 1) / 2;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < half; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t a = e / K, b = e - a * K, e2 = K * K - 1 - e;
+        const float v1 = M[e], v2 = M[e2];
+        // after the swap M[e] holds the old M[e2]; (a, b) is upper iff b >= a
+        M[e] = b >= a ? v2 : 0.0f;
+        const int64_t a2 = e2 / K, b2 = e2 - a2 * K;
+        if (e2 != e) M[e2] = b2 >= a2 ? v1 : 0.0f;
+    }
+}
+
+// Output error of a given W_hat through the search kernel: dW = RN16(W_hat - W)
+// is written as the "weights", and every group's parameters are those of a
+// quantizer whose clamp range is the single code z = 0 (qmax = 0, clamp flag
+// set), so the kernel's W_hat is 0 and it contracts -dW against X.
+__global__ void weight_diff_kernel(const __half *__restrict__ W, const __half *__restrict__ W_hat, int64_t total,
+                                   __half *__restrict__ dW) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        dW[i] = __float2half_rn(__fsub_rn(__half2float(W_hat[i]), __half2float(W[i])));
+}
+__global__ void zero_code_params_kernel(uint2 *__restrict__ params, int64_t total) {
+    QParams p;
+    p.r = 1.0f;
+    p.sh = 1.0f;
+    p.z = 0.0f;
+    p.clamp = true;
+    const uint2 v = pack_qparams(p);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        params[i] = v;
+}
+__global__ void fill_kernel(float *__restrict__ x, int64_t total, float v) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        x[i] = v;
+}
+
+// The GPTQ column sweep, one warp per row of W, binary32, bit for bit the
+// sequence of the definition:
+//   w = RN32(W s); for k = 0 .. K-1:
+//     at a group's first column: the group's parameters from its current w
+//     q  = clamp(rint(w_k r) + z, 0, qmax)         (one FMA with 1.5 2^23)
+//     wq = RN32((q - z) sh);  e = RN32(RN32(w_k - wq) / U_kk)
+//     w_j = fmaf(-e, U_kj, w_j), j > k             (packed pairs, FFMA2)
+// The row lives in shared memory; the last warp streams U's rows (from the
+// 16-byte boundary at or below the diagonal) into a ring that every row warp
+// of the block reads.  At the end each warp packs its codes and writes the
+// fp16 W_hat = RN16(RN32(wq RN32(1/s))); scales and zeros are written as each
+// group starts.
+namespace gsw {
+constexpr int MAX_ROWS = 8;
+struct Args {
+    const __half *W;
+    int64_t N, K;
+    const float *s, *U;
+    int group, G, bits, sym, rows, ring;     // rows per block, ring depth
+    float qmax;
+    uint32_t *codes;
+    __half *scales, *zeros, *W_hat;
+    uint64_t timeout_ns;
+};
+inline size_t smem_bytes(int64_t K, int rows, int ring) {
+    return (size_t)ring * K * 4 + (size_t)rows * K * 5 + 2 * 8 * 8 + 256;
+}
+}  // namespace gsw
+
+__global__ void __launch_bounds__((gsw::MAX_ROWS + 1) * 32, 1) gptq_sweep_kernel(const gsw::Args A) {
+    extern __shared__ uint8_t smem_raw[];
+    const int64_t K = A.K;
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float *ring = reinterpret_cast<float *>(base);                        // [ring][K]
+    float *wrow = ring + (size_t)A.ring * K;                              // [rows][K]
+    uint8_t *qrow = reinterpret_cast<uint8_t *>(wrow + (size_t)A.rows * K);   // [rows][K]
+    uint64_t *full = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(qrow + (size_t)A.rows * K) + 7) & ~uintptr_t(7));
+    uint64_t *empty = full + 8;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row0 = (int64_t)blockIdx.x * A.rows;
+    const int active = (int)(A.N - row0 < A.rows ? A.N - row0 : A.rows);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < A.ring; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], active); }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == gsw::MAX_ROWS) {                 // producer: U rows into the ring
+        if (lane == 0) {
+            int st = 0;
+            uint32_t ph = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                if (!mbar_wait_bounded(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
+                const int64_t c0 = k & ~int64_t(3);
+                const uint32_t bytes = (uint32_t)((K - c0) * 4);
+                mbar_arrive_expect_tx(&full[st], bytes);
+                bulk_load(ring + (size_t)st * K + c0, A.U + k * K + c0, bytes, &full[st]);
+                if (++st == A.ring) { st = 0; ph ^= 1u; }
+            }
+        }
+    } else if (warp < active) {
+        const int64_t n = row0 + warp;
+        float *w = wrow + (size_t)warp * K;
+        uint8_t *qv = qrow + (size_t)warp * K;
+        for (int64_t k = 2 * lane; k < K; k += 64) {
+            const __half2 h = *reinterpret_cast<const __half2 *>(A.W + n * K + k);
+            const float2 f = __half22float2(h);
+            *reinterpret_cast<float2 *>(w + k) = make_float2(__fmul_rn(f.x, A.s[k]), __fmul_rn(f.y, A.s[k + 1]));
+        }
+        __syncwarp();
+        QParams prm{};
+        int st = 0;
+        uint32_t ph = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            if (k % A.group == 0) {
+                float mn = INFINITY, mx = -INFINITY;
+                for (int64_t j = k + lane; j < k + A.group; j += 32) { mn = fminf(mn, w[j]); mx = fmaxf(mx, w[j]); }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                }
+                prm = make_qparams(mn, mx, A.qmax, A.sym != 0);
+                if (lane == 0) {
+                    A.scales[n * A.G + k / A.group] = __float2half_rn(prm.sh);
+                    A.zeros[n * A.G + k / A.group] = __float2half_rn(prm.z);
+                }
+            }
+            if (!mbar_wait_warp(&full[st], ph, &abort_flag, A.timeout_ns)) break;
+            const float *Ur = ring + (size_t)st * K;
+            const float wk = w[k];
+            const float vlo = __fsub_rn(kMagic, prm.z), vhi = __fadd_rn(kMagic, __fsub_rn(A.qmax, prm.z));
+            const float v = fminf(fmaxf(__fmaf_rn(wk, prm.r, kMagic), vlo), vhi);
+            const float qf = __fsub_rn(v, vlo);                              // the code, exact
+            const float wq = __fmul_rn(__fsub_rn(qf, prm.z), prm.sh);
+            const float e = __fdiv_rn(__fsub_rn(wk, wq), Ur[k]);
+            const float2 ne = make_float2(-e, -e);
+            const int64_t p0 = (k + 1) >> 1;                                 // first pair touching j > k
+            for (int64_t p = p0 + lane; p < K / 2; p += 32) {
+                float2 wv = *reinterpret_cast<const float2 *>(w + 2 * p);
+                const float2 uv = *reinterpret_cast<const float2 *>(Ur + 2 * p);
+                float2 r2 = fma2_rn(ne, uv, wv);
+                if (2 * p == k) r2.x = wq;                                   // column k itself: its value is final
+                *reinterpret_cast<float2 *>(w + 2 * p) = r2;
+            }
+            if ((k & 1) && lane == 0) w[k] = wq;
+            if (lane == 0) qv[k] = (uint8_t)qf;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+            if (++st == A.ring) { st = 0; ph ^= 1u; }
+        }
+        __syncwarp();
+        // codes (least-significant first) and W_hat
+        const int c = A.bits == 2 ? 2 : 4, per = 32 / c;
+        for (int64_t wd = lane; wd < K / per; wd += 32) {
+            uint32_t v = 0;
+            for (int i = 0; i < per; ++i) v |= (uint32_t)qv[wd * per + i] << (c * i);
+            A.codes[n * (K / per) + wd] = v;
+        }
+        for (int64_t k = lane; k < K; k += 32)
+            A.W_hat[n * K + k] = __float2half_rn(__fmul_rn(w[k], __frcp_rn(A.s[k])));
+    }
+    if (abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+}
+
+// ===========================================================================
 // Self-test of the bounded wait: one thread waits on an mbarrier that nothing
 // ever arrives on.  The wait gives up after the library's limit, raises the
 // device timeout flag and returns -- the path every role of the search kernel

@@ -54,11 +54,14 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
-    p.add_argument("--op", choices=["search", "qlinear", "baselines"], default="search",
+    p.add_argument("--op", choices=["search", "qlinear", "baselines", "gptq"], default="search",
                    help="search: the AWQ scale-search path (the benchmark); qlinear: the quantized "
                         "linear layer on the packed output vs the fp16 GEMM; baselines: the pages' "
-                        "comparisons (RTN, fixed 2x, fp16 1%%, symmetric) on one layer")
+                        "comparisons (RTN, fixed 2x, fp16 1%%, symmetric) on one layer; gptq: AWQ "
+                        "followed by GPTQ error compensation, each stage timed")
     p.add_argument("--tokens", default="1,4,16", help="token counts for --op qlinear")
+    p.add_argument("--bits", type=int, default=0, help="w_bit for --op gptq (default: the config's)")
+    p.add_argument("--group", type=int, default=0, help="group size for --op gptq (default: the config's)")
     return p.parse_args()
 
 
@@ -576,6 +579,62 @@ def run_baselines(args):
     return 0
 
 
+def run_gptq(args):
+    """AWQ followed by GPTQ on one layer: each GPU stage timed on the device
+    (CUDA events, after warm-up, L2 flushed before each), and the output error
+    of RTN, AWQ, GPTQ alone and AWQ+GPTQ.  One JSON line."""
+    import torch
+
+    import awq_activation_aware_b200 as awq
+    from awq_activation_aware_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    cfg = synth.CONFIGS[args.config]
+    bits = args.bits or cfg.bits
+    group = args.group or cfg.group
+    W, X, _ = synth.generate(cfg)
+    Wd = torch.from_numpy(W).to(dev)
+    Xd = torch.from_numpy(X).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 3)
+
+    def timed(fn):
+        for _ in range(2):
+            flush.zero_()
+            out = fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b.record()
+            out = fn()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(b.elapsed_time(e))
+        return out, statistics.median(ts)
+
+    res, t_awq = timed(lambda: awq.quantize_layer(Wd, Xd, bits=bits, group=group))
+    s = res["s_best"]
+    H, t_h = timed(lambda: awq.gptq_hessian(Xd, s))
+    U, t_f = timed(lambda: awq.gptq_factor(H))
+    q, t_q = timed(lambda: awq.gptq_quantize(Wd, s, U, bits, group))
+    loss_both, t_l = timed(lambda: awq.output_error(Wd, q["W_hat"], Xd))
+    ones = torch.ones(cfg.K, dtype=torch.float32, device=dev)
+    plain = awq.gptq_layer(Wd, Xd, ones, bits, group)
+    awq.get_status()
+    N, K, T = cfg.N, cfg.K, cfg.T
+    print(json.dumps({
+        "op": "gptq", "config": cfg.name, "bits": bits, "group": group,
+        "losses": {"rtn": float(res["losses"][0]), "awq": float(res["losses"].min()), "gptq": float(plain["loss"]),
+                   "awq_gptq": float(loss_both)},
+        "ms": {"awq_search_and_pack": t_awq, "hessian": t_h, "factor": t_f, "sweep": t_q, "output_error": t_l},
+        "rates": {"hessian_tflops": 2.0 * K * K * T / 2 / (t_h * 1e-3) / 1e12,
+                  "factor_gflops": (2.0 / 3.0) * K ** 3 / (t_f * 1e-3) / 1e9,
+                  "sweep_tflops": 1.0 * N * K * K / (t_q * 1e-3) / 1e12},
+        "l2": "flushed (256 MiB write) before every timed call"}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -584,6 +643,8 @@ def main():
         return run_qlinear(args)
     if args.op == "baselines":
         return run_baselines(args)
+    if args.op == "gptq":
+        return run_gptq(args)
     return run_awq(args)
 
 

@@ -220,6 +220,51 @@ AWQ_API awq_status awq_channel_topk(const float *stat, int64_t K, int64_t k, uin
 AWQ_API awq_status awq_salient_scales(const uint8_t *mask, int64_t K, float factor, float *s,
                                       void *stream);
 
+/* Output error of any quantized weights W_hat (fp16 [N, K], e.g. from GPTQ):
+ *   loss = ||(W_hat - W) X^T||^2 / (N T), row_losses[n] = sum_t ((W_hat - W) X^T)[n, t]^2
+ * with (W_hat - W) rounded to fp16 and contracted on the tensor cores as in
+ * awq_search_layer.  ws >= awq_output_error_workspace_bytes(N, K, T), 256-byte
+ * aligned.  K % 64 == 0. */
+AWQ_API size_t awq_output_error_workspace_bytes(int64_t N, int64_t K, int64_t T);
+AWQ_API awq_status awq_output_error(const void *W, const void *W_hat, int64_t N, int64_t K,
+                                    const void *X, int64_t T, int64_t ldx, float *loss,
+                                    float *row_losses, void *ws, size_t ws_bytes, void *stream);
+
+/* AWQ followed by GPTQ error compensation ([AWQ-note] "Measures": AWQ and GPTQ
+ * are complementary, AWQ+GPTQ at INT2; [Notes-52] §4: round one column at a time
+ * and push its error into the weights not yet quantized, weighted by
+ * second-order statistics of the real input; [GPTQ-AWQ] "GPTQ": a column sweep
+ * with a Cholesky factor prepared once).  Three steps, all binary32:
+ *
+ * awq_gptq_hessian: H = 2 X'^T X' with x' = RN32(x RN32(1/s)) -- the input the
+ *   scaled layer sees (s = 1 for GPTQ alone, s_best for AWQ+GPTQ).
+ *   X fp16 [T, ldx];  s float [K];  H float [K, K] output (full, symmetric).
+ *
+ * awq_gptq_factor: U, the upper triangular factor with (H + damp mean(diag H) I)^-1
+ *   = U^T U (below the diagonal: 0).  Blocked Cholesky of the order-reversed
+ *   damped matrix and a blocked triangular inverse.  damp = 0.01 is the usual
+ *   choice.  A pivot that is not positive sets a device flag reported by
+ *   awq_get_status as AWQ_ERR_INVALID_ARG.  ws >= awq_gptq_factor_workspace_bytes(K).
+ *
+ * awq_gptq_quantize: per row of w = RN32(W s), for k = 0 .. K-1: at a group's
+ *   first column the group parameters of the quantizer of awq_quant_dequant from
+ *   the group's current weights; q_k = clamp(rint(w_k r) + z, 0, qmax);
+ *   wq = RN32((q_k - z) sh);  e = RN32(RN32(w_k - wq) / U_kk);
+ *   w_j = fmaf(-e, U_kj, w_j) for j > k.  Outputs the codes, scales and zeros
+ *   in awq_pack's layout (s is the layer's s: s_best for AWQ+GPTQ) and
+ *   W_hat = RN16(RN32(wq RN32(1/s))), fp16 [N, K].
+ *
+ * K % 64 == 0 and K <= 8192 (each row of W stays in shared memory during its
+ * sweep); larger K returns AWQ_ERR_INVALID_ARG. */
+AWQ_API awq_status awq_gptq_hessian(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s,
+                                    float *H, void *stream);
+AWQ_API size_t awq_gptq_factor_workspace_bytes(int64_t K);
+AWQ_API awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void *ws,
+                                   size_t ws_bytes, void *stream);
+AWQ_API awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const float *s,
+                                     const float *U, awq_qcfg q, uint32_t *codes, void *scales,
+                                     void *zeros, void *W_hat, void *stream);
+
 /* Steps a7-a8 -- argmin over the grid and packing ([AWQ-note] "Measures":
  * scale by the best alpha's s, group-quantize, keep the quantized weights and
  * the necessary metadata).
@@ -245,8 +290,9 @@ AWQ_API awq_status awq_pack_scales(const void *W, int64_t N, int64_t K, const fl
 
 /* Synchronises `stream`, then reports (and clears) errors raised on the device
  * since the last call: AWQ_ERR_TIMEOUT if a kernel's bounded wait ran out,
- * AWQ_ERR_INVALID_ARG if a kernel saw an alpha outside [0, 1] or a given scale
- * that is not positive and finite, AWQ_ERR_CUDA for
+ * AWQ_ERR_INVALID_ARG if a kernel saw an alpha outside [0, 1], a given scale
+ * that is not positive and finite, or a Hessian that is not positive definite,
+ * AWQ_ERR_CUDA for
  * a pending CUDA error.  AWQ_OK otherwise. */
 AWQ_API awq_status awq_get_status(void *stream);
 

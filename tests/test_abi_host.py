@@ -134,3 +134,21 @@ def test_variant_entry_points_reject_bad_arguments():
     assert L.awq_salient_scales(BOGUS, 64, ctypes.c_float(float("inf")), BOGUS, None) == 1
     assert L.awq_pack_scales(BOGUS, 4, 100, BOGUS, QCfg(4, 128, 0), BOGUS, BOGUS, BOGUS, None) == 1
     assert L.awq_pack_scales(BOGUS, 4, 128, BOGUS, QCfg(4, 128, 0), MISALIGNED, BOGUS, BOGUS, None) == 1
+
+
+def test_gptq_entry_points_reject_bad_arguments():
+    L = awq.lib()
+    assert L.awq_gptq_hessian(BOGUS, 16, 96, 96, BOGUS, BOGUS, None) == 1           # K % 64
+    assert L.awq_gptq_hessian(BOGUS, 16, 16384, 16384, BOGUS, BOGUS, None) == 1     # K > 8192
+    assert L.awq_gptq_hessian(MISALIGNED, 16, 128, 128, BOGUS, BOGUS, None) == 1
+    assert L.awq_gptq_factor_workspace_bytes(16384) == 0
+    assert L.awq_gptq_factor_workspace_bytes(4096) >= 4 * 4096 * 4096
+    ws = L.awq_gptq_factor_workspace_bytes(128)
+    assert L.awq_gptq_factor(BOGUS, 128, ctypes.c_float(-1.0), BOGUS, BOGUS, ws, None) == 1
+    assert L.awq_gptq_factor(BOGUS, 128, ctypes.c_float(0.01), BOGUS, BOGUS, ws - 1, None) == 5
+    assert L.awq_gptq_quantize(BOGUS, 4, 192, BOGUS, BOGUS, QCfg(4, 128, 1), BOGUS, BOGUS, BOGUS, BOGUS, None) == 1
+    assert L.awq_gptq_quantize(BOGUS, 4, 128, BOGUS, None, QCfg(4, 128, 1), BOGUS, BOGUS, BOGUS, BOGUS, None) == 1
+    assert L.awq_output_error_workspace_bytes(10, 100, 10) == 0
+    n = L.awq_output_error_workspace_bytes(256, 512, 512)
+    assert L.awq_output_error(BOGUS, BOGUS, 256, 512, BOGUS, 512, 500, BOGUS, None, BOGUS, n, None) == 1   # ldx < K
+    assert L.awq_output_error(BOGUS, BOGUS, 256, 512, BOGUS, 512, 512, BOGUS, None, BOGUS, n - 1, None) == 5

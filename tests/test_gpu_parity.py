@@ -510,3 +510,97 @@ def test_qlinear_on_symmetric_pack(awq):
     awq.get_status()
     ref = oracle.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, 4, 128)
     np.testing.assert_allclose(Y, ref, rtol=1e-4, atol=1e-4 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------------------
+# AWQ followed by GPTQ error compensation
+# ---------------------------------------------------------------------------
+def test_output_error_equals_the_search_loss(awq):
+    """The loss of a given W_hat through the search kernel: for W_hat from the
+    quantizer at s, the same number as the search at s (the same Delta W up to
+    sign, contracted in the same order), and the oracle's within 1e-3."""
+    W, X = gen(300, 512, 700, seed=111)
+    a = oracle.act_stats(X)
+    s = oracle.scales(a, 0.5)
+    Wd, Xd = dev(W), dev(X)
+    What = awq.quant_dequant(Wd, dev(s))
+    loss, rows = awq.output_error(Wd, What, Xd, row_losses=True)
+    grid, grows = awq.search_scales(Wd, Xd, dev(s[None]), row_losses=True)
+    awq.get_status()
+    assert float(loss) == float(grid[0])
+    assert torch.equal(rows, grows[0])
+    ref = oracle.output_error(W, host(What), X)
+    assert float(loss) == pytest.approx(ref["loss"], rel=LOSS_RTOL)
+    np.testing.assert_allclose(host(rows).astype(np.float64), ref["row_sums"], rtol=LOSS_RTOL)
+
+
+@pytest.mark.parametrize("T,K", [(512, 256), (700, 512), (64, 1024)])
+def test_gptq_hessian_matches_oracle(awq, T, K):
+    """binary32 accumulation in token order against the binary64 product:
+    |H - H_oracle| <= T 2^-24 (2 |X'|^T |X'|) (the standard summation bound)."""
+    W, X = gen(8, K, T, seed=112)
+    s = oracle.scales(oracle.act_stats(X), 0.4)
+    H = host(awq.gptq_hessian(dev(X), dev(s))).astype(np.float64)
+    awq.get_status()
+    ref = oracle.gptq_hessian(X, s)
+    rs = (np.float32(1.0) / s).astype(np.float32)
+    Xa = np.abs((X.astype(np.float32) * rs[None]).astype(np.float32)).astype(np.float64)
+    bound = T * 2.0 ** -24 * 2.0 * (Xa.T @ Xa)
+    assert np.all(np.abs(H - ref) <= bound)
+    assert np.array_equal(H, H.T)
+
+
+@pytest.mark.parametrize("K", [128, 512, 1024])
+def test_gptq_factor_matches_oracle(awq, K):
+    """U from the same binary32 H: U^T U inverts the damped H, and U agrees
+    with the oracle's binary64 factor to the accuracy binary32 Cholesky
+    allows for this conditioning (relative Frobenius error <= 64 K 2^-24 cond)."""
+    W, X = gen(8, K, 2 * K, seed=113)
+    H32 = oracle.gptq_hessian(X, np.ones(K, np.float32)).astype(np.float32)
+    U = host(awq.gptq_factor(dev(H32), 0.01)).astype(np.float64)
+    awq.get_status()
+    H = H32.astype(np.float64)
+    Hd = H + np.float32(0.01 * np.float32(np.mean(np.diag(H)))) * np.eye(K)
+    ref = oracle.gptq_factor(H, 0.01)
+    assert np.count_nonzero(np.tril(U, -1)) == 0
+    cond = np.linalg.cond(Hd)
+    err = np.linalg.norm(U - ref) / np.linalg.norm(ref)
+    assert err <= 64 * K * 2.0 ** -24 * cond, (err, cond)
+    resid = np.abs(U.T @ U @ Hd - np.eye(K)).max()
+    assert resid <= 64 * K * 2.0 ** -24 * cond, (resid, cond)
+
+
+@pytest.mark.parametrize("N,K,bits,group,sym", [(300, 512, 4, 128, False), (136, 1024, 2, 64, False),
+                                                (257, 768, 3, 128, True), (64, 256, 2, 64, True)])
+def test_gptq_sweep_bitexact(awq, N, K, bits, group, sym):
+    """The sweep against the oracle's, both fed the oracle's binary32 U: codes,
+    scales, zeros and W_hat bit for bit."""
+    W, X = gen(N, K, 2 * K, bits=bits, group=group, seed=N + K + 114)
+    a = oracle.act_stats(X)
+    s = oracle.scales(a, 0.5)
+    U32 = oracle.gptq_factor(oracle.gptq_hessian(X, s)).astype(np.float32)
+    out = awq.gptq_quantize(dev(W), dev(s), dev(U32), bits, group, zero_point=not sym)
+    awq.get_status()
+    ref = oracle.gptq(W, s, U32, bits, group, zero_point=not sym)
+    assert np.array_equal(host(out["codes"]).view(np.uint32), oracle.pack_codes(ref["q"], bits))
+    assert np.array_equal(host(out["scales"]).view(np.uint16), ref["sh"].view(np.uint16))
+    assert np.array_equal(host(out["zeros"]).astype(np.float32), ref["z"])
+    assert np.array_equal(host(out["W_hat"]).view(np.uint16), ref["what"].view(np.uint16))
+
+
+@pytest.mark.parametrize("bits,group", [(2, 64), (3, 128)])
+def test_awq_gptq_whole_path(awq, bits, group):
+    """AWQ's search, then GPTQ on the scaled layer, all on the GPU: the result
+    beats AWQ alone (the pages' premise), and its loss is the oracle's for the
+    GPU's own W_hat; the oracle's end-to-end run lands within 5% (its Hessian
+    and factor are binary64, so a few codes may differ)."""
+    cfg = synth.make_config(256, 512, 512, bits=bits, group=group, seed=11)
+    W, X, _ = synth.generate(cfg)
+    r = awq.awq_gptq(dev(W), dev(X), bits, group)
+    awq.get_status()
+    loss = float(r["loss"])
+    assert loss < float(host(r["awq_losses"]).min())
+    assert loss == pytest.approx(oracle.output_error(W, host(r["W_hat"]), X)["loss"], rel=LOSS_RTOL)
+    s_best = host(r["s_best"])
+    ref = oracle.gptq(W, s_best, oracle.gptq_factor(oracle.gptq_hessian(X, s_best)), bits, group)
+    assert loss == pytest.approx(oracle.output_error(W, ref["what"], X)["loss"], rel=0.05)
