@@ -109,7 +109,15 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::gptq_sweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<4, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<8, 4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<16, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess)
             return AWQ_ERR_CUDA;
         d.search_attr = true;
@@ -556,7 +564,7 @@ awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void
     if (awq_status e = last_launch()) return e;
     const int nb = (int)(K / awq::kGb);
     for (int p = 0; p < nb; ++p) {          // blocked Cholesky of the reversed, damped Hessian
-        awq::chol_diag_kernel<<<1, 256, 0, st>>>(A, K, p);
+        awq::chol_diag_kernel<<<1, awq::kGb, 0, st>>>(A, K, p);
         const int m = nb - p - 1;
         if (m > 0) {
             awq::chol_panel_kernel<<<m, awq::kGb, 0, st>>>(A, K, p);
@@ -564,9 +572,15 @@ awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void
         }
         if (awq_status e = last_launch()) return e;
     }
-    awq::trinv_diag_kernel<<<nb, awq::kGb, 0, st>>>(A, K, U);           // M = L^-1 into U's storage
-    for (int dd = 1; dd < nb; ++dd) awq::trinv_offdiag_kernel<<<nb - dd, 256, 0, st>>>(A, K, dd, U);
-    if (awq_status e = last_launch()) return e;
+    // M = L^-1 into U's storage: diagonal blocks, then block rows in order,
+    // the pending sums of the rows below kept in the blocks they will become
+    if (cudaMemsetAsync(U, 0, 4 * (size_t)K * K, st) != cudaSuccess) return AWQ_ERR_CUDA;
+    awq::trinv_diag_kernel<<<nb, awq::kGb, 0, st>>>(A, K, U);
+    for (int k = 0; k < nb; ++k) {
+        if (k > 0) awq::trinv_final_kernel<<<k, 256, 0, st>>>(K, k, U);
+        if (k + 1 < nb) awq::trinv_update_kernel<<<(nb - 1 - k) * (k + 1), 256, 0, st>>>(A, K, k, U);
+        if (awq_status e = last_launch()) return e;
+    }
     grid = blocks_for((K * K + 1) / 2, 256);
     if (grid > 8 * d.sms) grid = 8 * d.sms;
     awq::gptq_rotate_kernel<<<grid, 256, 0, st>>>(U, K);                 // U = P M P, upper part
@@ -599,14 +613,23 @@ awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const float *s
     A.zeros = (__half *)zeros;
     A.W_hat = (__half *)W_hat;
     A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
-    // as many rows per block as shared memory holds, next to a ring of U rows
-    A.ring = K <= 4096 ? 3 : 2;
-    A.rows = awq::gsw::MAX_ROWS;
-    while (A.rows > 1 && awq::gsw::smem_bytes(K, A.rows, A.ring) > (size_t)awq::qlv::SMEM_LIMIT) --A.rows;
-    const size_t smem = awq::gsw::smem_bytes(K, A.rows, A.ring);
+    // the block's 256 worker threads own column pairs of R rows in registers:
+    // pairs per thread and rows per block trade against each other, and past
+    // K = 4096 two-column batches keep the ring of U rows in shared memory
+    const int bw = K <= 4096 ? 4 : 2;
+    const int rows = K <= 2048 ? 8 : K <= 4096 ? 4 : 2;
+    A.ring = 2;                                  // deeper rings measured no faster: the batch's serial part bounds it
+    const size_t smem = awq::gsw::smem_bytes(K, rows, bw, A.ring);
     if (smem > (size_t)awq::qlv::SMEM_LIMIT) return AWQ_ERR_UNSUPPORTED;
-    const unsigned grid = (unsigned)((N + A.rows - 1) / A.rows);
-    awq::gptq_sweep_kernel<<<grid, (awq::gsw::MAX_ROWS + 1) * 32, smem, (cudaStream_t)stream>>>(A);
+    cudaStream_t st = (cudaStream_t)stream;
+#define AWQ_SWEEP(SLOTS, R, B)                                                                            \
+    awq::gptq_sweep_kernel<SLOTS, R, B><<<(unsigned)((N + R - 1) / R), awq::gsw::THREADS, smem, st>>>(A)
+    if (K <= 512) AWQ_SWEEP(1, 8, 4);
+    else if (K <= 1024) AWQ_SWEEP(2, 8, 4);
+    else if (K <= 2048) AWQ_SWEEP(4, 8, 4);
+    else if (K <= 4096) AWQ_SWEEP(8, 4, 4);
+    else AWQ_SWEEP(16, 2, 2);
+#undef AWQ_SWEEP
     return last_launch();
 }
 

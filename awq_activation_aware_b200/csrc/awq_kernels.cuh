@@ -1359,33 +1359,32 @@ __global__ void gptq_reverse_kernel(const float *__restrict__ H, int64_t K, cons
 }
 
 // Cholesky, step p of the blocked right-looking form on A (lower, row-major):
-// the diagonal block in shared memory, column by column.  A pivot that is not
-// positive raises the not-positive-definite flag (and is replaced by 1 so the
-// rest stays finite).
-__global__ void __launch_bounds__(256) chol_diag_kernel(float *__restrict__ A, int64_t K, int p) {
+// the diagonal block in shared memory, left-looking inside it -- thread r
+// forms column c's entry of its row as A[r][c] - sum_{m<c} L[r][m] L[c][m]
+// (fmaf in m order, the same sequence as subtracting each column's rank-one
+// update in turn), thread c takes the square root, the others divide.  A
+// pivot that is not positive raises the not-positive-definite flag (and is
+// replaced by 1 so the rest stays finite).
+__global__ void __launch_bounds__(kGb) chol_diag_kernel(float *__restrict__ A, int64_t K, int p) {
     __shared__ float L[kGb][kGb + 1];
     const int64_t o = (int64_t)p * kGb;
-    for (int e = threadIdx.x; e < kGb * kGb; e += 256) L[e / kGb][e % kGb] = A[(o + e / kGb) * K + o + e % kGb];
+    const int r = threadIdx.x;
+    for (int e = r; e < kGb * kGb; e += kGb) L[e / kGb][e % kGb] = A[(o + e / kGb) * K + o + e % kGb];
     __syncthreads();
     for (int c = 0; c < kGb; ++c) {
-        if (threadIdx.x == 0) {
-            float d = L[c][c];
-            if (!(d > 0.0f)) { atomicOr(&g_dev_error, kDevErrNotPD); d = 1.0f; }
-            L[c][c] = __fsqrt_rn(d);
+        float v = L[r][c];
+        if (r >= c)
+            for (int m = 0; m < c; ++m) v = __fmaf_rn(-L[r][m], L[c][m], v);
+        if (r == c) {
+            if (!(v > 0.0f)) { atomicOr(&g_dev_error, kDevErrNotPD); v = 1.0f; }
+            L[c][c] = __fsqrt_rn(v);
         }
         __syncthreads();
-        for (int r = c + 1 + threadIdx.x; r < kGb; r += 256) L[r][c] = __fdiv_rn(L[r][c], L[c][c]);
-        __syncthreads();
-        for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
-            const int r = e / kGb, q = e % kGb;
-            if (r > c && q > c && q <= r) L[r][q] = __fmaf_rn(-L[r][c], L[q][c], L[r][q]);
-        }
+        if (r > c) L[r][c] = __fdiv_rn(v, L[c][c]);
         __syncthreads();
     }
-    for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
-        const int r = e / kGb, q = e % kGb;
-        if (q <= r) A[(o + r) * K + o + q] = L[r][q];
-    }
+    for (int e = r; e < kGb * kGb; e += kGb)
+        if (e % kGb <= e / kGb) A[(o + e / kGb) * K + o + e % kGb] = L[e / kGb][e % kGb];
 }
 
 // Cholesky step p: the panel below the diagonal block, A[i][p] <- A[i][p] L_pp^-T,
@@ -1478,36 +1477,20 @@ __global__ void __launch_bounds__(kGb) trinv_diag_kernel(const float *__restrict
     for (int r = 0; r < kGb; ++r) M[(o + r) * K + o + c] = x[r];
 }
 
-// Off-diagonal blocks at block distance d (i = j + d):
-//   M[i][j] = -M[i][i] (sum_{k=j}^{i-1} L[i][k] M[k][j]),  k in order.
-__global__ void __launch_bounds__(256) trinv_offdiag_kernel(const float *__restrict__ L, int64_t K, int d,
-                                                            float *__restrict__ M) {
+// Off-diagonal blocks, right-looking: U's strictly lower blocks first hold
+// the pending sums S[i][j] = sum_{k=j}^{i-1} L[i][k] M[k][j], built one block
+// column k at a time (fmaf in k order, then m order within a tile), and
+// become M[i][j] = -M[i][i] S[i][j] when block row i is final.
+// Round k, step 1: block row k's off-diagonal blocks become final.
+__global__ void __launch_bounds__(256) trinv_final_kernel(int64_t K, int k, float *__restrict__ M) {
     __shared__ float Pa[kGb][kGb + 4], Qb[kGb][kGb + 4];
-    const int bj = blockIdx.x, bi = bj + d;
-    const int64_t i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb;
+    const int bj = blockIdx.x;
+    const int64_t i0 = (int64_t)k * kGb, j0 = (int64_t)bj * kGb;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    float acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-    for (int bk = bj; bk < bi; ++bk) {
-        const int64_t k0 = (int64_t)bk * kGb;
-        __syncthreads();
-        for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
-            Pa[e / kGb][e % kGb] = L[(i0 + e / kGb) * K + k0 + e % kGb];      // L[i][k] rows, k columns
-            Qb[e % kGb][e / kGb] = M[(k0 + e / kGb) * K + j0 + e % kGb];      // M[k][j] transposed: [j][k]
-        }
-        __syncthreads();
-        block_mm_nt(Pa, Qb, ty, tx, acc);
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+        Pa[e / kGb][e % kGb] = M[(i0 + e / kGb) * K + i0 + e % kGb];        // M[k][k]
+        Qb[e % kGb][e / kGb] = M[(i0 + e / kGb) * K + j0 + e % kGb];        // S[k][j], transposed
     }
-    // S = acc (64 x 64); M[i][j] = -M_ii S
-    __syncthreads();
-    for (int e = threadIdx.x; e < kGb * kGb; e += 256) Pa[e / kGb][e % kGb] = M[(i0 + e / kGb) * K + i0 + e % kGb];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) Qb[tx * 4 + b][ty * 4 + a] = acc[a][b];      // S transposed: [col][row]
     __syncthreads();
     float out[4][4];
 #pragma unroll
@@ -1519,6 +1502,31 @@ __global__ void __launch_bounds__(256) trinv_offdiag_kernel(const float *__restr
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b] = -out[a][b];
+}
+
+// Round k, step 2: S[i][j] += L[i][k] M[k][j] for every block row i > k and
+// block column j <= k, one block per CTA.
+__global__ void __launch_bounds__(256) trinv_update_kernel(const float *__restrict__ L, int64_t K, int k,
+                                                           float *__restrict__ M) {
+    __shared__ float Pa[kGb][kGb + 4], Qb[kGb][kGb + 4];
+    const int bi = k + 1 + blockIdx.x / (k + 1), bj = blockIdx.x % (k + 1);
+    const int64_t i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb, k0 = (int64_t)k * kGb;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    for (int e = threadIdx.x; e < kGb * kGb; e += 256) {
+        Pa[e / kGb][e % kGb] = L[(i0 + e / kGb) * K + k0 + e % kGb];        // L[i][k]
+        Qb[e % kGb][e / kGb] = M[(k0 + e / kGb) * K + j0 + e % kGb];        // M[k][j], transposed
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b];
+    block_mm_nt(Pa, Qb, ty, tx, acc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b] = acc[a][b];
 }
 
 // U = P M P restricted to the upper triangle, in place: element (a, b) and
@@ -1559,129 +1567,207 @@ __global__ void fill_kernel(float *__restrict__ x, int64_t total, float v) {
         x[i] = v;
 }
 
-// The GPTQ column sweep, one warp per row of W, binary32, bit for bit the
+// The GPTQ column sweep over R rows of W per block, binary32, bit for bit the
 // sequence of the definition:
 //   w = RN32(W s); for k = 0 .. K-1:
 //     at a group's first column: the group's parameters from its current w
 //     q  = clamp(rint(w_k r) + z, 0, qmax)         (one FMA with 1.5 2^23)
 //     wq = RN32((q - z) sh);  e = RN32(RN32(w_k - wq) / U_kk)
-//     w_j = fmaf(-e, U_kj, w_j), j > k             (packed pairs, FFMA2)
-// The row lives in shared memory; the last warp streams U's rows (from the
-// 16-byte boundary at or below the diagonal) into a ring that every row warp
-// of the block reads.  At the end each warp packs its codes and writes the
-// fp16 W_hat = RN16(RN32(wq RN32(1/s))); scales and zeros are written as each
-// group starts.
+//     w_j = fmaf(-e, U_kj, w_j), j > k
+// in batches of B consecutive columns (B divides the group size).  The 256
+// worker threads own column pairs (pair p goes to thread p mod 256) of all R
+// rows and keep those weights in registers.  Per batch: the owners of the
+// batch's pairs (and, at a group's start, of the group's pairs) publish those
+// weights to shared memory; row warp r settles the batch's B columns of row r
+// one after another (each taking the updates of the batch's earlier columns,
+// in order) and publishes its B errors; then every owner applies the B
+// updates to each of its later weights in column order -- the same fmaf
+// sequence per element as one column at a time.  Each pair of U is read once
+// per block and used for all R rows.  Warp 8 streams the batch's B rows of U
+// into a ring of slots, RING - 1 batches ahead.  Codes go to shared memory and
+// are packed at the end;
+// W_hat = RN16(RN32(wq RN32(1/s))) is written as each column settles.
 namespace gsw {
-constexpr int MAX_ROWS = 8;
+constexpr int WARPS = 8;                 // worker warps; also the row warps
+constexpr int THREADS = (WARPS + 1) * 32;
+constexpr int MAX_RING = 8;
 struct Args {
     const __half *W;
     int64_t N, K;
     const float *s, *U;
-    int group, G, bits, sym, rows, ring;     // rows per block, ring depth
+    int group, G, bits, sym;
+    int ring;                            // slots of B rows of U, 2..MAX_RING
     float qmax;
     uint32_t *codes;
     __half *scales, *zeros, *W_hat;
     uint64_t timeout_ns;
 };
-inline size_t smem_bytes(int64_t K, int rows, int ring) {
-    return (size_t)ring * K * 4 + (size_t)rows * K * 5 + 2 * 8 * 8 + 256;
+// shared memory: ring [ring][B][K] floats, published group weights [R][128],
+// errors [R][B], codes [R][K] bytes, barriers
+inline size_t smem_bytes(int64_t K, int R, int B, int ring) {
+    return (size_t)ring * B * K * 4 + (size_t)R * 128 * 4 + (size_t)R * B * 4 + (size_t)R * K + MAX_RING * 8 + 512;
 }
 }  // namespace gsw
 
-__global__ void __launch_bounds__((gsw::MAX_ROWS + 1) * 32, 1) gptq_sweep_kernel(const gsw::Args A) {
+template <int SLOTS, int R, int B>   // pairs per thread (K <= 512 SLOTS), rows per block, columns per batch
+__global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::Args A) {
+    using namespace gsw;
     extern __shared__ uint8_t smem_raw[];
     const int64_t K = A.K;
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    float *ring = reinterpret_cast<float *>(base);                        // [ring][K]
-    float *wrow = ring + (size_t)A.ring * K;                              // [rows][K]
-    uint8_t *qrow = reinterpret_cast<uint8_t *>(wrow + (size_t)A.rows * K);   // [rows][K]
-    uint64_t *full = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(qrow + (size_t)A.rows * K) + 7) & ~uintptr_t(7));
-    uint64_t *empty = full + 8;
+    const int RING = A.ring;
+    float *ring = reinterpret_cast<float *>(base);                         // [RING][B][K]
+    float *pub = ring + (size_t)RING * B * K;                              // [R][128]: weights of a group / a batch
+    float *err = pub + R * 128;                                            // [R][B]
+    uint8_t *qrow = reinterpret_cast<uint8_t *>(err + R * B);              // [R][K]
+    uint64_t *full = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(qrow + (size_t)R * K) + 7) & ~uintptr_t(7));
     __shared__ int abort_flag;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row0 = (int64_t)blockIdx.x * A.rows;
-    const int active = (int)(A.N - row0 < A.rows ? A.N - row0 : A.rows);
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < A.ring; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], active); }
+    __shared__ int stop;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int64_t row0 = (int64_t)blockIdx.x * R;
+    const int active = (int)(A.N - row0 < R ? A.N - row0 : R);
+    const int64_t nbatch = K / B;
+    // batch bi's B rows of U into slot bi % RING, from the 16-byte boundary at or
+    // below its first column k0 = B bi (a bulk copy needs it; K % 4 == 0)
+    auto issue = [&](int64_t bi) {
+        const int64_t k0 = bi * B, c0 = k0 & ~int64_t(3);
+        const int s = (int)(bi % RING);
+        const uint32_t bytes = (uint32_t)((K - c0) * 4);
+        mbar_arrive_expect_tx(&full[s], B * bytes);
+#pragma unroll
+        for (int m = 0; m < B; ++m)
+            bulk_load(ring + ((size_t)s * B + m) * K + c0, A.U + (k0 + m) * K + c0, bytes, &full[s]);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < RING; ++i) mbar_init(&full[i], 1);
         abort_flag = 0;
+        stop = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    if (warp == gsw::MAX_ROWS) {                 // producer: U rows into the ring
-        if (lane == 0) {
-            int st = 0;
-            uint32_t ph = 0;
-            for (int64_t k = 0; k < K; ++k) {
-                if (!mbar_wait_bounded(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
-                const int64_t c0 = k & ~int64_t(3);
-                const uint32_t bytes = (uint32_t)((K - c0) * 4);
-                mbar_arrive_expect_tx(&full[st], bytes);
-                bulk_load(ring + (size_t)st * K + c0, A.U + k * K + c0, bytes, &full[st]);
-                if (++st == A.ring) { st = 0; ph ^= 1u; }
+    if (tid == WARPS * 32)                       // the first RING - 1 batches
+        for (int64_t b = 0; b < RING - 1 && b < nbatch; ++b) issue(b);
+
+    // this thread's weights (workers only): pair p = tid + 256 i, rows 0..R-1
+    float2 wr[SLOTS][R];
+    if (warp < WARPS) {
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i) {
+            const int64_t p = tid + 256 * (int64_t)i;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float2 v = make_float2(0.0f, 0.0f);
+                if (2 * p < K && r < active) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(A.W + (row0 + r) * K + 2 * p));
+                    v = make_float2(__fmul_rn(f.x, A.s[2 * p]), __fmul_rn(f.y, A.s[2 * p + 1]));
+                }
+                wr[i][r] = v;
             }
         }
-    } else if (warp < active) {
-        const int64_t n = row0 + warp;
-        float *w = wrow + (size_t)warp * K;
-        uint8_t *qv = qrow + (size_t)warp * K;
-        for (int64_t k = 2 * lane; k < K; k += 64) {
-            const __half2 h = *reinterpret_cast<const __half2 *>(A.W + n * K + k);
-            const float2 f = __half22float2(h);
-            *reinterpret_cast<float2 *>(w + k) = make_float2(__fmul_rn(f.x, A.s[k]), __fmul_rn(f.y, A.s[k + 1]));
-        }
-        __syncwarp();
-        QParams prm{};
-        int st = 0;
-        uint32_t ph = 0;
-        for (int64_t k = 0; k < K; ++k) {
-            if (k % A.group == 0) {
-                float mn = INFINITY, mx = -INFINITY;
-                for (int64_t j = k + lane; j < k + A.group; j += 32) { mn = fminf(mn, w[j]); mx = fmaxf(mx, w[j]); }
+    }
+    QParams prm{};                               // row warp `warp`'s current group parameters
+    for (int64_t bi = 0; bi < nbatch; ++bi) {
+        const int64_t k0 = bi * B;
+        const int sl = (int)(bi % RING);
+        const uint32_t par = (uint32_t)((bi / RING) & 1);
+        const bool gstart = k0 % A.group == 0;
+        const int npub = gstart ? A.group : B;
+        // (a) owners publish the group's weights at its start, else the batch's
+        if (warp < WARPS) {
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            for (int i = 0; i < SLOTS; ++i) {
+                const int64_t p = tid + 256 * (int64_t)i;
+                if (2 * p >= k0 && 2 * p < k0 + npub) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r) *reinterpret_cast<float2 *>(pub + r * 128 + (2 * p - k0)) = wr[i][r];
+                }
+            }
+        }
+        __syncthreads();                         // every worker is past batch bi-1: its slot is free
+        if (tid == WARPS * 32 && bi + RING - 1 < nbatch) issue(bi + RING - 1);
+        // (b) row warp r settles the batch's columns of row r; every worker waits for the slot
+        bool ok = true;
+        if (warp < WARPS) ok = mbar_wait_warp(&full[sl], par, &abort_flag, A.timeout_ns);
+        if (ok && warp < active) {
+            const int r = warp;
+            const float *pw = pub + r * 128;
+            if (gstart) {
+                float mn = INFINITY, mx = -INFINITY;
+                for (int j = lane; j < A.group; j += 32) { mn = fminf(mn, pw[j]); mx = fmaxf(mx, pw[j]); }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 }
                 prm = make_qparams(mn, mx, A.qmax, A.sym != 0);
                 if (lane == 0) {
-                    A.scales[n * A.G + k / A.group] = __float2half_rn(prm.sh);
-                    A.zeros[n * A.G + k / A.group] = __float2half_rn(prm.z);
+                    A.scales[(row0 + r) * A.G + k0 / A.group] = __float2half_rn(prm.sh);
+                    A.zeros[(row0 + r) * A.G + k0 / A.group] = __float2half_rn(prm.z);
                 }
             }
-            if (!mbar_wait_warp(&full[st], ph, &abort_flag, A.timeout_ns)) break;
-            const float *Ur = ring + (size_t)st * K;
-            const float wk = w[k];
+            const float *Ub = ring + (size_t)sl * B * K;
             const float vlo = __fsub_rn(kMagic, prm.z), vhi = __fadd_rn(kMagic, __fsub_rn(A.qmax, prm.z));
-            const float v = fminf(fmaxf(__fmaf_rn(wk, prm.r, kMagic), vlo), vhi);
-            const float qf = __fsub_rn(v, vlo);                              // the code, exact
-            const float wq = __fmul_rn(__fsub_rn(qf, prm.z), prm.sh);
-            const float e = __fdiv_rn(__fsub_rn(wk, wq), Ur[k]);
-            const float2 ne = make_float2(-e, -e);
-            const int64_t p0 = (k + 1) >> 1;                                 // first pair touching j > k
-            for (int64_t p = p0 + lane; p < K / 2; p += 32) {
-                float2 wv = *reinterpret_cast<const float2 *>(w + 2 * p);
-                const float2 uv = *reinterpret_cast<const float2 *>(Ur + 2 * p);
-                float2 r2 = fma2_rn(ne, uv, wv);
-                if (2 * p == k) r2.x = wq;                                   // column k itself: its value is final
-                *reinterpret_cast<float2 *>(w + 2 * p) = r2;
+            float e[B];
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                float wk = pw[i];
+#pragma unroll
+                for (int m = 0; m < i; ++m) wk = __fmaf_rn(-e[m], Ub[m * K + k0 + i], wk);
+                const float v = fminf(fmaxf(__fmaf_rn(wk, prm.r, kMagic), vlo), vhi);
+                const float qf = __fsub_rn(v, vlo);
+                const float wq = __fmul_rn(__fsub_rn(qf, prm.z), prm.sh);
+                e[i] = __fdiv_rn(__fsub_rn(wk, wq), Ub[i * K + k0 + i]);
+                if (lane == i) {
+                    qrow[(size_t)r * K + k0 + i] = (uint8_t)qf;
+                    A.W_hat[(row0 + r) * K + k0 + i] = __float2half_rn(__fmul_rn(wq, __frcp_rn(A.s[k0 + i])));
+                    err[r * B + i] = e[i];
+                }
             }
-            if ((k & 1) && lane == 0) w[k] = wq;
-            if (lane == 0) qv[k] = (uint8_t)qf;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-            if (++st == A.ring) { st = 0; ph ^= 1u; }
         }
-        __syncwarp();
-        // codes (least-significant first) and W_hat
-        const int c = A.bits == 2 ? 2 : 4, per = 32 / c;
-        for (int64_t wd = lane; wd < K / per; wd += 32) {
-            uint32_t v = 0;
-            for (int i = 0; i < per; ++i) v |= (uint32_t)qv[wd * per + i] << (c * i);
-            A.codes[n * (K / per) + wd] = v;
+        if (!ok && lane == 0) atomicExch(&stop, 1);
+        __syncthreads();
+        if (stop) break;
+        // (c) every owner: the B updates of each later weight, in column order
+        if (warp < WARPS) {
+            const float *Ub = ring + (size_t)sl * B * K;
+            float ne[R][B];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int m = 0; m < B; ++m) ne[r][m] = r < active ? -err[r * B + m] : 0.0f;
+            const int64_t pstart = (k0 + B) / 2;
+#pragma unroll
+            for (int i = 0; i < SLOTS; ++i) {
+                const int64_t p = tid + 256 * (int64_t)i;
+                if (p >= pstart && 2 * p < K) {
+                    float2 u[B];
+#pragma unroll
+                    for (int m = 0; m < B; ++m) u[m] = *reinterpret_cast<const float2 *>(Ub + m * K + 2 * p);
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        float2 v = wr[i][r];
+#pragma unroll
+                        for (int m = 0; m < B; ++m) v = fma2_rn(make_float2(ne[r][m], ne[r][m]), u[m], v);
+                        wr[i][r] = v;
+                    }
+                }
+            }
         }
-        for (int64_t k = lane; k < K; k += 32)
-            A.W_hat[n * K + k] = __float2half_rn(__fmul_rn(w[k], __frcp_rn(A.s[k])));
     }
+    __syncthreads();
+    // codes (least-significant first)
+    if (!stop && warp < WARPS) {
+        const int c = A.bits == 2 ? 2 : 4, per = 32 / c;
+        const int64_t words = K / per;
+        for (int64_t e = tid; e < (int64_t)active * words; e += WARPS * 32) {
+            const int r = (int)(e / words);
+            const int64_t wd = e - (int64_t)r * words;
+            uint32_t v = 0;
+            for (int i = 0; i < per; ++i) v |= (uint32_t)qrow[(size_t)r * K + wd * per + i] << (c * i);
+            A.codes[(row0 + r) * words + wd] = v;
+        }
+    }
+    // copies still in flight (an abort) land before the block leaves
     if (abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
