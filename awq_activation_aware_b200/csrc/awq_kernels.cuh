@@ -22,6 +22,7 @@
 #include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cfloat>
 #include <cstdint>
 
@@ -304,6 +305,356 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
     }
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0) = *reinterpret_cast<const uint4 *>(&out[0]);
     *reinterpret_cast<uint4 *>(W_hat + n * K + k0 + 8) = *reinterpret_cast<const uint4 *>(&out[4]);
+}
+
+// ===========================================================================
+// The decode consumer on the tensor cores (4-bit containers: w_bit 3 and 4).
+// The same Y = sum_k x'(q - z) sh, with the products on tcgen05:
+//   A = (q - z) as bf16, exact (|q - z| <= 15), written into tensor memory by
+//       the producer warps (one byte permute makes two bf16 values 128 + q,
+//       one bf16 subtraction leaves q - z);
+//   B = x' split into three bf16 pieces, x' = hi + mid + lo exactly (8 + 8 + 8
+//       significand bits), one MMA row per piece and token;
+//   D = per quantization group, fp32 in tensor memory; the epilogue adds the
+//       three pieces and scales by the group's fp16 scale.
+// Up to 5 tokens (N = 16) or 10 (N = 32) per pass cost the same codes read.
+// Within each 8-column word the MMA's K order is the permute's pair order
+// (0,2),(4,6),(1,3),(5,7); the prep kernel stores x' in that order.
+// ===========================================================================
+namespace qmm {
+constexpr int ROWS = 128;                 // W rows per unit (MMA M)
+constexpr int SC = 256;                   // columns per stage: one 128-byte row of codes
+constexpr int WORDS = SC / 8;
+constexpr int PWARPS = 8;                 // producers: lane quadrant warp % 4, column half warp / 4
+constexpr int EWARP0 = 8;                 // epilogue: warps 8-11, lane quadrant warp - 8, one row per thread
+constexpr int MMA_WARP = 12, LOAD_WARP = 13;
+constexpr int THREADS = 14 * 32;
+constexpr int STAGES = 4;
+constexpr int A_COLS = SC / 2;            // tensor-memory columns of one A slot (2 bf16 per column)
+constexpr int TMEM_COLS = 512;
+constexpr int CODE_BYTES = ROWS * WORDS * 4;                  // 16 KiB, 128-byte swizzled
+constexpr int TT_MAX = 10;
+constexpr int SLOT_FLOATS = ROWS * 16;                        // one partial-sum slot: 128 rows x 16
+constexpr int Z_BYTES = ROWS * 4 * 2;                         // zeros: [128][up to 4 groups] fp16
+template <int NM> __host__ __device__ constexpr int b_bytes() { return NM * SC * 2; }   // NM x 256 bf16, 4 swizzled atoms
+template <int NM> __host__ __device__ constexpr int stage_bytes() { return CODE_BYTES + b_bytes<NM>() + 1024; }
+template <int NM> __host__ __device__ constexpr int d_bufs() { return (TMEM_COLS - 2 * A_COLS) / (4 * NM); }
+template <int NM> constexpr size_t smem_bytes() {
+    return (size_t)STAGES * stage_bytes<NM>() + 1024 + 512;
+}
+// The block whose unit range [units*b/grid, units*(b+1)/grid) holds unit u.
+__device__ __forceinline__ int64_t block_of(int64_t u, int64_t units, int64_t grid) {
+    return ((u + 1) * grid - 1) / units;
+}
+// word i (0..15) of four 16-byte chunks, i known at compile time
+__device__ __forceinline__ uint32_t word_of(const uint4 (&cw)[4], int i) {
+    const uint4 c = cw[i >> 2];
+    return (i & 3) == 0 ? c.x : (i & 3) == 1 ? c.y : (i & 3) == 2 ? c.z : c.w;
+}
+struct Args {
+    const __half *scales, *zeros;
+    int64_t N, K;
+    int G, group, gps, z_bytes, T;        // z_bytes: zero copy size (8, 4, or 2 = plain loads); T: tokens of this pass
+    int64_t n_steps, units;
+    int32_t b_row0;                       // row of this pass's pieces in the x' map
+    float *Y;                             // this pass's output rows, [T][N]
+    float *part;
+    unsigned *cnt;                        // [row blocks][4]
+    uint64_t timeout_ns;
+};
+}  // namespace qmm
+
+// x' = RN32(x RN32(1/s)) of one pass of TT tokens as bf16 pieces: row 3t + p
+// of the pass holds piece p (hi, mid, lo) of token t, columns in the MMA's K
+// order; rows past 3 T and columns past K are zero.  The pieces sum to x'
+// exactly: hi = RN(x'), mid = RN(x' - hi), lo = x' - hi - mid.
+__global__ void qmm_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t Kp, int64_t ldx,
+                                const float *__restrict__ s, int TT, int NM, int n_pass,
+                                __nv_bfloat16 *__restrict__ xb) {
+    const int perm[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+    const int64_t total = (int64_t)n_pass * NM * Kp;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / Kp, kk = i - row * Kp;
+        const int pass = (int)(row / NM), rr = (int)(row % NM);
+        const int t = rr / 3, piece = rr % 3;
+        const int64_t tok = (int64_t)pass * TT + t;
+        const int64_t col = (kk & ~int64_t(7)) + perm[kk & 7];
+        float v = 0.0f;
+        if (t < TT && tok < T && col < K) {
+            const float x = __fmul_rn(__half2float(X[tok * ldx + col]), __frcp_rn(s[col]));
+            const float hi = __bfloat162float(__float2bfloat16_rn(x));
+            const float r1 = __fsub_rn(x, hi);
+            const float mid = __bfloat162float(__float2bfloat16_rn(r1));
+            v = piece == 0 ? hi : piece == 1 ? mid : __fsub_rn(r1, mid);
+        }
+        xb[i] = __float2bfloat16_rn(v);
+    }
+}
+
+template <int NM>
+__global__ void __launch_bounds__(qmm::THREADS, 1)
+qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_xb,
+                   const qmm::Args A) {
+    using namespace qmm;
+    constexpr int D_COLS = 4 * NM;                 // up to 4 groups per stage
+    constexpr int DB = d_bufs<NM>();               // D buffers: 4 at N = 16, 2 at N = 32
+    constexpr int TT = NM / 3;
+    constexpr uint32_t IDESC = mma_idesc_bf16_f32(ROWS, NM);
+    constexpr uint32_t STAGE_BYTES = stage_bytes<NM>();
+    constexpr uint32_t TX_BYTES = CODE_BYTES + b_bytes<NM>();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES;
+    uint64_t *a_full = bars + 2 * STAGES, *a_empty = a_full + 2, *d_full = a_empty + 2, *d_empty = d_full + 4;
+    uint64_t *drain = d_empty + 4;
+    __shared__ uint32_t tmem_base_sm;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t grid = gridDim.x;
+    const int64_t u_begin = A.units * blockIdx.x / grid, u_end = A.units * (blockIdx.x + 1) / grid;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 33); mbar_init(&empty[i], PWARPS + 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&a_full[i], PWARPS); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < 4; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+        mbar_init(drain, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc_1(&tmem_base_sm, TMEM_COLS);
+        tmem_relinquish_1();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sm;
+
+    if (warp == LOAD_WARP) {                       // codes, x' pieces (TMA), zeros (cp.async)
+        if (lane == 0) { tma_prefetch_desc(&tmap_codes); tma_prefetch_desc(&tmap_xb); }
+        int st = 0;
+        uint32_t ph = 0;
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+        const int per = A.z_bytes / 2;                   // groups per copy; gps and per are powers of 2
+        const int lcpr = __ffs(A.gps / per) - 1;         // log2(copies per row)
+        for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0, ++rb) : 0)) {
+            if (!mbar_wait_warp<false>(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
+            uint8_t *stage = base + st * STAGE_BYTES;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[st], TX_BYTES);
+                tma_load_2d(stage, &tmap_codes, (int32_t)(j * WORDS), (int32_t)(rb * ROWS), &full[st]);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    tma_load_2d(stage + CODE_BYTES + a * NM * 128, &tmap_xb, (int32_t)(j * SC + a * 64), A.b_row0,
+                                &full[st]);
+            }
+            __half *zs = reinterpret_cast<__half *>(stage + CODE_BYTES + b_bytes<NM>());
+            const int64_t g0 = j * A.gps;
+            static_assert(ROWS == 128, "copy indexing takes 7 bits for the row");
+            if (A.z_bytes == 2) {
+                for (int e = lane; e < ROWS * A.gps; e += 32) {
+                    const int r = e / A.gps, g = e % A.gps;
+                    int64_t n = rb * ROWS + r;
+                    n = n < A.N ? n : A.N - 1;
+                    if (g0 + g < A.G) zs[e] = A.zeros[n * A.G + g0 + g];
+                }
+                mbar_arrive(&full[st]);
+            } else {
+                for (int e = lane; e < ROWS << lcpr; e += 32) {
+                    const int r = e >> lcpr, c = e & ((1 << lcpr) - 1);
+                    int64_t n = rb * ROWS + r;
+                    n = n < A.N ? n : A.N - 1;
+                    if (g0 + c * per >= A.G) continue;
+                    const __half *src = A.zeros + n * A.G + g0 + c * per;
+                    __half *dst = zs + r * A.gps + c * per;
+                    if (A.z_bytes == 8) cp_async_8(dst, src); else cp_async_4(dst, src);
+                }
+                cp_async_arrive_noinc(&full[st]);
+            }
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+    } else if (warp == MMA_WARP) {                 // one thread issues the MMAs
+        if (lane == 0) {
+            int st = 0, as = 0, db = 0;
+            uint32_t ph = 0, aph = 0, dph = 0;
+            for (int64_t u = u_begin; u < u_end; ++u) {
+                if (!mbar_wait_bounded<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
+                if (!mbar_wait_bounded<false>(&a_full[as], aph, &abort_flag, A.timeout_ns)) break;
+                if (!mbar_wait_bounded<false>(&d_empty[db], dph ^ 1u, &abort_flag, A.timeout_ns)) break;
+                tc_fence_after();
+                const uint32_t bsm = smem_u32(base + st * STAGE_BYTES + CODE_BYTES);
+#pragma unroll
+                for (int m = 0; m < SC / 16; ++m) {
+                    const int gi = (16 * m) / A.group;
+                    const uint64_t bd = sw128_kmajor_desc(bsm + (m / 4) * NM * 128 + (m % 4) * 32);
+                    mma_f16_ts(tmem + 2 * A_COLS + db * D_COLS + gi * NM, tmem + as * A_COLS + 8 * m, bd, IDESC,
+                               (16 * m) % A.group != 0);
+                }
+                mma_commit_1(&a_empty[as]);
+                mma_commit_1(&empty[st]);
+                mma_commit_1(&d_full[db]);
+                if (++st == STAGES) { st = 0; ph ^= 1u; }
+                if (++as == 2) { as = 0; aph ^= 1u; }
+                if (++db == DB) { db = 0; dph ^= 1u; }
+            }
+            mma_commit_1(drain);                   // every MMA issued has finished when this fires
+            mbar_wait_bounded(drain, 0, &abort_flag, A.timeout_ns);
+        }
+    } else if (warp < PWARPS) {                    // producers: A = (q - z) as bf16 pairs
+        const int q = warp & 3, h = warp >> 2;
+        const int rr = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int ngrp = A.group == 128 ? 1 : 2;   // groups of the thread's column half
+        int st = 0, as = 0;
+        uint32_t ph = 0, aph = 0;
+        int64_t j = u_begin % A.n_steps;
+        for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0) : 0)) {
+            if (!mbar_wait_warp<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
+            const uint8_t *stage = base + st * STAGE_BYTES;
+            uint4 cw[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                cw[c] = *reinterpret_cast<const uint4 *>(stage + sw128_offset(rr, 4 * h + c));
+            const __half *zs = reinterpret_cast<const __half *>(stage + CODE_BYTES + b_bytes<NM>());
+            uint32_t z2[2];
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                const int grp = ngrp == 1 ? h : 2 * h + gi;
+                const int gsafe = gi < ngrp ? grp : 0;
+                // a group past G (the last stage of a K that is not a multiple of 256) was
+                // not copied: zero 0 there, on codes the copy filled with 0
+                const bool valid = j * A.gps + gsafe < A.G;
+                const uint32_t zi = valid ? (uint32_t)__half2float(zs[rr * A.gps + gsafe]) : 0u;
+                const uint32_t zb = 0x4300u | zi;
+                z2[gi] = zb | (zb << 16);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
+            if (!mbar_wait_warp<false>(&a_empty[as], aph ^ 1u, &abort_flag, A.timeout_ns)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int half8 = 0; half8 < 2; ++half8) {
+                uint32_t v[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int wi = half8 * 8 + i;                      // word of the thread's half
+                    const uint32_t w = word_of(cw, wi);
+                    const uint32_t zz = z2[ngrp == 1 ? 0 : wi / 8];
+                    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+                    const uint32_t pr[4] = {__byte_perm(lo, 0x43434343u, 0x4140u), __byte_perm(lo, 0x43434343u, 0x4342u),
+                                            __byte_perm(hi, 0x43434343u, 0x4140u), __byte_perm(hi, 0x43434343u, 0x4342u)};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const __nv_bfloat162 d = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&pr[c]),
+                                                         *reinterpret_cast<const __nv_bfloat162 *>(&zz));
+                        v[4 * i + c] = *reinterpret_cast<const uint32_t *>(&d);
+                    }
+                }
+                tmem_st_32x32b_x32_sync(tmem + lane_base + as * A_COLS + 64 * h + 32 * half8, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (++as == 2) { as = 0; aph ^= 1u; }
+        }
+    } else {                                       // epilogue: one row per thread, every group of the stage
+        const int q = warp - EWARP0;
+        const int rr = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        float y[TT];
+#pragma unroll
+        for (int t = 0; t < TT; ++t) y[t] = 0.0f;
+        int db = 0;
+        uint32_t dph = 0;
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+        // scale of each group of unit (rb, j) for this row (0 past G)
+        auto load_sh = [&](int64_t urb, int64_t uj, float (&sh)[4]) {
+            int64_t n = urb * ROWS + rr;
+            n = n < A.N ? n : A.N - 1;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int64_t gg = uj * A.gps + g;
+                sh[g] = (g < A.gps && gg < A.G) ? __half2float(__ldg(A.scales + n * A.G + gg)) : 0.0f;
+            }
+        };
+        float sh[4], sh_n[4];
+        load_sh(rb, j, sh);
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            const int64_t nrb = j + 1 == A.n_steps ? rb + 1 : rb, nj = j + 1 == A.n_steps ? 0 : j + 1;
+            if (u + 1 < u_end) load_sh(nrb, nj, sh_n);
+            if (!mbar_wait_warp<false>(&d_full[db], dph, &abort_flag, A.timeout_ns)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                if (g >= A.gps) break;
+                float dv[NM];
+#pragma unroll
+                for (int c = 0; c < NM; c += 16) {
+                    float pc[16];
+                    tmem_ld_32x32b_x16_sync(tmem + lane_base + 2 * A_COLS + db * D_COLS + g * NM + c, pc);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dv[c + e] = pc[e];
+                }
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    y[t] = __fmaf_rn(sh[g], __fadd_rn(__fadd_rn(dv[3 * t], dv[3 * t + 1]), dv[3 * t + 2]), y[t]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (++db == DB) { db = 0; dph ^= 1u; }
+#pragma unroll
+            for (int g = 0; g < 4; ++g) sh[g] = sh_n[g];
+            if (j == A.n_steps - 1 || u == u_end - 1) {
+                // row block rb's segment ends: Y, or a partial sum and the fixup
+                const int64_t n = rb * ROWS + rr;
+                const int64_t rb_u0 = rb * A.n_steps, rb_u1 = rb_u0 + A.n_steps;
+                if (u_begin <= rb_u0 && u_end >= rb_u1) {
+                    if (n < A.N)
+#pragma unroll
+                        for (int t = 0; t < TT; ++t)
+                            if (t < A.T) A.Y[t * A.N + n] = y[t];
+                } else {
+                    float *mine = A.part + ((rb + blockIdx.x) * ROWS + rr) * 16;
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) mine[t] = y[t];
+                    __threadfence();
+                    __syncwarp();
+                    const int64_t b0 = block_of(rb_u0, A.units, grid), b1 = block_of(rb_u1 - 1, A.units, grid);
+                    unsigned old = 0;
+                    if (lane == 0) old = atomicAdd(&A.cnt[rb * 4 + q], 1u);
+                    old = __shfl_sync(0xffffffffu, old, 0);
+                    if (old == (unsigned)(b1 - b0)) {
+                        __threadfence();
+                        float tot[TT];
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) tot[t] = 0.0f;
+                        for (int64_t b = b0; b <= b1; ++b)
+#pragma unroll
+                            for (int t = 0; t < TT; ++t)
+                                tot[t] = __fadd_rn(tot[t], __ldcg(A.part + ((rb + b) * ROWS + rr) * 16 + t));
+                        if (n < A.N)
+#pragma unroll
+                            for (int t = 0; t < TT; ++t)
+                                if (t < A.T) A.Y[t * A.N + n] = tot[t];
+                        if (lane == 0) A.cnt[rb * 4 + q] = 0u;
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < TT; ++t) y[t] = 0.0f;
+            }
+            if (++j == A.n_steps) { j = 0; ++rb; }
+        }
+    }
+    if (abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == MMA_WARP) tmem_dealloc_1(tmem, TMEM_COLS);
 }
 
 // ===========================================================================

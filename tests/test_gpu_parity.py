@@ -330,7 +330,12 @@ def test_shared_input_joint_search(awq):
                                               (300, 512, 4, 2, 64), (64, 4096, 7, 4, 128),
                                               (136, 640, 2, 2, 128), (520, 256, 9, 4, 64),
                                               (4096, 3072, 1, 4, 128), (2048, 8192, 2, 4, 128),
-                                              (1000, 4096, 3, 2, 64)])
+                                              (1000, 4096, 3, 2, 64),
+                                              # tensor-core path: 16- and 32-row token tiles, two passes,
+                                              # zeros copied 8, 4 and 2 bytes at a time
+                                              (4096, 3072, 5, 4, 128), (2048, 8192, 6, 4, 128),
+                                              (3000, 4352, 12, 3, 64), (136, 640, 4, 4, 128),
+                                              (200, 384, 3, 3, 64)])
 def test_qlinear(awq, N, K, T, bits, group):
     W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
     a = oracle.act_stats(X)
