@@ -109,10 +109,18 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)awq::qmm::smem_bytes<16>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qmm::smem_bytes<16>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<32, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)awq::qmm::smem_bytes<32>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qmm::smem_bytes<32>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<48, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qmm::smem_bytes<48>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_mma_kernel<48, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qmm::smem_bytes<48>()) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -282,8 +290,8 @@ struct QmmPlan {
 };
 QmmPlan qmm_plan(int64_t T, int64_t K, int64_t N) {
     QmmPlan p;
-    p.NM = T <= 5 ? 16 : 32;
-    p.TT = p.NM / 3;
+    p.NM = T <= 5 ? 16 : T <= 10 ? 32 : 48;
+    p.TT = awq::qmm::tile_tokens(p.NM);
     p.n_pass = (int)((T + p.TT - 1) / p.TT);
     p.Kp = (K + awq::qmm::SC - 1) / awq::qmm::SC * awq::qmm::SC;
     p.row_blocks = (N + awq::qmm::ROWS - 1) / awq::qmm::ROWS;
@@ -328,7 +336,6 @@ awq_status qlinear_mma(const uint32_t *codes, const void *scales, const void *ze
     A.G = (int)(K / q.group_size);
     A.group = q.group_size;
     A.gps = awq::qmm::SC / q.group_size;
-    A.z_bytes = A.G % A.gps == 0 ? 2 * A.gps : (A.G % 2 == 0 ? 4 : 2);
     A.n_steps = P.Kp / awq::qmm::SC;
     A.units = P.row_blocks * A.n_steps;
     A.part = part;
@@ -340,12 +347,20 @@ awq_status qlinear_mma(const uint32_t *codes, const void *scales, const void *ze
         A.b_row0 = pass * P.NM;
         A.Y = Y + (int64_t)pass * P.TT * N;
         A.T = (int)(T - (int64_t)pass * P.TT < P.TT ? T - (int64_t)pass * P.TT : P.TT);
-        if (P.NM == 16)
-            awq::qlinear_mma_kernel<16><<<(unsigned)grid, awq::qmm::THREADS, awq::qmm::smem_bytes<16>(), st>>>(
-                tmap_codes, tmap_xb, A);
+        const unsigned g = (unsigned)grid;
+        const int T_ = awq::qmm::THREADS;
+        if (P.NM == 16 && A.gps == 2)
+            awq::qlinear_mma_kernel<16, 2><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
+        else if (P.NM == 16)
+            awq::qlinear_mma_kernel<16, 4><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
+        else if (P.NM == 32 && A.gps == 2)
+            awq::qlinear_mma_kernel<32, 2><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
+        else if (P.NM == 32)
+            awq::qlinear_mma_kernel<32, 4><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
+        else if (A.gps == 2)
+            awq::qlinear_mma_kernel<48, 2><<<g, T_, awq::qmm::smem_bytes<48>(), st>>>(tmap_codes, tmap_xb, A);
         else
-            awq::qlinear_mma_kernel<32><<<(unsigned)grid, awq::qmm::THREADS, awq::qmm::smem_bytes<32>(), st>>>(
-                tmap_codes, tmap_xb, A);
+            awq::qlinear_mma_kernel<48, 4><<<g, T_, awq::qmm::smem_bytes<48>(), st>>>(tmap_codes, tmap_xb, A);
         if (awq_status e = last_launch()) return e;
     }
     return AWQ_OK;

@@ -327,20 +327,33 @@ constexpr int SC = 256;                   // columns per stage: one 128-byte row
 constexpr int WORDS = SC / 8;
 constexpr int PWARPS = 8;                 // producers: lane quadrant warp % 4, column half warp / 4
 constexpr int EWARP0 = 8;                 // epilogue: warps 8-11, lane quadrant warp - 8, one row per thread
-constexpr int MMA_WARP = 12, LOAD_WARP = 13;
-constexpr int THREADS = 14 * 32;
-constexpr int STAGES = 4;
+constexpr int MMA_WARP = 12, LOAD_WARP = 13, BLOAD_WARP = 14;   // MMA issue; code loads; x' loads
+constexpr int THREADS = 15 * 32;
 constexpr int A_COLS = SC / 2;            // tensor-memory columns of one A slot (2 bf16 per column)
 constexpr int TMEM_COLS = 512;
 constexpr int CODE_BYTES = ROWS * WORDS * 4;                  // 16 KiB, 128-byte swizzled
-constexpr int TT_MAX = 10;
-constexpr int SLOT_FLOATS = ROWS * 16;                        // one partial-sum slot: 128 rows x 16
-constexpr int Z_BYTES = ROWS * 4 * 2;                         // zeros: [128][up to 4 groups] fp16
+constexpr int TT_MAX = 16;
+constexpr int SLOT_FLOATS = ROWS * TT_MAX;                    // one partial-sum slot: 128 rows x 16 tokens
 template <int NM> __host__ __device__ constexpr int b_bytes() { return NM * SC * 2; }   // NM x 256 bf16, 4 swizzled atoms
-template <int NM> __host__ __device__ constexpr int stage_bytes() { return CODE_BYTES + b_bytes<NM>() + 1024; }
-template <int NM> __host__ __device__ constexpr int d_bufs() { return (TMEM_COLS - 2 * A_COLS) / (4 * NM); }
+// Two rings: code tiles, freed as soon as the producers hold them in registers, deep
+// enough to cover the load latency of HBM under load; x' tiles, freed when the MMAs
+// that read them complete.
+template <int NM> __host__ __device__ constexpr int code_stages() { return NM == 16 ? 10 : 8; }
+// Token tiles: N = 3 x tokens rows of x' pieces per pass (5, 10 or 16 tokens).
+__host__ __device__ constexpr int tile_tokens(int NM) { return NM / 3; }
+constexpr int B_STAGES = 4;
+// Accumulator columns of one unit: one N-wide block per group of the stage.
+template <int NM, int GPS> __host__ __device__ constexpr int d_cols() { return GPS * NM; }
+template <int NM, int GPS> __host__ __device__ constexpr int a_slots() {
+    return 3 * A_COLS + 2 * d_cols<NM, GPS>() <= TMEM_COLS ? 3 : 2;
+}
+template <int NM, int GPS> __host__ __device__ constexpr int d_bufs() {
+    return (TMEM_COLS - a_slots<NM, GPS>() * A_COLS) / d_cols<NM, GPS>() > 4
+               ? 4
+               : (TMEM_COLS - a_slots<NM, GPS>() * A_COLS) / d_cols<NM, GPS>();
+}
 template <int NM> constexpr size_t smem_bytes() {
-    return (size_t)STAGES * stage_bytes<NM>() + 1024 + 512;
+    return (size_t)code_stages<NM>() * CODE_BYTES + (size_t)B_STAGES * b_bytes<NM>() + 1024 + 512;
 }
 // The block whose unit range [units*b/grid, units*(b+1)/grid) holds unit u.
 __device__ __forceinline__ int64_t block_of(int64_t u, int64_t units, int64_t grid) {
@@ -354,7 +367,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4 (&cw)[4], int i) {
 struct Args {
     const __half *scales, *zeros;
     int64_t N, K;
-    int G, group, gps, z_bytes, T;        // z_bytes: zero copy size (8, 4, or 2 = plain loads); T: tokens of this pass
+    int G, group, gps, T;                 // T: tokens of this pass
     int64_t n_steps, units;
     int32_t b_row0;                       // row of this pass's pieces in the x' map
     float *Y;                             // this pass's output rows, [T][N]
@@ -391,32 +404,39 @@ __global__ void qmm_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t
     }
 }
 
-template <int NM>
+template <int NM, int GPS>
 __global__ void __launch_bounds__(qmm::THREADS, 1)
 qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_xb,
                    const qmm::Args A) {
     using namespace qmm;
-    constexpr int D_COLS = 4 * NM;                 // up to 4 groups per stage
-    constexpr int DB = d_bufs<NM>();               // D buffers: 4 at N = 16, 2 at N = 32
-    constexpr int TT = NM / 3;
+    constexpr int CS = code_stages<NM>();
+    constexpr int BS = B_STAGES;
+    constexpr int D_COLS = d_cols<NM, GPS>();
+    constexpr int AS = a_slots<NM, GPS>();         // A slots in tensor memory
+    constexpr int DB = d_bufs<NM, GPS>();          // accumulator buffers
+    constexpr int MPG = 16 / GPS;                  // MMAs (K = 16 each) per group
+    constexpr int TT = tile_tokens(NM);
+    static_assert(AS * A_COLS + DB * D_COLS <= TMEM_COLS && DB >= 1, "tensor memory budget");
     constexpr uint32_t IDESC = mma_idesc_bf16_f32(ROWS, NM);
-    constexpr uint32_t STAGE_BYTES = stage_bytes<NM>();
-    constexpr uint32_t TX_BYTES = CODE_BYTES + b_bytes<NM>();
+    constexpr uint32_t B_BYTES = b_bytes<NM>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + STAGES;
-    uint64_t *a_full = bars + 2 * STAGES, *a_empty = a_full + 2, *d_full = a_empty + 2, *d_empty = d_full + 4;
-    uint64_t *drain = d_empty + 4;
+    uint8_t *bring = base + CS * CODE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(bring + BS * B_BYTES);
+    uint64_t *full = bars, *empty = bars + CS, *b_full = bars + 2 * CS, *b_empty = b_full + BS;
+    uint64_t *a_full = b_empty + BS, *a_empty = a_full + AS, *d_full = a_empty + AS, *d_empty = d_full + DB;
+    uint64_t *drain = d_empty + DB;
+    static_assert((2 * CS + 2 * BS + 2 * AS + 2 * DB + 1) * 8 <= 512, "barrier area");
     __shared__ uint32_t tmem_base_sm;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t grid = gridDim.x;
     const int64_t u_begin = A.units * blockIdx.x / grid, u_end = A.units * (blockIdx.x + 1) / grid;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 33); mbar_init(&empty[i], PWARPS + 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&a_full[i], PWARPS); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 4; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+        for (int i = 0; i < CS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], PWARPS); }
+        for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], PWARPS); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
         mbar_init(drain, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -430,71 +450,57 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
     tc_fence_after();
     const uint32_t tmem = tmem_base_sm;
 
-    if (warp == LOAD_WARP) {                       // codes, x' pieces (TMA), zeros (cp.async)
-        if (lane == 0) { tma_prefetch_desc(&tmap_codes); tma_prefetch_desc(&tmap_xb); }
-        int st = 0;
-        uint32_t ph = 0;
-        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-        const int per = A.z_bytes / 2;                   // groups per copy; gps and per are powers of 2
-        const int lcpr = __ffs(A.gps / per) - 1;         // log2(copies per row)
-        for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0, ++rb) : 0)) {
-            if (!mbar_wait_warp<false>(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
-            uint8_t *stage = base + st * STAGE_BYTES;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&full[st], TX_BYTES);
-                tma_load_2d(stage, &tmap_codes, (int32_t)(j * WORDS), (int32_t)(rb * ROWS), &full[st]);
+    if (warp == LOAD_WARP) {                       // code tiles (TMA)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_codes);
+            int st = 0;
+            uint32_t ph = 0;
+            int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+            for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0, ++rb) : 0)) {
+                if (!mbar_wait_bounded<false>(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
+                mbar_arrive_expect_tx(&full[st], CODE_BYTES);
+                tma_load_2d(base + st * CODE_BYTES, &tmap_codes, (int32_t)(j * WORDS), (int32_t)(rb * ROWS), &full[st]);
+                if (++st == CS) { st = 0; ph ^= 1u; }
+            }
+        }
+    } else if (warp == BLOAD_WARP) {               // x' pieces of the unit's 256 columns (TMA)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_xb);
+            int st = 0;
+            uint32_t ph = 0;
+            int64_t j = u_begin % A.n_steps;
+            for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0) : 0)) {
+                if (!mbar_wait_bounded<false>(&b_empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
+                uint8_t *bst = bring + st * B_BYTES;
+                mbar_arrive_expect_tx(&b_full[st], B_BYTES);
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
-                    tma_load_2d(stage + CODE_BYTES + a * NM * 128, &tmap_xb, (int32_t)(j * SC + a * 64), A.b_row0,
-                                &full[st]);
+                    tma_load_2d(bst + a * NM * 128, &tmap_xb, (int32_t)(j * SC + a * 64), A.b_row0, &b_full[st]);
+                if (++st == BS) { st = 0; ph ^= 1u; }
             }
-            __half *zs = reinterpret_cast<__half *>(stage + CODE_BYTES + b_bytes<NM>());
-            const int64_t g0 = j * A.gps;
-            static_assert(ROWS == 128, "copy indexing takes 7 bits for the row");
-            if (A.z_bytes == 2) {
-                for (int e = lane; e < ROWS * A.gps; e += 32) {
-                    const int r = e / A.gps, g = e % A.gps;
-                    int64_t n = rb * ROWS + r;
-                    n = n < A.N ? n : A.N - 1;
-                    if (g0 + g < A.G) zs[e] = A.zeros[n * A.G + g0 + g];
-                }
-                mbar_arrive(&full[st]);
-            } else {
-                for (int e = lane; e < ROWS << lcpr; e += 32) {
-                    const int r = e >> lcpr, c = e & ((1 << lcpr) - 1);
-                    int64_t n = rb * ROWS + r;
-                    n = n < A.N ? n : A.N - 1;
-                    if (g0 + c * per >= A.G) continue;
-                    const __half *src = A.zeros + n * A.G + g0 + c * per;
-                    __half *dst = zs + r * A.gps + c * per;
-                    if (A.z_bytes == 8) cp_async_8(dst, src); else cp_async_4(dst, src);
-                }
-                cp_async_arrive_noinc(&full[st]);
-            }
-            if (++st == STAGES) { st = 0; ph ^= 1u; }
         }
     } else if (warp == MMA_WARP) {                 // one thread issues the MMAs
         if (lane == 0) {
-            int st = 0, as = 0, db = 0;
-            uint32_t ph = 0, aph = 0, dph = 0;
+            int bs = 0, as = 0, db = 0;
+            uint32_t bph = 0, aph = 0, dph = 0;
             for (int64_t u = u_begin; u < u_end; ++u) {
-                if (!mbar_wait_bounded<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
+                if (!mbar_wait_bounded<false>(&b_full[bs], bph, &abort_flag, A.timeout_ns)) break;
                 if (!mbar_wait_bounded<false>(&a_full[as], aph, &abort_flag, A.timeout_ns)) break;
                 if (!mbar_wait_bounded<false>(&d_empty[db], dph ^ 1u, &abort_flag, A.timeout_ns)) break;
                 tc_fence_after();
-                const uint32_t bsm = smem_u32(base + st * STAGE_BYTES + CODE_BYTES);
+                // every offset below is a compile-time constant: the descriptor's start
+                // address field (address / 16) takes the byte offset / 16 directly
+                const uint64_t bd0 = sw128_kmajor_desc(smem_u32(bring + bs * B_BYTES));
+                const uint32_t d0 = tmem + AS * A_COLS + db * D_COLS, a0 = tmem + as * A_COLS;
 #pragma unroll
-                for (int m = 0; m < SC / 16; ++m) {
-                    const int gi = (16 * m) / A.group;
-                    const uint64_t bd = sw128_kmajor_desc(bsm + (m / 4) * NM * 128 + (m % 4) * 32);
-                    mma_f16_ts(tmem + 2 * A_COLS + db * D_COLS + gi * NM, tmem + as * A_COLS + 8 * m, bd, IDESC,
-                               (16 * m) % A.group != 0);
-                }
+                for (int m = 0; m < SC / 16; ++m)
+                    mma_f16_ts(d0 + (m / MPG) * NM, a0 + 8 * m,
+                               bd0 + (uint64_t)(((m / 4) * NM * 128 + (m % 4) * 32) >> 4), IDESC, m % MPG != 0);
                 mma_commit_1(&a_empty[as]);
-                mma_commit_1(&empty[st]);
+                mma_commit_1(&b_empty[bs]);
                 mma_commit_1(&d_full[db]);
-                if (++st == STAGES) { st = 0; ph ^= 1u; }
-                if (++as == 2) { as = 0; aph ^= 1u; }
+                if (++bs == BS) { bs = 0; bph ^= 1u; }
+                if (++as == AS) { as = 0; aph ^= 1u; }
                 if (++db == DB) { db = 0; dph ^= 1u; }
             }
             mma_commit_1(drain);                   // every MMA issued has finished when this fires
@@ -504,33 +510,39 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
         const int q = warp & 3, h = warp >> 2;
         const int rr = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int ngrp = A.group == 128 ? 1 : 2;   // groups of the thread's column half
+        constexpr int ngrp = GPS / 2;              // groups of the thread's column half
         int st = 0, as = 0;
         uint32_t ph = 0, aph = 0;
-        int64_t j = u_begin % A.n_steps;
-        for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0) : 0)) {
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+        // bf16 pair (128 + z, 128 + z) of each group of the thread's row and column half;
+        // a group past G (the last stage of a K that is not a multiple of 256) takes z = 0,
+        // against codes the copy filled with 0
+        auto load_z = [&](int64_t urb, int64_t uj, uint32_t (&z2)[2]) {
+            int64_t n = urb * ROWS + rr;
+            n = n < A.N ? n : A.N - 1;
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                const int64_t gg = uj * GPS + (ngrp == 1 ? h : 2 * h + gi);
+                const uint32_t zi =
+                    (gi < ngrp && gg < A.G) ? (uint32_t)__half2float(__ldg(A.zeros + n * A.G + gg)) : 0u;
+                const uint32_t zb = 0x4300u | zi;
+                z2[gi] = zb | (zb << 16);
+            }
+        };
+        uint32_t z2[2], z2n[2] = {0u, 0u};
+        load_z(rb, j, z2);
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            const int64_t nrb = j + 1 == A.n_steps ? rb + 1 : rb, nj = j + 1 == A.n_steps ? 0 : j + 1;
+            if (u + 1 < u_end) load_z(nrb, nj, z2n);
             if (!mbar_wait_warp<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
-            const uint8_t *stage = base + st * STAGE_BYTES;
+            const uint8_t *stage = base + st * CODE_BYTES;
             uint4 cw[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 cw[c] = *reinterpret_cast<const uint4 *>(stage + sw128_offset(rr, 4 * h + c));
-            const __half *zs = reinterpret_cast<const __half *>(stage + CODE_BYTES + b_bytes<NM>());
-            uint32_t z2[2];
-#pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                const int grp = ngrp == 1 ? h : 2 * h + gi;
-                const int gsafe = gi < ngrp ? grp : 0;
-                // a group past G (the last stage of a K that is not a multiple of 256) was
-                // not copied: zero 0 there, on codes the copy filled with 0
-                const bool valid = j * A.gps + gsafe < A.G;
-                const uint32_t zi = valid ? (uint32_t)__half2float(zs[rr * A.gps + gsafe]) : 0u;
-                const uint32_t zb = 0x4300u | zi;
-                z2[gi] = zb | (zb << 16);
-            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
-            if (++st == STAGES) { st = 0; ph ^= 1u; }
+            if (++st == CS) { st = 0; ph ^= 1u; }
             if (!mbar_wait_warp<false>(&a_empty[as], aph ^ 1u, &abort_flag, A.timeout_ns)) break;
             tc_fence_after();
 #pragma unroll
@@ -556,7 +568,11 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[as]);
-            if (++as == 2) { as = 0; aph ^= 1u; }
+            if (++as == AS) { as = 0; aph ^= 1u; }
+            z2[0] = z2n[0];
+            z2[1] = z2n[1];
+            rb = nrb;
+            j = nj;
         }
     } else {                                       // epilogue: one row per thread, every group of the stage
         const int q = warp - EWARP0;
@@ -569,16 +585,16 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
         uint32_t dph = 0;
         int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
         // scale of each group of unit (rb, j) for this row (0 past G)
-        auto load_sh = [&](int64_t urb, int64_t uj, float (&sh)[4]) {
+        auto load_sh = [&](int64_t urb, int64_t uj, float (&sh)[GPS]) {
             int64_t n = urb * ROWS + rr;
             n = n < A.N ? n : A.N - 1;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const int64_t gg = uj * A.gps + g;
-                sh[g] = (g < A.gps && gg < A.G) ? __half2float(__ldg(A.scales + n * A.G + gg)) : 0.0f;
+            for (int g = 0; g < GPS; ++g) {
+                const int64_t gg = uj * GPS + g;
+                sh[g] = gg < A.G ? __half2float(__ldg(A.scales + n * A.G + gg)) : 0.0f;
             }
         };
-        float sh[4], sh_n[4];
+        float sh[GPS], sh_n[GPS];
         load_sh(rb, j, sh);
         for (int64_t u = u_begin; u < u_end; ++u) {
             const int64_t nrb = j + 1 == A.n_steps ? rb + 1 : rb, nj = j + 1 == A.n_steps ? 0 : j + 1;
@@ -586,13 +602,12 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
             if (!mbar_wait_warp<false>(&d_full[db], dph, &abort_flag, A.timeout_ns)) break;
             tc_fence_after();
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                if (g >= A.gps) break;
+            for (int g = 0; g < GPS; ++g) {
                 float dv[NM];
 #pragma unroll
                 for (int c = 0; c < NM; c += 16) {
                     float pc[16];
-                    tmem_ld_32x32b_x16_sync(tmem + lane_base + 2 * A_COLS + db * D_COLS + g * NM + c, pc);
+                    tmem_ld_32x32b_x16_sync(tmem + lane_base + AS * A_COLS + db * D_COLS + g * NM + c, pc);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) dv[c + e] = pc[e];
                 }
@@ -605,7 +620,7 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
             if (lane == 0) mbar_arrive(&d_empty[db]);
             if (++db == DB) { db = 0; dph ^= 1u; }
 #pragma unroll
-            for (int g = 0; g < 4; ++g) sh[g] = sh_n[g];
+            for (int g = 0; g < GPS; ++g) sh[g] = sh_n[g];
             if (j == A.n_steps - 1 || u == u_end - 1) {
                 // row block rb's segment ends: Y, or a partial sum and the fixup
                 const int64_t n = rb * ROWS + rr;
@@ -616,7 +631,7 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
                         for (int t = 0; t < TT; ++t)
                             if (t < A.T) A.Y[t * A.N + n] = y[t];
                 } else {
-                    float *mine = A.part + ((rb + blockIdx.x) * ROWS + rr) * 16;
+                    float *mine = A.part + ((rb + blockIdx.x) * ROWS + rr) * TT_MAX;
 #pragma unroll
                     for (int t = 0; t < TT; ++t) mine[t] = y[t];
                     __threadfence();
@@ -633,7 +648,7 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
                         for (int64_t b = b0; b <= b1; ++b)
 #pragma unroll
                             for (int t = 0; t < TT; ++t)
-                                tot[t] = __fadd_rn(tot[t], __ldcg(A.part + ((rb + b) * ROWS + rr) * 16 + t));
+                                tot[t] = __fadd_rn(tot[t], __ldcg(A.part + ((rb + b) * ROWS + rr) * TT_MAX + t));
                         if (n < A.N)
 #pragma unroll
                             for (int t = 0; t < TT; ++t)

@@ -335,7 +335,9 @@ def test_shared_input_joint_search(awq):
                                               # zeros copied 8, 4 and 2 bytes at a time
                                               (4096, 3072, 5, 4, 128), (2048, 8192, 6, 4, 128),
                                               (3000, 4352, 12, 3, 64), (136, 640, 4, 4, 128),
-                                              (200, 384, 3, 3, 64)])
+                                              (200, 384, 3, 3, 64),
+                                              # 48-row token tiles: one pass of 16, two passes of 16 + 4
+                                              (1536, 2048, 16, 4, 128), (700, 1280, 20, 4, 64)])
 def test_qlinear(awq, N, K, T, bits, group):
     W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
     a = oracle.act_stats(X)
