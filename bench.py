@@ -496,6 +496,15 @@ def run_qlinear(args):
         del g
         return statistics.median(ts)
 
+    def path_and_launches(T):
+        # the library's dispatch: 4-bit containers past two tokens run on the tensor
+        # cores (x' split kernel + one pass per tile of 5, 10 or 16 tokens), the rest
+        # on the CUDA-core kernel (x' kernel + one pass per two tokens)
+        if cfg.bits != 2 and T > 2:
+            tt = 5 if T <= 5 else 10 if T <= 10 else 16
+            return "tcgen05", 1 + -(-T // tt)
+        return "cuda-core", 1 + (T + 1) // 2
+
     for T in [int(t) for t in args.tokens.split(",")]:
         Xt = Xd[:T].contiguous()
         ws = torch.empty(int(awq.lib().awq_qlinear_workspace_bytes(T, cfg.K, cfg.N)), dtype=torch.uint8, device=dev)
@@ -513,7 +522,7 @@ def run_qlinear(args):
                           "fp16_gemm_us": t_ref, "speedup_vs_fp16": t_ref / t_awq,
                           "awq_bytes": nbytes, "awq_GBps": gbs, "hbm_frac": gbs / hbm if hbm else None,
                           "hbm_peak_source": src, "layer_copies": [n_awq, n_ref],
-                          "launches": 1 + (T + 1) // 2}), flush=True)
+                          "path": path_and_launches(T)[0], "launches": path_and_launches(T)[1]}), flush=True)
     awq.get_status()
     return 0
 
