@@ -364,6 +364,65 @@ __device__ __forceinline__ uint32_t word_of(const uint4 (&cw)[4], int i) {
     const uint4 c = cw[i >> 2];
     return (i & 3) == 0 ? c.x : (i & 3) == 1 ? c.y : (i & 3) == 2 ? c.z : c.w;
 }
+// fp16 value o (0..7) of eight packed in 16 bytes
+__device__ __forceinline__ float half_at(const uint4 &v, int o) {
+    const uint32_t w = (o >> 1) == 0 ? v.x : (o >> 1) == 1 ? v.y : (o >> 1) == 2 ? v.z : v.w;
+    return __half2float(__ushort_as_half((unsigned short)((o & 1) ? (w >> 16) : (w & 0xFFFFu))));
+}
+// One row's fp16 values by group ([N][G] scales or zeros) for the units a block
+// walks through in order.  With G a multiple of 8 the thread reads 8 groups (16
+// bytes) at a time, one chunk ahead of use; otherwise one value per group at use.
+template <int GPS>
+struct RowGroups {
+    const __half *p;
+    int64_t N, n_steps;
+    int G, rr;
+    bool vec;
+    uint4 cur, nxt;
+    int64_t nrb;                          // chunk held in nxt: row block, chunk index
+    int nc;
+    __device__ __forceinline__ uint4 fetch(int64_t rb, int c) const {
+        int64_t n = rb * ROWS + rr;
+        n = n < N ? n : N - 1;
+        return __ldg(reinterpret_cast<const uint4 *>(p + n * G) + c);
+    }
+    // the chunk after (nrb, nc): a row block's chunks end at its n_steps * GPS groups
+    // (= G when G is a multiple of 8, since K is then a multiple of 256)
+    __device__ __forceinline__ void next_chunk() {
+        if ((int64_t)(nc + 1) * 8 < n_steps * GPS) {
+            ++nc;
+        } else {
+            ++nrb;
+            nc = 0;
+        }
+    }
+    __device__ __forceinline__ void begin(int64_t rb, int64_t j) {
+        vec = G % 8 == 0;
+        if (vec) {
+            nrb = rb;
+            nc = (int)((j * GPS) >> 3);
+            cur = fetch(nrb, nc);
+            next_chunk();
+            nxt = fetch(nrb, nc);
+        }
+    }
+    // called on reaching unit (., j), for every unit after the first
+    __device__ __forceinline__ void enter(int64_t j) {
+        if (vec && ((j * GPS) & 7) == 0) {
+            cur = nxt;
+            next_chunk();
+            nxt = fetch(nrb, nc);
+        }
+    }
+    __device__ __forceinline__ float get(int64_t rb, int64_t j, int g) const {
+        const int64_t gg = j * GPS + g;
+        if (vec) return half_at(cur, (int)(gg & 7));
+        if (gg >= G) return 0.0f;         // past G: codes and x' are zero there too
+        int64_t n = rb * ROWS + rr;
+        n = n < N ? n : N - 1;
+        return __half2float(__ldg(p + n * G + gg));
+    }
+};
 struct Args {
     const __half *scales, *zeros;
     int64_t N, K;
@@ -514,26 +573,10 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
         int st = 0, as = 0;
         uint32_t ph = 0, aph = 0;
         int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-        // bf16 pair (128 + z, 128 + z) of each group of the thread's row and column half;
-        // a group past G (the last stage of a K that is not a multiple of 256) takes z = 0,
-        // against codes the copy filled with 0
-        auto load_z = [&](int64_t urb, int64_t uj, uint32_t (&z2)[2]) {
-            int64_t n = urb * ROWS + rr;
-            n = n < A.N ? n : A.N - 1;
-#pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                const int64_t gg = uj * GPS + (ngrp == 1 ? h : 2 * h + gi);
-                const uint32_t zi =
-                    (gi < ngrp && gg < A.G) ? (uint32_t)__half2float(__ldg(A.zeros + n * A.G + gg)) : 0u;
-                const uint32_t zb = 0x4300u | zi;
-                z2[gi] = zb | (zb << 16);
-            }
-        };
-        uint32_t z2[2], z2n[2] = {0u, 0u};
-        load_z(rb, j, z2);
+        RowGroups<GPS> zr{A.zeros, A.N, A.n_steps, A.G, rr};
+        zr.begin(rb, j);
         for (int64_t u = u_begin; u < u_end; ++u) {
-            const int64_t nrb = j + 1 == A.n_steps ? rb + 1 : rb, nj = j + 1 == A.n_steps ? 0 : j + 1;
-            if (u + 1 < u_end) load_z(nrb, nj, z2n);
+            if (u != u_begin) zr.enter(j);
             if (!mbar_wait_warp<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
             const uint8_t *stage = base + st * CODE_BYTES;
             uint4 cw[4];
@@ -543,6 +586,14 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
             if (++st == CS) { st = 0; ph ^= 1u; }
+            // bf16 pair (128 + z, 128 + z) of each group of the thread's row and column half
+            uint32_t z2[2];
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                const uint32_t zi = gi < ngrp ? (uint32_t)zr.get(rb, j, ngrp == 1 ? h : 2 * h + gi) : 0u;
+                const uint32_t zb = 0x4300u | zi;
+                z2[gi] = zb | (zb << 16);
+            }
             if (!mbar_wait_warp<false>(&a_empty[as], aph ^ 1u, &abort_flag, A.timeout_ns)) break;
             tc_fence_after();
 #pragma unroll
@@ -569,10 +620,10 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[as]);
             if (++as == AS) { as = 0; aph ^= 1u; }
-            z2[0] = z2n[0];
-            z2[1] = z2n[1];
-            rb = nrb;
-            j = nj;
+            if (++j == A.n_steps) {
+                j = 0;
+                ++rb;
+            }
         }
     } else {                                       // epilogue: one row per thread, every group of the stage
         const int q = warp - EWARP0;
@@ -584,21 +635,10 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
         int db = 0;
         uint32_t dph = 0;
         int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-        // scale of each group of unit (rb, j) for this row (0 past G)
-        auto load_sh = [&](int64_t urb, int64_t uj, float (&sh)[GPS]) {
-            int64_t n = urb * ROWS + rr;
-            n = n < A.N ? n : A.N - 1;
-#pragma unroll
-            for (int g = 0; g < GPS; ++g) {
-                const int64_t gg = uj * GPS + g;
-                sh[g] = gg < A.G ? __half2float(__ldg(A.scales + n * A.G + gg)) : 0.0f;
-            }
-        };
-        float sh[GPS], sh_n[GPS];
-        load_sh(rb, j, sh);
+        RowGroups<GPS> sr{A.scales, A.N, A.n_steps, A.G, rr};
+        sr.begin(rb, j);
         for (int64_t u = u_begin; u < u_end; ++u) {
-            const int64_t nrb = j + 1 == A.n_steps ? rb + 1 : rb, nj = j + 1 == A.n_steps ? 0 : j + 1;
-            if (u + 1 < u_end) load_sh(nrb, nj, sh_n);
+            if (u != u_begin) sr.enter(j);
             if (!mbar_wait_warp<false>(&d_full[db], dph, &abort_flag, A.timeout_ns)) break;
             tc_fence_after();
 #pragma unroll
@@ -611,16 +651,15 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
 #pragma unroll
                     for (int e = 0; e < 16; ++e) dv[c + e] = pc[e];
                 }
+                const float shg = sr.get(rb, j, g);
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
-                    y[t] = __fmaf_rn(sh[g], __fadd_rn(__fadd_rn(dv[3 * t], dv[3 * t + 1]), dv[3 * t + 2]), y[t]);
+                    y[t] = __fmaf_rn(shg, __fadd_rn(__fadd_rn(dv[3 * t], dv[3 * t + 1]), dv[3 * t + 2]), y[t]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&d_empty[db]);
             if (++db == DB) { db = 0; dph ^= 1u; }
-#pragma unroll
-            for (int g = 0; g < GPS; ++g) sh[g] = sh_n[g];
             if (j == A.n_steps - 1 || u == u_end - 1) {
                 // row block rb's segment ends: Y, or a partial sum and the fixup
                 const int64_t n = rb * ROWS + rr;
