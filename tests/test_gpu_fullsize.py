@@ -89,3 +89,47 @@ def test_fullsize_layer(awq, name):
     assert np.all((z >= 0) & (z <= qmax) & (z == np.round(z)))
     # the premise on LLM-shaped layers: the best alpha beats plain RTN
     assert losses_h[best] < losses_h[0]
+
+
+_layers = {}
+
+
+def layer(name):
+    """The seeded layer of a benchmark config, generated once per test session."""
+    if name not in _layers:
+        _layers[name] = synth.generate(synth.CONFIGS[name])
+    return _layers[name]
+
+
+@pytest.mark.parametrize("name", ["attn4096", "mlp_up28672"])
+@pytest.mark.parametrize("T", [1, 2, 4, 16])
+def test_fullsize_qlinear(awq, name, T):
+    """The decode layer at the benchmark's sizes and token counts (the CUDA-core kernel
+    at one and two tokens, the tensor-core kernel at 4 and 16), on sampled rows.  The
+    expected rows come from the oracle's own pack of those rows."""
+    cfg = synth.CONFIGS[name]
+    W, X, _ = layer(name)
+    alphas = synth.default_alphas()
+    losses = np.linspace(1.0, 0.5, len(alphas))                  # chooses the last alpha
+    Wd = torch.from_numpy(W).cuda()
+    a = awq.act_stats(torch.from_numpy(X).cuda())
+    a_h = a.cpu().numpy()
+    out = awq.pack(Wd, a, torch.from_numpy(alphas).cuda(), torch.from_numpy(losses.astype(np.float32)).cuda(),
+                   cfg.bits, cfg.group)
+    Xt = np.ascontiguousarray(X[:T])
+    Y = awq.qlinear(out["codes"], out["scales"], out["zeros"], out["s_best"], torch.from_numpy(Xt).cuda(),
+                    cfg.bits, cfg.group).cpu().numpy()
+    awq.get_status()
+    del Wd
+    rows = sample_rows(cfg.N, cfg.seed + T)
+    pk = oracle.pack(W, a_h, cfg.bits, cfg.group, alphas, losses, rows=rows)
+    ref = oracle.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], Xt, cfg.bits, cfg.group)
+    # binary32 accumulation against the binary64 sum: bound by the sum of |terms|
+    q = oracle.unpack_codes(pk["codes"], cfg.K, cfg.bits).astype(np.float64)
+    gi = np.arange(cfg.K) // cfg.group
+    wq = np.abs((q - pk["zeros"].astype(np.float64)[:, gi]) * pk["scales"].astype(np.float64)[:, gi])
+    xs = np.abs(Xt.astype(np.float32) * (np.float32(1) / pk["s_best"]).astype(np.float32)).astype(np.float64)
+    bound = xs @ wq.T
+    assert Y.shape == (T, cfg.N)
+    assert np.all(np.abs(Y[:, rows] - ref) <= 2e-6 * bound + 1e-30)
+    assert np.all(np.isfinite(Y))
