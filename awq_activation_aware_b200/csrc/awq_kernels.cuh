@@ -1993,7 +1993,8 @@ __global__ void fill_kernel(float *__restrict__ x, int64_t total, float v) {
 // are packed at the end;
 // W_hat = RN16(RN32(wq RN32(1/s))) is written as each column settles.
 namespace gsw {
-constexpr int WARPS = 8;                 // worker warps; also the row warps
+constexpr int WARPS = 8;                 // worker warps; the first R are also the row warps
+constexpr int OWNERS = WARPS * 32;       // worker threads: thread t owns column pairs t + OWNERS i
 constexpr int THREADS = (WARPS + 1) * 32;
 constexpr int MAX_RING = 8;
 struct Args {
@@ -2014,7 +2015,7 @@ inline size_t smem_bytes(int64_t K, int R, int B, int ring) {
 }
 }  // namespace gsw
 
-template <int SLOTS, int R, int B>   // pairs per thread (K <= 512 SLOTS), rows per block, columns per batch
+template <int SLOTS, int R, int B>   // pairs per thread (K <= 2 OWNERS SLOTS), rows per block, columns per batch
 __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::Args A) {
     using namespace gsw;
     extern __shared__ uint8_t smem_raw[];
@@ -2053,12 +2054,12 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
     if (tid == WARPS * 32)                       // the first RING - 1 batches
         for (int64_t b = 0; b < RING - 1 && b < nbatch; ++b) issue(b);
 
-    // this thread's weights (workers only): pair p = tid + 256 i, rows 0..R-1
+    // this thread's weights (workers only): pair p = tid + OWNERS i, rows 0..R-1
     float2 wr[SLOTS][R];
     if (warp < WARPS) {
 #pragma unroll
         for (int i = 0; i < SLOTS; ++i) {
-            const int64_t p = tid + 256 * (int64_t)i;
+            const int64_t p = tid + OWNERS * (int64_t)i;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 float2 v = make_float2(0.0f, 0.0f);
@@ -2081,7 +2082,7 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
         if (warp < WARPS) {
 #pragma unroll
             for (int i = 0; i < SLOTS; ++i) {
-                const int64_t p = tid + 256 * (int64_t)i;
+                const int64_t p = tid + OWNERS * (int64_t)i;
                 if (2 * p >= k0 && 2 * p < k0 + npub) {
 #pragma unroll
                     for (int r = 0; r < R; ++r) *reinterpret_cast<float2 *>(pub + r * 128 + (2 * p - k0)) = wr[i][r];
@@ -2090,7 +2091,9 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
         }
         __syncthreads();                         // every worker is past batch bi-1: its slot is free
         if (tid == WARPS * 32 && bi + RING - 1 < nbatch) issue(bi + RING - 1);
-        // (b) row warp r settles the batch's columns of row r; every worker waits for the slot
+        // (b) row warp r settles the batch's columns of row r; every worker waits for the slot.
+        // Lane i < B reads s of column k0 + i first, so the load is off the column chain.
+        const float s_lane = (warp < active && lane < B) ? __ldg(A.s + k0 + lane) : 1.0f;
         bool ok = true;
         if (warp < WARPS) ok = mbar_wait_warp(&full[sl], par, &abort_flag, A.timeout_ns);
         if (ok && warp < active) {
@@ -2113,6 +2116,7 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
             const float *Ub = ring + (size_t)sl * B * K;
             const float vlo = __fsub_rn(kMagic, prm.z), vhi = __fadd_rn(kMagic, __fsub_rn(A.qmax, prm.z));
             float e[B];
+            float q_l = 0.0f, wq_l = 0.0f, e_l = 0.0f;   // lane i keeps column k0 + i's results
 #pragma unroll
             for (int i = 0; i < B; ++i) {
                 float wk = pw[i];
@@ -2123,10 +2127,15 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
                 const float wq = __fmul_rn(__fsub_rn(qf, prm.z), prm.sh);
                 e[i] = __fdiv_rn(__fsub_rn(wk, wq), Ub[i * K + k0 + i]);
                 if (lane == i) {
-                    qrow[(size_t)r * K + k0 + i] = (uint8_t)qf;
-                    A.W_hat[(row0 + r) * K + k0 + i] = __float2half_rn(__fmul_rn(wq, __frcp_rn(A.s[k0 + i])));
-                    err[r * B + i] = e[i];
+                    q_l = qf;
+                    wq_l = wq;
+                    e_l = e[i];
                 }
+            }
+            if (lane < B) {
+                qrow[(size_t)r * K + k0 + lane] = (uint8_t)q_l;
+                A.W_hat[(row0 + r) * K + k0 + lane] = __float2half_rn(__fmul_rn(wq_l, __frcp_rn(s_lane)));
+                err[r * B + lane] = e_l;
             }
         }
         if (!ok && lane == 0) atomicExch(&stop, 1);
@@ -2143,7 +2152,7 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
             const int64_t pstart = (k0 + B) / 2;
 #pragma unroll
             for (int i = 0; i < SLOTS; ++i) {
-                const int64_t p = tid + 256 * (int64_t)i;
+                const int64_t p = tid + OWNERS * (int64_t)i;
                 if (p >= pstart && 2 * p < K) {
                     float2 u[B];
 #pragma unroll
