@@ -127,9 +127,9 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<4, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::gptq_sweep_kernel<8, 4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<8, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::gptq_sweep_kernel<16, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(awq::gptq_sweep_kernel<16, 4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess)
             return AWQ_ERR_CUDA;
         d.search_attr = true;
@@ -741,7 +741,7 @@ awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const float *s
     // pairs per thread and rows per block trade against each other, and past
     // K = 4096 two-column batches keep the ring of U rows in shared memory
     const int bw = K <= 4096 ? 4 : 2;
-    const int rows = K <= 2048 ? 8 : K <= 4096 ? 4 : 2;
+    const int rows = K <= 4096 ? 8 : 4;
     A.ring = 2;                                  // deeper rings measured no faster: the batch's serial part bounds it
     const size_t smem = awq::gsw::smem_bytes(K, rows, bw, A.ring);
     if (smem > (size_t)awq::qlv::SMEM_LIMIT) return AWQ_ERR_UNSUPPORTED;
@@ -751,8 +751,8 @@ awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const float *s
     if (K <= 512) AWQ_SWEEP(1, 8, 4);
     else if (K <= 1024) AWQ_SWEEP(2, 8, 4);
     else if (K <= 2048) AWQ_SWEEP(4, 8, 4);
-    else if (K <= 4096) AWQ_SWEEP(8, 4, 4);
-    else AWQ_SWEEP(16, 2, 2);
+    else if (K <= 4096) AWQ_SWEEP(8, 8, 4);
+    else AWQ_SWEEP(16, 4, 2);
 #undef AWQ_SWEEP
     return last_launch();
 }

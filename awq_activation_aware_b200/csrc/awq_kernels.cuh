@@ -1995,7 +1995,8 @@ __global__ void fill_kernel(float *__restrict__ x, int64_t total, float v) {
 namespace gsw {
 constexpr int WARPS = 8;                 // worker warps; the first R are also the row warps
 constexpr int OWNERS = WARPS * 32;       // worker threads: thread t owns column pairs t + OWNERS i
-constexpr int THREADS = (WARPS + 1) * 32;
+constexpr int THREADS = WARPS * 32;      // two warps per scheduler: up to 255 registers a thread
+constexpr int ISSUER = OWNERS - 1;       // the worker thread that also issues the copies of U rows
 constexpr int MAX_RING = 8;
 struct Args {
     const __half *W;
@@ -2051,7 +2052,7 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
         fence_mbar_init();
     }
     __syncthreads();
-    if (tid == WARPS * 32)                       // the first RING - 1 batches
+    if (tid == ISSUER)                           // the first RING - 1 batches
         for (int64_t b = 0; b < RING - 1 && b < nbatch; ++b) issue(b);
 
     // this thread's weights (workers only): pair p = tid + OWNERS i, rows 0..R-1
@@ -2090,7 +2091,7 @@ __global__ void __launch_bounds__(gsw::THREADS, 1) gptq_sweep_kernel(const gsw::
             }
         }
         __syncthreads();                         // every worker is past batch bi-1: its slot is free
-        if (tid == WARPS * 32 && bi + RING - 1 < nbatch) issue(bi + RING - 1);
+        if (tid == ISSUER && bi + RING - 1 < nbatch) issue(bi + RING - 1);
         // (b) row warp r settles the batch's columns of row r; every worker waits for the slot.
         // Lane i < B reads s of column k0 + i first, so the load is off the column chain.
         const float s_lane = (warp < active && lane < B) ? __ldg(A.s + k0 + lane) : 1.0f;
