@@ -688,7 +688,7 @@ awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void
     if (awq_status e = last_launch()) return e;
     const int nb = (int)(K / awq::kGb);
     for (int p = 0; p < nb; ++p) {          // blocked Cholesky of the reversed, damped Hessian
-        awq::chol_diag_kernel<<<1, awq::kGb, 0, st>>>(A, K, p);
+        awq::chol_diag_kernel<<<1, awq::kCholDiagThreads, 0, st>>>(A, K, p);
         const int m = nb - p - 1;
         if (m > 0) {
             awq::chol_panel_kernel<<<m, awq::kGb, 0, st>>>(A, K, p);

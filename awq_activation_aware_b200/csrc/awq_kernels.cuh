@@ -1764,32 +1764,54 @@ __global__ void gptq_reverse_kernel(const float *__restrict__ H, int64_t K, cons
 }
 
 // Cholesky, step p of the blocked right-looking form on A (lower, row-major):
-// the diagonal block in shared memory, left-looking inside it -- thread r
-// forms column c's entry of its row as A[r][c] - sum_{m<c} L[r][m] L[c][m]
-// (fmaf in m order, the same sequence as subtracting each column's rank-one
-// update in turn), thread c takes the square root, the others divide.  A
-// pivot that is not positive raises the not-positive-definite flag (and is
-// replaced by 1 so the rest stays finite).
-__global__ void __launch_bounds__(kGb) chol_diag_kernel(float *__restrict__ A, int64_t K, int p) {
-    __shared__ float L[kGb][kGb + 1];
+// the diagonal block, right-looking inside it.  Thread (r, q) holds row r's
+// entries k = q, q + 4, ... in registers.  Column c: the owner of (c, c) takes
+// the square root, the owners of (r, c) below divide by it, and every entry
+// c < k <= r subtracts L[r][c] L[k][c] (fmaf).  Each entry so receives
+// fmaf(-L[r][m], L[k][m], .) for m = 0, 1, ... in order, the sequence of forming
+// A[r][k] - sum_m L[r][m] L[k][m] left to right.  A pivot that is not positive
+// raises the not-positive-definite flag (and is replaced by 1 so the rest stays
+// finite).
+constexpr int kCholDiagThreads = 4 * kGb;
+__global__ void __launch_bounds__(kCholDiagThreads) chol_diag_kernel(float *__restrict__ A, int64_t K, int p) {
+    __shared__ float col[2][kGb];                // column c of L, by parity of c
     const int64_t o = (int64_t)p * kGb;
-    const int r = threadIdx.x;
-    for (int e = r; e < kGb * kGb; e += kGb) L[e / kGb][e % kGb] = A[(o + e / kGb) * K + o + e % kGb];
-    __syncthreads();
+    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
+    float acc[kGb / 4];
+#pragma unroll
+    for (int i = 0; i < kGb / 4; ++i) {
+        const int k = 4 * i + q;
+        acc[i] = k <= r ? A[(o + r) * K + o + k] : 0.0f;
+    }
+#pragma unroll
     for (int c = 0; c < kGb; ++c) {
-        float v = L[r][c];
-        if (r >= c)
-            for (int m = 0; m < c; ++m) v = __fmaf_rn(-L[r][m], L[c][m], v);
-        if (r == c) {
+        float *cl = col[c & 1];
+        if (r == c && q == (c & 3)) {
+            float v = acc[c >> 2];
             if (!(v > 0.0f)) { atomicOr(&g_dev_error, kDevErrNotPD); v = 1.0f; }
-            L[c][c] = __fsqrt_rn(v);
+            acc[c >> 2] = __fsqrt_rn(v);
+            cl[c] = acc[c >> 2];
         }
         __syncthreads();
-        if (r > c) L[r][c] = __fdiv_rn(v, L[c][c]);
+        if (r > c && q == (c & 3)) {
+            acc[c >> 2] = __fdiv_rn(acc[c >> 2], cl[c]);
+            cl[r] = acc[c >> 2];
+        }
         __syncthreads();
+        if (r > c) {
+            const float lrc = cl[r];
+#pragma unroll
+            for (int i = 0; i < kGb / 4; ++i) {
+                const int k = 4 * i + q;
+                if (k > c && k <= r) acc[i] = __fmaf_rn(-lrc, cl[k], acc[i]);
+            }
+        }
     }
-    for (int e = r; e < kGb * kGb; e += kGb)
-        if (e % kGb <= e / kGb) A[(o + e / kGb) * K + o + e % kGb] = L[e / kGb][e % kGb];
+#pragma unroll
+    for (int i = 0; i < kGb / 4; ++i) {
+        const int k = 4 * i + q;
+        if (k <= r) A[(o + r) * K + o + k] = acc[i];
+    }
 }
 
 // Cholesky step p: the panel below the diagonal block, A[i][p] <- A[i][p] L_pp^-T,
@@ -1816,25 +1838,44 @@ __global__ void __launch_bounds__(kGb) chol_panel_kernel(float *__restrict__ A, 
 }
 
 // 64 x 64 x 64 block product on shared-memory tiles: acc[a][b] += sum_m P[r][m] Q[c][m]
-// for this thread's 4 x 4 patch (rows ty*4+a of P, rows tx*4+b of Q), m in order.
+// for this thread's 4 x 4 patch, rows r = ty*4+a of P and rows c = tx+16b of Q (a
+// warp's 16 Q rows then fall in distinct bank groups), m in order; 16-byte loads
+// of 4 consecutive m.  Tiles are 16-byte aligned with rows of kGb + 4 floats.
+__device__ __forceinline__ int mm_col(int tx, int b) { return tx + 16 * b; }
 __device__ __forceinline__ void block_mm_nt(const float (*P)[kGb + 4], const float (*Q)[kGb + 4], int ty, int tx,
                                             float (&acc)[4][4]) {
-#pragma unroll 8
-    for (int m = 0; m < kGb; ++m) {
-        float pv[4], qv[4];
+#pragma unroll 2
+    for (int m = 0; m < kGb; m += 4) {
+        float4 pv[4], qv[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) { pv[a] = P[ty * 4 + a][m]; qv[a] = Q[tx * 4 + a][m]; }
+        for (int a = 0; a < 4; ++a) {
+            pv[a] = *reinterpret_cast<const float4 *>(&P[ty * 4 + a][m]);
+            qv[a] = *reinterpret_cast<const float4 *>(&Q[mm_col(tx, a)][m]);
+        }
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a], qv[b], acc[a][b]);
+            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a].x, qv[b].x, acc[a][b]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a].y, qv[b].y, acc[a][b]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a].z, qv[b].z, acc[a][b]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(pv[a].w, qv[b].w, acc[a][b]);
     }
 }
 
 // Cholesky step p: trailing update A[i][j] -= L[i][p] L[j][p]^T for the lower
 // blocks p < j <= i, one block per CTA.
 __global__ void __launch_bounds__(256) chol_update_kernel(float *__restrict__ A, int64_t K, int p) {
-    __shared__ float Pi[kGb][kGb + 4], Pj[kGb][kGb + 4];
+    __shared__ __align__(16) float Pi[kGb][kGb + 4];
+    __shared__ __align__(16) float Pj[kGb][kGb + 4];
     int bi, bj;
     lower_block(blockIdx.x, bi, bj);
     bi += p + 1;
@@ -1856,7 +1897,7 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float *__restrict__ A,
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            float *d = &A[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b];
+            float *d = &A[(i0 + ty * 4 + a) * K + j0 + mm_col(tx, b)];
             *d = __fsub_rn(*d, acc[a][b]);
         }
 }
@@ -1888,7 +1929,8 @@ __global__ void __launch_bounds__(kGb) trinv_diag_kernel(const float *__restrict
 // become M[i][j] = -M[i][i] S[i][j] when block row i is final.
 // Round k, step 1: block row k's off-diagonal blocks become final.
 __global__ void __launch_bounds__(256) trinv_final_kernel(int64_t K, int k, float *__restrict__ M) {
-    __shared__ float Pa[kGb][kGb + 4], Qb[kGb][kGb + 4];
+    __shared__ __align__(16) float Pa[kGb][kGb + 4];
+    __shared__ __align__(16) float Qb[kGb][kGb + 4];
     const int bj = blockIdx.x;
     const int64_t i0 = (int64_t)k * kGb, j0 = (int64_t)bj * kGb;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -1906,14 +1948,15 @@ __global__ void __launch_bounds__(256) trinv_final_kernel(int64_t K, int k, floa
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b] = -out[a][b];
+        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + mm_col(tx, b)] = -out[a][b];
 }
 
 // Round k, step 2: S[i][j] += L[i][k] M[k][j] for every block row i > k and
 // block column j <= k, one block per CTA.
 __global__ void __launch_bounds__(256) trinv_update_kernel(const float *__restrict__ L, int64_t K, int k,
                                                            float *__restrict__ M) {
-    __shared__ float Pa[kGb][kGb + 4], Qb[kGb][kGb + 4];
+    __shared__ __align__(16) float Pa[kGb][kGb + 4];
+    __shared__ __align__(16) float Qb[kGb][kGb + 4];
     const int bi = k + 1 + blockIdx.x / (k + 1), bj = blockIdx.x % (k + 1);
     const int64_t i0 = (int64_t)bi * kGb, j0 = (int64_t)bj * kGb, k0 = (int64_t)k * kGb;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -1926,12 +1969,12 @@ __global__ void __launch_bounds__(256) trinv_update_kernel(const float *__restri
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b];
+        for (int b = 0; b < 4; ++b) acc[a][b] = M[(i0 + ty * 4 + a) * K + j0 + mm_col(tx, b)];
     block_mm_nt(Pa, Qb, ty, tx, acc);
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + tx * 4 + b] = acc[a][b];
+        for (int b = 0; b < 4; ++b) M[(i0 + ty * 4 + a) * K + j0 + mm_col(tx, b)] = acc[a][b];
 }
 
 // U = P M P restricted to the upper triangle, in place: element (a, b) and
