@@ -332,10 +332,8 @@ awq_status qlinear_mma(const uint32_t *codes, const void *scales, const void *ze
     A.scales = (const __half *)scales;
     A.zeros = (const __half *)zeros;
     A.N = N;
-    A.K = K;
     A.G = (int)(K / q.group_size);
-    A.group = q.group_size;
-    A.gps = awq::qmm::SC / q.group_size;
+    const int gps = awq::qmm::SC / q.group_size;   // groups per 256-column stage: 2 or 4
     A.n_steps = P.Kp / awq::qmm::SC;
     A.units = P.row_blocks * A.n_steps;
     A.part = part;
@@ -349,15 +347,15 @@ awq_status qlinear_mma(const uint32_t *codes, const void *scales, const void *ze
         A.T = (int)(T - (int64_t)pass * P.TT < P.TT ? T - (int64_t)pass * P.TT : P.TT);
         const unsigned g = (unsigned)grid;
         const int T_ = awq::qmm::THREADS;
-        if (P.NM == 16 && A.gps == 2)
+        if (P.NM == 16 && gps == 2)
             awq::qlinear_mma_kernel<16, 2><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
         else if (P.NM == 16)
             awq::qlinear_mma_kernel<16, 4><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
-        else if (P.NM == 32 && A.gps == 2)
+        else if (P.NM == 32 && gps == 2)
             awq::qlinear_mma_kernel<32, 2><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
         else if (P.NM == 32)
             awq::qlinear_mma_kernel<32, 4><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
-        else if (A.gps == 2)
+        else if (gps == 2)
             awq::qlinear_mma_kernel<48, 2><<<g, T_, awq::qmm::smem_bytes<48>(), st>>>(tmap_codes, tmap_xb, A);
         else
             awq::qlinear_mma_kernel<48, 4><<<g, T_, awq::qmm::smem_bytes<48>(), st>>>(tmap_codes, tmap_xb, A);

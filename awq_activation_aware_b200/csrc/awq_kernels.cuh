@@ -425,8 +425,8 @@ struct RowGroups {
 };
 struct Args {
     const __half *scales, *zeros;
-    int64_t N, K;
-    int G, group, gps, T;                 // T: tokens of this pass
+    int64_t N;
+    int G, T;                             // groups per row; tokens of this pass
     int64_t n_steps, units;
     int32_t b_row0;                       // row of this pass's pieces in the x' map
     float *Y;                             // this pass's output rows, [T][N]
