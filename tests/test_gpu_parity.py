@@ -332,7 +332,7 @@ def test_shared_input_joint_search(awq):
                                               (4096, 3072, 1, 4, 128), (2048, 8192, 2, 4, 128),
                                               (1000, 4096, 3, 2, 64),
                                               # tensor-core path: 16- and 32-row token tiles, two passes,
-                                              # zeros copied 8, 4 and 2 bytes at a time
+                                              # G a multiple of 8 (16-byte reads of scales and zeros) or not
                                               (4096, 3072, 5, 4, 128), (2048, 8192, 6, 4, 128),
                                               (3000, 4352, 12, 3, 64), (136, 640, 4, 4, 128),
                                               (200, 384, 3, 3, 64),
