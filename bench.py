@@ -526,12 +526,7 @@ def run_qlinear(args):
         return statistics.median(ts)
 
     def path_and_launches(T):
-        # the library's dispatch: 4-bit containers past two tokens run on the tensor
-        # cores (x' split kernel + one pass per tile of 5, 10 or 16 tokens), the rest
-        # on the CUDA-core kernel (x' kernel + one pass per two tokens)
-        if cfg.bits != 2 and T > 2:
-            tt = 5 if T <= 5 else 10 if T <= 10 else 16
-            return "tcgen05", 1 + -(-T // tt)
+        # the library's dispatch: the CUDA-core kernel (x' kernel + one pass per two tokens)
         return "cuda-core", 1 + (T + 1) // 2
 
     for T in [int(t) for t in args.tokens.split(",")]:

@@ -307,18 +307,15 @@ AWQ_API awq_status awq_get_status(void *stream);
  *   X   fp16 [T, ldx] (the layer's input, not yet divided by s)
  *   Y   float [T, N] output, row-major
  *   ws  device workspace of ws_bytes >= awq_qlinear_workspace_bytes(T, K, N),
- *       256-byte aligned (x' as binary32 or as three bf16 pieces, partial sums
- *       of row blocks split across thread blocks, arrival counters);
- *       overwritten by every call
+ *       256-byte aligned (x' as binary32, partial sums of row blocks split
+ *       across thread blocks, arrival counters); overwritten by every call
  * Requires K % 64 == 0.  Built for small T (decode), where streaming the
- * packed codes from HBM is the cost.  One or two tokens, and 2-bit containers,
- * run on the CUDA cores, two tokens a pass.  3-bit and 4-bit codes with T >= 3
- * run on the tensor cores: (q - z) exact in bf16 against x' split into three
- * bf16 pieces whose sum is x' exactly, so every product is exact, with up to
- * 16 tokens a pass.  Each pass re-reads the codes.  The summation order
- * depends on T and the device's SM count, not on timing: repeated calls on one
- * device give identical Y.  Calls that share a workspace must be ordered (one
- * stream). */
+ * packed codes from HBM is the cost.  Runs on the CUDA cores, two tokens a
+ * pass, each pass re-reading the codes.  The summation order depends on the
+ * device's SM count, not on timing: repeated calls on one device give
+ * identical Y.  Calls that share a workspace must be ordered (one stream).
+ * The workspace size also covers a tensor-core form of the same product
+ * that the library builds but does not dispatch at present. */
 AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
 AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
                                const float *s_best, int64_t N, int64_t K, awq_qcfg q,
