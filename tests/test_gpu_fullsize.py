@@ -104,9 +104,8 @@ def layer(name):
 @pytest.mark.parametrize("name", ["attn4096", "mlp_up28672"])
 @pytest.mark.parametrize("T", [1, 2, 4, 16])
 def test_fullsize_qlinear(awq, name, T):
-    """The decode layer at the benchmark's sizes and token counts (the CUDA-core kernel
-    at one and two tokens, the tensor-core kernel at 4 and 16), on sampled rows.  The
-    expected rows come from the oracle's own pack of those rows."""
+    """The decode layer at the benchmark's sizes and decode token counts, on sampled
+    rows.  The expected rows come from the oracle's own pack of those rows."""
     cfg = synth.CONFIGS[name]
     W, X, _ = layer(name)
     alphas = synth.default_alphas()

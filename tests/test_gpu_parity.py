@@ -331,12 +331,11 @@ def test_shared_input_joint_search(awq):
                                               (136, 640, 2, 2, 128), (520, 256, 9, 4, 64),
                                               (4096, 3072, 1, 4, 128), (2048, 8192, 2, 4, 128),
                                               (1000, 4096, 3, 2, 64),
-                                              # tensor-core path: 16- and 32-row token tiles, two passes,
-                                              # G a multiple of 8 (16-byte reads of scales and zeros) or not
+                                              # 5 to 20 tokens (several passes), G a multiple of 8 or not,
+                                              # K not a multiple of 256
                                               (4096, 3072, 5, 4, 128), (2048, 8192, 6, 4, 128),
                                               (3000, 4352, 12, 3, 64), (136, 640, 4, 4, 128),
                                               (200, 384, 3, 3, 64),
-                                              # 48-row token tiles: one pass of 16, two passes of 16 + 4
                                               (1536, 2048, 16, 4, 128), (700, 1280, 20, 4, 64)])
 def test_qlinear(awq, N, K, T, bits, group):
     W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
