@@ -494,8 +494,10 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
     if (threadIdx.x == 0) {
         for (int i = 0; i < CS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], PWARPS); }
         for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
-        for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], PWARPS); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+        // tensor-memory hand-offs count every lane: each arrives after its own tcgen05
+        // wait and fence, with no warp-level sync in between
+        for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], PWARPS * 32); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4 * 32); }
         mbar_init(drain, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -617,8 +619,7 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
                 tmem_st_32x32b_x32_sync(tmem + lane_base + as * A_COLS + 64 * h + 32 * half8, v);
             }
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[as]);
+            mbar_arrive(&a_full[as]);
             if (++as == AS) { as = 0; aph ^= 1u; }
             if (++j == A.n_steps) {
                 j = 0;
@@ -657,8 +658,7 @@ qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_
                     y[t] = __fmaf_rn(shg, __fadd_rn(__fadd_rn(dv[3 * t], dv[3 * t + 1]), dv[3 * t + 2]), y[t]);
             }
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[db]);
+            mbar_arrive(&d_empty[db]);
             if (++db == DB) { db = 0; dph ^= 1u; }
             if (j == A.n_steps - 1 || u == u_end - 1) {
                 // row block rb's segment ends: Y, or a partial sum and the fixup
