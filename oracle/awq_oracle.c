@@ -81,6 +81,18 @@ uint16_t awq_oracle_rn16(double x)
     return sign | (uint16_t)((E + 15) << 10) | mant;
 }
 
+/* The zero point as stored: the integer rint(-min/scale), saturated to the
+ * largest finite binary16 magnitude (the zeros are kept in fp16), rounded to
+ * binary16 (integers above 2048 are not all representable), and +0 in place
+ * of -0.  The search, the packer and every consumer use this stored value. */
+static double stored_zero(double z)
+{
+    if (z > 65504.0) z = 65504.0;
+    if (z < -65504.0) z = -65504.0;
+    z = awq_oracle_h2d(awq_oracle_rn16(z));
+    return z == 0.0 ? 0.0 : z;
+}
+
 /* ------------------------------------------------------------------ */
 /* Step a1: activation statistics                                      */
 /*   [AWQ-note] "Measures": collect each layer's input X and take its  */
@@ -131,7 +143,11 @@ void awq_oracle_scales(const float *a, int64_t K, float alpha, float *s)
 /*   mn,mx  = min, max of w'_k over the group                          */
 /* asymmetric (zero_point = 1):                                         */
 /*   scale  = RN32(RN32(mx - mn) / qmax)                               */
-/*   z      = clamp(rint(-mn * r), 0, qmax)   (zero point, a code)     */
+/*   z      = RN16(sat(rint(-mn * r)))  (zero point = round(-min/scale),*/
+/*            not clamped to the codes; sat() keeps it inside the      */
+/*            finite fp16 range +-65504 it is stored in, and the       */
+/*            stored fp16 value is the z used below, so the stored     */
+/*            metadata reproduce what exactly; never -0)               */
 /* symmetric (zero_point = 0; [AWQ-note] "Measures": the INT3 grid of  */
 /* step max|w| / (2^(b-1) - 1)):                                        */
 /*   scale  = RN32(max(-mn, mx) / (2^(b-1) - 1)),  z = 2^(b-1)          */
@@ -190,9 +206,7 @@ void awq_oracle_quantize(const uint16_t *W, int64_t N, int64_t K, const float *s
             float r = rn32(1.0 / sh);
             double z;
             if (zero_point) {
-                z = nearbyint(-(double)mn * (double)r);    /* exact product */
-                if (!(z > 0.0)) z = 0.0;        /* a code in [0, qmax]: never -0 */
-                if (z > qmax) z = qmax;
+                z = stored_zero(nearbyint(-(double)mn * (double)r));    /* exact product */
             } else {
                 z = qsym + 1.0;                 /* 2^(b-1): the middle code */
             }
@@ -297,9 +311,7 @@ void awq_oracle_gptq(const uint16_t *W, int64_t N, int64_t K, const float *s, co
                 sh = awq_oracle_h2d(shb);
                 r = rn32(1.0 / sh);
                 if (zero_point) {
-                    z = nearbyint(-(double)mn * r);
-                    if (!(z > 0.0)) z = 0.0;
-                    if (z > qmax) z = qmax;
+                    z = stored_zero(nearbyint(-(double)mn * r));
                 } else {
                     z = qsym + 1.0;
                 }

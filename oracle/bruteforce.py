@@ -42,6 +42,14 @@ def mean_abs(column) -> np.float32:
     return f32(float(tot) / len(column))
 
 
+def stored_zero(z: int) -> float:
+    """zero = round(-min/scale) as kept in the fp16 zeros: saturated to the
+    largest finite binary16 magnitude, then the nearest binary16 (above 2048
+    not every integer is one).  The codes and W_hat use this stored value."""
+    z = min(max(z, -65504), 65504)
+    return to_f16(z) + 0.0          # + 0.0: a zero point of -0 is stored as +0
+
+
 def quantize_group(w, s, bits, sym=False, keep=None):
     """One group: w (binary16 values as floats), s (float32).  Returns q, sh, z, what.
 
@@ -65,12 +73,11 @@ def quantize_group(w, s, bits, sym=False, keep=None):
     if sym:
         z = 1 << (bits - 1)
     else:
-        z = round(-float(mn) * float(r))    # exact product (24 x 24 bits); round(): ties to even
-        z = min(max(z, 0), qmax)
+        z = stored_zero(round(-float(mn) * float(r)))   # exact product (24 x 24 bits); round(): ties to even
     q, what = [], []
     for k in range(len(w)):
         t = float(wp[k]) * float(r)         # exact product
-        qk = min(max(round(t) + z, 0), qmax)
+        qk = int(min(max(round(t) + z, 0), qmax))
         rs = f32(f32(1.0) / s[k])
         deq = f32(f32(qk - z) * f32(sh))
         what.append(float(w[k]) if keep[k] else to_f16(float(f32(deq * rs))))

@@ -124,7 +124,8 @@ def test_notes52_example_through_group_quantizer(oracle_mod):
 @pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (2, 64)])
 def test_round_trip_exact_codes(oracle_mod, bits, group):
     """W built from chosen codes/scales/zeros (each group holds codes 0 and
-    qmax, scales powers of two) is recovered exactly at alpha = 0, and Ŵ = W."""
+    qmax, scales powers of two) is recovered exactly at alpha = 0, and Ŵ = W --
+    also for zero points outside [0, qmax], i.e. groups that do not span zero."""
     rng = np.random.default_rng(bits * 100 + group)
     N, K = 6, 2 * group
     qmax = (1 << bits) - 1
@@ -135,6 +136,7 @@ def test_round_trip_exact_codes(oracle_mod, bits, group):
             pos = rng.choice(group, 2, replace=False) + gi * group
             q[n, pos[0]], q[n, pos[1]] = 0, qmax
     z = rng.integers(0, qmax + 1, size=(N, G))
+    z[:, 0] = rng.integers(-3 * qmax, 4 * qmax + 1, size=N)   # groups that do not span zero too
     sh = 2.0 ** rng.integers(-9, -3, size=(N, G))
     W = np.empty((N, K))
     for n in range(N):
@@ -148,6 +150,58 @@ def test_round_trip_exact_codes(oracle_mod, bits, group):
     assert np.array_equal(r["z"], z.astype(np.float32))
     assert np.array_equal(r["sh"].astype(np.float64), sh)
     assert np.array_equal(r["what"], W16)
+
+
+def test_one_signed_group_golden(oracle_mod):
+    """A group that does not span zero, worked by hand from the affine formula
+    zero = round(-min/scale), q = clamp(round(w/scale) + zero, 0, qmax)
+    (tests/golden/one_signed_group_int4.json): the zero point leaves the code
+    range ([1, 2] gives zero -15) and the codes still cover 0..15.  A zero
+    point clamped to the codes would saturate every code instead."""
+    g = _gold("one_signed_group_int4.json")
+    for W_vals, part in ((g["W"], g), (g["mirrored"]["W"], g["mirrored"])):
+        W = np.array([W_vals], dtype=np.float16)
+        s = np.array(g["s"], dtype=np.float32)
+        r = oracle_mod.quantize(W, s, bits=g["bits"], group=g["group"])
+        assert float(r["sh"][0, 0]) == g["working"]["sh"]
+        assert hex(int(r["sh"].view(np.uint16)[0, 0])) == g["working"]["sh_fp16_bits"]
+        assert float(r["z"][0, 0]) == part["zero"]
+        assert r["q"][0].tolist() == part["q"]
+        assert r["what"][0].astype(np.float64).tolist() == part["W_hat"]
+        Q, SH, Z, WH = bruteforce.quantize([list(map(float, W_vals))], [np.float32(v) for v in s],
+                                           g["bits"], g["group"])
+        assert Q == [part["q"]] and Z == [[part["zero"]]] and WH == [part["W_hat"]]
+    assert g["zero_clamped_to_codes"]["W_hat"] != g["W_hat"]
+
+
+def test_large_zero_points_against_bruteforce(oracle_mod):
+    """Groups far from zero push |zero| past 2048, where not every integer is a
+    binary16 value, and past 65504, where the fp16 zeros saturate: the oracle
+    and the independent restatement agree bit for bit, the stored zero is a
+    binary16 value, and the stored scale and zero reproduce W_hat."""
+    rows = [
+        [64.0, 64.5, 64.25, 64.0625, 64.125, 64.375, 64.4375, 64.3125],      # |zero| < 2048
+        [128.0, 128.5, 128.25, 128.125, 128.375, 128.0, 128.5, 128.25],     # 2048 < |zero| < 4096
+        [-1000.0, -999.5, -999.0, -998.5, -1000.0, -999.0, -999.5, -998.5],
+        [3.0, 3.0, 3.0, 3.0, 3.0, 3.0, 3.0, 3.0],                           # constant: zero saturates
+        [0.25, 0.25, 0.25, 0.25, 0.25, 0.25, 0.25, 0.25],
+    ]
+    W = np.array(rows, dtype=np.float16)
+    assert np.array_equal(W.astype(np.float64), np.array(rows))
+    for bits in (2, 3, 4):
+        s = np.ones(8, dtype=np.float32)
+        r = oracle_mod.quantize(W, s, bits, 8)
+        Q, SH, Z, WH = bruteforce.quantize(rows, [np.float32(1.0)] * 8, bits, 8)
+        assert r["q"].tolist() == Q
+        assert r["z"].tolist() == Z
+        assert r["sh"].astype(np.float64).tolist() == SH
+        assert r["what"].astype(np.float64).tolist() == WH
+        z = r["z"][:, 0].astype(np.float64)
+        assert np.array_equal(z.astype(np.float16).astype(np.float64), z)
+        assert np.abs(z).max() == 65504.0 and np.any(np.abs(z) > 2048)
+        sh = r["sh"].astype(np.float32)
+        deq = ((r["q"].astype(np.float32) - r["z"].astype(np.float32)) * sh).astype(np.float32)
+        assert np.array_equal(deq.astype(np.float16), r["what"])
 
 
 def test_ties_round_to_even(oracle_mod):
@@ -559,7 +613,7 @@ def test_gptq_sweep_against_scalar_restatement(oracle_mod):
                 scale = np.float32(np.float32(mx - mn) / np.float32(qmax))
                 sh = bf.to_f16(min(max(float(scale), 2.0 ** -24), 65504.0))
                 r = np.float32(np.float32(1.0) / np.float32(sh))
-                z = min(max(round(-float(mn) * float(r)), 0), qmax)
+                z = bf.stored_zero(round(-float(mn) * float(r)))
             qk = min(max(round(float(w[k]) * float(r)) + z, 0), qmax)
             wq = np.float32(np.float32(qk - z) * np.float32(sh))
             e = np.float32(np.float32(w[k] - wq) / U[k, k])
