@@ -109,14 +109,6 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qmm::smem_bytes<16>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qmm::smem_bytes<16>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<32, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qmm::smem_bytes<32>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_mma_kernel<32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qmm::smem_bytes<32>()) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -180,34 +172,6 @@ bool encode_codes_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(codes), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// Packed codes [rows][words] as boxes of 32 words (128 bytes) x 128 rows,
-// 128-byte swizzle (the tensor-core decode path reads rows across lanes).
-bool encode_codes_map_sw128(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64_t words) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)words * 4};
-    cuuint32_t box[2] = {(cuuint32_t)awq::qmm::WORDS, (cuuint32_t)awq::qmm::ROWS};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(codes), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-// bf16 [rows][cols] as boxes of 64 columns x box_rows rows, 128-byte swizzle.
-bool encode_bf16_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -277,87 +241,7 @@ size_t qlinear_ws_simt(int64_t T, int64_t K, int64_t N) {
     return ql_xs_bytes(T, K) + ql_part_bytes(N) +
            round_up(sizeof(unsigned) * (size_t)ql_row_blocks(N) * awq::qlv::RGROUPS, 256);
 }
-// The tensor-core path: x' pieces [passes][NM][Kp] bf16, partial sums of split
-// 128-row blocks, arrival counters per block and lane quadrant.
-struct QmmPlan {
-    int NM, TT, n_pass;
-    int64_t Kp, row_blocks;
-    size_t xb_bytes, part_bytes, cnt_bytes;
-};
-QmmPlan qmm_plan(int64_t T, int64_t K, int64_t N) {
-    QmmPlan p;
-    // 16 or 32 rows of x' pieces (5 or 10 tokens) a pass.  The 48-row tile (16 tokens)
-    // gave an intermittent wrong element on the 28672 x 8192 layer at 16 tokens and is
-    // not dispatched until that is understood.
-    p.NM = T <= 5 ? 16 : 32;
-    p.TT = awq::qmm::tile_tokens(p.NM);
-    p.n_pass = (int)((T + p.TT - 1) / p.TT);
-    p.Kp = (K + awq::qmm::SC - 1) / awq::qmm::SC * awq::qmm::SC;
-    p.row_blocks = (N + awq::qmm::ROWS - 1) / awq::qmm::ROWS;
-    p.xb_bytes = round_up(2 * (size_t)p.n_pass * p.NM * p.Kp, 1024);
-    p.part_bytes = round_up(sizeof(float) * (size_t)(p.row_blocks + kQlMaxGrid) * awq::qmm::SLOT_FLOATS, 256);
-    p.cnt_bytes = round_up(sizeof(unsigned) * (size_t)p.row_blocks * 4, 256);
-    return p;
-}
-size_t qlinear_ws(int64_t T, int64_t K, int64_t N) {
-    const QmmPlan p = qmm_plan(T, K, N);
-    const size_t mma = p.xb_bytes + p.part_bytes + p.cnt_bytes;
-    const size_t simt = qlinear_ws_simt(T, K, N);
-    return mma > simt ? mma : simt;
-}
-
-// The decode consumer on the tensor cores (4-bit containers).
-[[maybe_unused]] awq_status qlinear_mma(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best, int64_t N,
-                       int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y, void *ws,
-                       const DevInfo &d, cudaStream_t st) {
-    const QmmPlan P = qmm_plan(T, K, N);
-    uint8_t *w8 = static_cast<uint8_t *>(ws);
-    __nv_bfloat16 *xb = reinterpret_cast<__nv_bfloat16 *>(w8);
-    float *part = reinterpret_cast<float *>(w8 + P.xb_bytes);
-    unsigned *cnt = reinterpret_cast<unsigned *>(w8 + P.xb_bytes + P.part_bytes);
-    {
-        int grid = blocks_for((int64_t)P.n_pass * P.NM * P.Kp, 256);
-        if (grid > 8 * d.sms) grid = 8 * d.sms;
-        awq::qmm_prep_kernel<<<grid, 256, 0, st>>>((const __half *)X, T, K, P.Kp, ldx, s_best, P.TT, P.NM, P.n_pass,
-                                                   xb);
-        if (awq_status e = last_launch()) return e;
-        if (cudaMemsetAsync(cnt, 0, P.cnt_bytes, st) != cudaSuccess) return AWQ_ERR_CUDA;
-    }
-    CUtensorMap tmap_codes, tmap_xb;
-    if (!encode_codes_map_sw128(&tmap_codes, codes, N, K / 8) ||
-        !encode_bf16_map(&tmap_xb, xb, (int64_t)P.n_pass * P.NM, P.Kp, P.NM))
-        return AWQ_ERR_CUDA;
-    awq::qmm::Args A;
-    A.scales = (const __half *)scales;
-    A.zeros = (const __half *)zeros;
-    A.N = N;
-    A.G = (int)(K / q.group_size);
-    const int gps = awq::qmm::SC / q.group_size;   // groups per 256-column stage: 2 or 4
-    A.n_steps = P.Kp / awq::qmm::SC;
-    A.units = P.row_blocks * A.n_steps;
-    A.part = part;
-    A.cnt = cnt;
-    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
-    int64_t grid = d.sms < kQlMaxGrid ? d.sms : kQlMaxGrid;
-    if (grid > A.units) grid = A.units;
-    for (int pass = 0; pass < P.n_pass; ++pass) {
-        A.b_row0 = pass * P.NM;
-        A.Y = Y + (int64_t)pass * P.TT * N;
-        A.T = (int)(T - (int64_t)pass * P.TT < P.TT ? T - (int64_t)pass * P.TT : P.TT);
-        const unsigned g = (unsigned)grid;
-        const int T_ = awq::qmm::THREADS;
-        if (P.NM == 16 && gps == 2)
-            awq::qlinear_mma_kernel<16, 2><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
-        else if (P.NM == 16)
-            awq::qlinear_mma_kernel<16, 4><<<g, T_, awq::qmm::smem_bytes<16>(), st>>>(tmap_codes, tmap_xb, A);
-        else if (gps == 2)
-            awq::qlinear_mma_kernel<32, 2><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
-        else
-            awq::qlinear_mma_kernel<32, 4><<<g, T_, awq::qmm::smem_bytes<32>(), st>>>(tmap_codes, tmap_xb, A);
-        if (awq_status e = last_launch()) return e;
-    }
-    return AWQ_OK;
-}
+size_t qlinear_ws(int64_t T, int64_t K, int64_t N) { return qlinear_ws_simt(T, K, N); }
 
 // a8 for a given s: codes, fp16 scales and zeros.
 awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, uint32_t *codes,
@@ -813,10 +697,6 @@ awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *ze
     DevInfo d;
     if (awq_status e = device_info(d)) return e;
     cudaStream_t st = (cudaStream_t)stream;
-    // Every call runs on the CUDA-core kernel.  The tensor-core kernel (qlinear_mma) is
-    // parity-green in single runs and twice as fast from three tokens on, but repeated
-    // runs gave an intermittent wrong element on the 28672 x 8192 layer; it is not
-    // dispatched until that is understood.
     const bool c2 = q.bits == 2;
     const int64_t cpw = c2 ? 16 : 8;                       // codes per 32-bit word
     const int64_t sc = awq::qlv::WORDS * cpw;              // columns per stage

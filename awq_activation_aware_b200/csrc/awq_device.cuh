@@ -37,23 +37,30 @@ constexpr float kMaxScale = 65504.0f;                  // largest finite fp16
 // Per-(row, group) quantizer parameters derived from the group's min and max of
 // w' = RN32(w*s) ([QAS-QA] §9: zero_point = True, q_group_size, w_bit):
 //   scale = RN32(RN32(mx - mn) / qmax), sh = RN16(clamp(scale, 2^-24, 65504)),
-//   r = RN32(1/sh), z = clamp(rint(-mn * r), 0, qmax),
-// where every product inside rint is exact (rint is the only rounding of
-// w'/scale).  RN32(x + kMagic) with x an exact product is kMagic + rint(x) for
-// |x| <= 2^22 and is monotone in x, so one FMA with kMagic evaluates rint of an
-// exact product, and clamping in that shifted domain clamps the code.
+//   r = RN32(1/sh), z = RN16(sat(rint(-mn * r))),
+// i.e. zero = round(-min/scale), not clamped to the codes: it is saturated to
+// +-65504 and rounded to fp16 because the zeros are stored in fp16, and that
+// stored value is the z the codes and W_hat use.  Every product inside rint is
+// exact (rint is the only rounding of w'/scale).  RN32(x + kMagic) with x an
+// exact product is kMagic + rint(x) for |x| <= 2^22 and is monotone in x, so
+// one FMA with kMagic evaluates rint of an exact product, and clamping in that
+// shifted domain clamps the code (|z| <= 65504 keeps kMagic - z and
+// kMagic + qmax - z inside [2^23, 2^24), where binary32 spacing is 1).
 // `clamp` records whether any code of the group needs clamping:
 // rint(mn r) + z < 0 or rint(mx r) + z > qmax.  The rounding is monotone in w',
 // so when neither end needs it no element of the group does.
 struct QParams {
     float r;     // reciprocal of the stored fp16 scale
     float sh;    // the stored fp16 scale, as binary32
-    float z;     // zero point, an integer in [0, qmax] (never -0)
+    float z;     // zero point: an fp16 integer value in [-65504, 65504] (never -0)
     bool clamp;  // some code of the group leaves [0, qmax] before clamping
 };
 
+constexpr float kZeroLo = 12517408.0f;   // kMagic - 65504
+constexpr float kZeroHi = 12648416.0f;   // kMagic + 65504
+
 // Group parameters from the group's range [mn, mx] of w' = RN32(w s).
-//   asymmetric: scale = RN32(RN32(mx - mn) / qmax), z = clamp(rint(-mn r), 0, qmax)
+//   asymmetric: scale = RN32(RN32(mx - mn) / qmax), z = RN16(sat(rint(-mn r)))
 //   symmetric (sym): scale = RN32(max(-mn, mx) / (2^(b-1) - 1)), z = 2^(b-1)
 //     with qmax = 2^b - 1, so 2^(b-1) = (qmax + 1) / 2
 // then sh = RN16(clamp(scale)), r = RN32(1 / sh).
@@ -64,12 +71,14 @@ __device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax, 
     scale = fminf(fmaxf(scale, kMinScale), kMaxScale);
     p.sh = __half2float(__float2half_rn(scale));
     p.r = __frcp_rn(p.sh);
-    const float top = __fadd_rn(kMagic, qmax);
     if (sym) {
         p.z = mid;
     } else {
+        // vz - kMagic is exact and +0 when vz == kMagic; saturating in the
+        // shifted domain also covers |mn r| > 2^22, where vz is no longer
+        // kMagic + rint but still lies beyond the saturation bound.
         const float vz = __fmaf_rn(-mn, p.r, kMagic);
-        p.z = __fsub_rn(fminf(fmaxf(vz, kMagic), top), kMagic);
+        p.z = __half2float(__float2half_rn(__fsub_rn(fminf(fmaxf(vz, kZeroLo), kZeroHi), kMagic)));
     }
     const float vmn = __fmaf_rn(mn, p.r, kMagic);
     const float vmx = __fmaf_rn(mx, p.r, kMagic);
@@ -78,20 +87,20 @@ __device__ __forceinline__ QParams make_qparams(float mn, float mx, float qmax, 
 }
 
 // Compact 8-byte form kept in the search workspace: r as binary32, then the
-// fp16 scale and the fp16 zero point whose sign bit carries the clamp flag
-// (so one half2 -> float2 conversion unpacks both).
+// fp16 scale, whose sign bit carries the clamp flag (the scale is positive),
+// and the fp16 zero point (so one half2 -> float2 conversion unpacks both).
 __device__ __forceinline__ uint2 pack_qparams(const QParams &p) {
-    const uint32_t shb = __half_as_ushort(__float2half_rn(p.sh));
-    const uint32_t zb = __half_as_ushort(__float2half_rn(p.z)) | (p.clamp ? 0x8000u : 0u);
+    const uint32_t shb = __half_as_ushort(__float2half_rn(p.sh)) | (p.clamp ? 0x8000u : 0u);
+    const uint32_t zb = __half_as_ushort(__float2half_rn(p.z));
     return make_uint2(__float_as_uint(p.r), shb | (zb << 16));
 }
 __device__ __forceinline__ QParams unpack_qparams(uint2 v) {
     QParams p;
     p.r = __uint_as_float(v.x);
     const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
-    p.sh = f.x;
-    p.z = fabsf(f.y);
-    p.clamp = (v.y >> 31) != 0;
+    p.sh = fabsf(f.x);
+    p.z = f.y;
+    p.clamp = (v.y & 0x8000u) != 0;
     return p;
 }
 

@@ -308,410 +308,6 @@ quant_dequant_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G,
 }
 
 // ===========================================================================
-// The decode consumer on the tensor cores (4-bit containers: w_bit 3 and 4).
-// The same Y = sum_k x'(q - z) sh, with the products on tcgen05:
-//   A = (q - z) as bf16, exact (|q - z| <= 15), written into tensor memory by
-//       the producer warps (one byte permute makes two bf16 values 128 + q,
-//       one bf16 subtraction leaves q - z);
-//   B = x' split into three bf16 pieces, x' = hi + mid + lo exactly (8 + 8 + 8
-//       significand bits), one MMA row per piece and token;
-//   D = per quantization group, fp32 in tensor memory; the epilogue adds the
-//       three pieces and scales by the group's fp16 scale.
-// Up to 5 tokens (N = 16) or 10 (N = 32) per pass cost the same codes read.
-// Within each 8-column word the MMA's K order is the permute's pair order
-// (0,2),(4,6),(1,3),(5,7); the prep kernel stores x' in that order.
-// ===========================================================================
-namespace qmm {
-constexpr int ROWS = 128;                 // W rows per unit (MMA M)
-constexpr int SC = 256;                   // columns per stage: one 128-byte row of codes
-constexpr int WORDS = SC / 8;
-constexpr int PWARPS = 8;                 // producers: lane quadrant warp % 4, column half warp / 4
-constexpr int EWARP0 = 8;                 // epilogue: warps 8-11, lane quadrant warp - 8, one row per thread
-constexpr int MMA_WARP = 12, LOAD_WARP = 13, BLOAD_WARP = 14;   // MMA issue; code loads; x' loads
-constexpr int THREADS = 15 * 32;
-constexpr int A_COLS = SC / 2;            // tensor-memory columns of one A slot (2 bf16 per column)
-constexpr int TMEM_COLS = 512;
-constexpr int CODE_BYTES = ROWS * WORDS * 4;                  // 16 KiB, 128-byte swizzled
-constexpr int TT_MAX = 16;
-constexpr int SLOT_FLOATS = ROWS * TT_MAX;                    // one partial-sum slot: 128 rows x 16 tokens
-template <int NM> __host__ __device__ constexpr int b_bytes() { return NM * SC * 2; }   // NM x 256 bf16, 4 swizzled atoms
-// Two rings: code tiles, freed as soon as the producers hold them in registers, deep
-// enough to cover the load latency of HBM under load; x' tiles, freed when the MMAs
-// that read them complete.
-template <int NM> __host__ __device__ constexpr int code_stages() { return NM == 16 ? 10 : 8; }
-// Token tiles: N = 3 x tokens rows of x' pieces per pass (5, 10 or 16 tokens).
-__host__ __device__ constexpr int tile_tokens(int NM) { return NM / 3; }
-constexpr int B_STAGES = 4;
-// Accumulator columns of one unit: one N-wide block per group of the stage.
-template <int NM, int GPS> __host__ __device__ constexpr int d_cols() { return GPS * NM; }
-template <int NM, int GPS> __host__ __device__ constexpr int a_slots() {
-    return 3 * A_COLS + 2 * d_cols<NM, GPS>() <= TMEM_COLS ? 3 : 2;
-}
-template <int NM, int GPS> __host__ __device__ constexpr int d_bufs() {
-    return (TMEM_COLS - a_slots<NM, GPS>() * A_COLS) / d_cols<NM, GPS>() > 4
-               ? 4
-               : (TMEM_COLS - a_slots<NM, GPS>() * A_COLS) / d_cols<NM, GPS>();
-}
-template <int NM> constexpr size_t smem_bytes() {
-    return (size_t)code_stages<NM>() * CODE_BYTES + (size_t)B_STAGES * b_bytes<NM>() + 1024 + 512;
-}
-// The block whose unit range [units*b/grid, units*(b+1)/grid) holds unit u.
-__device__ __forceinline__ int64_t block_of(int64_t u, int64_t units, int64_t grid) {
-    return ((u + 1) * grid - 1) / units;
-}
-// word i (0..15) of four 16-byte chunks, i known at compile time
-__device__ __forceinline__ uint32_t word_of(const uint4 (&cw)[4], int i) {
-    const uint4 c = cw[i >> 2];
-    return (i & 3) == 0 ? c.x : (i & 3) == 1 ? c.y : (i & 3) == 2 ? c.z : c.w;
-}
-// fp16 value o (0..7) of eight packed in 16 bytes
-__device__ __forceinline__ float half_at(const uint4 &v, int o) {
-    const uint32_t w = (o >> 1) == 0 ? v.x : (o >> 1) == 1 ? v.y : (o >> 1) == 2 ? v.z : v.w;
-    return __half2float(__ushort_as_half((unsigned short)((o & 1) ? (w >> 16) : (w & 0xFFFFu))));
-}
-// One row's fp16 values by group ([N][G] scales or zeros) for the units a block
-// walks through in order.  With G a multiple of 8 the thread reads 8 groups (16
-// bytes) at a time, one chunk ahead of use; otherwise one value per group at use.
-template <int GPS>
-struct RowGroups {
-    const __half *p;
-    int64_t N, n_steps;
-    int G, rr;
-    bool vec;
-    uint4 cur, nxt;
-    int64_t nrb;                          // chunk held in nxt: row block, chunk index
-    int nc;
-    __device__ __forceinline__ uint4 fetch(int64_t rb, int c) const {
-        int64_t n = rb * ROWS + rr;
-        n = n < N ? n : N - 1;
-        return __ldg(reinterpret_cast<const uint4 *>(p + n * G) + c);
-    }
-    // the chunk after (nrb, nc): a row block's chunks end at its n_steps * GPS groups
-    // (= G when G is a multiple of 8, since K is then a multiple of 256)
-    __device__ __forceinline__ void next_chunk() {
-        if ((int64_t)(nc + 1) * 8 < n_steps * GPS) {
-            ++nc;
-        } else {
-            ++nrb;
-            nc = 0;
-        }
-    }
-    __device__ __forceinline__ void begin(int64_t rb, int64_t j) {
-        vec = G % 8 == 0;
-        if (vec) {
-            nrb = rb;
-            nc = (int)((j * GPS) >> 3);
-            cur = fetch(nrb, nc);
-            next_chunk();
-            nxt = fetch(nrb, nc);
-        }
-    }
-    // called on reaching unit (., j), for every unit after the first
-    __device__ __forceinline__ void enter(int64_t j) {
-        if (vec && ((j * GPS) & 7) == 0) {
-            cur = nxt;
-            next_chunk();
-            nxt = fetch(nrb, nc);
-        }
-    }
-    __device__ __forceinline__ float get(int64_t rb, int64_t j, int g) const {
-        const int64_t gg = j * GPS + g;
-        if (vec) return half_at(cur, (int)(gg & 7));
-        if (gg >= G) return 0.0f;         // past G: codes and x' are zero there too
-        int64_t n = rb * ROWS + rr;
-        n = n < N ? n : N - 1;
-        return __half2float(__ldg(p + n * G + gg));
-    }
-};
-struct Args {
-    const __half *scales, *zeros;
-    int64_t N;
-    int G, T;                             // groups per row; tokens of this pass
-    int64_t n_steps, units;
-    int32_t b_row0;                       // row of this pass's pieces in the x' map
-    float *Y;                             // this pass's output rows, [T][N]
-    float *part;
-    unsigned *cnt;                        // [row blocks][4]
-    uint64_t timeout_ns;
-};
-}  // namespace qmm
-
-// x' = RN32(x RN32(1/s)) of one pass of TT tokens as bf16 pieces: row 3t + p
-// of the pass holds piece p (hi, mid, lo) of token t, columns in the MMA's K
-// order; rows past 3 T and columns past K are zero.  The pieces sum to x'
-// exactly: hi = RN(x'), mid = RN(x' - hi), lo = x' - hi - mid.
-__global__ void qmm_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t Kp, int64_t ldx,
-                                const float *__restrict__ s, int TT, int NM, int n_pass,
-                                __nv_bfloat16 *__restrict__ xb) {
-    const int perm[8] = {0, 2, 4, 6, 1, 3, 5, 7};
-    const int64_t total = (int64_t)n_pass * NM * Kp;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = i / Kp, kk = i - row * Kp;
-        const int pass = (int)(row / NM), rr = (int)(row % NM);
-        const int t = rr / 3, piece = rr % 3;
-        const int64_t tok = (int64_t)pass * TT + t;
-        const int64_t col = (kk & ~int64_t(7)) + perm[kk & 7];
-        float v = 0.0f;
-        if (t < TT && tok < T && col < K) {
-            const float x = __fmul_rn(__half2float(X[tok * ldx + col]), __frcp_rn(s[col]));
-            const float hi = __bfloat162float(__float2bfloat16_rn(x));
-            const float r1 = __fsub_rn(x, hi);
-            const float mid = __bfloat162float(__float2bfloat16_rn(r1));
-            v = piece == 0 ? hi : piece == 1 ? mid : __fsub_rn(r1, mid);
-        }
-        xb[i] = __float2bfloat16_rn(v);
-    }
-}
-
-template <int NM, int GPS>
-__global__ void __launch_bounds__(qmm::THREADS, 1)
-qlinear_mma_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_xb,
-                   const qmm::Args A) {
-    using namespace qmm;
-    constexpr int CS = code_stages<NM>();
-    constexpr int BS = B_STAGES;
-    constexpr int D_COLS = d_cols<NM, GPS>();
-    constexpr int AS = a_slots<NM, GPS>();         // A slots in tensor memory
-    constexpr int DB = d_bufs<NM, GPS>();          // accumulator buffers
-    constexpr int MPG = 16 / GPS;                  // MMAs (K = 16 each) per group
-    constexpr int TT = tile_tokens(NM);
-    static_assert(AS * A_COLS + DB * D_COLS <= TMEM_COLS && DB >= 1, "tensor memory budget");
-    constexpr uint32_t IDESC = mma_idesc_bf16_f32(ROWS, NM);
-    constexpr uint32_t B_BYTES = b_bytes<NM>();
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *bring = base + CS * CODE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(bring + BS * B_BYTES);
-    uint64_t *full = bars, *empty = bars + CS, *b_full = bars + 2 * CS, *b_empty = b_full + BS;
-    uint64_t *a_full = b_empty + BS, *a_empty = a_full + AS, *d_full = a_empty + AS, *d_empty = d_full + DB;
-    uint64_t *drain = d_empty + DB;
-    static_assert((2 * CS + 2 * BS + 2 * AS + 2 * DB + 1) * 8 <= 512, "barrier area");
-    __shared__ uint32_t tmem_base_sm;
-    __shared__ int abort_flag;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t grid = gridDim.x;
-    const int64_t u_begin = A.units * blockIdx.x / grid, u_end = A.units * (blockIdx.x + 1) / grid;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < CS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], PWARPS); }
-        for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
-        // tensor-memory hand-offs count every lane: each arrives after its own tcgen05
-        // wait and fence, with no warp-level sync in between
-        for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], PWARPS * 32); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4 * 32); }
-        mbar_init(drain, 1);
-        abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == MMA_WARP) {
-        tmem_alloc_1(&tmem_base_sm, TMEM_COLS);
-        tmem_relinquish_1();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_base_sm;
-
-    if (warp == LOAD_WARP) {                       // code tiles (TMA)
-        if (lane == 0) {
-            tma_prefetch_desc(&tmap_codes);
-            int st = 0;
-            uint32_t ph = 0;
-            int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-            for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0, ++rb) : 0)) {
-                if (!mbar_wait_bounded<false>(&empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
-                mbar_arrive_expect_tx(&full[st], CODE_BYTES);
-                tma_load_2d(base + st * CODE_BYTES, &tmap_codes, (int32_t)(j * WORDS), (int32_t)(rb * ROWS), &full[st]);
-                if (++st == CS) { st = 0; ph ^= 1u; }
-            }
-        }
-    } else if (warp == BLOAD_WARP) {               // x' pieces of the unit's 256 columns (TMA)
-        if (lane == 0) {
-            tma_prefetch_desc(&tmap_xb);
-            int st = 0;
-            uint32_t ph = 0;
-            int64_t j = u_begin % A.n_steps;
-            for (int64_t u = u_begin; u < u_end; ++u, (++j == A.n_steps ? (j = 0) : 0)) {
-                if (!mbar_wait_bounded<false>(&b_empty[st], ph ^ 1u, &abort_flag, A.timeout_ns)) break;
-                uint8_t *bst = bring + st * B_BYTES;
-                mbar_arrive_expect_tx(&b_full[st], B_BYTES);
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-                    tma_load_2d(bst + a * NM * 128, &tmap_xb, (int32_t)(j * SC + a * 64), A.b_row0, &b_full[st]);
-                if (++st == BS) { st = 0; ph ^= 1u; }
-            }
-        }
-    } else if (warp == MMA_WARP) {                 // one thread issues the MMAs
-        if (lane == 0) {
-            int bs = 0, as = 0, db = 0;
-            uint32_t bph = 0, aph = 0, dph = 0;
-            for (int64_t u = u_begin; u < u_end; ++u) {
-                if (!mbar_wait_bounded<false>(&b_full[bs], bph, &abort_flag, A.timeout_ns)) break;
-                if (!mbar_wait_bounded<false>(&a_full[as], aph, &abort_flag, A.timeout_ns)) break;
-                if (!mbar_wait_bounded<false>(&d_empty[db], dph ^ 1u, &abort_flag, A.timeout_ns)) break;
-                tc_fence_after();
-                // every offset below is a compile-time constant: the descriptor's start
-                // address field (address / 16) takes the byte offset / 16 directly
-                const uint64_t bd0 = sw128_kmajor_desc(smem_u32(bring + bs * B_BYTES));
-                const uint32_t d0 = tmem + AS * A_COLS + db * D_COLS, a0 = tmem + as * A_COLS;
-#pragma unroll
-                for (int m = 0; m < SC / 16; ++m)
-                    mma_f16_ts(d0 + (m / MPG) * NM, a0 + 8 * m,
-                               bd0 + (uint64_t)(((m / 4) * NM * 128 + (m % 4) * 32) >> 4), IDESC, m % MPG != 0);
-                mma_commit_1(&a_empty[as]);
-                mma_commit_1(&b_empty[bs]);
-                mma_commit_1(&d_full[db]);
-                if (++bs == BS) { bs = 0; bph ^= 1u; }
-                if (++as == AS) { as = 0; aph ^= 1u; }
-                if (++db == DB) { db = 0; dph ^= 1u; }
-            }
-            mma_commit_1(drain);                   // every MMA issued has finished when this fires
-            mbar_wait_bounded(drain, 0, &abort_flag, A.timeout_ns);
-        }
-    } else if (warp < PWARPS) {                    // producers: A = (q - z) as bf16 pairs
-        const int q = warp & 3, h = warp >> 2;
-        const int rr = 32 * q + lane;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        constexpr int ngrp = GPS / 2;              // groups of the thread's column half
-        int st = 0, as = 0;
-        uint32_t ph = 0, aph = 0;
-        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-        RowGroups<GPS> zr{A.zeros, A.N, A.n_steps, A.G, rr};
-        zr.begin(rb, j);
-        for (int64_t u = u_begin; u < u_end; ++u) {
-            if (u != u_begin) zr.enter(j);
-            if (!mbar_wait_warp<false>(&full[st], ph, &abort_flag, A.timeout_ns)) break;
-            const uint8_t *stage = base + st * CODE_BYTES;
-            uint4 cw[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                cw[c] = *reinterpret_cast<const uint4 *>(stage + sw128_offset(rr, 4 * h + c));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-            if (++st == CS) { st = 0; ph ^= 1u; }
-            // bf16 pair (128 + z, 128 + z) of each group of the thread's row and column half
-            uint32_t z2[2];
-#pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                const uint32_t zi = gi < ngrp ? (uint32_t)zr.get(rb, j, ngrp == 1 ? h : 2 * h + gi) : 0u;
-                const uint32_t zb = 0x4300u | zi;
-                z2[gi] = zb | (zb << 16);
-            }
-            if (!mbar_wait_warp<false>(&a_empty[as], aph ^ 1u, &abort_flag, A.timeout_ns)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int half8 = 0; half8 < 2; ++half8) {
-                uint32_t v[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int wi = half8 * 8 + i;                      // word of the thread's half
-                    const uint32_t w = word_of(cw, wi);
-                    const uint32_t zz = z2[ngrp == 1 ? 0 : wi / 8];
-                    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-                    const uint32_t pr[4] = {__byte_perm(lo, 0x43434343u, 0x4140u), __byte_perm(lo, 0x43434343u, 0x4342u),
-                                            __byte_perm(hi, 0x43434343u, 0x4140u), __byte_perm(hi, 0x43434343u, 0x4342u)};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const __nv_bfloat162 d = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&pr[c]),
-                                                         *reinterpret_cast<const __nv_bfloat162 *>(&zz));
-                        v[4 * i + c] = *reinterpret_cast<const uint32_t *>(&d);
-                    }
-                }
-                tmem_st_32x32b_x32_sync(tmem + lane_base + as * A_COLS + 64 * h + 32 * half8, v);
-            }
-            tc_fence_before();
-            mbar_arrive(&a_full[as]);
-            if (++as == AS) { as = 0; aph ^= 1u; }
-            if (++j == A.n_steps) {
-                j = 0;
-                ++rb;
-            }
-        }
-    } else {                                       // epilogue: one row per thread, every group of the stage
-        const int q = warp - EWARP0;
-        const int rr = 32 * q + lane;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        float y[TT];
-#pragma unroll
-        for (int t = 0; t < TT; ++t) y[t] = 0.0f;
-        int db = 0;
-        uint32_t dph = 0;
-        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
-        RowGroups<GPS> sr{A.scales, A.N, A.n_steps, A.G, rr};
-        sr.begin(rb, j);
-        for (int64_t u = u_begin; u < u_end; ++u) {
-            if (u != u_begin) sr.enter(j);
-            if (!mbar_wait_warp<false>(&d_full[db], dph, &abort_flag, A.timeout_ns)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int g = 0; g < GPS; ++g) {
-                float dv[NM];
-#pragma unroll
-                for (int c = 0; c < NM; c += 16) {
-                    float pc[16];
-                    tmem_ld_32x32b_x16_sync(tmem + lane_base + AS * A_COLS + db * D_COLS + g * NM + c, pc);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) dv[c + e] = pc[e];
-                }
-                const float shg = sr.get(rb, j, g);
-#pragma unroll
-                for (int t = 0; t < TT; ++t)
-                    y[t] = __fmaf_rn(shg, __fadd_rn(__fadd_rn(dv[3 * t], dv[3 * t + 1]), dv[3 * t + 2]), y[t]);
-            }
-            tc_fence_before();
-            mbar_arrive(&d_empty[db]);
-            if (++db == DB) { db = 0; dph ^= 1u; }
-            if (j == A.n_steps - 1 || u == u_end - 1) {
-                // row block rb's segment ends: Y, or a partial sum and the fixup
-                const int64_t n = rb * ROWS + rr;
-                const int64_t rb_u0 = rb * A.n_steps, rb_u1 = rb_u0 + A.n_steps;
-                if (u_begin <= rb_u0 && u_end >= rb_u1) {
-                    if (n < A.N)
-#pragma unroll
-                        for (int t = 0; t < TT; ++t)
-                            if (t < A.T) A.Y[t * A.N + n] = y[t];
-                } else {
-                    float *mine = A.part + ((rb + blockIdx.x) * ROWS + rr) * TT_MAX;
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) mine[t] = y[t];
-                    __threadfence();
-                    __syncwarp();
-                    const int64_t b0 = block_of(rb_u0, A.units, grid), b1 = block_of(rb_u1 - 1, A.units, grid);
-                    unsigned old = 0;
-                    if (lane == 0) old = atomicAdd(&A.cnt[rb * 4 + q], 1u);
-                    old = __shfl_sync(0xffffffffu, old, 0);
-                    if (old == (unsigned)(b1 - b0)) {
-                        __threadfence();
-                        float tot[TT];
-#pragma unroll
-                        for (int t = 0; t < TT; ++t) tot[t] = 0.0f;
-                        for (int64_t b = b0; b <= b1; ++b)
-#pragma unroll
-                            for (int t = 0; t < TT; ++t)
-                                tot[t] = __fadd_rn(tot[t], __ldcg(A.part + ((rb + b) * ROWS + rr) * TT_MAX + t));
-                        if (n < A.N)
-#pragma unroll
-                            for (int t = 0; t < TT; ++t)
-                                if (t < A.T) A.Y[t * A.N + n] = tot[t];
-                        if (lane == 0) A.cnt[rb * 4 + q] = 0u;
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < TT; ++t) y[t] = 0.0f;
-            }
-            if (++j == A.n_steps) { j = 0; ++rb; }
-        }
-    }
-    if (abort_flag) {
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == MMA_WARP) tmem_dealloc_1(tmem, TMEM_COLS);
-}
-
-// ===========================================================================
 // Quantizer variants and baselines ([AWQ-note] "Measures": RTN, a fixed scale
 // of 2 on the salient channels, and keeping 1% of the channels in FP16,
 // chosen by activation or by weight magnitude).

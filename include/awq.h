@@ -61,8 +61,10 @@ typedef enum {
 /* Quantizer configuration ([QAS-QA] §9 quant_config):
  *   bits        w_bit, one of 2, 3, 4  (codes 0 .. 2^bits - 1)
  *   group_size  q_group_size along K, one of 64, 128
- *   zero_point  1: asymmetric groups with a zero-point code
- *                  (scale = (max w' - min w') / qmax, z = clamp(rint(-min w' / scale)))
+ *   zero_point  1: asymmetric groups with a zero point
+ *                  (scale = (max w' - min w') / qmax, z = round(-min w' / scale), the
+ *                  codes clamped to [0, qmax] but not z: a group that does not span
+ *                  zero has z outside [0, qmax])
  *               0: symmetric absmax groups ([AWQ-note] "Measures": the INT3
  *                  grid of step max|w| / (2^(b-1) - 1)): scale = max|w'| / (2^(bits-1) - 1)
  *                  and the zero fixed at the middle code 2^(bits-1), stored in
@@ -101,7 +103,9 @@ AWQ_API awq_status awq_alpha_scales(const float *a, int64_t K, const float *alph
  *   per row n and group G of group_size columns:
  *     w'    = RN32(w * s)
  *     scale = RN32(RN32(max w' - min w') / qmax),  sh = RN16(clamp(scale, 2^-24, 65504))
- *     r     = RN32(1 / sh),  z = clamp(rint(-min w' * r), 0, qmax)
+ *     r     = RN32(1 / sh),  z = RN16(sat(rint(-min w' * r)))
+ *             (z saturated to +-65504 and rounded to fp16, the format `zeros`
+ *             stores; that stored z is the one used below, and -0 is stored as +0)
  *     q     = clamp(rint(w' * r) + z, 0, qmax)
  *     w_hat = RN16(RN32(RN32((q - z) * sh) * RN32(1 / s)))
  *   (the products inside rint are exact: rint is their only rounding)
@@ -274,7 +278,8 @@ AWQ_API awq_status awq_gptq_quantize(const void *W, int64_t N, int64_t K, const 
  *             c = 2 for bits 2 (16 per word); code of column k at bit c*(k mod 32/c)
  *             of word k/(32/c) (least significant first)
  *   scales    fp16 [N, K/group_size] output: sh per group
- *   zeros     fp16 [N, K/group_size] output: z per group (an integer code)
+ *   zeros     fp16 [N, K/group_size] output: z per group, an integer (outside
+ *             [0, 2^bits - 1] for a group that does not span zero)
  * The argmin runs on the device; nothing is read back to the host.
  * Dequantization: w_hat = RN16(RN32(RN32((code - zero) * scale) * RN32(1/s_best))). */
 AWQ_API awq_status awq_pack(const void *W, int64_t N, int64_t K, const float *a, awq_qcfg q,
@@ -313,9 +318,7 @@ AWQ_API awq_status awq_get_status(void *stream);
  * packed codes from HBM is the cost.  Runs on the CUDA cores, two tokens a
  * pass, each pass re-reading the codes.  The summation order depends on the
  * device's SM count, not on timing: repeated calls on one device give
- * identical Y.  Calls that share a workspace must be ordered (one stream).
- * The workspace size also covers a tensor-core form of the same product
- * that the library builds but does not dispatch at present. */
+ * identical Y.  Calls that share a workspace must be ordered (one stream). */
 AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
 AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
                                const float *s_best, int64_t N, int64_t K, awq_qcfg q,

@@ -64,6 +64,26 @@ def dequantize(q, scales, zeros, s_best, group):
     return (deq * rs[None, :]).astype(np.float32).astype(np.float16)
 
 
+def plant_groups(W, group):
+    """Rows whose groups exercise every branch of the zero point and the code
+    clamp: an all-zero row, a constant group near zero, one-signed rows (zero
+    points below 0 and above qmax), a group far from zero (|zero| > 2048, not
+    every integer an fp16 value), a constant group far from zero (the fp16
+    zero saturates at 65504), and a huge single weight."""
+    plants = [
+        lambda r: r.fill(0),
+        lambda r: r.__setitem__(slice(0, group), np.float16(0.013)),
+        lambda r: r.__setitem__(slice(None), np.abs(r) + np.float16(0.5)),
+        lambda r: r.__setitem__(slice(None), -np.abs(r) - np.float16(0.5)),
+        lambda r: r.__setitem__(5, np.float16(60000.0)),
+        lambda r: r.__setitem__(slice(0, group), np.float16(128.0) + np.abs(r[:group]) * np.float16(8.0)),
+        lambda r: r.__setitem__(slice(group, 2 * group), np.float16(3.0)),
+    ]
+    for n, plant in enumerate(plants[:W.shape[0]]):
+        plant(W[n])
+    return W
+
+
 def assert_alpha_choice(best_gpu, losses_oracle):
     best_o = oracle.argmin(losses_oracle)
     if best_gpu != best_o:
@@ -139,11 +159,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(awq):
 @pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (2, 64), (4, 64), (2, 128)])
 def test_quant_dequant_bit_exact(awq, bits, group):
     W, X = gen(96, 512, 64, bits=bits, group=group, seed=bits * 10 + group)
-    W[0, :] = 0                                  # all-zero row
-    W[1, :group] = np.float16(0.013)             # constant group
-    W[2, :] = np.abs(W[2, :]) + np.float16(0.5)  # all-positive row: zero point clamps to 0
-    W[3, :] = -np.abs(W[3, :]) - np.float16(0.5) # all-negative row: zero point clamps to qmax
-    W[4, 5] = np.float16(60000.0)                # huge outlier weight
+    plant_groups(W, group)
     a = oracle.act_stats(X)
     Wd = dev(W)
     for al in (0.0, 0.25, 0.5, 0.95):
@@ -202,14 +218,11 @@ def test_search_losses(awq, N, K, T, bits, group, seed):
 
 
 def test_search_degenerate_groups(awq):
-    """Rows whose groups need the code clamp (one-signed rows, a constant
-    group, a huge weight), so the producer's clamp path runs."""
+    """Rows whose groups need the code clamp or have zero points outside
+    [0, qmax] (one-signed rows, constant groups, a group far from zero, a huge
+    weight), so the producer's clamp path runs."""
     W, X = gen(160, 512, 600, seed=12, outlier_frac=0.02)
-    W[0, :] = 0
-    W[1, :128] = np.float16(0.013)
-    W[2, :] = np.abs(W[2, :]) + np.float16(0.5)
-    W[3, :] = -np.abs(W[3, :]) - np.float16(0.5)
-    W[4, 5] = np.float16(60000.0)
+    plant_groups(W, 128)
     W[130, :] = np.abs(W[130, :]) + np.float16(0.25)
     alphas = synth.default_alphas()
     a = oracle.act_stats(X)
@@ -250,6 +263,7 @@ def test_search_repeatable_and_workspace_reuse(awq):
                                             (32, 128, 2, 128), (48, 192, 4, 64)])
 def test_pack_bit_exact(awq, N, K, bits, group):
     W, X = gen(N, K, 64, bits=bits, group=group, seed=N + K)
+    plant_groups(W, group)
     a = oracle.act_stats(X)
     alphas = synth.default_alphas()
     rng = np.random.default_rng(N)
@@ -339,6 +353,7 @@ def test_shared_input_joint_search(awq):
                                               (1536, 2048, 16, 4, 128), (700, 1280, 20, 4, 64)])
 def test_qlinear(awq, N, K, T, bits, group):
     W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
+    plant_groups(W, group)
     a = oracle.act_stats(X)
     alphas = synth.default_alphas()
     losses = np.linspace(1.0, 0.5, 20).astype(np.float32)      # chooses alpha = 0.95
@@ -584,6 +599,7 @@ def test_gptq_sweep_bitexact(awq, N, K, bits, group, sym):
     scales, zeros and W_hat bit for bit (K = 4096 and 8192 take the 2-column
     batches, whose first column is not on a 16-byte boundary every time)."""
     W, X = gen(N, K, min(2 * K, 1024), bits=bits, group=group, seed=N + K + 114)
+    plant_groups(W, group)
     a = oracle.act_stats(X)
     s = oracle.scales(a, 0.5)
     U32 = oracle.gptq_factor(oracle.gptq_hessian(X, s)).astype(np.float32)
