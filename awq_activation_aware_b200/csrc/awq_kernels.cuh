@@ -439,7 +439,7 @@ struct Smem {
     uint64_t x_full[XS], x_empty[XS];
     uint64_t a_full[AS], a_empty[AS];
     uint64_t w_full[WS], w_empty[WS];
-    uint64_t acc_full, acc_empty, drain;
+    uint64_t acc_full[NJ], acc_empty[NJ], drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -531,8 +531,10 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             mbar_init(&S.a_empty[i], 1);
         }
         for (int i = 0; i < WS; ++i) { mbar_init(&S.w_full[i], 1); mbar_init(&S.w_empty[i], NUM_PROD_WARPS); }
-        mbar_init(&S.acc_full, 1);
-        mbar_init(&S.acc_empty, 2 * NUM_EPI_WARPS);
+        for (int j = 0; j < NJ; ++j) {
+            mbar_init(&S.acc_full[j], 1);
+            mbar_init(&S.acc_empty[j], 2 * NUM_EPI_WARPS);
+        }
         mbar_init(&S.drain, 1);
         S.abort_flag = 0;
         fence_mbar_init();
@@ -610,31 +612,40 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         if (lane == 0) {
             int xs = 0, as = 0;
             uint32_t xph = 0, aph = 0, accph = 0;
+            // The two accumulators are handed over separately: accumulator j of a
+            // unit is committed right after its last MMAs and reused by the next
+            // unit as soon as the epilogue has drained it, so one accumulator's
+            // drain overlaps the other's MMAs.
             for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
-                if (!mbar_wait_bounded(&S.acc_empty, accph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
-                tc_fence_after();
-                for (int kb = 0; kb < A.n_kb; ++kb) {
+                for (int kb = 0; kb < A.n_kb && !aborted; ++kb) {
                     if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
                         !mbar_wait_bounded(&S.x_full[xs], xph, abort_flag, A.timeout_ns)) { aborted = true; break; }
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(&S.a[as][0]);
                     const uint32_t x_base = smem_u32(&S.x[xs][0]);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
+                    for (int j = 0; j < NJ; ++j) {
+                        if (kb == 0) {
+                            if (!mbar_wait_bounded(&S.acc_empty[j], accph ^ 1u, abort_flag, A.timeout_ns)) {
+                                aborted = true;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
 #pragma unroll
-                        for (int j = 0; j < NJ; ++j) {
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
                             const uint64_t bdesc = sw128_kmajor_desc(x_base + j * X_J_BYTES + kk * 32);
                             mma_f16_ss_pair(tmem + j * BN, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                         }
+                        if (kb + 1 == A.n_kb) mma_commit_pair_mc(&S.acc_full[j], PAIR_MASK);
                     }
+                    if (aborted) break;
                     mma_commit_pair_mc(&S.x_empty[xs], PAIR_MASK);
                     mma_commit_pair_mc(&S.a_empty[as], PAIR_MASK);
                     if (++xs == XS) { xs = 0; xph ^= 1u; }
                     if (++as == AS) { as = 0; aph ^= 1u; }
                 }
-                if (aborted) break;
-                mma_commit_pair_mc(&S.acc_full, PAIR_MASK);
                 accph ^= 1u;
             }
             mma_commit_pair(&S.drain);                  // every pair MMA of this thread done before teardown
@@ -643,29 +654,32 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     } else if (warp < NUM_EPI_WARPS) {
         uint32_t accph = 0;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t acc_empty_l = mapa_shared(smem_u32(&S.acc_empty), 0);
-        for (int64_t u = pair; u < A.n_units; u += npairs) {
+        for (int64_t u = pair; u < A.n_units && !aborted; u += npairs) {
             const UnitIdx ui = unit_index(u, A);
-            if (!mbar_wait_warp(&S.acc_full, accph, abort_flag, A.timeout_ns, 256)) { aborted = true; break; }
-            tc_fence_after();
             float2 sum2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-            for (int c = 0; c < TMEM_COLS; c += 64) {
-                float v[64];
-                tmem_ld_32x32b_x64_sync(tmem + lane_base + c, v);
+            for (int j = 0; j < NJ; ++j) {
+                if (!mbar_wait_warp(&S.acc_full[j], accph, abort_flag, A.timeout_ns, 256)) { aborted = true; break; }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = j * BN; c < (j + 1) * BN; c += 64) {
+                    float v[64];
+                    tmem_ld_32x32b_x64_sync(tmem + lane_base + c, v);
 #pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    const float2 e = make_float2(v[i], v[i + 1]);
-                    sum2 = fma2_rn(e, e, sum2);
+                    for (int i = 0; i < 64; i += 2) {
+                        const float2 e = make_float2(v[i], v[i + 1]);
+                        sum2 = fma2_rn(e, e, sum2);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader) mbar_arrive(&S.acc_empty[j]);
+                    else mbar_arrive_cluster(mapa_shared(smem_u32(&S.acc_empty[j]), 0));
                 }
             }
+            if (aborted) break;
             const float sum = __fadd_rn(sum2.x, sum2.y);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (leader) mbar_arrive(&S.acc_empty);
-                else mbar_arrive_cluster(acc_empty_l);
-            }
             const int64_t n = (int64_t)ui.nb * PM + rank * BM + warp * 32 + lane;
             if (n < A.N) A.partial[((int64_t)ui.alpha * A.n_tb + ui.tb) * A.N + n] = sum;
             accph ^= 1u;

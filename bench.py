@@ -12,6 +12,10 @@ summed over ranks (each rank quantizes its own layer: weak scaling, no
 collective on the data path).  Inputs live in HBM before the timed region and
 L2 is flushed between steps (the layer's W and X fit in the 126 MB L2).
 
+Beside ``value`` the line carries ``layers_per_s`` (whole-job layers per
+second), the search kernel's ``roofline`` and, in ``hbm_kernels``, the warm
+per-launch HBM rates of the statistics and packing kernels.
+
 ``--impl reference`` times the CPU oracle as it stands on this host's cores over
 a bounded row sample of the same layer (rank 0 only).
 """
@@ -52,6 +56,7 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=12)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-hbm", action="store_true", help="skip the warm HBM-kernel rates")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     p.add_argument("--op", choices=["search", "qlinear", "baselines", "gptq"], default="search",
@@ -277,11 +282,63 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(cfg, len(alphas)),
+            "layers_per_s": (rows_n / cfg.N) / t,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def hbm_kernel_rates(awq, torch, cfg, Xd, Wd, s_best, peaks, reps=3):
+    """Warm per-launch rates of the two HBM-bound kernels of the path.
+
+    act_stats (reads X) and pack_kernel (awq_pack_scales: reads W and s_best,
+    writes codes, scales and zeros) each run over a sequence of distinct copies
+    of their input, together more than 4x the 126 MB L2, so every launch reads
+    HBM as a model's layers do; CUDA events bracket each launch on the stream.
+    Bytes are the algorithmic ones (each input byte read once, each output
+    byte written once)."""
+    budget = 512 << 20
+    per = 16 if cfg.bits == 2 else 8
+    x_bytes = cfg.T * cfg.K * 2
+    w_bytes = cfg.N * cfg.K * 2
+    Xs = [Xd.clone() for _ in range(max(2, -(-budget // x_bytes)))]
+    Ws = [Wd.clone() for _ in range(max(2, -(-budget // w_bytes)))]
+    stream = torch.cuda.current_stream()
+
+    def per_launch_s(calls):
+        for fn in calls:
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+        ts = []
+        for _ in range(reps):
+            torch.cuda._sleep(20_000_000)           # the host queues every launch before the first runs
+            for (b, e), fn in zip(evs, calls):
+                b.record(stream)
+                fn()
+                e.record(stream)
+            torch.cuda.synchronize()
+            ts += [b.elapsed_time(e) * 1e-3 for b, e in evs]
+        return statistics.median(ts)
+
+    t_stats = per_launch_s([(lambda x=x: awq.act_stats(x)) for x in Xs])
+    t_pack = per_launch_s([(lambda w=w: awq.pack_scales(w, s_best, cfg.bits, cfg.group)) for w in Ws])
+    awq.get_status()
+    del Xs, Ws
+    hbm = peaks.get("hbm_gbs")
+    stats_bytes = x_bytes + cfg.K * 4
+    pack_bytes = w_bytes + cfg.K * 4 + cfg.N * cfg.K // per * 4 + 2 * cfg.N * (cfg.K // cfg.group) * 2
+
+    def entry(kernel, nbytes, t):
+        gbs = nbytes / t / 1e9
+        return {"kernel": kernel, "us": t * 1e6, "bytes": nbytes, "GBps": gbs,
+                "frac": gbs / hbm if hbm else None}
+    return {"act_stats": entry("act_stats_kernel", stats_bytes, t_stats),
+            "pack": entry("pack_kernel", pack_bytes, t_pack),
+            "peak_GBps": hbm,
+            "how": "median per-launch CUDA-event time over distinct input copies (> 4x L2), warm"}
 
 
 def rank_layer_config(base, rank):
@@ -349,6 +406,9 @@ def run_awq(args):
         sampler.start()
     torch.cuda.synchronize()
     barrier(world)
+    # a GPU-side pause lets the host queue the steps ahead of the device, so no
+    # step waits on the host's launch calls (the pause is outside every event pair)
+    torch.cuda._sleep(40_000_000)
     for i in range(K):
         flush.zero_()
         ev[i][0].record(stream)
@@ -440,6 +500,10 @@ def run_awq(args):
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "overlap": "double-buffered: H2D and D2H on their own streams, overlapping compute"}
 
+    hbm_rates = None
+    if not args.no_hbm:
+        hbm_rates = hbm_kernel_rates(awq, torch, cfg, Xd, Wd, out["s_best"], peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cv, dt, rows_n = cpu_measure(cfg, W, X, alphas_np, args)
@@ -452,9 +516,10 @@ def run_awq(args):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-                "config": config_dict(cfg, n_alpha, {"parallelism": f"{world} independent layers"
-                                                     if world > 1 else "1 GPU"}),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "config": config_dict(cfg, n_alpha),
+                "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "1 GPU",
+                "layers_per_s": world / (ms_per_step * 1e-3),
+                "roofline": roofline, "hbm_kernels": hbm_rates, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": LAUNCHES_PER_STEP * K, "clocks": clocks,
                 "pct_of_peak": 100.0 * value / peak}
         print(json.dumps(line), flush=True)
