@@ -72,6 +72,7 @@ def lib():
     L.awq_search_workspace_bytes.argtypes = [i64, i64, i64, QCfg, i32]
     L.awq_search_workspace_bytes.restype = ctypes.c_size_t
     L.awq_search_layer.argtypes = [P, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P, ctypes.c_size_t, P]
+    L.awq_search_layer_part.argtypes = [P, i64, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P, ctypes.c_size_t, P]
     L.awq_pack.argtypes = [P, i64, i64, P, QCfg, P, P, i32, P, P, P, P, P, P]
     L.awq_get_status.argtypes = [P]
     L.awq_set_wait_timeout_ms.argtypes = [ctypes.c_uint32]
@@ -171,11 +172,15 @@ def search_workspace_bytes(N, K, T, bits=4, group=128, n_alpha=20, zero_point=Tr
 
 def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torch.Tensor, bits: int = 4,
                  group: int = 128, workspace: torch.Tensor | None = None, row_losses: bool = False,
-                 losses_out: torch.Tensor | None = None, stream=None, zero_point: bool = True):
+                 losses_out: torch.Tensor | None = None, stream=None, zero_point: bool = True,
+                 rows_total: int | None = None):
     """Per-alpha MSE of the layer output, ||(W_hat_alpha - W) X^T||^2 / (N T).
 
     Returns ``losses`` (float32 [n_alpha]) or ``(losses, row_losses)`` with
-    row_losses float32 [n_alpha, N] holding unnormalised per-row sums."""
+    row_losses float32 [n_alpha, N] holding unnormalised per-row sums.  With
+    ``rows_total``, W is one part of a layer of that many rows and the losses
+    are normalised by rows_total T (awq_search_layer_part): the parts' losses
+    add up to the layer's."""
     _rowmajor(X, "X")
     if not W.is_contiguous():
         raise ValueError("W must be contiguous")
@@ -187,12 +192,15 @@ def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torc
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     losses = losses_out if losses_out is not None else torch.empty(n, dtype=torch.float32, device=W.device)
     rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
-    _check(lib().awq_search_layer(
-        _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X"), T, X.stride(0),
-        _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point), _dev(alphas, torch.float32, "alphas"), n,
-        _dev(losses, torch.float32, "losses"),
-        _dev(rl, torch.float32, "row_losses") if rl is not None else None,
-        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)), "awq_search_layer")
+    rest = (_dev(X, torch.float16, "X"), T, X.stride(0), _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point),
+            _dev(alphas, torch.float32, "alphas"), n, _dev(losses, torch.float32, "losses"),
+            _dev(rl, torch.float32, "row_losses") if rl is not None else None,
+            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    if rows_total is None:
+        _check(lib().awq_search_layer(_dev(W, torch.float16, "W"), N, K, *rest), "awq_search_layer")
+    else:
+        _check(lib().awq_search_layer_part(_dev(W, torch.float16, "W"), N, int(rows_total), K, *rest),
+               "awq_search_layer_part")
     return (losses, rl) if row_losses else losses
 
 

@@ -109,6 +109,8 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -246,17 +248,21 @@ size_t qlinear_ws(int64_t T, int64_t K, int64_t N) { return qlinear_ws_simt(T, K
 // a8 for a given s: codes, fp16 scales and zeros.
 awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, uint32_t *codes,
                        void *scales, void *zeros, cudaStream_t st) {
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
     const int G = (int)(K / q.group_size);
-    const int lpr = q.group_size / awq::kGpCols;
     const int sym = q.zero_point ? 0 : 1;
-    const int64_t rows_per_block = awq::kGpThreads / lpr;
-    const unsigned grid = (unsigned)(((N + rows_per_block - 1) / rows_per_block) * G);
-    if (lpr == 2)
-        awq::pack_kernel<2><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s, codes,
-                                                             (__half *)scales, (__half *)zeros);
+    // one warp per item of 8 rows x 256 columns, at most 8 blocks per SM (the rest loop)
+    const int64_t items = (N + awq::kPkRows - 1) / awq::kPkRows * ((K + awq::kPkCols - 1) / awq::kPkCols);
+    const int64_t warps_per_block = awq::kPkThreads / 32;
+    int64_t grid = (items + warps_per_block - 1) / warps_per_block;
+    if (grid > 8 * (int64_t)d.sms) grid = 8 * (int64_t)d.sms;
+    if (q.group_size == 128)
+        awq::pack_kernel<16><<<(unsigned)grid, awq::kPkThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s,
+                                                                        codes, (__half *)scales, (__half *)zeros);
     else
-        awq::pack_kernel<1><<<grid, awq::kGpThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s, codes,
-                                                             (__half *)scales, (__half *)zeros);
+        awq::pack_kernel<8><<<(unsigned)grid, awq::kPkThreads, 0, st>>>((const __half *)W, N, K, G, q.bits, sym, s,
+                                                                       codes, (__half *)scales, (__half *)zeros);
     return last_launch();
 }
 
@@ -264,21 +270,24 @@ awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_
 // parameters, the tensor-core search against X, the loss reduction.
 awq_status run_search(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, int group,
                       float qmax, const float *s_tab, const float *rs_tab, int n_alpha, const uint2 *params,
-                      float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st);
+                      float *partial, float *losses, float *row_losses, int64_t norm_rows, const DevInfo &d,
+                      cudaStream_t st);
 
 awq_status search_core(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, awq_qcfg q,
                        const float *s_tab, const float *rs_tab, int n_alpha, const uint8_t *mask, uint2 *params,
-                       float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st) {
+                       float *partial, float *losses, float *row_losses, int64_t norm_rows, const DevInfo &d,
+                       cudaStream_t st) {
     // a3 (group parameters for every alpha)
     if (awq_status e = launch_group_params(W, N, K, q, s_tab, n_alpha, mask, params, st)) return e;
     return run_search(W, N, K, X, T, ldx, q.group_size, (float)((1 << q.bits) - 1), s_tab, rs_tab, n_alpha, params,
-                      partial, losses, row_losses, d, st);
+                      partial, losses, row_losses, norm_rows, d, st);
 }
 
 // a4-a6 with the group parameters already in the workspace.
 awq_status run_search(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx, int group,
                       float qmax, const float *s_tab, const float *rs_tab, int n_alpha, const uint2 *params,
-                      float *partial, float *losses, float *row_losses, const DevInfo &d, cudaStream_t st) {
+                      float *partial, float *losses, float *row_losses, int64_t norm_rows, const DevInfo &d,
+                      cudaStream_t st) {
     // a4-a6: the tensor-core search on CTA pairs
     CUtensorMap tmap_x, tmap_w;
     if (!encode_rows_map(&tmap_x, X, T, K, ldx, awq::srch2::HN) ||
@@ -311,7 +320,8 @@ awq_status run_search(const void *W, int64_t N, int64_t K, const void *X, int64_
     if (pe && cudaEventRecord(pe, st) != cudaSuccess) return AWQ_ERR_CUDA;
 
     // a6: deterministic reduction to per-alpha MSE (and optional per-row sums)
-    awq::loss_reduce_kernel<<<n_alpha, awq::kLossThreads, 0, st>>>(partial, N, T, A.n_tb, losses, row_losses);
+    awq::loss_reduce_kernel<<<n_alpha, awq::kLossThreads, 0, st>>>(partial, N, T, A.n_tb, norm_rows, losses,
+                                                                   row_losses);
     return last_launch();
 }
 
@@ -395,7 +405,15 @@ size_t awq_search_workspace_bytes(int64_t N, int64_t K, int64_t T, awq_qcfg q, i
 awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, int64_t T, int64_t ldx,
                             const float *a, awq_qcfg q, const float *alphas, int32_t n_alpha, float *losses,
                             float *row_losses, void *ws, size_t ws_bytes, void *stream) {
+    return awq_search_layer_part(W, N, N, K, X, T, ldx, a, q, alphas, n_alpha, losses, row_losses, ws, ws_bytes,
+                                 stream);
+}
+
+awq_status awq_search_layer_part(const void *W, int64_t N, int64_t rows_total, int64_t K, const void *X, int64_t T,
+                                 int64_t ldx, const float *a, awq_qcfg q, const float *alphas, int32_t n_alpha,
+                                 float *losses, float *row_losses, void *ws, size_t ws_bytes, void *stream) {
     if (!W || !X || !a || !alphas || !losses) return AWQ_ERR_INVALID_ARG;
+    if (rows_total < N || rows_total > kMaxDim) return AWQ_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(X) || !aligned16(a) || !aligned16(alphas) || !aligned16(losses) ||
         (row_losses && !aligned16(row_losses)))
         return AWQ_ERR_INVALID_ARG;
@@ -421,7 +439,7 @@ awq_status awq_search_layer(const void *W, int64_t N, int64_t K, const void *X, 
         if (awq_status e = last_launch()) return e;
     }
     return search_core(W, N, K, X, T, ldx, q, s_tab, rs_tab, n_alpha, nullptr, params, partial, losses, row_losses,
-                       d, st);
+                       rows_total, d, st);
 }
 
 
@@ -481,7 +499,8 @@ awq_status awq_search_scales(const void *W, int64_t N, int64_t K, const void *X,
         Xs = Xm;
         ld = K;
     }
-    return search_core(W, N, K, Xs, T, ld, q, s_tab, rs_tab, n_s, mask, params, partial, losses, row_losses, d, st);
+    return search_core(W, N, K, Xs, T, ld, q, s_tab, rs_tab, n_s, mask, params, partial, losses, row_losses, N, d,
+                       st);
 }
 
 awq_status awq_salient_scales(const uint8_t *mask, int64_t K, float factor, float *s, void *stream) {
@@ -530,7 +549,7 @@ awq_status awq_output_error(const void *W, const void *W_hat, int64_t N, int64_t
     awq::fill_kernel<<<blocks_for(K, 256), 256, 0, st>>>(s_tab, K, 1.0f);
     awq::fill_kernel<<<blocks_for(K, 256), 256, 0, st>>>(rs_tab, K, 1.0f);
     if (awq_status e = last_launch()) return e;
-    return run_search(dW, N, K, X, T, ldx, 64, 0.0f, s_tab, rs_tab, 1, params, partial, loss, row_losses, d, st);
+    return run_search(dW, N, K, X, T, ldx, 64, 0.0f, s_tab, rs_tab, 1, params, partial, loss, row_losses, N, d, st);
 }
 
 awq_status awq_gptq_hessian(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s, float *H, void *stream) {
@@ -727,7 +746,9 @@ awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *ze
     A.units = row_blocks * A.n_steps;
     A.gps = (int)(sc / q.group_size);
     A.sz_mode = A.G % 8 == 0 ? 16 : (A.G % 2 == 0 ? 4 : 2);
-    const int tt = T == 1 ? 1 : 2;
+    // tokens per pass: 1, 2, or 4 (every pass reads the codes once; a last pass
+    // with fewer tokens reads the zero rows that pad x')
+    const int tt = T == 1 ? 1 : (T == 2 || c2) ? 2 : awq::qlv::TOKENS;   // 2-bit words: at most 2 tokens
     A.n_stages = awq::qlv::ring_stages((int)sc, tt, A.gps);
     const size_t smem = (size_t)A.n_stages * awq::qlv::stage_bytes((int)sc, tt, A.gps) + awq::qlv::fixed_smem();
     A.part = part;
@@ -736,16 +757,15 @@ awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *ze
     // one block per SM, each streaming an equal share of the units
     int64_t grid = d.sms < kQlMaxGrid ? d.sms : kQlMaxGrid;
     if (grid > A.units) grid = A.units;
-    for (int64_t t0 = 0; t0 < T; t0 += awq::qlv::TOKENS) {
+    for (int64_t t0 = 0; t0 < T; t0 += tt) {
         A.xs = xs + t0 * Kp;
         A.Y = Y + t0 * N;
-        A.T = (int)(T - t0 < awq::qlv::TOKENS ? T - t0 : awq::qlv::TOKENS);
-        // one token alone takes the single-token kernel; an odd last token of a
-        // longer batch reads the zero row that pads x'
+        A.T = (int)(T - t0 < tt ? T - t0 : tt);
 #define AWQ_QL_LAUNCH(CB, TT) \
     awq::qlinear_gemv_kernel<CB, TT><<<(unsigned)grid, awq::qlv::THREADS, smem, st>>>(tmap, A)
-        if (T == 1) { if (c2) AWQ_QL_LAUNCH(2, 1); else AWQ_QL_LAUNCH(4, 1); }
-        else { if (c2) AWQ_QL_LAUNCH(2, 2); else AWQ_QL_LAUNCH(4, 2); }
+        if (tt == 1) { if (c2) AWQ_QL_LAUNCH(2, 1); else AWQ_QL_LAUNCH(4, 1); }
+        else if (tt == 2) { if (c2) AWQ_QL_LAUNCH(2, 2); else AWQ_QL_LAUNCH(4, 2); }
+        else AWQ_QL_LAUNCH(4, 4);
 #undef AWQ_QL_LAUNCH
         if (awq_status e = last_launch()) return e;
     }

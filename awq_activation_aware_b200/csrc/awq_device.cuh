@@ -190,6 +190,52 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
     return v;
 }
 
+// Sixteen streaming 16-byte loads at p, p + stride, ..., p + 15 stride (bytes),
+// issued back to back from one asm statement, so all sixteen are in flight
+// before any result is used.
+__device__ __forceinline__ void ldg_stream_v4x16(const void *p, int64_t stride, uint4 (&v)[16]) {
+    uint32_t r[64];
+    asm volatile(
+        "{\n\t.reg .b64 a;\n\t"
+        "mov.b64 a, %64;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%4, %5, %6, %7}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%8, %9, %10, %11}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%12, %13, %14, %15}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%16, %17, %18, %19}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%20, %21, %22, %23}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%24, %25, %26, %27}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%28, %29, %30, %31}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%32, %33, %34, %35}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%36, %37, %38, %39}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%40, %41, %42, %43}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%44, %45, %46, %47}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%48, %49, %50, %51}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%52, %53, %54, %55}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%56, %57, %58, %59}, [a];\n\t"
+        "add.s64 a, a, %65;\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%60, %61, %62, %63}, [a];\n\t"
+        "}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "l"(p), "l"(stride));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+}
+
 // ----- mbarrier -------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -38,22 +38,34 @@ namespace cg = cooperative_groups;
 //
 // A cluster of 8 CTAs owns a slab of 64 columns; each CTA reads every 8th
 // group of 32 rows with 16-byte loads (8 threads cover one 128-byte row
-// segment), accumulates |x| in binary64 -- exact, since every fp16 value is a
-// multiple of 2^-24 and the sums stay below 2^29 -- reduces its 16 row lanes
-// in shared memory, and CTA 0 of the cluster sums the 8 partial vectors
-// through distributed shared memory.  No workspace, one launch.
+// segment, 16 loads issued per batch), accumulates |x| in binary64 -- exact,
+// since every fp16 value is a multiple of 2^-24 and the sums stay below 2^29,
+// so the order of the additions cannot change them -- reduces its row lanes
+// by warp shuffles and shared memory, and CTA 0 of the cluster sums the 8
+// partial vectors through distributed shared memory.  No workspace, one launch.
 // ===========================================================================
 constexpr int kStatsCols = 64;
 constexpr int kStatsTPR = 8;                       // threads per row segment (128 bytes)
 constexpr int kStatsThreads = 256;
+constexpr int kStatsWarps = kStatsThreads / 32;
 constexpr int kStatsRowsPerCta = kStatsThreads / kStatsTPR;   // 32
 constexpr int kStatsCluster = 8;
-constexpr int kStatsUnroll = 8;
+constexpr int kStatsUnroll = 16;                   // loads per batch
+
+__device__ __forceinline__ void stats_accumulate(const uint4 &v, double (&acc)[8]) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(__habs2(h[e]));
+        acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
+        acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
+    }
+}
 
 __global__ void __cluster_dims__(kStatsCluster, 1, 1) __launch_bounds__(kStatsThreads)
 act_stats_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx,
                  float *__restrict__ a) {
-    __shared__ double red[kStatsRowsPerCta][kStatsCols + 1];
+    __shared__ double red[kStatsWarps][kStatsCols];
     __shared__ double part[kStatsCols];
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -70,39 +82,31 @@ act_stats_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx
     int64_t t = (int64_t)rank * kStatsRowsPerCta + rl;
     if (active) {
         for (; t + (kStatsUnroll - 1) * rstride < T; t += kStatsUnroll * rstride) {
+            static_assert(kStatsUnroll == 16, "one batch is one ldg_stream_v4x16");
             uint4 v[kStatsUnroll];
+            ldg_stream_v4x16(X + t * ldx + col0, rstride * ldx * 2, v);
 #pragma unroll
-            for (int u = 0; u < kStatsUnroll; ++u)
-                v[u] = ldg_stream_v4(X + (t + u * rstride) * ldx + col0);
-#pragma unroll
-            for (int u = 0; u < kStatsUnroll; ++u) {
-                const __half2 *h = reinterpret_cast<const __half2 *>(&v[u]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 f = __half22float2(__habs2(h[e]));
-                    acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
-                    acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
-                }
-            }
+            for (int u = 0; u < kStatsUnroll; ++u) stats_accumulate(v[u], acc);
         }
-        for (; t < T; t += rstride) {
-            uint4 v = ldg_stream_v4(X + t * ldx + col0);
-            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float2 f = __half22float2(__habs2(h[e]));
-                acc[2 * e] = __dadd_rn(acc[2 * e], (double)f.x);
-                acc[2 * e + 1] = __dadd_rn(acc[2 * e + 1], (double)f.y);
-            }
-        }
+        for (; t < T; t += rstride) stats_accumulate(ldg_stream_v4(X + t * ldx + col0), acc);
     }
+    // the warp's 4 row lanes by shuffles, the 8 warps in shared memory, the
+    // cluster's 8 CTAs through distributed shared memory
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[rl][cc * 8 + e] = acc[e];
+    for (int e = 0; e < 8; ++e) {
+        acc[e] = __dadd_rn(acc[e], __shfl_xor_sync(0xffffffffu, acc[e], 8));
+        acc[e] = __dadd_rn(acc[e], __shfl_xor_sync(0xffffffffu, acc[e], 16));
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) < kStatsTPR) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[warp][cc * 8 + e] = acc[e];
+    }
     __syncthreads();
     if (threadIdx.x < kStatsCols) {
         double s = 0.0;
 #pragma unroll
-        for (int r = 0; r < kStatsRowsPerCta; ++r) s = __dadd_rn(s, red[r][threadIdx.x]);
+        for (int w = 0; w < kStatsWarps; ++w) s = __dadd_rn(s, red[w][threadIdx.x]);
         part[threadIdx.x] = s;
     }
     cluster.sync();
@@ -165,19 +169,23 @@ __device__ __forceinline__ void load_row64(const __half *src, float (&w)[kGpCols
     }
 }
 
-// min and max of w[k] * s[k] over the lane's 64 columns (s in shared memory).
+// min and max of w[k] * s[k] over the lane's 64 columns (s in shared memory),
+// in four independent chains so that consecutive min/max operations do not
+// wait on one another (min and max are exact, so the grouping is free).
 __device__ __forceinline__ void minmax64(const float (&w)[kGpCols], const float *s_sm, float &mn, float &mx) {
-    float lo = INFINITY, hi = -INFINITY;
+    float lo[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+    float hi[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int q = 0; q < kGpCols / 4; ++q) {
         const float4 sv = *reinterpret_cast<const float4 *>(s_sm + 4 * q);
         const float2 p0 = mul2_rn(make_float2(w[4 * q], w[4 * q + 1]), make_float2(sv.x, sv.y));
         const float2 p1 = mul2_rn(make_float2(w[4 * q + 2], w[4 * q + 3]), make_float2(sv.z, sv.w));
-        lo = fmin3(lo, fminf(p0.x, p0.y), fminf(p1.x, p1.y));
-        hi = fmax3(hi, fmaxf(p0.x, p0.y), fmaxf(p1.x, p1.y));
+        // two three-input operations per four products and per bound
+        lo[q & 3] = fmin3(fmin3(lo[q & 3], p0.x, p0.y), p1.x, p1.y);
+        hi[q & 3] = fmax3(fmax3(hi[q & 3], p0.x, p0.y), p1.x, p1.y);
     }
-    mn = lo;
-    mx = hi;
+    mn = fminf(fmin3(lo[0], lo[1], lo[2]), lo[3]);
+    mx = fmaxf(fmax3(hi[0], hi[1], hi[2]), hi[3]);
 }
 
 // The same over the channels not held in fp16 (keep: one flag byte per column
@@ -196,7 +204,7 @@ __device__ __forceinline__ void minmax64_kept(const float (&w)[kGpCols], const f
 }
 
 template <int LPR>   // lanes per row = group_size / 64
-__global__ void __launch_bounds__(kGpThreads)
+__global__ void __launch_bounds__(kGpThreads, 3)
 group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int64_t K, int G,
                     const float *__restrict__ s_tab, int n_alpha, float qmax, int sym,
                     const uint8_t *__restrict__ mask, uint2 *__restrict__ params) {
@@ -224,20 +232,43 @@ group_params_kernel(const __half *__restrict__ W, int64_t N, int64_t N_pad, int6
 #pragma unroll
         for (int e = 0; e < kGpCols; ++e) w[e] = 0.0f;
     }
-    for (int ai = 0; ai < n_alpha; ++ai) {
-        float mn, mx;
-        if (mask)
-            minmax64_kept(w, s_sm + (ai * LPR + half) * kStride, keep_sm + half * kGpCols, mn, mx);
-        else
-            minmax64(w, s_sm + (ai * LPR + half) * kStride, mn, mx);
-        if (LPR == 2) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    // two alphas per iteration: their chains (products, min/max, the divide and
+    // reciprocal of the parameters) are independent and interleave
+    for (int a0 = 0; a0 < n_alpha; a0 += 2) {
+        const int na = n_alpha - a0 < 2 ? 1 : 2;
+        float mn[2], mx[2];
+#pragma unroll
+        for (int d = 0; d < 2; ++d) {
+            const int ai = d < na ? a0 + d : a0;
+            if (mask)
+                minmax64_kept(w, s_sm + (ai * LPR + half) * kStride, keep_sm + half * kGpCols, mn[d], mx[d]);
+            else
+                minmax64(w, s_sm + (ai * LPR + half) * kStride, mn[d], mx[d]);
         }
-        if (mn > mx) { mn = 0.0f; mx = 0.0f; }          // every channel of the group kept in fp16
-        if (half == 0 && n < N_pad)
-            params[((int64_t)ai * G + grp) * N_pad + n] = active ? pack_qparams(make_qparams(mn, mx, qmax, sym != 0))
-                                                                 : make_uint2(0, 0);
+#pragma unroll
+        for (int d = 0; d < 2; ++d) {
+            if (LPR == 2) {
+                mn[d] = fminf(mn[d], __shfl_xor_sync(0xffffffffu, mn[d], 1));
+                mx[d] = fmaxf(mx[d], __shfl_xor_sync(0xffffffffu, mx[d], 1));
+            }
+            if (mn[d] > mx[d]) { mn[d] = 0.0f; mx[d] = 0.0f; }   // every channel of the group kept in fp16
+        }
+        if (LPR == 2) {
+            // the row's two lanes share the work: lane `half` derives and stores alpha a0 + half
+            const float lo_ = half ? mn[1] : mn[0], hi_ = half ? mx[1] : mx[0];
+            const uint2 v = active ? pack_qparams(make_qparams(lo_, hi_, qmax, sym != 0)) : make_uint2(0, 0);
+            if (half < na && n < N_pad) params[((int64_t)(a0 + half) * G + grp) * N_pad + n] = v;
+        } else {
+            uint2 v[2];
+#pragma unroll
+            for (int d = 0; d < 2; ++d)
+                v[d] = active ? pack_qparams(make_qparams(mn[d], mx[d], qmax, sym != 0)) : make_uint2(0, 0);
+            if (n < N_pad) {
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+                    if (d < na) params[((int64_t)(a0 + d) * G + grp) * N_pad + n] = v[d];
+            }
+        }
     }
 }
 
@@ -746,12 +777,13 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 
 // ===========================================================================
 // a6 (reduction). losses[i] = RN32(sum over token blocks and rows of the
-// partials, in binary64 and a fixed order, / (N T)); optional per-row sums.
-// One block per alpha.
+// partials, in binary64 and a fixed order, / (R T)), R = N for a whole layer
+// or the layer's row count when these N rows are one part of it; optional
+// per-row sums.  One block per alpha.
 // ===========================================================================
 constexpr int kLossThreads = 1024;
 __global__ void __launch_bounds__(kLossThreads)
-loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int n_tb,
+loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int n_tb, int64_t norm_rows,
                    float *__restrict__ losses, float *__restrict__ row_losses) {
     const int ai = blockIdx.x;
     const float *p = partial + (int64_t)ai * n_tb * N;
@@ -779,7 +811,7 @@ loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int 
         if ((int)threadIdx.x < off) red[threadIdx.x] = __dadd_rn(red[threadIdx.x], red[threadIdx.x + off]);
         __syncthreads();
     }
-    if (threadIdx.x == 0) losses[ai] = __double2float_rn(red[0] / ((double)N * (double)T));
+    if (threadIdx.x == 0) losses[ai] = __double2float_rn(red[0] / ((double)norm_rows * (double)T));
 }
 
 // ===========================================================================
@@ -821,83 +853,138 @@ __global__ void best_scale_kernel(const float *__restrict__ a, int64_t K,
 // a8. Pack: per (row, group) recompute w' = RN32(w s_best), the group's
 // parameters and every code; store codes LSB-first, the fp16 scale and zero
 // ([AWQ-note] "Measures": keep the quantized weights and their metadata).
-// Same layout as group_params_kernel: a block owns one column group and
-// 128 / LPR rows, a lane holds 64 consecutive weights, s_best is staged in
-// shared memory.  A lane's 64 codes are 8 words of 4-bit containers
-// (w_bit 3/4) or 4 words of 2-bit containers (w_bit 2).
+// A warp takes items of 8 rows x 256 columns; lane l holds columns 8l..8l+7
+// of each row, so every load instruction of the warp reads 512 contiguous
+// bytes of one row and every code store writes the row's words contiguously.
+// A group of g columns is GL = g/8 neighbouring lanes.  Its min and max go
+// through a reduce-scatter over those lanes (lane i of a group ends with row
+// i mod 8's values), each lane computes the parameters of that one row, and
+// the lanes of the group read them back by shuffles.  HBM-bound: W is read
+// once, codes, scales and zeros are written once.
 // ===========================================================================
-template <int LPR>
-__global__ void __launch_bounds__(kGpThreads)
+constexpr int kPkThreads = 256;
+constexpr int kPkRows = 8;               // rows per warp item
+constexpr int kPkCols = 256;             // columns per warp item (8 per lane)
+
+// min over the GL lanes of this lane's group of v[i], for i = this lane's row
+// (lane index within the group mod 8); max likewise.
+template <int GL>
+__device__ __forceinline__ void group_reduce_scatter(float (&lo)[kPkRows], float (&hi)[kPkRows], float &mn, float &mx) {
+    const int gl = threadIdx.x & (GL - 1);
+#pragma unroll
+    for (int half = kPkRows / 2; half >= 1; half >>= 1) {
+        const bool upper = (gl & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float slo = upper ? lo[i] : lo[i + half], shi = upper ? hi[i] : hi[i + half];
+            const float klo = upper ? lo[i + half] : lo[i], khi = upper ? hi[i + half] : hi[i];
+            lo[i] = fminf(klo, __shfl_xor_sync(0xffffffffu, slo, half));
+            hi[i] = fmaxf(khi, __shfl_xor_sync(0xffffffffu, shi, half));
+        }
+    }
+    mn = lo[0];
+    mx = hi[0];
+    if (GL == 16) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    }
+}
+
+template <int GL>   // lanes per group = group_size / 8
+__global__ void __launch_bounds__(kPkThreads)
 pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits, int sym,
             const float *__restrict__ s_best, uint32_t *__restrict__ codes,
             __half *__restrict__ scales, __half *__restrict__ zeros) {
-    __shared__ __align__(16) float s_sm[LPR * (kGpCols + 4)];
-    constexpr int kRowsPerBlock = kGpThreads / LPR;
-    constexpr int kStride = kGpCols + 4;
-    const int grp = blockIdx.x % G;
-    const int64_t n0 = (int64_t)(blockIdx.x / G) * kRowsPerBlock;
-    const int64_t k0 = (int64_t)grp * (kGpCols * LPR);
-    for (int i = threadIdx.x; i < LPR * kGpCols; i += kGpThreads)
-        s_sm[(i / kGpCols) * kStride + i % kGpCols] = __ldg(s_best + k0 + i);
-    __syncthreads();
-    const int half = threadIdx.x % LPR;
-    const int64_t n = n0 + threadIdx.x / LPR;
-    const bool active = n < N;
+    const int lane = threadIdx.x & 31;
+    const int gl = lane & (GL - 1);
+    const int gbase = lane & ~(GL - 1);
     const float qmax = (float)((1 << bits) - 1);
-    float w[kGpCols];
-    if (active) {
-        load_row64(W + n * K + k0 + half * kGpCols, w);
-    } else {
+    const int64_t n_ct = (K + kPkCols - 1) / kPkCols;
+    const int64_t n_items = (N + kPkRows - 1) / kPkRows * n_ct;
+    const int64_t wid = ((int64_t)blockIdx.x * kPkThreads + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * kPkThreads) >> 5;
+    for (int64_t item = wid; item < n_items; item += n_warps) {
+        const int64_t rb = item / n_ct, ct = item - rb * n_ct;
+        const int64_t n0 = rb * kPkRows;
+        const int64_t col = ct * kPkCols + lane * 8;
+        const bool colok = col < K;           // K is a multiple of the group: whole groups are in or out
+        uint4 raw[kPkRows];
 #pragma unroll
-        for (int e = 0; e < kGpCols; ++e) w[e] = 0.0f;
-    }
-    const float *sp = s_sm + half * kStride;
+        for (int r = 0; r < kPkRows; ++r)
+            raw[r] = (colok && n0 + r < N) ? ldg_stream_v4(W + (n0 + r) * K + col) : make_uint4(0u, 0u, 0u, 0u);
+        float sv[8];
+        if (colok) {
+            const float4 s0 = __ldg(reinterpret_cast<const float4 *>(s_best + col));
+            const float4 s1 = __ldg(reinterpret_cast<const float4 *>(s_best + col + 4));
+            sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+            sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+        } else {
 #pragma unroll
-    for (int q = 0; q < kGpCols / 4; ++q) {
-        const float4 sv = *reinterpret_cast<const float4 *>(sp + 4 * q);
-        const float2 p0 = mul2_rn(make_float2(w[4 * q], w[4 * q + 1]), make_float2(sv.x, sv.y));
-        const float2 p1 = mul2_rn(make_float2(w[4 * q + 2], w[4 * q + 3]), make_float2(sv.z, sv.w));
-        w[4 * q] = p0.x; w[4 * q + 1] = p0.y; w[4 * q + 2] = p1.x; w[4 * q + 3] = p1.y;   // now w'
-    }
-    float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < kGpCols; e += 2) {
-        mn = fmin3(mn, w[e], w[e + 1]);
-        mx = fmax3(mx, w[e], w[e + 1]);
-    }
-    if (LPR == 2) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    }
-    const QParams p = make_qparams(mn, mx, qmax, sym != 0);
-    if (!active) return;
-    const int64_t col = k0 + half * kGpCols;
-    if (bits == 2) {
-        uint32_t word[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v |= quant_code(w[16 * j + e], p, qmax, p.clamp) << (2 * e);
-            word[j] = v;
+            for (int e = 0; e < 8; ++e) sv[e] = 1.0f;
         }
-        *reinterpret_cast<uint4 *>(codes + n * (K / 16) + col / 16) = make_uint4(word[0], word[1], word[2], word[3]);
-    } else {
-        uint32_t word[8];
+        float wp[kPkRows][8];                  // w' = RN32(w s)
+        float lo[kPkRows], hi[kPkRows];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            uint32_t v = 0;
+        for (int r = 0; r < kPkRows; ++r) {
+            const __half2 *h = reinterpret_cast<const __half2 *>(&raw[r]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v |= quant_code(w[8 * j + e], p, qmax, p.clamp) << (4 * e);
-            word[j] = v;
+            for (int e = 0; e < 4; ++e) {
+                const float2 p = mul2_rn(__half22float2(h[e]), make_float2(sv[2 * e], sv[2 * e + 1]));
+                wp[r][2 * e] = p.x;
+                wp[r][2 * e + 1] = p.y;
+            }
+            lo[r] = fminf(fmin3(fmin3(wp[r][0], wp[r][1], wp[r][2]), fmin3(wp[r][3], wp[r][4], wp[r][5]), wp[r][6]), wp[r][7]);
+            hi[r] = fmaxf(fmax3(fmax3(wp[r][0], wp[r][1], wp[r][2]), fmax3(wp[r][3], wp[r][4], wp[r][5]), wp[r][6]), wp[r][7]);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(codes + n * (K / 8) + col / 8);
-        dst[0] = make_uint4(word[0], word[1], word[2], word[3]);
-        dst[1] = make_uint4(word[4], word[5], word[6], word[7]);
-    }
-    if (half == 0) {
-        scales[n * G + grp] = __float2half_rn(p.sh);
-        zeros[n * G + grp] = __float2half_rn(p.z);
+        float mn, mx;
+        group_reduce_scatter<GL>(lo, hi, mn, mx);
+        // this lane's row of its group: gl mod 8
+        const QParams mine = make_qparams(mn, mx, qmax, sym != 0);
+        const uint2 mine_p = pack_qparams(mine);
+        const int64_t grp = col / (GL * 8);
+        // Codes packed by integer multiply-adds: with v_e = RN32(w'_e r + kMagic)
+        // (clamped when the group needs it), q_e = bits(v_e) - base, base =
+        // bits(kMagic) - z, and the word sum_e q_e B^e (B = 16 or 4) equals
+        // sum_e bits(v_e) B^e - base sum_e B^e modulo 2^32 -- exact, since the
+        // word itself fits in 32 bits.
+        const uint32_t B = bits == 2 ? 4u : 16u;
+        const uint32_t geom = bits == 2 ? 0x5555u : 0x11111111u;      // sum_{e<8} B^e
+#pragma unroll
+        for (int r = 0; r < kPkRows; ++r) {
+            const int src = gbase + r;
+            const uint2 pv = make_uint2(__shfl_sync(0xffffffffu, mine_p.x, src), __shfl_sync(0xffffffffu, mine_p.y, src));
+            const QParams p = unpack_qparams(pv);
+            const int64_t n = n0 + r;
+            const uint32_t base = (uint32_t)(__float_as_int(kMagic) - (int)p.z);
+            uint32_t acc = 0u, mult = 1u;
+            if (__any_sync(0xffffffffu, p.clamp)) {        // some group of this row needs the code clamp
+                const float vlo = __fsub_rn(kMagic, p.z), vhi = __fadd_rn(kMagic, __fsub_rn(qmax, p.z));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float v = fminf(fmaxf(__fmaf_rn(wp[r][e], p.r, kMagic), vlo), vhi);
+                    acc += (uint32_t)__float_as_uint(v) * mult;
+                    mult *= B;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    acc += (uint32_t)__float_as_uint(__fmaf_rn(wp[r][e], p.r, kMagic)) * mult;
+                    mult *= B;
+                }
+            }
+            uint32_t v = acc - base * geom;
+            if (bits == 2) {
+                v |= __shfl_down_sync(0xffffffffu, v, 1) << 16;      // 16 codes per word: lane pairs
+                if (colok && n < N && (lane & 1) == 0) codes[n * (K / 16) + col / 16] = v;
+            } else {
+                if (colok && n < N) codes[n * (K / 8) + col / 8] = v;
+            }
+        }
+        const int64_t n = n0 + gl;
+        if (colok && gl < kPkRows && n < N) {
+            scales[n * G + grp] = __float2half_rn(mine.sh);
+            zeros[n * G + grp] = __float2half_rn(mine.z);
+        }
     }
 }
 
@@ -920,7 +1007,7 @@ constexpr int RPW = ROWS / RGROUPS;
 constexpr int CWARPS = 2 * RGROUPS;      // consumer warps: a row group x a column half
 constexpr int THREADS = (CWARPS + 1) * 32;
 constexpr int MAX_STAGES = 4;
-constexpr int TOKENS = 2;                // tokens per pass (activations stay in registers)
+constexpr int TOKENS = 4;                // most tokens per pass (activations stay in registers)
 constexpr int WORDS = 128;               // code words per row per stage (512 B)
 constexpr int CODE_BYTES = ROWS * WORDS * 4;                 // 32 KiB
 constexpr int MAX_STAGE_COLS = WORDS * 16;                   // columns per stage at 2 bits
@@ -1162,15 +1249,12 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
             const uint8_t *stage = base + st * STAGE_BYTES;
             if (j * SC + lane_col < A.K) {                       // lanes past K hold zero fill
                 const __half *sz = reinterpret_cast<const __half *>(stage + TX_BYTES);
-                uint2 w[RPW];
                 float sh[RPW];
-                float2 noff[RPW];                                // -(2^23 + z), twice
+                float noff[RPW];                                 // -(2^23 + z)
 #pragma unroll
                 for (int r = 0; r < RPW; ++r) {
-                    w[r] = *reinterpret_cast<const uint2 *>(stage + ((rg * RPW + r) * WORDS + hh * 64 + 2 * lane) * 4);
                     sh[r] = __half2float(sz[(rg * RPW + r) * gps + gl]);
-                    const float nz = -__fadd_rn(8388608.0f, __half2float(sz[(ROWS + rg * RPW + r) * gps + gl]));
-                    noff[r] = make_float2(nz, nz);
+                    noff[r] = -__fadd_rn(8388608.0f, __half2float(sz[(ROWS + rg * RPW + r) * gps + gl]));
                 }
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -1186,7 +1270,9 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
 #pragma unroll
                     for (int r = 0; r < RPW; ++r) {
                         float d[CPW];
-                        dequant_word<CB>(i == 0 ? w[r].x : w[r].y, noff[r], d);
+                        const uint32_t wr =
+                            *reinterpret_cast<const uint32_t *>(stage + ((rg * RPW + r) * WORDS + hh * 64 + 2 * lane + i) * 4);
+                        dequant_word<CB>(wr, make_float2(noff[r], noff[r]), d);
 #pragma unroll
                         for (int t = 0; t < TT; ++t) {
                             float2 s2 = mul2_rn(make_float2(x[t][0], x[t][1]), make_float2(d[0], d[1]));

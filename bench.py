@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-hbm", action="store_true", help="skip the warm HBM-kernel rates")
+    p.add_argument("--shard", choices=["layers", "rows"], default="layers",
+                   help="layers: each rank quantizes its own layer (weak scaling, no collective); rows: the "
+                        "ranks split one layer's rows and all-reduce the per-alpha losses (strong scaling)")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows of W in the oracle sample (0 = auto)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     p.add_argument("--op", choices=["search", "qlinear", "baselines", "gptq"], default="search",
@@ -358,8 +361,23 @@ def run_awq(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist_init(world, "nccl")
-    cfg = rank_layer_config(synth.CONFIGS[args.config], rank)
-    W, X, _ = synth.generate(cfg)
+    rows_mode = args.shard == "rows"
+    if rows_mode:
+        # one layer, its rows split across the ranks; the all-reduce of the
+        # per-alpha losses is inside every step (awq_activation_aware_b200.sharded)
+        from awq_activation_aware_b200 import sharded
+        base = synth.CONFIGS[args.config]
+        W_full, X, _ = synth.generate(base)
+        r0, r1 = sharded.shard_rows(base.N, world, rank)
+        W = np.ascontiguousarray(W_full[r0:r1])
+        del W_full
+        cfg = synth.LayerConfig(**{**base.as_dict(), "N": r1 - r0})
+        if cfg.N < 1:
+            raise SystemExit(f"--shard rows: rank {rank} holds no rows of the {base.N}-row layer")
+        layer_flops = 2.0 * base.N * base.K * base.T * len(synth.default_alphas())
+    else:
+        cfg = rank_layer_config(synth.CONFIGS[args.config], rank)
+        W, X, _ = synth.generate(cfg)
     alphas_np = synth.default_alphas()
     n_alpha = len(alphas_np)
     flops = 2.0 * cfg.N * cfg.K * cfg.T * n_alpha
@@ -385,7 +403,11 @@ def run_awq(args):
         a = awq.act_stats(Xd)
         if prof is not None:
             awq.profile_next_search(*prof)
-        awq.search_layer(Wd, Xd, a, alphas, cfg.bits, cfg.group, workspace=ws, losses_out=losses)
+        awq.search_layer(Wd, Xd, a, alphas, cfg.bits, cfg.group, workspace=ws, losses_out=losses,
+                         rows_total=base.N if rows_mode else None)
+        if rows_mode and world > 1:
+            import torch.distributed as dist
+            dist.all_reduce(losses, op=dist.ReduceOp.SUM)
         awq.pack(Wd, a, alphas, losses, cfg.bits, cfg.group, out=out)
 
     for _ in range(max(args.warmup, 0)):
@@ -422,7 +444,8 @@ def run_awq(args):
     search_ms = [b.elapsed_time(e) for b, e in sev]
     total_ms, search_avg = reduce_max([sum(step_ms), sum(search_ms) / K], world, dev)
     ms_per_step = total_ms / K
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    job_flops = layer_flops if rows_mode else world * flops
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
     long_region = total_ms > 1000.0
@@ -444,7 +467,7 @@ def run_awq(args):
     # compute; the timed region spans the first H2D to the last D2H.  L2 is flushed
     # before every step's compute.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not rows_mode:
         d2h = (n_alpha * 4 + 4 + cfg.K * 4 + cfg.N * cfg.K // per * 4 + 2 * cfg.N * cfg.K // cfg.group * 2)
         h2d = W_h.numel() * 2 + X_h.numel() * 2
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -515,10 +538,13 @@ def run_awq(args):
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-                "config": config_dict(cfg, n_alpha),
-                "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "1 GPU",
-                "layers_per_s": world / (ms_per_step * 1e-3),
+                "scaling": "strong" if rows_mode else "weak", "vs_baseline": None, "dtype": "f16",
+                "data": "synthetic",
+                "config": config_dict(base if rows_mode else cfg, n_alpha),
+                "parallelism": (f"one layer's rows split over {world} GPUs, all-reduce of {n_alpha} losses"
+                                if rows_mode else
+                                f"{world} independent layers, one per GPU" if world > 1 else "1 GPU"),
+                "layers_per_s": (1 if rows_mode else world) / (ms_per_step * 1e-3),
                 "roofline": roofline, "hbm_kernels": hbm_rates, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": LAUNCHES_PER_STEP * K, "clocks": clocks,
                 "pct_of_peak": 100.0 * value / peak}
@@ -591,8 +617,10 @@ def run_qlinear(args):
         return statistics.median(ts)
 
     def path_and_launches(T):
-        # the library's dispatch: the CUDA-core kernel (x' kernel + one pass per two tokens)
-        return "cuda-core", 1 + (T + 1) // 2
+        # the library's dispatch: the x' kernel, then one pass of the CUDA-core kernel per
+        # 1, 2 or 4 tokens (4-bit codes) / 1 or 2 tokens (2-bit codes)
+        per = 1 if T == 1 else 2 if (T == 2 or cfg.bits == 2) else 4
+        return "cuda-core", 1 + -(-T // per)
 
     for T in [int(t) for t in args.tokens.split(",")]:
         Xt = Xd[:T].contiguous()

@@ -152,6 +152,23 @@ AWQ_API awq_status awq_search_layer(const void *W, int64_t N, int64_t K,
                             float *losses, float *row_losses,
                             void *ws, size_t ws_bytes, void *stream);
 
+/* Steps a2-a6 for one part of a layer whose rows are split among several
+ * callers -- typically one process per GPU, each holding rows [r0, r0 + N) of
+ * the layer's W ([AWQ-note] "Measures": the error is a sum over the layer's
+ * output rows, so the parts' errors add up).  Identical to awq_search_layer
+ * except that the losses are normalised by the layer's row count:
+ *   losses[i] = sum over these N rows of ||((W_hat_i - W) X^T)[n, :]||^2 / (rows_total T)
+ * so that summing `losses` over the parts (e.g. one all-reduce of n_alpha
+ * floats) gives the layer's MSE, after which every part takes the same argmin
+ * (awq_pack on the summed losses) and packs its own rows.
+ *   rows_total  the layer's row count, N <= rows_total < 2^31
+ * Other arguments, the workspace and the errors are those of awq_search_layer
+ * (sized by awq_search_workspace_bytes for this part's N). */
+AWQ_API awq_status awq_search_layer_part(const void *W, int64_t N, int64_t rows_total, int64_t K,
+                                         const void *X, int64_t T, int64_t ldx, const float *a, awq_qcfg q,
+                                         const float *alphas, int32_t n_alpha, float *losses,
+                                         float *row_losses, void *ws, size_t ws_bytes, void *stream);
+
 /* Size of the scratch array built into the library for
  * awq_search_layer_noalloc: 32 MiB of device memory. */
 #define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -256,6 +256,31 @@ def test_search_repeatable_and_workspace_reuse(awq):
     assert np.array_equal(l1, l2)
 
 
+@pytest.mark.parametrize("N,cut", [(600, 256), (1000, 768)])
+def test_search_layer_part_sums_to_the_layer(awq, N, cut):
+    """A layer split into two row parts (as across two GPUs): the parts'
+    losses, normalised by the layer's row count, add up to the layer's losses,
+    and packing each part with the summed losses gives the layer's codes,
+    scales and zeros for those rows."""
+    from awq_activation_aware_b200 import sharded
+    W, X = gen(N, 512, 700, seed=N + cut, outlier_frac=0.02)
+    a = oracle.act_stats(X)
+    alphas = synth.default_alphas()
+    Ad, Xd = dev(a), dev(X)
+    whole = host(awq.search_layer(dev(W), Xd, Ad, dev(alphas), 4, 128))
+    parts = [np.ascontiguousarray(W[:cut]), np.ascontiguousarray(W[cut:])]
+    summed = sum(host(awq.search_layer(dev(Wp), Xd, Ad, dev(alphas), 4, 128, rows_total=N)).astype(np.float64)
+                 for Wp in parts)
+    awq.get_status()
+    np.testing.assert_allclose(summed, whole, rtol=1e-5)
+    np.testing.assert_allclose(summed, oracle.search(W, X, a, 4, 128, alphas)["losses"], rtol=LOSS_RTOL)
+    ref = awq.pack(dev(W), Ad, dev(alphas), dev(summed.astype(np.float32)), 4, 128)
+    got = [awq.pack(dev(Wp), Ad, dev(alphas), dev(summed.astype(np.float32)), 4, 128) for Wp in parts]
+    for k in ("codes", "scales", "zeros"):
+        assert np.array_equal(np.concatenate([host(g[k]) for g in got]), host(ref[k])), k
+    assert sharded.shard_rows(N, 2, 0)[1] % sharded.ROW_UNIT == 0
+
+
 # ---------------------------------------------------------------------------
 # a7-a8: argmin + pack
 # ---------------------------------------------------------------------------

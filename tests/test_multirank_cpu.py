@@ -93,3 +93,83 @@ def test_reference_arm_other_ranks_do_no_work():
     r = _run_reference({"WORLD_SIZE": "2", "RANK": "1"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+# ---------------------------------------------------------------------------
+# One layer's rows split across ranks (awq_activation_aware_b200.sharded):
+# the plumbing runs with two gloo ranks, with the library's kernels stood in
+# for by the oracle on the CPU (each stand-in follows the C ABI's definition,
+# awq_search_layer_part normalising by the layer's row count).
+# ---------------------------------------------------------------------------
+def _row_split_worker(rank, world, port, q, N, K, T, unit):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, str(ROOT))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from awq_activation_aware_b200 import sharded, synth
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    W, X, _ = synth.generate(synth.make_config(N, K, T, seed=31, outlier_frac=0.03))
+    r0, r1 = sharded.shard_rows(N, world, rank, unit=unit)
+
+    def fake_stats(Xt):
+        return torch.from_numpy(oracle.act_stats(Xt.numpy()))
+
+    def fake_search(Wp, Xt, a, al, bits, group, workspace=None, zero_point=True, rows_total=None):
+        r = oracle.search(Wp.numpy(), Xt.numpy(), a.numpy(), bits, group, al.numpy(), zero_point=zero_point)
+        return torch.from_numpy((r["row_sums"].sum(axis=1) / (rows_total * Xt.shape[0])).astype(np.float32))
+
+    def fake_pack(Wp, a, al, losses, bits, group, zero_point=True):
+        pk = oracle.pack(Wp.numpy(), a.numpy(), bits, group, al.numpy(), losses.numpy().astype(np.float64),
+                         zero_point=zero_point)
+        return {"best_idx": torch.tensor([pk["best"]]), "codes": torch.from_numpy(pk["codes"])}
+
+    sharded.act_stats, sharded.search_layer, sharded.pack = fake_stats, fake_search, fake_pack
+    al = torch.from_numpy(synth.default_alphas())
+    res = sharded.quantize_layer_rows(torch.from_numpy(np.ascontiguousarray(W[r0:r1])), torch.from_numpy(X), N,
+                                      alphas=al)
+    dist.destroy_process_group()
+    q.put((rank, r0, r1, res["losses"].numpy().tolist(),
+           int(res["best_idx"][0]) if "best_idx" in res else None,
+           res["codes"].numpy() if "codes" in res else None))
+
+
+@pytest.mark.parametrize("N,unit", [(200, 64), (200, 256)])
+def test_row_split_two_ranks_matches_whole_layer(N, unit):
+    """Two ranks: the all-reduced losses equal the whole layer's MSE, both
+    ranks take the same argmin, and the parts' codes are the whole layer's
+    rows.  With 256-row units the second rank holds no rows and still takes
+    part in the all-reduce."""
+    import numpy as np
+
+    import oracle
+    from awq_activation_aware_b200 import synth
+    K, T = 256, 48
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_row_split_worker, args=(r, 2, port, q, N, K, T, unit)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=300) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    W, X, _ = synth.generate(synth.make_config(N, K, T, seed=31, outlier_frac=0.03))
+    al = synth.default_alphas()
+    a = oracle.act_stats(X)
+    whole = oracle.search(W, X, a, 4, 128, al)
+    full_pack = oracle.pack(W, a, 4, 128, al, whole["losses"])
+    assert res[0][2] == res[1][1] and res[0][1] == 0 and res[1][2] == N
+    for rank, r0, r1, losses, best, codes in res:
+        np.testing.assert_allclose(losses, whole["losses"], rtol=1e-6)
+        assert losses == res[0][3]                       # the same bits on every rank
+        if r1 > r0:
+            assert best == full_pack["best"]
+            assert np.array_equal(codes, full_pack["codes"][r0:r1])
+        else:
+            assert codes is None
