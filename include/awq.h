@@ -190,7 +190,11 @@ AWQ_API awq_status awq_search_layer_part(const void *W, int64_t N, int64_t rows_
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on that device.
+ *     that first call before any stream capture on that device.  The cached
+ *     address belongs to the device's current primary context: after
+ *     cudaDeviceReset (or anything else that destroys that context) it is no
+ *     longer valid, so do not call this entry point on that device again in
+ *     the same process.
  *   - Layers whose awq_search_workspace_bytes(...) exceeds
  *     AWQ_NOALLOC_SCRATCH_BYTES are rejected with AWQ_ERR_WORKSPACE before
  *     anything is launched.  (The 4096 x 4096, T = 4096, 20-alpha layer needs

@@ -204,6 +204,18 @@ def test_large_zero_points_against_bruteforce(oracle_mod):
         assert np.array_equal(deq.astype(np.float16), r["what"])
 
 
+def test_zero_point_of_a_group_starting_at_zero_is_plus_zero(oracle_mod):
+    """A group whose minimum is exactly +0 has zero point rint(-0 * r) = -0; the
+    fp16 zeros store it as +0 (bits 0x0000), like any other zero, and the brute
+    force's stored value is +0 too."""
+    W = np.array([[0.0, 1.0, 2.0, 3.0, 0.5, 1.5, 2.5, 3.5]], dtype=np.float16)
+    s = np.ones(8, dtype=np.float32)
+    pk = oracle_mod.pack_scales(W, s, 4, 8)
+    assert int(pk["zeros"].view(np.uint16)[0, 0]) == 0x0000
+    _, _, Z, _ = bruteforce.quantize([list(map(float, W[0]))], [np.float32(1.0)] * 8, 4, 8)
+    assert Z[0][0] == 0 and math.copysign(1.0, Z[0][0]) == 1.0
+
+
 def test_ties_round_to_even(oracle_mod):
     # scale = 15/15 = 1; the values k + 1/2 land exactly on ties
     W = np.array([[0.0, 15.0, 0.5, 1.5, 2.5, 3.5, 10.5, 11.5]], dtype=np.float16)
