@@ -80,6 +80,8 @@ def lib():
     L.awq_qlinear_workspace_bytes.argtypes = [i64, i64, i64]
     L.awq_qlinear_workspace_bytes.restype = ctypes.c_size_t
     L.awq_qlinear.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
+    L.awq_qlinear_tc.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
+    L.awq_qlinear_cc.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
     L.awq_qlinear.restype = ctypes.c_int
     L.awq_selftest_bounded_wait.argtypes = [P]
     L.awq_selftest_bounded_wait.restype = ctypes.c_int
@@ -90,7 +92,7 @@ def lib():
     for fn in ("awq_act_stats", "awq_alpha_scales", "awq_quant_dequant", "awq_search_layer", "awq_pack",
                "awq_get_status", "awq_quant_dequant_masked", "awq_search_scales", "awq_channel_topk",
                "awq_pack_scales", "awq_salient_scales", "awq_output_error", "awq_gptq_hessian", "awq_gptq_factor",
-               "awq_gptq_quantize"):
+               "awq_gptq_quantize", "awq_qlinear_tc", "awq_qlinear_cc"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
     return L
@@ -250,20 +252,24 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, alphas: torch.Tensor | None
 
 def qlinear(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, s_best: torch.Tensor,
             X: torch.Tensor, bits: int = 4, group: int = 128, workspace: torch.Tensor | None = None,
-            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+            out: torch.Tensor | None = None, stream=None, tensor_cores: bool | None = None) -> torch.Tensor:
     """Y = X W_hat^T straight from the packed codes (the layer's input X is fp16 [T, K];
-    1/s_best is folded into it).  Returns float32 [T, N]."""
+    1/s_best is folded into it).  Returns float32 [T, N].  tensor_cores None calls
+    awq_qlinear (which picks the kernel by T), True awq_qlinear_tc (tcgen05), False
+    awq_qlinear_cc (CUDA cores)."""
     _rowmajor(X, "X")
     N = codes.shape[0]
     T, K = X.shape
     need = int(lib().awq_qlinear_workspace_bytes(T, K, N))
     ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
     Y = out if out is not None else torch.empty((T, N), dtype=torch.float32, device=X.device)
-    _check(lib().awq_qlinear(_dev(codes, torch.int32, "codes"), _dev(scales, torch.float16, "scales"),
-                             _dev(zeros, torch.float16, "zeros"), _dev(s_best, torch.float32, "s_best"), N, K,
-                             _qcfg(bits, group), _dev(X, torch.float16, "X"), T, X.stride(0),
-                             _dev(Y, torch.float32, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
-                             _stream(stream)), "awq_qlinear")
+    name = {None: "awq_qlinear", True: "awq_qlinear_tc", False: "awq_qlinear_cc"}[tensor_cores]
+    fn = getattr(lib(), name)
+    _check(fn(_dev(codes, torch.int32, "codes"), _dev(scales, torch.float16, "scales"),
+              _dev(zeros, torch.float16, "zeros"), _dev(s_best, torch.float32, "s_best"), N, K,
+              _qcfg(bits, group), _dev(X, torch.float16, "X"), T, X.stride(0),
+              _dev(Y, torch.float32, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+              _stream(stream)), name)
     return Y
 
 

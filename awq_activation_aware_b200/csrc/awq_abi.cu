@@ -111,6 +111,12 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qtc::smem_bytes<16>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qtc::smem_bytes<32>()) != cudaSuccess ||
+            cudaFuncSetAttribute(awq::qlinear_tc_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::qtc::smem_bytes<48>()) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -178,6 +184,34 @@ bool encode_codes_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64
     return r == CUDA_SUCCESS;
 }
 
+// Packed code words [rows][words] as boxes of box_words (128 bytes) x box_rows, 128-byte swizzle.
+bool encode_words_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64_t words, int box_words,
+                      int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)words * 4};
+    cuuint32_t box[2] = {(cuuint32_t)box_words, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(codes), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+// bf16 [rows][cols] as boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool encode_bf16_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int blocks_for(int64_t threads_total, int block) {
     int64_t b = (threads_total + block - 1) / block;
     return (int)(b < 1 ? 1 : b);
@@ -230,6 +264,7 @@ awq_status noalloc_scratch(void **out) {
 // widest stage), the partial sums of row blocks split across blocks, and the
 // per row block arrival counters.
 constexpr int64_t kQlMaxGrid = 1024;
+constexpr int64_t kQlTcMinTokens = 3;      // awq_qlinear: tensor cores from 3 tokens on
 int64_t ql_rows_pad(int64_t T) { return (T + awq::qlv::TOKENS - 1) / awq::qlv::TOKENS * awq::qlv::TOKENS; }
 int64_t ql_cols_pad(int64_t K, int64_t sc) { return (K + sc - 1) / sc * sc; }
 size_t ql_xs_bytes(int64_t T, int64_t K) {
@@ -243,7 +278,38 @@ size_t qlinear_ws_simt(int64_t T, int64_t K, int64_t N) {
     return ql_xs_bytes(T, K) + ql_part_bytes(N) +
            round_up(sizeof(unsigned) * (size_t)ql_row_blocks(N) * awq::qlv::RGROUPS, 256);
 }
-size_t qlinear_ws(int64_t T, int64_t K, int64_t N) { return qlinear_ws_simt(T, K, N); }
+// The tensor-core path: x' pieces bf16 [passes][NR][Kp], group sums fp32
+// [passes][K/64 or fewer groups][16], and per-chunk partial sums fp32
+// [chunks][TT][N] when K is split into chunks.
+struct QtcPlan {
+    int NR, TT, n_pass, n_chunks;
+    int64_t Kp, chunk, units;
+    size_t xb_bytes, gs_bytes, part_bytes;
+};
+QtcPlan qtc_plan(int64_t T, int64_t K, int64_t N, int group) {
+    QtcPlan p;
+    p.NR = T <= 5 ? 16 : T <= 10 ? 32 : 48;
+    p.TT = awq::qtc::tile_tokens(p.NR);
+    p.n_pass = (int)((T + p.TT - 1) / p.TT);
+    p.Kp = (K + 63) / 64 * 64;
+    const int64_t rb = (N + awq::qtc::ROWS - 1) / awq::qtc::ROWS;
+    p.chunk = awq::qtc::CHUNK;                              // at most 8 groups a unit: the epilogue prefetches them
+    p.n_chunks = (int)((K + p.chunk - 1) / p.chunk);
+    p.units = rb * p.n_chunks;
+    p.xb_bytes = round_up(2 * (size_t)p.n_pass * p.NR * p.Kp, 1024);
+    p.gs_bytes = round_up(4 * (size_t)p.n_pass * (size_t)(K / group) * 16, 256);
+    p.part_bytes = p.n_chunks > 1 ? round_up(4 * (size_t)p.n_chunks * p.TT * N, 256) : 0;
+    return p;
+}
+size_t qtc_ws_bound(int64_t T, int64_t K, int64_t N) {
+    // the largest plan over group sizes: 64-column groups
+    const QtcPlan p = qtc_plan(T, K, N, 64);
+    return p.xb_bytes + p.gs_bytes + p.part_bytes;
+}
+size_t qlinear_ws(int64_t T, int64_t K, int64_t N) {
+    const size_t a = qlinear_ws_simt(T, K, N), b = qtc_ws_bound(T, K, N);
+    return a > b ? a : b;
+}
 
 // a8 for a given s: codes, fp16 scales and zeros.
 awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_qcfg q, uint32_t *codes,
@@ -252,7 +318,7 @@ awq_status launch_pack(const void *W, int64_t N, int64_t K, const float *s, awq_
     if (awq_status e = device_info(d)) return e;
     const int G = (int)(K / q.group_size);
     const int sym = q.zero_point ? 0 : 1;
-    // one warp per item of 8 rows x 256 columns, at most 8 blocks per SM (the rest loop)
+    // one warp per item of 4 rows x 256 columns, at most 8 blocks per SM (the rest loop)
     const int64_t items = (N + awq::kPkRows - 1) / awq::kPkRows * ((K + awq::kPkCols - 1) / awq::kPkCols);
     const int64_t warps_per_block = awq::kPkThreads / 32;
     int64_t grid = (items + warps_per_block - 1) / warps_per_block;
@@ -702,9 +768,9 @@ size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N) {
     return qlinear_ws(T, K, N);
 }
 
-awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
-                                  int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
-                                  void *ws, size_t ws_bytes, void *stream) {
+awq_status awq_qlinear_cc(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
+                          int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
+                          void *ws, size_t ws_bytes, void *stream) {
     if (!codes || !scales || !zeros || !s_best || !X || !Y) return AWQ_ERR_INVALID_ARG;
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(s_best) || !aligned16(X) ||
         !aligned16(Y))
@@ -770,6 +836,90 @@ awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *ze
         if (awq_status e = last_launch()) return e;
     }
     return AWQ_OK;
+}
+
+awq_status awq_qlinear_tc(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
+                          int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
+                          void *ws, size_t ws_bytes, void *stream) {
+    if (!codes || !scales || !zeros || !s_best || !X || !Y) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(s_best) || !aligned16(X) ||
+        !aligned16(Y))
+        return AWQ_ERR_INVALID_ARG;
+    if (!valid_qcfg(q) || N < 1 || N > kMaxDim || T < 1 || T > kMaxDim || K < 64 || K > kMaxDim || K % 64 ||
+        K % q.group_size || ldx < K || ldx % 8)
+        return AWQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qlinear_ws(T, K, N) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    const QtcPlan P = qtc_plan(T, K, N, q.group_size);
+    const int G = (int)(K / q.group_size);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    __nv_bfloat16 *xb = reinterpret_cast<__nv_bfloat16 *>(w8);
+    float *gsum = reinterpret_cast<float *>(w8 + P.xb_bytes);
+    float *part = reinterpret_cast<float *>(w8 + P.xb_bytes + P.gs_bytes);
+    {
+        int grid = blocks_for((int64_t)P.n_pass * P.NR * P.Kp, 256);
+        if (grid > 8 * d.sms) grid = 8 * d.sms;
+        awq::qtc_prep_kernel<<<grid, 256, 0, st>>>((const __half *)X, T, K, P.Kp, ldx, s_best, P.TT, P.NR, P.n_pass,
+                                                   xb);
+        if (awq_status e = last_launch()) return e;
+        int grid2 = blocks_for((int64_t)P.n_pass * G * 16 * 16, 256);       // 16 lanes per group sum
+        if (grid2 > 8 * d.sms) grid2 = 8 * d.sms;
+        awq::qtc_gsum_kernel<<<grid2, 256, 0, st>>>((const __half *)X, T, K, ldx, s_best, P.TT, P.n_pass, G,
+                                                    q.group_size, gsum);
+        if (awq_status e = last_launch()) return e;
+    }
+    const int cpw = q.bits == 2 ? 16 : 8;
+    CUtensorMap tmap_codes, tmap_b;
+    if (!encode_words_map(&tmap_codes, codes, N, K / cpw, awq::qtc::CODE_ROW_BYTES / 4, awq::qtc::ROWS) ||
+        !encode_bf16_map(&tmap_b, xb, (int64_t)P.n_pass * P.NR, P.Kp, P.NR))
+        return AWQ_ERR_CUDA;
+    awq::qtc::Args A;
+    A.scales = (const __half *)scales;
+    A.zeros = (const __half *)zeros;
+    A.N = N;
+    A.K = K;
+    A.G = G;
+    A.group = q.group_size;
+    A.cpw = cpw;
+    A.chunk = P.chunk;
+    A.n_chunks = P.n_chunks;
+    A.units = P.units;
+    A.part = part;
+    A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+    const int64_t grid = P.units < d.sms ? P.units : d.sms;
+    for (int pass = 0; pass < P.n_pass; ++pass) {
+        A.gsum = gsum + (int64_t)pass * G * 16;
+        A.Y = Y + (int64_t)pass * P.TT * N;
+        A.T = (int)(T - (int64_t)pass * P.TT < P.TT ? T - (int64_t)pass * P.TT : P.TT);
+        A.b_row0 = pass * P.NR;
+        const unsigned g = (unsigned)grid;
+        if (P.NR == 16)
+            awq::qlinear_tc_kernel<16><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<16>(), st>>>(tmap_codes, tmap_b, A);
+        else if (P.NR == 32)
+            awq::qlinear_tc_kernel<32><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<32>(), st>>>(tmap_codes, tmap_b, A);
+        else
+            awq::qlinear_tc_kernel<48><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<48>(), st>>>(tmap_codes, tmap_b, A);
+        if (awq_status e = last_launch()) return e;
+        if (P.n_chunks > 1) {
+            int grid3 = blocks_for((int64_t)A.T * N, 256);
+            if (grid3 > 8 * d.sms) grid3 = 8 * d.sms;
+            awq::qtc_reduce_kernel<<<grid3, 256, 0, st>>>(part, P.n_chunks, P.TT, A.T, N, A.Y);
+            if (awq_status e = last_launch()) return e;
+        }
+    }
+    return AWQ_OK;
+}
+
+// From kQlTcMinTokens tokens on, one tensor-core pass reads the codes once for
+// up to 16 tokens, where the CUDA-core kernel reads them once per 2 or 4.
+awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
+                       int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
+                       void *ws, size_t ws_bytes, void *stream) {
+    if (T >= kQlTcMinTokens)
+        return awq_qlinear_tc(codes, scales, zeros, s_best, N, K, q, X, T, ldx, Y, ws, ws_bytes, stream);
+    return awq_qlinear_cc(codes, scales, zeros, s_best, N, K, q, X, T, ldx, Y, ws, ws_bytes, stream);
 }
 
 awq_status awq_selftest_bounded_wait(void *stream) {

@@ -527,8 +527,7 @@ __device__ __forceinline__ void tmem_relinquish_1() {
 __device__ __forceinline__ void tmem_dealloc_1(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-// D (+)= A * B^T with A (M x 16, 16-bit) read from tensor memory at `a_tmem`
-// and B (N x 16, K-major) from shared memory.
+// D (+)= A * B^T with A (M x 16) in tensor memory and B (N x 16) K-major in shared memory.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                            uint32_t accumulate) {
     asm volatile(
@@ -543,19 +542,19 @@ __device__ __forceinline__ void mma_commit_1(uint64_t *bar) {
                  : "memory");
 }
 // 32 lanes x 32 consecutive 32-bit columns from registers (thread i writes
-// lane quadrant base + i), then wait until the stores are done.
-__device__ __forceinline__ void tmem_st_32x32b_x32_sync(uint32_t taddr, const uint32_t (&v)[32]) {
+// lane quadrant base + i); tmem_wait_st waits until this thread's stores are done.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
         "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
         "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
         "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // 32 lanes x 16 consecutive fp32 columns into registers (load and wait in one statement).
 __device__ __forceinline__ void tmem_ld_32x32b_x16_sync(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];

@@ -853,21 +853,22 @@ __global__ void best_scale_kernel(const float *__restrict__ a, int64_t K,
 // a8. Pack: per (row, group) recompute w' = RN32(w s_best), the group's
 // parameters and every code; store codes LSB-first, the fp16 scale and zero
 // ([AWQ-note] "Measures": keep the quantized weights and their metadata).
-// A warp takes items of 8 rows x 256 columns; lane l holds columns 8l..8l+7
+// A warp takes items of 4 rows x 256 columns; lane l holds columns 8l..8l+7
 // of each row, so every load instruction of the warp reads 512 contiguous
 // bytes of one row and every code store writes the row's words contiguously.
 // A group of g columns is GL = g/8 neighbouring lanes.  Its min and max go
 // through a reduce-scatter over those lanes (lane i of a group ends with row
-// i mod 8's values), each lane computes the parameters of that one row, and
+// i mod 4's values), each lane computes the parameters of that one row, and
 // the lanes of the group read them back by shuffles.  HBM-bound: W is read
 // once, codes, scales and zeros are written once.
 // ===========================================================================
 constexpr int kPkThreads = 256;
-constexpr int kPkRows = 8;               // rows per warp item
+constexpr int kPkRows = 4;               // rows per warp item (4: fewer registers, more warps resident)
 constexpr int kPkCols = 256;             // columns per warp item (8 per lane)
 
 // min over the GL lanes of this lane's group of v[i], for i = this lane's row
-// (lane index within the group mod 8); max likewise.
+// (lane index within the group mod kPkRows); max likewise.  kPkRows <= 8 = the
+// smallest group's lane count.
 template <int GL>
 __device__ __forceinline__ void group_reduce_scatter(float (&lo)[kPkRows], float (&hi)[kPkRows], float &mn, float &mx) {
     const int gl = threadIdx.x & (GL - 1);
@@ -884,9 +885,10 @@ __device__ __forceinline__ void group_reduce_scatter(float (&lo)[kPkRows], float
     }
     mn = lo[0];
     mx = hi[0];
-    if (GL == 16) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+#pragma unroll
+    for (int o = kPkRows; o < GL; o <<= 1) {              // the group's remaining lanes hold the same rows
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
 }
 
@@ -938,7 +940,7 @@ pack_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int G, int bits,
         }
         float mn, mx;
         group_reduce_scatter<GL>(lo, hi, mn, mx);
-        // this lane's row of its group: gl mod 8
+        // this lane's row of its group: gl mod kPkRows
         const QParams mine = make_qparams(mn, mx, qmax, sym != 0);
         const uint2 mine_p = pack_qparams(mine);
         const int64_t grp = col / (GL * 8);
@@ -1342,6 +1344,479 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
     }
     __syncthreads();
+}
+
+// ===========================================================================
+// The decode consumer on the tensor cores (row n1, any w_bit).  The same
+// definition as the CUDA-core kernel,
+//   Y[t, n] = sum_k x'[t, k] (q[n, k] - z[n, g]) sh[n, g],   x' = RN32(x RN32(1/s)),
+// evaluated as Y = sum_g sh (D_g - z S_g) with
+//   D_g[n, t] = sum_{k in g} q[n, k] x'[t, k]   on tcgen05 (kind::f16, bf16 operands, fp32 accumulate),
+//   S_g[t]    = RN32(sum_{k in g} x'[t, k])     in binary64 by the prep kernel.
+// Both MMA operands hold exact values: A = q (an integer below 16, exact in
+// bf16) and B = x' split into three bf16 pieces whose sum is x' exactly
+// (8 + 8 + 8 significant bits), one B row per piece and token.  So every
+// product the tensor core forms is exact and only the fp32 accumulation
+// rounds; no step depends on the range of the zero point.
+//
+// Work unit: 128 weight rows x one chunk of K (a multiple of 512 columns);
+// the units go round-robin to one persistent CTA per SM.  A TMA warp loads
+// code stages of 128 bytes of every row of the unit (16 KiB: 256 columns at
+// 4-bit containers, 512 at 2-bit; a 6-deep ring keeps about 96 KiB in flight
+// per SM) and, per 64-column sub-stage, the B tile (NR = 16, 32 or 48 rows x
+// 64 bf16, 128-byte swizzle).  Eight producer warps turn each sub-stage's
+// codes into the bf16 A tile (128 x 64, 128-byte swizzle); one thread issues
+// the four MMAs of a sub-stage into the accumulator of its quantization group
+// (a ring of 4 in tensor memory); four epilogue warps (one row per thread)
+// read each finished group, add its three piece sums, and accumulate
+// sh (D - z S) per token.  A
+// unit's sums go to Y directly (one chunk) or to per-chunk partials that a
+// second kernel adds in chunk order, so Y does not depend on timing.
+// ===========================================================================
+// Row r's 64 codes starting at 16-byte chunk `chunk0` of a 128-byte-swizzled
+// code tile (two chunks of 4-bit codes or one of 2-bit codes) as 32 bf16x2
+// words for the A operand in tensor memory (column i holds A columns 2i and
+// 2i + 1, the lower in the low half).  Each 8-column chunk of A holds its codes
+// in the order (0, 4, 1, 5, 2, 6, 3, 7): pair e is (code e, code e + 4), which
+// one mask of the word (shifted by e code widths) places in the two halves of a
+// 32-bit word under the bf16 exponent of 128; a bf16x2 subtraction of 128 then
+// leaves the exact codes.  The B operand's columns follow the same order.  The
+// 8 rows of a quarter warp read 8 distinct chunk positions of the swizzle.
+template <int CB>
+__device__ __forceinline__ void qtc_convert_half(const uint8_t *ct, int r, int chunk0, uint32_t (&v)[32]) {
+    const __nv_bfloat162 off = __floats2bfloat162_rn(128.0f, 128.0f);
+    constexpr uint32_t mask = CB == 4 ? 0x000F000Fu : 0x00030003u;
+    constexpr int NCH = CB == 4 ? 2 : 1;
+    uint32_t w[4 * NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(ct + r * 128 + (((chunk0 + c) ^ (r & 7)) << 4));
+        w[4 * c] = q.x; w[4 * c + 1] = q.y; w[4 * c + 2] = q.z; w[4 * c + 3] = q.w;
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {                                        // 8-column chunk h
+        uint32_t x;
+        if (CB == 4) x = w[h];
+        else x = __byte_perm(w[h >> 1], 0u, (h & 1) ? 0x4342u : 0x4140u);   // codes 0-3 in byte 0, codes 4-7 in byte 2
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t u = ((x >> (CB * e)) & mask) | 0x43004300u;
+            const __nv_bfloat162 b = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&u), off);
+            v[4 * h + e] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+    }
+}
+
+namespace qtc {
+constexpr int ROWS = 128;                  // weight rows per unit (MMA M)
+constexpr int SK = 128;                    // K columns per sub-stage (8 MMAs of K 16; one or two groups)
+constexpr int CODE_ROW_BYTES = 128;        // codes per row per code stage: 256 (4-bit) or 512 (2-bit) columns
+constexpr int CS = 8;                      // code ring depth (16 KiB stages)
+constexpr int AS_MAX = 6, NB_MAX = 8;
+constexpr int TMEM_COLS = 512;
+constexpr int PROD_WARP0 = 8, NUM_PROD_WARPS = 8, EPI_WARP0 = 4;
+constexpr int LOAD_WARP = 0, MMA_WARP = 1, ALLOC_WARP = 2, B_LOAD_WARP = 3;   // warp 2 also issues MMAs
+constexpr int THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;     // 512
+constexpr int CODE_BYTES = ROWS * CODE_ROW_BYTES;               // 16 KiB
+constexpr int CHUNK = 512;                                      // K columns per unit
+constexpr int MAXG = CHUNK / 64;                                // groups per unit at most
+__host__ __device__ constexpr int tile_tokens(int nr) { return nr == 16 ? 5 : nr == 32 ? 10 : 16; }
+// Tensor memory: sub-stage slots of A (64 columns each) at the top, the
+// accumulators (one per group, NR columns each) below them.
+__host__ __device__ constexpr int a_slots(int nr) { return nr == 48 ? 4 : 6; }
+__host__ __device__ constexpr int a_col0(int nr) { return TMEM_COLS - a_slots(nr) * 64; }
+__host__ __device__ constexpr int acc_slots(int nr) { return nr == 16 ? 8 : nr == 32 ? 4 : 5; }
+static_assert(acc_slots(16) * 16 <= a_col0(16) && acc_slots(32) * 32 <= a_col0(32) &&
+              acc_slots(48) * 48 <= a_col0(48), "tensor-memory layout");
+
+// Sub-stage slot i holds A in tensor memory and the B tile (NR x 128 bf16, two
+// 128-byte-swizzled boxes of 64 columns) in shared memory; one MMA commit
+// (slot_empty) releases both.
+template <int NR>
+struct Smem {
+    uint8_t codes[CS][CODE_BYTES];         // every tile 1024-byte aligned
+    uint8_t b[a_slots(NR)][NR * SK * 2];   // box 0 at 0, box 1 at NR x 128 bytes: 1024-byte aligned
+    float gs[2][MAXG * 16];                // group sums of the current / next unit (epilogue)
+    uint64_t c_full[CS], c_empty[CS];
+    uint64_t a_full[AS_MAX], b_full[AS_MAX], slot_empty[AS_MAX];
+    uint64_t acc_full[NB_MAX], acc_empty[NB_MAX];
+    uint64_t drain[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+template <int NR>
+constexpr size_t smem_bytes() { return sizeof(Smem<NR>) + 1024; }
+static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448 && smem_bytes<48>() <= 232448,
+              "decode shared memory above the 227 KiB a CTA may use");
+
+struct Args {
+    const __half *scales, *zeros;          // [N][G]
+    const float *gsum;                     // S: [G][16] for this pass
+    float *Y;                              // this pass's output rows [T][N] (one chunk) ...
+    float *part;                           // ... or partials [chunks][TT][N]
+    int64_t N, K;
+    int G, group, cpw;                     // groups, group size, codes per 32-bit word (8 or 16)
+    int T;                                 // tokens of this pass (<= TT)
+    int b_row0;                            // first B row of this pass in the B map
+    int64_t chunk;                         // K columns per chunk (CHUNK)
+    int n_chunks;
+    int64_t units;                         // row blocks x chunks
+    uint64_t timeout_ns;
+};
+}  // namespace qtc
+
+// x' = RN32(x RN32(1/s)) split into three bf16 pieces, stored as the B rows of
+// every pass: row piece * TT + t of pass p holds piece `piece` of token
+// p TT + t; within each 8-column chunk column p holds x' of column
+// (p / 2) + 4 (p % 2), the order of the A tile's codes (qtc_convert); rows past
+// 3 TT, tokens past T and columns past K are zero.
+__global__ void qtc_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t Kp, int64_t ldx,
+                                const float *__restrict__ s, int TT, int NR, int n_pass,
+                                __nv_bfloat16 *__restrict__ xb) {
+    const int64_t total = (int64_t)n_pass * NR * Kp;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t kb = i % Kp, rowg = i / Kp;
+        const int64_t k = (kb & ~int64_t(7)) + ((kb & 7) >> 1) + 4 * (kb & 1);
+        const int row = (int)(rowg % NR), pass = (int)(rowg / NR);
+        const int piece = row / TT, t = row % TT;
+        const int64_t tok = (int64_t)pass * TT + t;
+        float v = 0.0f;
+        if (piece < 3 && tok < T && k < K) {
+            const float xp = __fmul_rn(__half2float(X[tok * ldx + k]), __frcp_rn(s[k]));
+            const __nv_bfloat16 h = __float2bfloat16_rn(xp);
+            const float r1 = __fsub_rn(xp, __bfloat162float(h));                 // exact
+            const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+            const float r2 = __fsub_rn(r1, __bfloat162float(m));                 // exact, <= 8 bits
+            v = piece == 0 ? __bfloat162float(h) : piece == 1 ? __bfloat162float(m) : r2;
+        }
+        xb[i] = __float2bfloat16_rn(v);                                          // exact for every piece
+    }
+}
+
+// S[p][g][t] = RN32(sum over the group's columns of x'[p TT + t, k]) in
+// binary64 (16 slots per group; tokens past the pass or past T give 0).  16
+// lanes per output: lane j sums columns j * group/16 .. + group/16 - 1, then the
+// 16 partial sums are added by shuffles (total threads a multiple of 32).
+__global__ void qtc_gsum_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx,
+                                const float *__restrict__ s, int TT, int n_pass, int G, int group,
+                                float *__restrict__ gsum) {
+    const int64_t total = (int64_t)n_pass * G * 16 * 16;
+    const int per = group / 16;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int j = (int)(i & 15);
+        const int64_t o = i >> 4;
+        const int t = (int)(o % 16);
+        const int64_t pg = o / 16;
+        const int g = (int)(pg % G), pass = (int)(pg / G);
+        const int64_t tok = (int64_t)pass * TT + t;
+        double acc = 0.0;
+        if (t < TT && tok < T) {
+            const int64_t kb = (int64_t)g * group + (int64_t)j * per;
+            for (int c = 0; c < per; ++c)
+                acc = __dadd_rn(acc, (double)__fmul_rn(__half2float(X[tok * ldx + kb + c]), __frcp_rn(s[kb + c])));
+        }
+#pragma unroll
+        for (int o2 = 8; o2 >= 1; o2 >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o2));
+        if (j == 0) gsum[o] = __double2float_rn(acc);
+    }
+}
+
+// Y[t, n] = sum over chunks, in chunk order, of the partial sums.
+__global__ void qtc_reduce_kernel(const float *__restrict__ part, int n_chunks, int TT, int T, int64_t N,
+                                  float *__restrict__ Y) {
+    const int64_t total = (int64_t)T * N;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / N, n = i - t * N;
+        const float *p0 = part + t * N + n;
+        const int64_t cs = (int64_t)TT * N;                          // one chunk's stride
+        float y = 0.0f;
+        int c = 0;
+        for (; c + 4 <= n_chunks; c += 4) {                          // loads issued together, added in chunk order
+            const float v0 = p0[c * cs], v1 = p0[(c + 1) * cs], v2 = p0[(c + 2) * cs], v3 = p0[(c + 3) * cs];
+            y = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(y, v0), v1), v2), v3);
+        }
+        for (; c < n_chunks; ++c) y = __fadd_rn(y, p0[c * cs]);
+        Y[i] = y;
+    }
+}
+
+template <int NR>
+__global__ void __launch_bounds__(qtc::THREADS, 1)
+qlinear_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_b,
+                  const qtc::Args A) {
+    using namespace qtc;
+    constexpr int TT = tile_tokens(NR);
+    constexpr uint32_t IDESC = mma_idesc_bf16_f32(ROWS, NR);
+    extern __shared__ uint8_t smem_raw[];
+    using SmemT = Smem<NR>;
+    SmemT &S = *reinterpret_cast<SmemT *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = &S.abort_flag;
+    constexpr int NB = acc_slots(NR), AS = a_slots(NR), A_COL0 = a_col0(NR);
+    const int spc = CODE_ROW_BYTES * 8 / (32 / A.cpw) / SK;       // sub-stages per code stage: 2 (4-bit) or 4 (2-bit)
+    const int kpg = A.group / 16;                                 // MMAs per group: 4 or 8
+    const int64_t grid = gridDim.x;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < CS; ++i) { mbar_init(&S.c_full[i], 1); mbar_init(&S.c_empty[i], 4 * spc); }
+        for (int i = 0; i < AS; ++i) { mbar_init(&S.a_full[i], 4); mbar_init(&S.b_full[i], 1); mbar_init(&S.slot_empty[i], 1); }
+        for (int i = 0; i < NB; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 4); }
+        mbar_init(&S.drain[0], 1);
+        mbar_init(&S.drain[1], 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == ALLOC_WARP) {
+        tmem_alloc_1(&S.tmem_base, TMEM_COLS);
+        tmem_relinquish_1();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    bool aborted = false;
+
+    // unit u: columns [k0, k0 + cols) of row block rb, in subs sub-stages (the
+    // last one of 64 columns when cols is an odd multiple of 64)
+    auto unit_span = [&](int64_t u, int64_t &rb, int64_t &k0, int &cols, int &subs) {
+        rb = u / A.n_chunks;
+        const int64_t kc = u - rb * A.n_chunks;
+        k0 = kc * A.chunk;
+        cols = (int)(A.K - k0 < A.chunk ? A.K - k0 : A.chunk);   // a multiple of 64
+        subs = (cols + SK - 1) / SK;
+    };
+
+    if (warp == LOAD_WARP) {
+        // the code stream from HBM: 128 bytes of each of the unit's 128 rows per stage
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_codes);
+            int cs = 0;
+            uint32_t cph = 0;
+            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
+                int64_t rb, k0;
+                int cols, subs;
+                unit_span(u, rb, k0, cols, subs);
+                for (int sub = 0; sub < subs; sub += spc) {
+                    if (!mbar_wait_bounded(&S.c_empty[cs], cph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    mbar_arrive_expect_tx(&S.c_full[cs], CODE_BYTES);
+                    tma_load_2d(&S.codes[cs][0], &tmap_codes, (int32_t)((k0 + (int64_t)sub * SK) / A.cpw),
+                                (int32_t)(rb * ROWS), &S.c_full[cs]);
+                    if (++cs == CS) { cs = 0; cph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == B_LOAD_WARP) {
+        // the B tiles (x' pieces, L2-resident): two boxes of 64 columns per sub-stage slot
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_b);
+            int bs = 0;
+            uint32_t bph = 0;
+            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
+                int64_t rb, k0;
+                int cols, subs;
+                unit_span(u, rb, k0, cols, subs);
+                for (int sub = 0; sub < subs; ++sub) {
+                    if (!mbar_wait_bounded(&S.slot_empty[bs], bph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    mbar_arrive_expect_tx(&S.b_full[bs], (uint32_t)(NR * SK * 2));
+                    const int32_t x = (int32_t)(k0 + (int64_t)sub * SK);
+                    tma_load_2d(&S.b[bs][0], &tmap_b, x, A.b_row0, &S.b_full[bs]);
+                    tma_load_2d(&S.b[bs][NR * 128], &tmap_b, x + 64, A.b_row0, &S.b_full[bs]);
+                    if (++bs == AS) { bs = 0; bph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == MMA_WARP || warp == ALLOC_WARP) {
+        // Two issuing threads, one per warp: thread mt takes the sub-stages of
+        // parity mt (each holds whole groups, so every group's MMAs are issued by
+        // one thread in order), and the two threads' issue latencies overlap.
+        // Each thread follows the whole sequence of slots and accumulators.
+        if (lane == 0) {
+            const int mt = warp == MMA_WARP ? 0 : 1;
+            const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(&S.b[0][0]));
+            int as = 0, nb = 0;
+            uint32_t aph = 0, accph = 0, gsub = 0;
+            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
+                int64_t rb, k0;
+                int cols, subs;
+                unit_span(u, rb, k0, cols, subs);
+                for (int sub = 0; sub < subs && !aborted; ++sub, ++gsub) {
+                    const bool mine = (int)(gsub & 1u) == mt;
+                    const int ng = (cols - sub * SK < SK ? cols - sub * SK : SK) / A.group;   // groups in this sub-stage
+                    if (mine) {
+                        if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
+                            !mbar_wait_bounded(&S.b_full[as], aph, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                        tc_fence_after();
+                    }
+                    const uint32_t a_tmem = tmem + (uint32_t)(A_COL0 + as * 64);
+                    const uint64_t bdesc = bdesc0 + (uint64_t)((as * NR * SK * 2) >> 4);   // start address field
+                    for (int gl = 0; gl < ng; ++gl) {
+                        if (mine) {
+                            if (!mbar_wait_bounded(&S.acc_empty[nb], accph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                            tc_fence_after();
+                            const uint32_t d_tmem = tmem + (uint32_t)(nb * NR);
+                            for (int kk = 0; kk < kpg; ++kk) {
+                                const int kq = gl * kpg + kk;                 // K step of the sub-stage: box kq / 4, 32 bytes each
+                                mma_f16_ts(d_tmem, a_tmem + (uint32_t)(kq * 8),
+                                           bdesc + (uint64_t)((((kq >> 2) * NR * 128) + (kq & 3) * 32) >> 4), IDESC,
+                                           kk != 0 ? 1u : 0u);
+                            }
+                            mma_commit_1(&S.acc_full[nb]);
+                        }
+                        if (++nb == NB) { nb = 0; accph ^= 1u; }
+                    }
+                    if (mine && !aborted) mma_commit_1(&S.slot_empty[as]);
+                    if (++as == AS) { as = 0; aph ^= 1u; }
+                }
+            }
+            mma_commit_1(&S.drain[mt]);                               // every MMA of this thread done before teardown
+            mbar_wait_bounded(&S.drain[mt], 0, abort_flag, A.timeout_ns);
+        }
+    } else if (warp >= PROD_WARP0) {
+        // Two sets of 4 producer warps take the sub-stages in turn (set gsub % 2);
+        // within a set, warp q writes the rows of tensor-memory lane quadrant q,
+        // one row per thread, into A slot gsub % AS (two halves of 64 columns,
+        // qtc_convert_half).  A code stage is released once every warp of each of
+        // its sub-stages has read it (the unit's last sub-stage of a partial stage
+        // arrives for the missing ones).
+        const int pset = (warp - PROD_WARP0) >> 2, q4 = warp & 3;
+        const int r = q4 * 32 + lane;                                 // the thread's row of the unit
+        const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+        int cs = 0, as = 0;
+        uint32_t cph = 0, aph = 0, gsub = 0;
+        for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
+            int64_t rb, k0;
+            int cols, subs;
+            unit_span(u, rb, k0, cols, subs);
+            int sc = 0;                                               // sub-stage within the code stage
+            for (int sub = 0; sub < subs; ++sub, ++gsub) {
+                const bool stage_end = sc == spc - 1 || sub == subs - 1;
+                if ((int)(gsub & 1u) == pset) {
+                    if (!mbar_wait_warp(&S.c_full[cs], cph, abort_flag, A.timeout_ns) ||
+                        !mbar_wait_warp(&S.slot_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                    tc_fence_after();
+                    const uint32_t dst = tmem + lane_base + (uint32_t)(A_COL0 + as * 64);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t v[32];
+                        if (A.cpw == 8) qtc_convert_half<4>(&S.codes[cs][0], r, 4 * sc + 2 * h, v);
+                        else qtc_convert_half<2>(&S.codes[cs][0], r, 2 * sc + h, v);
+                        tmem_st_32x32b_x32(dst + (uint32_t)(32 * h), v);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&S.a_full[as]);
+                        const int n_arrive = sub == subs - 1 ? spc - sc : 1;   // a partial last stage: the missing ones too
+                        for (int k = 0; k < n_arrive; ++k) mbar_arrive(&S.c_empty[cs]);
+                    }
+                }
+                if (++as == AS) { as = 0; aph ^= 1u; }
+                if (++sc == spc || stage_end) { sc = 0; if (++cs == CS) { cs = 0; cph ^= 1u; } }
+            }
+        }
+    } else if (warp >= EPI_WARP0) {
+        // Per unit: the scale and zero of this thread's row for each group come
+        // from global memory one unit ahead (registers), the unit's group sums
+        // (one float per thread) through a double buffer in shared memory, so no
+        // group waits on a global load.
+        const int q4 = warp - EPI_WARP0;                              // TMEM lane quadrant
+        const int et = threadIdx.x - EPI_WARP0 * 32;                  // 0 .. 127
+        const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+        int nb = 0;
+        uint32_t accph = 0;
+        __half2 szc[MAXG], szn[MAXG];                                 // (scale, zero) per group
+        float gsn = 0.0f;
+        auto fetch = [&](int64_t uu, __half2 (&dst)[MAXG], float &gsv) {
+            int64_t rb_, k0_;
+            int cols_, subs_;
+            unit_span(uu, rb_, k0_, cols_, subs_);
+            const int64_t nn = rb_ * ROWS + q4 * 32 + lane;
+            const int groups_ = cols_ / A.group, g0_ = (int)(k0_ / A.group);
+#pragma unroll
+            for (int gi = 0; gi < MAXG; ++gi)
+                dst[gi] = (nn < A.N && gi < groups_) ? __halves2half2(A.scales[nn * A.G + g0_ + gi], A.zeros[nn * A.G + g0_ + gi])
+                                                     : __float2half2_rn(0.0f);
+            const int gg = et >> 4, tt = et & 15;                      // thread et: group gg, token slot tt
+            gsv = gg < groups_ ? A.gsum[(int64_t)(g0_ + gg) * 16 + tt] : 0.0f;
+        };
+        int buf = 0;
+        if (blockIdx.x < A.units) {
+            float g0v;
+            fetch(blockIdx.x, szc, g0v);
+            S.gs[0][et] = g0v;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // Every epilogue warp runs every unit and reaches every named barrier,
+        // also after an abort (then it only skips the waits and the work), so
+        // the barrier cannot strand the others.
+        for (int64_t u = blockIdx.x; u < A.units; u += grid) {
+            int64_t rb, k0;
+            int cols, subs;
+            unit_span(u, rb, k0, cols, subs);
+            const bool more = u + grid < A.units;
+            if (more && !aborted) fetch(u + grid, szn, gsn);         // in flight during this unit
+            const int64_t n = rb * ROWS + q4 * 32 + lane;
+            const bool row_ok = n < A.N;
+            float y[TT];
+#pragma unroll
+            for (int t = 0; t < TT; ++t) y[t] = 0.0f;
+            const int groups = cols / A.group;
+            const float *gsu = &S.gs[buf][0];
+#pragma unroll
+            for (int gi = 0; gi < MAXG; ++gi) {
+                if (gi >= groups || aborted) break;
+                const float2 szf = __half22float2(szc[gi]);
+                if (!mbar_wait_warp(&S.acc_full[nb], accph, abort_flag, A.timeout_ns, 128)) { aborted = true; break; }
+                tc_fence_after();
+                // the accumulator's NR columns: B row piece * TT + t  (x16 or x32 loads, then x16 for NR = 48)
+                float d[NR];
+                if constexpr (NR == 16) {
+                    tmem_ld_32x32b_x16_sync(tmem + lane_base + (uint32_t)(nb * NR), *reinterpret_cast<float(*)[16]>(&d[0]));
+                } else {
+                    tmem_ld_32x32b_x32_sync(tmem + lane_base + (uint32_t)(nb * NR), *reinterpret_cast<float(*)[32]>(&d[0]));
+                    if constexpr (NR == 48)
+                        tmem_ld_32x32b_x16_sync(tmem + lane_base + (uint32_t)(nb * NR + 32),
+                                                *reinterpret_cast<float(*)[16]>(&d[32]));
+                }
+                tc_fence_before();
+                __syncwarp();                                          // every lane's reads are complete (wait::ld)
+                if (lane == 0) mbar_arrive(&S.acc_empty[nb]);
+                if (++nb == NB) { nb = 0; accph ^= 1u; }
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+                    const float dt = __fadd_rn(__fadd_rn(d[t], d[TT + t]), d[2 * TT + t]);
+                    y[t] = __fmaf_rn(szf.x, __fmaf_rn(-szf.y, gsu[gi * 16 + t], dt), y[t]);
+                }
+            }
+            if (row_ok && !aborted) {
+                const int64_t kc = u - rb * A.n_chunks;
+                float *dst = A.n_chunks == 1 ? A.Y : A.part + kc * (int64_t)TT * A.N;
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    if (t < A.T) dst[(int64_t)t * A.N + n] = y[t];
+            }
+            // hand the next unit's values over: registers, and the other group-sum buffer
+            if (more) {
+#pragma unroll
+                for (int gi = 0; gi < MAXG; ++gi) szc[gi] = szn[gi];
+                S.gs[buf ^ 1][et] = gsn;
+            }
+            buf ^= 1;
+            asm volatile("bar.sync 1, 128;" ::: "memory");        // the 4 epilogue warps only
+        }
+    }
+
+    if (aborted || *abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == ALLOC_WARP) {
+        tc_fence_after();
+        tmem_dealloc_1(tmem, TMEM_COLS);
+    }
 }
 
 // ===========================================================================

@@ -293,14 +293,15 @@ def run_reference(args):
     return 0
 
 
-def hbm_kernel_rates(awq, torch, cfg, Xd, Wd, s_best, peaks, reps=3):
+def hbm_kernel_rates(awq, torch, cfg, Xd, Wd, s_best, peaks, reps=5):
     """Warm per-launch rates of the two HBM-bound kernels of the path.
 
     act_stats (reads X) and pack_kernel (awq_pack_scales: reads W and s_best,
     writes codes, scales and zeros) each run over a sequence of distinct copies
     of their input, together more than 4x the 126 MB L2, so every launch reads
-    HBM as a model's layers do; CUDA events bracket each launch on the stream.
-    Bytes are the algorithmic ones (each input byte read once, each output
+    HBM as a model's layers do; CUDA events bracket the whole sequence on the
+    stream and a launch's time is the sequence time over its launches.  Bytes
+    are the algorithmic ones (each input byte read once, each output
     byte written once)."""
     budget = 512 << 20
     per = 16 if cfg.bits == 2 else 8
@@ -311,19 +312,21 @@ def hbm_kernel_rates(awq, torch, cfg, Xd, Wd, s_best, peaks, reps=3):
     stream = torch.cuda.current_stream()
 
     def per_launch_s(calls):
+        # average launch duration over the back-to-back sequence (events around the
+        # whole sequence, so no event sits between two launches); median over reps
         for fn in calls:
             fn()
         torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
         ts = []
         for _ in range(reps):
+            b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda._sleep(20_000_000)           # the host queues every launch before the first runs
-            for (b, e), fn in zip(evs, calls):
-                b.record(stream)
+            b.record(stream)
+            for fn in calls:
                 fn()
-                e.record(stream)
+            e.record(stream)
             torch.cuda.synchronize()
-            ts += [b.elapsed_time(e) * 1e-3 for b, e in evs]
+            ts.append(b.elapsed_time(e) * 1e-3 / len(calls))
         return statistics.median(ts)
 
     t_stats = per_launch_s([(lambda x=x: awq.act_stats(x)) for x in Xs])
@@ -341,7 +344,8 @@ def hbm_kernel_rates(awq, torch, cfg, Xd, Wd, s_best, peaks, reps=3):
     return {"act_stats": entry("act_stats_kernel", stats_bytes, t_stats),
             "pack": entry("pack_kernel", pack_bytes, t_pack),
             "peak_GBps": hbm,
-            "how": "median per-launch CUDA-event time over distinct input copies (> 4x L2), warm"}
+            "how": "average launch duration over a back-to-back sequence of distinct input copies "
+                   "(> 4x L2), CUDA events around the sequence, median of 5"}
 
 
 def rank_layer_config(base, rank):
@@ -617,25 +621,33 @@ def run_qlinear(args):
         return statistics.median(ts)
 
     def path_and_launches(T):
-        # the library's dispatch: the x' kernel, then one pass of the CUDA-core kernel per
-        # 1, 2 or 4 tokens (4-bit codes) / 1 or 2 tokens (2-bit codes)
-        per = 1 if T == 1 else 2 if (T == 2 or cfg.bits == 2) else 4
-        return "cuda-core", 1 + -(-T // per)
+        # the library's dispatch.  Below 3 tokens: the x' kernel, then one pass of the
+        # CUDA-core kernel per 1 or 2 tokens.  From 3 tokens: the B-operand and
+        # group-sum kernels, then per pass of 5, 10 or 16 tokens the tensor-core kernel
+        # and (K split in chunks of 512 columns) the chunk reduction.
+        if T < 3:
+            return "cuda-core", 1 + -(-T // (1 if T == 1 else 2))
+        tt = 5 if T <= 5 else 10 if T <= 10 else 16
+        return "tensor-core", 2 + -(-T // tt) * (1 + (cfg.K > 512))
 
     for T in [int(t) for t in args.tokens.split(",")]:
         Xt = Xd[:T].contiguous()
         ws = torch.empty(int(awq.lib().awq_qlinear_workspace_bytes(T, cfg.K, cfg.N)), dtype=torch.uint8, device=dev)
         Y = torch.empty((T, cfg.N), dtype=torch.float32, device=dev)
         Yh = torch.empty((T, cfg.N), dtype=torch.float16, device=dev)
-        t_awq = per_call_us([
-            (lambda c=c: awq.qlinear(c["codes"], c["scales"], c["zeros"], c["s_best"], Xt, cfg.bits, cfg.group,
-                                     workspace=ws, out=Y)) for c in copies])
-        awq.get_status()
+        def timed(tc):
+            t = per_call_us([
+                (lambda c=c: awq.qlinear(c["codes"], c["scales"], c["zeros"], c["s_best"], Xt, cfg.bits, cfg.group,
+                                         workspace=ws, out=Y, tensor_cores=tc)) for c in copies])
+            awq.get_status()
+            return t
+        t_awq, t_cc, t_tc = timed(None), timed(False), timed(True)
         t_ref = per_call_us([(lambda w=w: torch.matmul(Xt, w.t(), out=Yh)) for w in refs])
         nbytes = (cfg.N * cfg.K // per * 4 + 2 * 2 * cfg.N * cfg.K // cfg.group + cfg.K * 4 + T * cfg.K * 2
                   + T * cfg.N * 4)
         gbs = nbytes / (t_awq * 1e-6) / 1e9
         print(json.dumps({"op": "qlinear", "config": cfg.name, "tokens": T, "awq_us": t_awq,
+                          "cuda_core_us": t_cc, "tensor_core_us": t_tc,
                           "fp16_gemm_us": t_ref, "speedup_vs_fp16": t_ref / t_awq,
                           "awq_bytes": nbytes, "awq_GBps": gbs, "hbm_frac": gbs / hbm if hbm else None,
                           "hbm_peak_source": src, "layer_copies": [n_awq, n_ref],

@@ -336,15 +336,39 @@ AWQ_API awq_status awq_get_status(void *stream);
  *       256-byte aligned (x' as binary32, partial sums of row blocks split
  *       across thread blocks, arrival counters); overwritten by every call
  * Requires K % 64 == 0.  Built for small T (decode), where streaming the
- * packed codes from HBM is the cost.  Runs on the CUDA cores, two tokens a
- * pass, each pass re-reading the codes.  The summation order depends on the
- * device's SM count, not on timing: repeated calls on one device give
- * identical Y.  Calls that share a workspace must be ordered (one stream). */
+ * packed codes from HBM is the cost.  awq_qlinear runs awq_qlinear_cc below 3
+ * tokens and awq_qlinear_tc from 3 tokens on; either may be called directly.
+ * Calls that share a workspace must be ordered (one stream). */
 AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
 AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
                                const float *s_best, int64_t N, int64_t K, awq_qcfg q,
                                const void *X, int64_t T, int64_t ldx, float *Y,
                                void *ws, size_t ws_bytes, void *stream);
+
+/* The product on the CUDA cores: binary32 multiply-adds, one, two or four
+ * tokens a pass (two for 2-bit codes), each pass re-reading the codes.  The
+ * summation order depends on the device's SM count, not on timing: repeated
+ * calls on one device give identical Y. */
+AWQ_API awq_status awq_qlinear_cc(const uint32_t *codes, const void *scales, const void *zeros,
+                                  const float *s_best, int64_t N, int64_t K, awq_qcfg q,
+                                  const void *X, int64_t T, int64_t ldx, float *Y,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* The same product on the tensor cores (tcgen05), for any T.  Identical
+ * arguments, workspace (awq_qlinear_workspace_bytes covers both) and result
+ * definition as awq_qlinear, evaluated as
+ *   Y[t, n] = sum_g sh[n, g] (D_g[n, t] - z[n, g] S_g[t]),
+ *   D_g = sum_{k in g} q[n, k] x'[t, k]   (bf16 operands, fp32 accumulation:
+ *         q is exact in bf16 and x' is split into three bf16 pieces whose sum
+ *         is x' exactly, so every product is exact),
+ *   S_g = RN32(sum_{k in g} x'[t, k]) in binary64.
+ * Passes of up to 5, 10 or 16 tokens each read the codes once; K is split into
+ * chunks whose partial sums are added in chunk order, so repeated calls on one
+ * device give identical Y.  Calls that share a workspace must be ordered. */
+AWQ_API awq_status awq_qlinear_tc(const uint32_t *codes, const void *scales, const void *zeros,
+                                  const float *s_best, int64_t N, int64_t K, awq_qcfg q,
+                                  const void *X, int64_t T, int64_t ldx, float *Y,
+                                  void *ws, size_t ws_bytes, void *stream);
 
 /* Self-test of device-side failure detection (no counterpart on the pages: it
  * checks the library, not the method).  Launches one warp that waits on a

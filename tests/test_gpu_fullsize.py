@@ -103,7 +103,8 @@ def layer(name):
 
 @pytest.mark.parametrize("name", ["attn4096", "mlp_up28672"])
 @pytest.mark.parametrize("T", [1, 2, 4, 16])
-def test_fullsize_qlinear(awq, name, T):
+@pytest.mark.parametrize("tc", [False, True], ids=["cuda_cores", "tensor_cores"])
+def test_fullsize_qlinear(awq, name, T, tc):
     """The decode layer at the benchmark's sizes and decode token counts, on sampled
     rows.  The expected rows come from the oracle's own pack of those rows."""
     cfg = synth.CONFIGS[name]
@@ -117,7 +118,7 @@ def test_fullsize_qlinear(awq, name, T):
                    cfg.bits, cfg.group)
     Xt = np.ascontiguousarray(X[:T])
     Y = awq.qlinear(out["codes"], out["scales"], out["zeros"], out["s_best"], torch.from_numpy(Xt).cuda(),
-                    cfg.bits, cfg.group).cpu().numpy()
+                    cfg.bits, cfg.group, tensor_cores=tc).cpu().numpy()
     awq.get_status()
     del Wd
     rows = sample_rows(cfg.N, cfg.seed + T)

@@ -376,7 +376,8 @@ def test_shared_input_joint_search(awq):
                                               (3000, 4352, 12, 3, 64), (136, 640, 4, 4, 128),
                                               (200, 384, 3, 3, 64),
                                               (1536, 2048, 16, 4, 128), (700, 1280, 20, 4, 64)])
-def test_qlinear(awq, N, K, T, bits, group):
+@pytest.mark.parametrize("tc", [False, True, None], ids=["cuda_cores", "tensor_cores", "dispatch"])
+def test_qlinear(awq, N, K, T, bits, group, tc):
     W, X = gen(N, K, T, bits=bits, group=group, seed=N + T, outlier_frac=0.02)
     plant_groups(W, group)
     a = oracle.act_stats(X)
@@ -384,7 +385,7 @@ def test_qlinear(awq, N, K, T, bits, group):
     losses = np.linspace(1.0, 0.5, 20).astype(np.float32)      # chooses alpha = 0.95
     pk = oracle.pack(W, a, bits, group, alphas, losses.astype(np.float64))
     Y = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]), dev(pk["s_best"]),
-                         dev(X), bits, group))
+                         dev(X), bits, group, tensor_cores=tc))
     awq.get_status()
     ref = oracle.qlinear(pk["codes"], pk["scales"], pk["zeros"], pk["s_best"], X, bits, group)
     # binary32 accumulation: bound by the sum of |terms|
@@ -394,9 +395,9 @@ def test_qlinear(awq, N, K, T, bits, group):
     xs = np.abs(X.astype(np.float32) * (np.float32(1) / pk["s_best"]).astype(np.float32)).astype(np.float64)
     bound = xs @ wq.T
     assert np.all(np.abs(Y - ref) <= 2e-6 * bound + 1e-30)
-    # row blocks split across thread blocks are summed in a fixed order
+    # row blocks (and K chunks) split across thread blocks are summed in a fixed order
     Y2 = host(awq.qlinear(dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]),
-                          dev(pk["s_best"]), dev(X), bits, group))
+                          dev(pk["s_best"]), dev(X), bits, group, tensor_cores=tc))
     assert np.array_equal(Y, Y2)
 
 
