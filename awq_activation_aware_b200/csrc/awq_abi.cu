@@ -56,6 +56,40 @@ SearchWs search_ws_layout(int64_t N, int64_t K, int64_t T, int group, int n_alph
     w.total = off;
     return w;
 }
+// One pass of the tensor-core decode, launched so that it may start while the
+// prep grid before it on the stream still runs (programmatic dependent launch):
+// its code stream, tensor-memory allocation and barrier set-up overlap the prep,
+// and the roles that read the prep's outputs wait for it (griddepcontrol.wait).
+template <int NR, int CB, int GPS>
+cudaError_t launch_qtc(unsigned grid, cudaStream_t st, const CUtensorMap &tmap_codes, const CUtensorMap &tmap_b,
+                       const awq::qtc::Args &A) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(awq::qtc::THREADS);
+    cfg.dynamicSmemBytes = awq::qtc::smem_bytes<NR>();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, awq::qlinear_tc_kernel<NR, CB, GPS>, tmap_codes, tmap_b, A);
+}
+
+// The dynamic shared memory of the tensor-core decode instantiations.
+template <int NR>
+bool qtc_attrs() {
+    const int b = (int)awq::qtc::smem_bytes<NR>();
+    return cudaFuncSetAttribute(awq::qlinear_tc_kernel<NR, 4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(awq::qlinear_tc_kernel<NR, 4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(awq::qlinear_tc_kernel<NR, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(awq::qlinear_tc_kernel<NR, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) ==
+               cudaSuccess;
+}
+
 
 awq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
 
@@ -111,12 +145,7 @@ awq_status device_info(DevInfo &out) {
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qtc::smem_bytes<16>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qtc::smem_bytes<32>()) != cudaSuccess ||
-            cudaFuncSetAttribute(awq::qlinear_tc_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)awq::qtc::smem_bytes<48>()) != cudaSuccess ||
+            !qtc_attrs<16>() || !qtc_attrs<32>() || !qtc_attrs<48>() ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -184,7 +213,8 @@ bool encode_codes_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64
     return r == CUDA_SUCCESS;
 }
 
-// Packed code words [rows][words] as boxes of box_words (128 bytes) x box_rows, 128-byte swizzle.
+// Packed code words [rows][words] as boxes of box_words x box_rows: 32 words
+// (128 bytes) with the 128-byte swizzle, 16 words (64 bytes) with the 64-byte one.
 bool encode_words_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64_t words, int box_words,
                       int box_rows) {
     EncodeTiledFn fn = encode_fn();
@@ -194,8 +224,9 @@ bool encode_words_map(CUtensorMap *m, const uint32_t *codes, int64_t rows, int64
     cuuint32_t box[2] = {(cuuint32_t)box_words, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(codes), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_words == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 // bf16 [rows][cols] as boxes of 64 columns x box_rows rows, 128-byte swizzle.
@@ -264,7 +295,7 @@ awq_status noalloc_scratch(void **out) {
 // widest stage), the partial sums of row blocks split across blocks, and the
 // per row block arrival counters.
 constexpr int64_t kQlMaxGrid = 1024;
-constexpr int64_t kQlTcMinTokens = 3;      // awq_qlinear: tensor cores from 3 tokens on
+constexpr int64_t kQlTcMinTokens = 2;      // awq_qlinear: tensor cores from 2 tokens on
 int64_t ql_rows_pad(int64_t T) { return (T + awq::qlv::TOKENS - 1) / awq::qlv::TOKENS * awq::qlv::TOKENS; }
 int64_t ql_cols_pad(int64_t K, int64_t sc) { return (K + sc - 1) / sc * sc; }
 size_t ql_xs_bytes(int64_t T, int64_t K) {
@@ -279,12 +310,12 @@ size_t qlinear_ws_simt(int64_t T, int64_t K, int64_t N) {
            round_up(sizeof(unsigned) * (size_t)ql_row_blocks(N) * awq::qlv::RGROUPS, 256);
 }
 // The tensor-core path: x' pieces bf16 [passes][NR][Kp], group sums fp32
-// [passes][K/64 or fewer groups][16], and per-chunk partial sums fp32
-// [chunks][TT][N] when K is split into chunks.
+// [passes][K/64 or fewer groups][16], partial sums of row blocks split across
+// blocks fp32 [(row blocks + grid) * 128][16] and their arrival counters.
 struct QtcPlan {
-    int NR, TT, n_pass, n_chunks;
-    int64_t Kp, chunk, units;
-    size_t xb_bytes, gs_bytes, part_bytes;
+    int NR, TT, n_pass;
+    int64_t Kp, row_blocks, n_steps, units;
+    size_t xb_bytes, gs_bytes, part_bytes, cnt_bytes;
 };
 QtcPlan qtc_plan(int64_t T, int64_t K, int64_t N, int group) {
     QtcPlan p;
@@ -292,19 +323,19 @@ QtcPlan qtc_plan(int64_t T, int64_t K, int64_t N, int group) {
     p.TT = awq::qtc::tile_tokens(p.NR);
     p.n_pass = (int)((T + p.TT - 1) / p.TT);
     p.Kp = (K + 63) / 64 * 64;
-    const int64_t rb = (N + awq::qtc::ROWS - 1) / awq::qtc::ROWS;
-    p.chunk = awq::qtc::CHUNK;                              // at most 8 groups a unit: the epilogue prefetches them
-    p.n_chunks = (int)((K + p.chunk - 1) / p.chunk);
-    p.units = rb * p.n_chunks;
+    p.row_blocks = (N + awq::qtc::ROWS - 1) / awq::qtc::ROWS;
+    p.n_steps = (K + awq::qtc::SC - 1) / awq::qtc::SC;
+    p.units = p.row_blocks * p.n_steps;
     p.xb_bytes = round_up(2 * (size_t)p.n_pass * p.NR * p.Kp, 1024);
     p.gs_bytes = round_up(4 * (size_t)p.n_pass * (size_t)(K / group) * 16, 256);
-    p.part_bytes = p.n_chunks > 1 ? round_up(4 * (size_t)p.n_chunks * p.TT * N, 256) : 0;
+    p.part_bytes = round_up(sizeof(float) * (size_t)(p.row_blocks + kQlMaxGrid) * awq::qtc::SLOT_FLOATS, 256);
+    p.cnt_bytes = round_up(sizeof(unsigned) * (size_t)p.row_blocks * 4, 256);
     return p;
 }
 size_t qtc_ws_bound(int64_t T, int64_t K, int64_t N) {
     // the largest plan over group sizes: 64-column groups
     const QtcPlan p = qtc_plan(T, K, N, 64);
-    return p.xb_bytes + p.gs_bytes + p.part_bytes;
+    return p.xb_bytes + p.gs_bytes + p.part_bytes + p.cnt_bytes;
 }
 size_t qlinear_ws(int64_t T, int64_t K, int64_t N) {
     const size_t a = qlinear_ws_simt(T, K, N), b = qtc_ws_bound(T, K, N);
@@ -858,62 +889,60 @@ awq_status awq_qlinear_tc(const uint32_t *codes, const void *scales, const void 
     __nv_bfloat16 *xb = reinterpret_cast<__nv_bfloat16 *>(w8);
     float *gsum = reinterpret_cast<float *>(w8 + P.xb_bytes);
     float *part = reinterpret_cast<float *>(w8 + P.xb_bytes + P.gs_bytes);
+    unsigned *cnt = reinterpret_cast<unsigned *>(w8 + P.xb_bytes + P.gs_bytes + P.part_bytes);
     {
-        int grid = blocks_for((int64_t)P.n_pass * P.NR * P.Kp, 256);
+        const int64_t work = std::max((int64_t)P.n_pass * P.NR * P.Kp, (int64_t)P.n_pass * G * 16 * 16);
+        int grid = blocks_for(work, 256);
         if (grid > 8 * d.sms) grid = 8 * d.sms;
         awq::qtc_prep_kernel<<<grid, 256, 0, st>>>((const __half *)X, T, K, P.Kp, ldx, s_best, P.TT, P.NR, P.n_pass,
-                                                   xb);
-        if (awq_status e = last_launch()) return e;
-        int grid2 = blocks_for((int64_t)P.n_pass * G * 16 * 16, 256);       // 16 lanes per group sum
-        if (grid2 > 8 * d.sms) grid2 = 8 * d.sms;
-        awq::qtc_gsum_kernel<<<grid2, 256, 0, st>>>((const __half *)X, T, K, ldx, s_best, P.TT, P.n_pass, G,
-                                                    q.group_size, gsum);
+                                                   G, q.group_size, xb, gsum, cnt, P.row_blocks * 4);
         if (awq_status e = last_launch()) return e;
     }
-    const int cpw = q.bits == 2 ? 16 : 8;
+    const bool c2 = q.bits == 2;
+    const int cpw = c2 ? 16 : 8;
     CUtensorMap tmap_codes, tmap_b;
-    if (!encode_words_map(&tmap_codes, codes, N, K / cpw, awq::qtc::CODE_ROW_BYTES / 4, awq::qtc::ROWS) ||
+    if (!encode_words_map(&tmap_codes, codes, N, K / cpw, c2 ? 16 : 32, awq::qtc::ROWS) ||
         !encode_bf16_map(&tmap_b, xb, (int64_t)P.n_pass * P.NR, P.Kp, P.NR))
         return AWQ_ERR_CUDA;
     awq::qtc::Args A;
     A.scales = (const __half *)scales;
     A.zeros = (const __half *)zeros;
     A.N = N;
-    A.K = K;
     A.G = G;
-    A.group = q.group_size;
-    A.cpw = cpw;
-    A.chunk = P.chunk;
-    A.n_chunks = P.n_chunks;
+    A.n_steps = P.n_steps;
     A.units = P.units;
     A.part = part;
+    A.cnt = cnt;
     A.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
-    const int64_t grid = P.units < d.sms ? P.units : d.sms;
+    int64_t grid = d.sms < kQlMaxGrid ? d.sms : kQlMaxGrid;
+    if (grid > P.units) grid = P.units;
+    const bool g64 = q.group_size == 64;
     for (int pass = 0; pass < P.n_pass; ++pass) {
         A.gsum = gsum + (int64_t)pass * G * 16;
         A.Y = Y + (int64_t)pass * P.TT * N;
         A.T = (int)(T - (int64_t)pass * P.TT < P.TT ? T - (int64_t)pass * P.TT : P.TT);
         A.b_row0 = pass * P.NR;
         const unsigned g = (unsigned)grid;
-        if (P.NR == 16)
-            awq::qlinear_tc_kernel<16><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<16>(), st>>>(tmap_codes, tmap_b, A);
-        else if (P.NR == 32)
-            awq::qlinear_tc_kernel<32><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<32>(), st>>>(tmap_codes, tmap_b, A);
-        else
-            awq::qlinear_tc_kernel<48><<<g, awq::qtc::THREADS, awq::qtc::smem_bytes<48>(), st>>>(tmap_codes, tmap_b, A);
+        cudaError_t err;
+#define AWQ_QTC_LAUNCH(NR, CB, GPS) err = launch_qtc<NR, CB, GPS>(g, st, tmap_codes, tmap_b, A)
+#define AWQ_QTC_BY_CODE(NR)                                                   \
+    do {                                                                      \
+        if (c2) { if (g64) AWQ_QTC_LAUNCH(NR, 2, 4); else AWQ_QTC_LAUNCH(NR, 2, 2); } \
+        else { if (g64) AWQ_QTC_LAUNCH(NR, 4, 4); else AWQ_QTC_LAUNCH(NR, 4, 2); }    \
+    } while (0)
+        if (P.NR == 16) AWQ_QTC_BY_CODE(16);
+        else if (P.NR == 32) AWQ_QTC_BY_CODE(32);
+        else AWQ_QTC_BY_CODE(48);
+#undef AWQ_QTC_BY_CODE
+#undef AWQ_QTC_LAUNCH
+        if (err != cudaSuccess) return AWQ_ERR_CUDA;
         if (awq_status e = last_launch()) return e;
-        if (P.n_chunks > 1) {
-            int grid3 = blocks_for((int64_t)A.T * N, 256);
-            if (grid3 > 8 * d.sms) grid3 = 8 * d.sms;
-            awq::qtc_reduce_kernel<<<grid3, 256, 0, st>>>(part, P.n_chunks, P.TT, A.T, N, A.Y);
-            if (awq_status e = last_launch()) return e;
-        }
     }
     return AWQ_OK;
 }
 
 // From kQlTcMinTokens tokens on, one tensor-core pass reads the codes once for
-// up to 16 tokens, where the CUDA-core kernel reads them once per 2 or 4.
+// up to 16 tokens, where the CUDA-core kernel reads them once per 1, 2 or 4.
 awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
                        int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
                        void *ws, size_t ws_bytes, void *stream) {

@@ -515,6 +515,13 @@ __host__ __device__ constexpr uint32_t mma_idesc_f16_f32(int M, int N) {
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// ----- programmatic dependent launch ---------------------------------------
+// Wait until the grids this one depends on have completed and their writes are
+// visible (a no-op when the launch had no programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid be scheduled before this one completes.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----- tcgen05, one CTA (cta_group::1) --------------------------------------
 __device__ __forceinline__ void tmem_alloc_1(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),

@@ -1373,108 +1373,175 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
 // unit's sums go to Y directly (one chunk) or to per-chunk partials that a
 // second kernel adds in chunk order, so Y does not depend on timing.
 // ===========================================================================
-// Row r's 64 codes starting at 16-byte chunk `chunk0` of a 128-byte-swizzled
-// code tile (two chunks of 4-bit codes or one of 2-bit codes) as 32 bf16x2
-// words for the A operand in tensor memory (column i holds A columns 2i and
-// 2i + 1, the lower in the low half).  Each 8-column chunk of A holds its codes
-// in the order (0, 4, 1, 5, 2, 6, 3, 7): pair e is (code e, code e + 4), which
-// one mask of the word (shifted by e code widths) places in the two halves of a
-// 32-bit word under the bf16 exponent of 128; a bf16x2 subtraction of 128 then
-// leaves the exact codes.  The B operand's columns follow the same order.  The
-// 8 rows of a quarter warp read 8 distinct chunk positions of the swizzle.
+// ---------------------------------------------------------------------------
+// The decode consumer on the tensor cores (qlinear_tc_kernel), [AWQ-note]
+// "Tiny Chat" (dequantization inside the kernel) with reading 22's exact
+// products:
+//   Y[t, n] = sum_g sh[n, g] (D_g[n, t] - z[n, g] S_g[t]),
+//   D_g[n, t] = sum_{k in g} q[n, k] x'[t, k]   (tcgen05, bf16 operands, fp32 accumulation)
+//   S_g[t] = RN32(sum_{k in g} x'[t, k]) in binary64 (qtc_gsum_kernel).
+// q is exact in bf16 and x' = hi + mid + lo exactly (three bf16 pieces, the B
+// rows), so every product is exact and only the fp32 accumulation rounds.
+// ---------------------------------------------------------------------------
+
+// The 8 codes of one 8-column chunk (code e in bits CB e .. of x) as 4 bf16x2
+// words of A: word e holds (code e, code e + 4).  One mask places the two codes
+// in the two halves under the bf16 exponent of 128, one bf16x2 subtraction of
+// 128 leaves them exactly.  The B operand's columns follow the same order
+// (column 2e of the chunk is x' of column e, column 2e + 1 that of e + 4).
 template <int CB>
-__device__ __forceinline__ void qtc_convert_half(const uint8_t *ct, int r, int chunk0, uint32_t (&v)[32]) {
+__device__ __forceinline__ void qtc_chunk_bf16(uint32_t x, uint32_t *v) {
     const __nv_bfloat162 off = __floats2bfloat162_rn(128.0f, 128.0f);
     constexpr uint32_t mask = CB == 4 ? 0x000F000Fu : 0x00030003u;
-    constexpr int NCH = CB == 4 ? 2 : 1;
-    uint32_t w[4 * NCH];
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(ct + r * 128 + (((chunk0 + c) ^ (r & 7)) << 4));
-        w[4 * c] = q.x; w[4 * c + 1] = q.y; w[4 * c + 2] = q.z; w[4 * c + 3] = q.w;
-    }
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {                                        // 8-column chunk h
-        uint32_t x;
-        if (CB == 4) x = w[h];
-        else x = __byte_perm(w[h >> 1], 0u, (h & 1) ? 0x4342u : 0x4140u);   // codes 0-3 in byte 0, codes 4-7 in byte 2
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t u = ((x >> (CB * e)) & mask) | 0x43004300u;
-            const __nv_bfloat162 b = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&u), off);
-            v[4 * h + e] = *reinterpret_cast<const uint32_t *>(&b);
-        }
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t u = ((x >> (CB * e)) & mask) | 0x43004300u;
+        const __nv_bfloat162 b = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&u), off);
+        v[e] = *reinterpret_cast<const uint32_t *>(&b);
     }
 }
 
 namespace qtc {
-constexpr int ROWS = 128;                  // weight rows per unit (MMA M)
-constexpr int SK = 128;                    // K columns per sub-stage (8 MMAs of K 16; one or two groups)
-constexpr int CODE_ROW_BYTES = 128;        // codes per row per code stage: 256 (4-bit) or 512 (2-bit) columns
-constexpr int CS = 8;                      // code ring depth (16 KiB stages)
-constexpr int AS_MAX = 6, NB_MAX = 8;
+constexpr int ROWS = 128;                 // W rows per unit (MMA M)
+constexpr int SC = 256;                   // K columns per unit: 16 MMAs of K 16
+constexpr int A_COLS = SC / 2;            // tensor-memory columns of one A slot (2 bf16 per column)
 constexpr int TMEM_COLS = 512;
-constexpr int PROD_WARP0 = 8, NUM_PROD_WARPS = 8, EPI_WARP0 = 4;
-constexpr int LOAD_WARP = 0, MMA_WARP = 1, ALLOC_WARP = 2, B_LOAD_WARP = 3;   // warp 2 also issues MMAs
-constexpr int THREADS = (PROD_WARP0 + NUM_PROD_WARPS) * 32;     // 512
-constexpr int CODE_BYTES = ROWS * CODE_ROW_BYTES;               // 16 KiB
-constexpr int CHUNK = 512;                                      // K columns per unit
-constexpr int MAXG = CHUNK / 64;                                // groups per unit at most
+constexpr int CODE_BYTES = ROWS * 128;    // one unit's codes: 128 (4-bit) or 64 (2-bit) bytes a row
+constexpr int TT_MAX = 16;
+constexpr int SLOT_FLOATS = ROWS * TT_MAX;                    // one partial-sum slot: 128 rows x 16 tokens
+constexpr int PWARPS = 8;                 // producers: lane quadrant warp % 4, column half warp / 4
+constexpr int EWARP0 = 8;                 // epilogue: warps 8-11, lane quadrant warp - 8, one row per thread
+constexpr int MMA_WARP = 12, LOAD_WARP = 13, BLOAD_WARP = 14, MMA_WARP2 = 15;   // MMA issue (two warps); code loads; B loads
+constexpr int THREADS = 16 * 32;
+// Token tiles: N = 16, 32 or 48 rows of x' pieces per pass (5, 10 or 16 tokens).
 __host__ __device__ constexpr int tile_tokens(int nr) { return nr == 16 ? 5 : nr == 32 ? 10 : 16; }
-// Tensor memory: sub-stage slots of A (64 columns each) at the top, the
-// accumulators (one per group, NR columns each) below them.
-__host__ __device__ constexpr int a_slots(int nr) { return nr == 48 ? 4 : 6; }
-__host__ __device__ constexpr int a_col0(int nr) { return TMEM_COLS - a_slots(nr) * 64; }
-__host__ __device__ constexpr int acc_slots(int nr) { return nr == 16 ? 8 : nr == 32 ? 4 : 5; }
-static_assert(acc_slots(16) * 16 <= a_col0(16) && acc_slots(32) * 32 <= a_col0(32) &&
-              acc_slots(48) * 48 <= a_col0(48), "tensor-memory layout");
-
-// Sub-stage slot i holds A in tensor memory and the B tile (NR x 128 bf16, two
-// 128-byte-swizzled boxes of 64 columns) in shared memory; one MMA commit
-// (slot_empty) releases both.
-template <int NR>
-struct Smem {
-    uint8_t codes[CS][CODE_BYTES];         // every tile 1024-byte aligned
-    uint8_t b[a_slots(NR)][NR * SK * 2];   // box 0 at 0, box 1 at NR x 128 bytes: 1024-byte aligned
-    float gs[2][MAXG * 16];                // group sums of the current / next unit (epilogue)
-    uint64_t c_full[CS], c_empty[CS];
-    uint64_t a_full[AS_MAX], b_full[AS_MAX], slot_empty[AS_MAX];
-    uint64_t acc_full[NB_MAX], acc_empty[NB_MAX];
-    uint64_t drain[2];
-    uint32_t tmem_base;
-    int abort_flag;
-};
-template <int NR>
-constexpr size_t smem_bytes() { return sizeof(Smem<NR>) + 1024; }
+template <int NR> __host__ __device__ constexpr int b_bytes() { return NR * SC * 2; }   // 4 swizzled boxes of NR x 64
+// Two rings: code tiles, freed as soon as the producers hold them in registers,
+// deep enough to cover the load latency of HBM under load; B tiles, freed when
+// the MMAs that read them complete.
+template <int NR> __host__ __device__ constexpr int code_stages() { return NR == 16 ? 10 : NR == 32 ? 8 : 7; }
+constexpr int B_STAGES = 4;
+// Accumulator columns of one unit: one NR-wide block per group of the unit.
+template <int NR, int GPS> __host__ __device__ constexpr int d_cols() { return GPS * NR; }
+template <int NR, int GPS> __host__ __device__ constexpr int a_slots() {
+    return 3 * A_COLS + 2 * d_cols<NR, GPS>() <= TMEM_COLS ? 3 : 2;
+}
+template <int NR, int GPS> __host__ __device__ constexpr int d_bufs() {
+    return (TMEM_COLS - a_slots<NR, GPS>() * A_COLS) / d_cols<NR, GPS>() > 4
+               ? 4
+               : (TMEM_COLS - a_slots<NR, GPS>() * A_COLS) / d_cols<NR, GPS>();
+}
+// Group sums S of the epilogue: per epilogue warp, two slots of 4 groups x 16 tokens.
+constexpr int S_AREA_BYTES = 4 * 2 * 64 * 4;
+template <int NR> constexpr size_t smem_bytes() {
+    return (size_t)code_stages<NR>() * CODE_BYTES + (size_t)B_STAGES * b_bytes<NR>() + 1024 + 512 + S_AREA_BYTES;
+}
 static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448 && smem_bytes<48>() <= 232448,
               "decode shared memory above the 227 KiB a CTA may use");
-
+// The block whose unit range [units*b/grid, units*(b+1)/grid) holds unit u.
+__device__ __forceinline__ int64_t block_of(int64_t u, int64_t units, int64_t grid) {
+    return ((u + 1) * grid - 1) / units;
+}
+// word i (0..4 NCH - 1) of NCH 16-byte chunks, i known at compile time
+template <int NCH>
+__device__ __forceinline__ uint32_t word_of(const uint4 (&cw)[NCH], int i) {
+    const uint4 c = cw[i >> 2];
+    return (i & 3) == 0 ? c.x : (i & 3) == 1 ? c.y : (i & 3) == 2 ? c.z : c.w;
+}
+// fp16 value o (0..7) of eight packed in 16 bytes
+__device__ __forceinline__ float half_at(const uint4 &v, int o) {
+    const uint32_t w = (o >> 1) == 0 ? v.x : (o >> 1) == 1 ? v.y : (o >> 1) == 2 ? v.z : v.w;
+    return __half2float(__ushort_as_half((unsigned short)((o & 1) ? (w >> 16) : (w & 0xFFFFu))));
+}
+// One row's fp16 values by group ([N][G] scales or zeros) for the units a block
+// walks through in order.  With G a multiple of 8 the thread reads 8 groups (16
+// bytes) at a time, one chunk ahead of use; otherwise one value per group at use.
+template <int GPS>
+struct RowGroups {
+    const __half *p;
+    int64_t N, n_steps;
+    int G, rr;
+    bool vec;
+    uint4 cur, nxt;
+    int64_t nrb;                          // chunk held in nxt: row block, chunk index
+    int nc;
+    __device__ __forceinline__ uint4 fetch(int64_t rb, int c) const {
+        int64_t n = rb * ROWS + rr;
+        n = n < N ? n : N - 1;
+        return __ldg(reinterpret_cast<const uint4 *>(p + n * G) + c);
+    }
+    // the chunk after (nrb, nc): a row block's chunks end at its n_steps * GPS
+    // groups (= G when G is a multiple of 8, since K is then a multiple of 256)
+    __device__ __forceinline__ void next_chunk() {
+        if ((int64_t)(nc + 1) * 8 < n_steps * GPS) {
+            ++nc;
+        } else {
+            ++nrb;
+            nc = 0;
+        }
+    }
+    __device__ __forceinline__ void begin(int64_t rb, int64_t j) {
+        vec = G % 8 == 0;
+        if (vec) {
+            nrb = rb;
+            nc = (int)((j * GPS) >> 3);
+            cur = fetch(nrb, nc);
+            next_chunk();
+            nxt = fetch(nrb, nc);
+        }
+    }
+    // called on reaching unit (., j), for every unit after the first
+    __device__ __forceinline__ void enter(int64_t j) {
+        if (vec && ((j * GPS) & 7) == 0) {
+            cur = nxt;
+            next_chunk();
+            nxt = fetch(nrb, nc);
+        }
+    }
+    __device__ __forceinline__ float get(int64_t rb, int64_t j, int g) const {
+        const int64_t gg = j * GPS + g;
+        if (vec) return half_at(cur, (int)(gg & 7));
+        int64_t n = rb * ROWS + rr;
+        n = n < N ? n : N - 1;
+        return __half2float(__ldg(p + n * G + gg));
+    }
+};
 struct Args {
     const __half *scales, *zeros;          // [N][G]
-    const float *gsum;                     // S: [G][16] for this pass
-    float *Y;                              // this pass's output rows [T][N] (one chunk) ...
-    float *part;                           // ... or partials [chunks][TT][N]
-    int64_t N, K;
-    int G, group, cpw;                     // groups, group size, codes per 32-bit word (8 or 16)
-    int T;                                 // tokens of this pass (<= TT)
-    int b_row0;                            // first B row of this pass in the B map
-    int64_t chunk;                         // K columns per chunk (CHUNK)
-    int n_chunks;
-    int64_t units;                         // row blocks x chunks
+    const float *gsum;                     // S of this pass: [G][16]
+    int64_t N;
+    int G, T;                              // groups per row; tokens of this pass (<= TT)
+    int64_t n_steps, units;                // units per row block (K / 256, rounded up); row blocks x n_steps
+    int32_t b_row0;                        // first B row of this pass in the B map
+    float *Y;                              // this pass's output rows [T][N]
+    float *part;                           // partial sums of split row blocks: [(row blocks + grid) * 128][16]
+    unsigned *cnt;                         // arrivals per row block and lane quadrant [row blocks][4]
     uint64_t timeout_ns;
 };
 }  // namespace qtc
 
-// x' = RN32(x RN32(1/s)) split into three bf16 pieces, stored as the B rows of
-// every pass: row piece * TT + t of pass p holds piece `piece` of token
-// p TT + t; within each 8-column chunk column p holds x' of column
-// (p / 2) + 4 (p % 2), the order of the A tile's codes (qtc_convert); rows past
-// 3 TT, tokens past T and columns past K are zero.
+// The operands the main kernel reads besides the codes, in one launch:
+//   xb: x' = RN32(x RN32(1/s)) split into three bf16 pieces, stored as the B rows
+//       of every pass: row piece * TT + t of pass p holds piece `piece` of token
+//       p TT + t; within each 8-column chunk column c holds x' of column
+//       (c / 2) + 4 (c % 2), the order of A's codes (qtc_chunk_bf16); rows past
+//       3 TT, tokens past T and columns past K are zero;
+//   gsum: S[p][g][t] = RN32(sum over the group's columns of x'[p TT + t, k]) in
+//       binary64 (16 slots per group; tokens past the pass or past T give 0).  16
+//       lanes per value: lane j sums columns j * group/16 .. + group/16 - 1, then
+//       the 16 partial sums are added by shuffles (that loop's thread count is a
+//       multiple of 32, and so is the grid's);
+//   cnt: the main kernel's arrival counters, cleared.
+// The main kernel may start early (programmatic dependent launch): its roles
+// that read these wait for this grid with griddepcontrol.wait.
 __global__ void qtc_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t Kp, int64_t ldx,
-                                const float *__restrict__ s, int TT, int NR, int n_pass,
-                                __nv_bfloat16 *__restrict__ xb) {
+                                const float *__restrict__ s, int TT, int NR, int n_pass, int G, int group,
+                                __nv_bfloat16 *__restrict__ xb, float *__restrict__ gsum,
+                                unsigned *__restrict__ cnt, int64_t n_cnt) {
+    griddep_launch_dependents();
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, nth = (int64_t)gridDim.x * blockDim.x;
     const int64_t total = (int64_t)n_pass * NR * Kp;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t i = tid; i < total; i += nth) {
         const int64_t kb = i % Kp, rowg = i / Kp;
         const int64_t k = (kb & ~int64_t(7)) + ((kb & 7) >> 1) + 4 * (kb & 1);
         const int row = (int)(rowg % NR), pass = (int)(rowg / NR);
@@ -1491,18 +1558,9 @@ __global__ void qtc_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t
         }
         xb[i] = __float2bfloat16_rn(v);                                          // exact for every piece
     }
-}
-
-// S[p][g][t] = RN32(sum over the group's columns of x'[p TT + t, k]) in
-// binary64 (16 slots per group; tokens past the pass or past T give 0).  16
-// lanes per output: lane j sums columns j * group/16 .. + group/16 - 1, then the
-// 16 partial sums are added by shuffles (total threads a multiple of 32).
-__global__ void qtc_gsum_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t ldx,
-                                const float *__restrict__ s, int TT, int n_pass, int G, int group,
-                                float *__restrict__ gsum) {
-    const int64_t total = (int64_t)n_pass * G * 16 * 16;
+    const int64_t gtotal = (int64_t)n_pass * G * 16 * 16;
     const int per = group / 16;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t i = tid; i < gtotal; i += nth) {
         const int j = (int)(i & 15);
         const int64_t o = i >> 4;
         const int t = (int)(o % 16);
@@ -1519,301 +1577,334 @@ __global__ void qtc_gsum_kernel(const __half *__restrict__ X, int64_t T, int64_t
         for (int o2 = 8; o2 >= 1; o2 >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o2));
         if (j == 0) gsum[o] = __double2float_rn(acc);
     }
+    for (int64_t i = tid; i < n_cnt; i += nth) cnt[i] = 0u;
 }
 
-// Y[t, n] = sum over chunks, in chunk order, of the partial sums.
-__global__ void qtc_reduce_kernel(const float *__restrict__ part, int n_chunks, int TT, int T, int64_t N,
-                                  float *__restrict__ Y) {
-    const int64_t total = (int64_t)T * N;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = i / N, n = i - t * N;
-        const float *p0 = part + t * N + n;
-        const int64_t cs = (int64_t)TT * N;                          // one chunk's stride
-        float y = 0.0f;
-        int c = 0;
-        for (; c + 4 <= n_chunks; c += 4) {                          // loads issued together, added in chunk order
-            const float v0 = p0[c * cs], v1 = p0[(c + 1) * cs], v2 = p0[(c + 2) * cs], v3 = p0[(c + 3) * cs];
-            y = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(y, v0), v1), v2), v3);
-        }
-        for (; c < n_chunks; ++c) y = __fadd_rn(y, p0[c * cs]);
-        Y[i] = y;
-    }
-}
-
-template <int NR>
+// One pass (up to TT tokens) of the packed layer on the tensor cores.  Persistent:
+// block b takes the contiguous units [units b / grid, units (b + 1) / grid) of the
+// list (row block of 128 rows, step of 256 columns), row-block major, so every
+// block streams the same number of code bytes.  Roles:
+//   warp 13: the codes, one 2-D TMA tile per unit (128 rows x 128 or 64 bytes,
+//            swizzled), into a ring of code_stages tiles;
+//   warp 14: the unit's B tile, 4 boxes of NR x 64 bf16 (128-byte swizzle);
+//   warps 0-7: producers; warp w converts columns 128 (w / 4) .. + 127 of the rows
+//            of lane quadrant w % 4 (one row per thread) into A slot as of tensor
+//            memory with tcgen05.st, after releasing the code tile;
+//   warps 12 and 15: one thread each issues the 16 MMAs of every other unit (A
+//            from tensor memory, B from shared memory) into one accumulator per
+//            group, then commits;
+//   warps 8-11: epilogue; each thread drains its row's accumulators, applies
+//            sh (D - z S) and, at the end of its row block's segment, writes Y or
+//            a partial sum that the last block to arrive adds in block order.
+template <int NR, int CB, int GPS>
 __global__ void __launch_bounds__(qtc::THREADS, 1)
 qlinear_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_b,
                   const qtc::Args A) {
     using namespace qtc;
+    constexpr int CS = code_stages<NR>();
+    constexpr int BS = B_STAGES;
+    constexpr int D_COLS = d_cols<NR, GPS>();
+    constexpr int AS = a_slots<NR, GPS>();         // A slots in tensor memory
+    constexpr int DB = d_bufs<NR, GPS>();          // accumulator buffers
+    constexpr int MPG = 16 / GPS;                  // MMAs (K 16 each) per group
+    // Issuing threads.  A thread that takes every other unit waits on an
+    // accumulator buffer's d_empty for every other release of it; its parity
+    // wait is unambiguous only if the buffer ring holds two or more buffers.
+    constexpr int NISSUE = DB >= 2 ? 2 : 1;
     constexpr int TT = tile_tokens(NR);
+    constexpr int NCH = CB == 4 ? 4 : 2;           // 16-byte code chunks of a producer thread per unit
+    static_assert(AS * A_COLS + DB * D_COLS <= TMEM_COLS && DB >= 1, "tensor memory budget");
+    static_assert(3 * TT <= NR, "three pieces per token");
     constexpr uint32_t IDESC = mma_idesc_bf16_f32(ROWS, NR);
+    constexpr uint32_t B_BYTES = b_bytes<NR>();
+    constexpr uint32_t CODE_TX = ROWS * (CB == 4 ? 128 : 64);
     extern __shared__ uint8_t smem_raw[];
-    using SmemT = Smem<NR>;
-    SmemT &S = *reinterpret_cast<SmemT *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *bring = base + CS * CODE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(bring + BS * B_BYTES);
+    uint64_t *full = bars, *empty = bars + CS, *b_full = bars + 2 * CS, *b_empty = b_full + BS;
+    uint64_t *a_full = b_empty + BS, *a_empty = a_full + AS, *d_full = a_empty + AS, *d_empty = d_full + DB;
+    uint64_t *drain = d_empty + DB;                // one per issuing thread
+    static_assert((2 * CS + 2 * BS + 2 * AS + 2 * DB + 2) * 8 <= 512, "barrier area");
+    float *s_area = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + 512);
+    __shared__ uint32_t tmem_base_sm;
+    __shared__ int abort_sm;
+    volatile int *abort_flag = &abort_sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    volatile int *abort_flag = &S.abort_flag;
-    constexpr int NB = acc_slots(NR), AS = a_slots(NR), A_COL0 = a_col0(NR);
-    const int spc = CODE_ROW_BYTES * 8 / (32 / A.cpw) / SK;       // sub-stages per code stage: 2 (4-bit) or 4 (2-bit)
-    const int kpg = A.group / 16;                                 // MMAs per group: 4 or 8
     const int64_t grid = gridDim.x;
-
+    const int64_t u_begin = A.units * blockIdx.x / grid, u_end = A.units * (blockIdx.x + 1) / grid;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < CS; ++i) { mbar_init(&S.c_full[i], 1); mbar_init(&S.c_empty[i], 4 * spc); }
-        for (int i = 0; i < AS; ++i) { mbar_init(&S.a_full[i], 4); mbar_init(&S.b_full[i], 1); mbar_init(&S.slot_empty[i], 1); }
-        for (int i = 0; i < NB; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 4); }
-        mbar_init(&S.drain[0], 1);
-        mbar_init(&S.drain[1], 1);
-        S.abort_flag = 0;
+        for (int i = 0; i < CS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], PWARPS); }
+        for (int i = 0; i < BS; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], PWARPS); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < DB; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
+        abort_sm = 0;
         fence_mbar_init();
     }
-    if (warp == ALLOC_WARP) {
-        tmem_alloc_1(&S.tmem_base, TMEM_COLS);
+    if (warp == MMA_WARP) {
+        tmem_alloc_1(&tmem_base_sm, TMEM_COLS);
         tmem_relinquish_1();
-        tc_fence_before();
     }
+    tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = S.tmem_base;
+    const uint32_t tmem = tmem_base_sm;
     bool aborted = false;
 
-    // unit u: columns [k0, k0 + cols) of row block rb, in subs sub-stages (the
-    // last one of 64 columns when cols is an odd multiple of 64)
-    auto unit_span = [&](int64_t u, int64_t &rb, int64_t &k0, int &cols, int &subs) {
-        rb = u / A.n_chunks;
-        const int64_t kc = u - rb * A.n_chunks;
-        k0 = kc * A.chunk;
-        cols = (int)(A.K - k0 < A.chunk ? A.K - k0 : A.chunk);   // a multiple of 64
-        subs = (cols + SK - 1) / SK;
-    };
-
-    if (warp == LOAD_WARP) {
-        // the code stream from HBM: 128 bytes of each of the unit's 128 rows per stage
+    if (warp == LOAD_WARP) {                       // code tiles (TMA)
         if (lane == 0) {
             tma_prefetch_desc(&tmap_codes);
-            int cs = 0;
-            uint32_t cph = 0;
-            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
-                int64_t rb, k0;
-                int cols, subs;
-                unit_span(u, rb, k0, cols, subs);
-                for (int sub = 0; sub < subs; sub += spc) {
-                    if (!mbar_wait_bounded(&S.c_empty[cs], cph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
-                    mbar_arrive_expect_tx(&S.c_full[cs], CODE_BYTES);
-                    tma_load_2d(&S.codes[cs][0], &tmap_codes, (int32_t)((k0 + (int64_t)sub * SK) / A.cpw),
-                                (int32_t)(rb * ROWS), &S.c_full[cs]);
-                    if (++cs == CS) { cs = 0; cph ^= 1u; }
-                }
+            int st = 0;
+            uint32_t ph = 0;
+            int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+            for (int64_t u = u_begin; u < u_end; ++u) {
+                if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                mbar_arrive_expect_tx(&full[st], CODE_TX);
+                tma_load_2d(base + st * CODE_BYTES, &tmap_codes, (int32_t)(j * (SC * CB / 32)), (int32_t)(rb * ROWS),
+                            &full[st]);
+                if (++st == CS) { st = 0; ph ^= 1u; }
+                if (++j == A.n_steps) { j = 0; ++rb; }
             }
         }
-    } else if (warp == B_LOAD_WARP) {
-        // the B tiles (x' pieces, L2-resident): two boxes of 64 columns per sub-stage slot
+    } else if (warp == BLOAD_WARP) {               // x' pieces of the unit's 256 columns (TMA)
         if (lane == 0) {
             tma_prefetch_desc(&tmap_b);
-            int bs = 0;
-            uint32_t bph = 0;
-            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
-                int64_t rb, k0;
-                int cols, subs;
-                unit_span(u, rb, k0, cols, subs);
-                for (int sub = 0; sub < subs; ++sub) {
-                    if (!mbar_wait_bounded(&S.slot_empty[bs], bph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
-                    mbar_arrive_expect_tx(&S.b_full[bs], (uint32_t)(NR * SK * 2));
-                    const int32_t x = (int32_t)(k0 + (int64_t)sub * SK);
-                    tma_load_2d(&S.b[bs][0], &tmap_b, x, A.b_row0, &S.b_full[bs]);
-                    tma_load_2d(&S.b[bs][NR * 128], &tmap_b, x + 64, A.b_row0, &S.b_full[bs]);
-                    if (++bs == AS) { bs = 0; bph ^= 1u; }
-                }
+            griddep_wait();                        // x' pieces written by the prep grid
+            int st = 0;
+            uint32_t ph = 0;
+            int64_t j = u_begin % A.n_steps;
+            for (int64_t u = u_begin; u < u_end; ++u) {
+                if (!mbar_wait_bounded(&b_empty[st], ph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+                uint8_t *bst = bring + st * B_BYTES;
+                mbar_arrive_expect_tx(&b_full[st], B_BYTES);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    tma_load_2d(bst + a * NR * 128, &tmap_b, (int32_t)(j * SC + a * 64), A.b_row0, &b_full[st]);
+                if (++st == BS) { st = 0; ph ^= 1u; }
+                if (++j == A.n_steps) j = 0;
             }
         }
-    } else if (warp == MMA_WARP || warp == ALLOC_WARP) {
-        // Two issuing threads, one per warp: thread mt takes the sub-stages of
-        // parity mt (each holds whole groups, so every group's MMAs are issued by
-        // one thread in order), and the two threads' issue latencies overlap.
-        // Each thread follows the whole sequence of slots and accumulators.
+    } else if (warp == MMA_WARP || warp == MMA_WARP2) {   // two threads issue the MMAs, units in turn
         if (lane == 0) {
+            // thread mt takes the units u_begin + mt, u_begin + mt + NISSUE, ...: each
+            // unit's MMAs come from one thread in order, and the two threads' issue
+            // latencies overlap.  Both follow every unit's slots and phases.
             const int mt = warp == MMA_WARP ? 0 : 1;
-            const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(&S.b[0][0]));
-            int as = 0, nb = 0;
-            uint32_t aph = 0, accph = 0, gsub = 0;
-            for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
-                int64_t rb, k0;
-                int cols, subs;
-                unit_span(u, rb, k0, cols, subs);
-                for (int sub = 0; sub < subs && !aborted; ++sub, ++gsub) {
-                    const bool mine = (int)(gsub & 1u) == mt;
-                    const int ng = (cols - sub * SK < SK ? cols - sub * SK : SK) / A.group;   // groups in this sub-stage
-                    if (mine) {
-                        if (!mbar_wait_bounded(&S.a_full[as], aph, abort_flag, A.timeout_ns) ||
-                            !mbar_wait_bounded(&S.b_full[as], aph, abort_flag, A.timeout_ns)) { aborted = true; break; }
-                        tc_fence_after();
-                    }
-                    const uint32_t a_tmem = tmem + (uint32_t)(A_COL0 + as * 64);
-                    const uint64_t bdesc = bdesc0 + (uint64_t)((as * NR * SK * 2) >> 4);   // start address field
-                    for (int gl = 0; gl < ng; ++gl) {
-                        if (mine) {
-                            if (!mbar_wait_bounded(&S.acc_empty[nb], accph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
-                            tc_fence_after();
-                            const uint32_t d_tmem = tmem + (uint32_t)(nb * NR);
-                            for (int kk = 0; kk < kpg; ++kk) {
-                                const int kq = gl * kpg + kk;                 // K step of the sub-stage: box kq / 4, 32 bytes each
-                                mma_f16_ts(d_tmem, a_tmem + (uint32_t)(kq * 8),
-                                           bdesc + (uint64_t)((((kq >> 2) * NR * 128) + (kq & 3) * 32) >> 4), IDESC,
-                                           kk != 0 ? 1u : 0u);
-                            }
-                            mma_commit_1(&S.acc_full[nb]);
-                        }
-                        if (++nb == NB) { nb = 0; accph ^= 1u; }
-                    }
-                    if (mine && !aborted) mma_commit_1(&S.slot_empty[as]);
-                    if (++as == AS) { as = 0; aph ^= 1u; }
-                }
-            }
-            mma_commit_1(&S.drain[mt]);                               // every MMA of this thread done before teardown
-            mbar_wait_bounded(&S.drain[mt], 0, abort_flag, A.timeout_ns);
-        }
-    } else if (warp >= PROD_WARP0) {
-        // Two sets of 4 producer warps take the sub-stages in turn (set gsub % 2);
-        // within a set, warp q writes the rows of tensor-memory lane quadrant q,
-        // one row per thread, into A slot gsub % AS (two halves of 64 columns,
-        // qtc_convert_half).  A code stage is released once every warp of each of
-        // its sub-stages has read it (the unit's last sub-stage of a partial stage
-        // arrives for the missing ones).
-        const int pset = (warp - PROD_WARP0) >> 2, q4 = warp & 3;
-        const int r = q4 * 32 + lane;                                 // the thread's row of the unit
-        const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-        int cs = 0, as = 0;
-        uint32_t cph = 0, aph = 0, gsub = 0;
-        for (int64_t u = blockIdx.x; u < A.units && !aborted; u += grid) {
-            int64_t rb, k0;
-            int cols, subs;
-            unit_span(u, rb, k0, cols, subs);
-            int sc = 0;                                               // sub-stage within the code stage
-            for (int sub = 0; sub < subs; ++sub, ++gsub) {
-                const bool stage_end = sc == spc - 1 || sub == subs - 1;
-                if ((int)(gsub & 1u) == pset) {
-                    if (!mbar_wait_warp(&S.c_full[cs], cph, abort_flag, A.timeout_ns) ||
-                        !mbar_wait_warp(&S.slot_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+            int bs = 0, as = 0, db = 0;
+            uint32_t bph = 0, aph = 0, dph = 0;
+            for (int64_t u = u_begin; u < u_end && mt < NISSUE; ++u) {
+                if ((int)((u - u_begin) % NISSUE) == mt) {
+                    if (!mbar_wait_bounded(&b_full[bs], bph, abort_flag, A.timeout_ns) ||
+                        !mbar_wait_bounded(&a_full[as], aph, abort_flag, A.timeout_ns) ||
+                        !mbar_wait_bounded(&d_empty[db], dph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
                     tc_fence_after();
-                    const uint32_t dst = tmem + lane_base + (uint32_t)(A_COL0 + as * 64);
+                    // every offset below is a compile-time constant: the descriptor's start
+                    // address field (address / 16) takes the byte offset / 16 directly
+                    const uint64_t bd0 = sw128_kmajor_desc(smem_u32(bring + bs * B_BYTES));
+                    const uint32_t d0 = tmem + AS * A_COLS + db * D_COLS, a0 = tmem + as * A_COLS;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t v[32];
-                        if (A.cpw == 8) qtc_convert_half<4>(&S.codes[cs][0], r, 4 * sc + 2 * h, v);
-                        else qtc_convert_half<2>(&S.codes[cs][0], r, 2 * sc + h, v);
-                        tmem_st_32x32b_x32(dst + (uint32_t)(32 * h), v);
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&S.a_full[as]);
-                        const int n_arrive = sub == subs - 1 ? spc - sc : 1;   // a partial last stage: the missing ones too
-                        for (int k = 0; k < n_arrive; ++k) mbar_arrive(&S.c_empty[cs]);
-                    }
+                    for (int m = 0; m < SC / 16; ++m)
+                        mma_f16_ts(d0 + (m / MPG) * NR, a0 + 8 * m,
+                                   bd0 + (uint64_t)(((m / 4) * NR * 128 + (m % 4) * 32) >> 4), IDESC, m % MPG != 0);
+                    mma_commit_1(&a_empty[as]);
+                    mma_commit_1(&b_empty[bs]);
+                    mma_commit_1(&d_full[db]);
                 }
+                if (++bs == BS) { bs = 0; bph ^= 1u; }
                 if (++as == AS) { as = 0; aph ^= 1u; }
-                if (++sc == spc || stage_end) { sc = 0; if (++cs == CS) { cs = 0; cph ^= 1u; } }
+                if (++db == DB) { db = 0; dph ^= 1u; }
             }
+            mma_commit_1(&drain[mt]);              // every MMA this thread issued has finished when this fires
+            mbar_wait_bounded(&drain[mt], 0, abort_flag, A.timeout_ns);
         }
-    } else if (warp >= EPI_WARP0) {
-        // Per unit: the scale and zero of this thread's row for each group come
-        // from global memory one unit ahead (registers), the unit's group sums
-        // (one float per thread) through a double buffer in shared memory, so no
-        // group waits on a global load.
-        const int q4 = warp - EPI_WARP0;                              // TMEM lane quadrant
-        const int et = threadIdx.x - EPI_WARP0 * 32;                  // 0 .. 127
-        const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-        int nb = 0;
-        uint32_t accph = 0;
-        __half2 szc[MAXG], szn[MAXG];                                 // (scale, zero) per group
-        float gsn = 0.0f;
-        auto fetch = [&](int64_t uu, __half2 (&dst)[MAXG], float &gsv) {
-            int64_t rb_, k0_;
-            int cols_, subs_;
-            unit_span(uu, rb_, k0_, cols_, subs_);
-            const int64_t nn = rb_ * ROWS + q4 * 32 + lane;
-            const int groups_ = cols_ / A.group, g0_ = (int)(k0_ / A.group);
+    } else if (warp < PWARPS) {                    // producers: A = q as bf16 pairs
+        const int q = warp & 3, h = warp >> 2;
+        const int rr = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int st = 0, as = 0;
+        uint32_t ph = 0, aph = 0;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            if (!mbar_wait_warp(&full[st], ph, abort_flag, A.timeout_ns)) { aborted = true; break; }
+            const uint8_t *stage = base + st * CODE_BYTES;
+            uint4 cw[NCH];
 #pragma unroll
-            for (int gi = 0; gi < MAXG; ++gi)
-                dst[gi] = (nn < A.N && gi < groups_) ? __halves2half2(A.scales[nn * A.G + g0_ + gi], A.zeros[nn * A.G + g0_ + gi])
-                                                     : __float2half2_rn(0.0f);
-            const int gg = et >> 4, tt = et & 15;                      // thread et: group gg, token slot tt
-            gsv = gg < groups_ ? A.gsum[(int64_t)(g0_ + gg) * 16 + tt] : 0.0f;
-        };
-        int buf = 0;
-        if (blockIdx.x < A.units) {
-            float g0v;
-            fetch(blockIdx.x, szc, g0v);
-            S.gs[0][et] = g0v;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // Every epilogue warp runs every unit and reaches every named barrier,
-        // also after an abort (then it only skips the waits and the work), so
-        // the barrier cannot strand the others.
-        for (int64_t u = blockIdx.x; u < A.units; u += grid) {
-            int64_t rb, k0;
-            int cols, subs;
-            unit_span(u, rb, k0, cols, subs);
-            const bool more = u + grid < A.units;
-            if (more && !aborted) fetch(u + grid, szn, gsn);         // in flight during this unit
-            const int64_t n = rb * ROWS + q4 * 32 + lane;
-            const bool row_ok = n < A.N;
-            float y[TT];
+            for (int c = 0; c < NCH; ++c) {
+                // 4-bit: 128-byte rows, 128-byte swizzle; 2-bit: 64-byte rows, 64-byte swizzle
+                const uint32_t off = CB == 4 ? (uint32_t)rr * 128u + ((uint32_t)((4 * h + c) ^ (rr & 7)) << 4)
+                                             : (uint32_t)rr * 64u + ((uint32_t)((2 * h + c) ^ ((rr >> 1) & 3)) << 4);
+                cw[c] = *reinterpret_cast<const uint4 *>(stage + off);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+            if (++st == CS) { st = 0; ph ^= 1u; }
+            if (!mbar_wait_warp(&a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
+            tc_fence_after();
 #pragma unroll
-            for (int t = 0; t < TT; ++t) y[t] = 0.0f;
-            const int groups = cols / A.group;
-            const float *gsu = &S.gs[buf][0];
+            for (int half8 = 0; half8 < 2; ++half8) {  // 64 columns: tensor-memory columns 64 h + 32 half8 ..
+                uint32_t v[32];
+                if (CB == 4) {
 #pragma unroll
-            for (int gi = 0; gi < MAXG; ++gi) {
-                if (gi >= groups || aborted) break;
-                const float2 szf = __half22float2(szc[gi]);
-                if (!mbar_wait_warp(&S.acc_full[nb], accph, abort_flag, A.timeout_ns, 128)) { aborted = true; break; }
-                tc_fence_after();
-                // the accumulator's NR columns: B row piece * TT + t  (x16 or x32 loads, then x16 for NR = 48)
-                float d[NR];
-                if constexpr (NR == 16) {
-                    tmem_ld_32x32b_x16_sync(tmem + lane_base + (uint32_t)(nb * NR), *reinterpret_cast<float(*)[16]>(&d[0]));
+                    for (int i = 0; i < 8; ++i) qtc_chunk_bf16<4>(word_of<NCH>(cw, half8 * 8 + i), &v[4 * i]);
                 } else {
-                    tmem_ld_32x32b_x32_sync(tmem + lane_base + (uint32_t)(nb * NR), *reinterpret_cast<float(*)[32]>(&d[0]));
-                    if constexpr (NR == 48)
-                        tmem_ld_32x32b_x16_sync(tmem + lane_base + (uint32_t)(nb * NR + 32),
-                                                *reinterpret_cast<float(*)[16]>(&d[32]));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t w = word_of<NCH>(cw, half8 * 4 + i);   // 16 codes: two chunks
+                        qtc_chunk_bf16<2>(__byte_perm(w, 0u, 0x4140u), &v[8 * i]);
+                        qtc_chunk_bf16<2>(__byte_perm(w, 0u, 0x4342u), &v[8 * i + 4]);
+                    }
                 }
-                tc_fence_before();
-                __syncwarp();                                          // every lane's reads are complete (wait::ld)
-                if (lane == 0) mbar_arrive(&S.acc_empty[nb]);
-                if (++nb == NB) { nb = 0; accph ^= 1u; }
+                tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)(as * A_COLS + 64 * h + 32 * half8), v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (++as == AS) { as = 0; aph ^= 1u; }
+        }
+    } else if (warp >= EWARP0 && warp < EWARP0 + 4) {   // epilogue: one row per thread
+        const int q = warp - EWARP0;
+        const int rr = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        griddep_wait();                            // group sums and counters written by the prep grid
+        float y[TT];
 #pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    const float dt = __fadd_rn(__fadd_rn(d[t], d[TT + t]), d[2 * TT + t]);
-                    y[t] = __fmaf_rn(szf.x, __fmaf_rn(-szf.y, gsu[gi * 16 + t], dt), y[t]);
+        for (int t = 0; t < TT; ++t) y[t] = 0.0f;
+        int db = 0;
+        uint32_t dph = 0;
+        int64_t rb = u_begin / A.n_steps, j = u_begin - rb * A.n_steps;
+        RowGroups<GPS> sr{A.scales, A.N, A.n_steps, A.G, rr}, zr{A.zeros, A.N, A.n_steps, A.G, rr};
+        if (u_begin < u_end) {
+            sr.begin(rb, j);
+            zr.begin(rb, j);
+        }
+        // The unit's group sums S_g[t] (the same for every row) through this warp's
+        // two shared-memory slots of 64 values (group e / 16, token slot e % 16):
+        // lane l loads values l and l + 32 of the unit two ahead into registers and
+        // stores them one unit later, so no load latency sits on a unit.
+        float *sw = s_area + q * 128;
+        auto s_load = [&](int64_t jj, float &v0, float &v1) {
+            const int g0 = lane >> 4, g1 = 2 + (lane >> 4);
+            const int64_t a0 = jj * GPS + g0, a1 = jj * GPS + g1;
+            v0 = (g0 < GPS && a0 < A.G) ? __ldg(A.gsum + a0 * 16 + (lane & 15)) : 0.0f;
+            v1 = (g1 < GPS && a1 < A.G) ? __ldg(A.gsum + a1 * 16 + (lane & 15)) : 0.0f;
+        };
+        auto next_step = [&](int64_t jj) { return jj + 1 == A.n_steps ? int64_t(0) : jj + 1; };
+        int64_t j_next = next_step(j), j_next2 = next_step(j_next);   // steps of the next two units
+        float p0 = 0.0f, p1 = 0.0f;
+        if (u_begin < u_end) {
+            float c0, c1;
+            s_load(j, c0, c1);
+            sw[lane] = c0;
+            sw[lane + 32] = c1;
+            s_load(j_next, p0, p1);
+        }
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            const int slot = (int)((u - u_begin) & 1);
+            __syncwarp();                          // every lane is done with the other slot
+            if (u + 1 < u_end) {
+                sw[(slot ^ 1) * 64 + lane] = p0;
+                sw[(slot ^ 1) * 64 + lane + 32] = p1;
+            }
+            if (u + 2 < u_end) s_load(j_next2, p0, p1);
+            __syncwarp();                          // this unit's slot is complete
+            const float *su = sw + slot * 64;
+            j_next = j_next2;
+            j_next2 = next_step(j_next2);
+            if (u != u_begin) {
+                sr.enter(j);
+                zr.enter(j);
+            }
+            if (!mbar_wait_warp(&d_full[db], dph, abort_flag, A.timeout_ns, 64)) { aborted = true; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < GPS; ++g) {
+                // dt[t] = (hi + mid) + lo: accumulator columns t, TT + t, 2 TT + t
+                float dt[TT];
+                const uint32_t dcol = tmem + lane_base + (uint32_t)(AS * A_COLS + db * D_COLS + g * NR);
+                if constexpr (NR == 48) {          // TT = 16: one 16-column load per piece
+                    float pc[16];
+                    tmem_ld_32x32b_x16_sync(dcol, pc);
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) dt[t] = pc[t];
+                    tmem_ld_32x32b_x16_sync(dcol + 16, pc);
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
+                    tmem_ld_32x32b_x16_sync(dcol + 32, pc);
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
+                } else {
+                    float dv[NR];
+#pragma unroll
+                    for (int c = 0; c < NR; c += 16)
+                        tmem_ld_32x32b_x16_sync(dcol + c, *reinterpret_cast<float(*)[16]>(&dv[c]));
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(__fadd_rn(dv[t], dv[TT + t]), dv[2 * TT + t]);
+                }
+                const int64_t gg = j * GPS + g;
+                if (gg < A.G) {                    // past G the codes and x' are zero: no term
+                    const float shg = sr.get(rb, j, g), zg = zr.get(rb, j, g);
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) y[t] = __fmaf_rn(shg, __fmaf_rn(-zg, su[g * 16 + t], dt[t]), y[t]);
                 }
             }
-            if (row_ok && !aborted) {
-                const int64_t kc = u - rb * A.n_chunks;
-                float *dst = A.n_chunks == 1 ? A.Y : A.part + kc * (int64_t)TT * A.N;
+            tc_fence_before();
+            __syncwarp();                          // every lane's reads are complete (wait::ld)
+            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (++db == DB) { db = 0; dph ^= 1u; }
+            if (j == A.n_steps - 1 || u == u_end - 1) {
+                // row block rb's segment ends: Y, or a partial sum and the fixup
+                const int64_t n = rb * ROWS + rr;
+                const int64_t rb_u0 = rb * A.n_steps, rb_u1 = rb_u0 + A.n_steps;
+                if (u_begin <= rb_u0 && u_end >= rb_u1) {
+                    if (n < A.N)
 #pragma unroll
-                for (int t = 0; t < TT; ++t)
-                    if (t < A.T) dst[(int64_t)t * A.N + n] = y[t];
-            }
-            // hand the next unit's values over: registers, and the other group-sum buffer
-            if (more) {
+                        for (int t = 0; t < TT; ++t)
+                            if (t < A.T) A.Y[t * A.N + n] = y[t];
+                } else {
+                    float *mine = A.part + ((rb + blockIdx.x) * ROWS + rr) * TT_MAX;
 #pragma unroll
-                for (int gi = 0; gi < MAXG; ++gi) szc[gi] = szn[gi];
-                S.gs[buf ^ 1][et] = gsn;
+                    for (int t = 0; t < TT; ++t) mine[t] = y[t];
+                    __threadfence();
+                    __syncwarp();
+                    const int64_t b0 = block_of(rb_u0, A.units, grid), b1 = block_of(rb_u1 - 1, A.units, grid);
+                    unsigned old = 0;
+                    if (lane == 0) old = atomicAdd(&A.cnt[rb * 4 + q], 1u);
+                    old = __shfl_sync(0xffffffffu, old, 0);
+                    if (old == (unsigned)(b1 - b0)) {
+                        __threadfence();
+                        float tot[TT];
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) tot[t] = 0.0f;
+                        for (int64_t b = b0; b <= b1; ++b)
+#pragma unroll
+                            for (int t = 0; t < TT; ++t)
+                                tot[t] = __fadd_rn(tot[t], __ldcg(A.part + ((rb + b) * ROWS + rr) * TT_MAX + t));
+                        if (n < A.N)
+#pragma unroll
+                            for (int t = 0; t < TT; ++t)
+                                if (t < A.T) A.Y[t * A.N + n] = tot[t];
+                        if (lane == 0) A.cnt[rb * 4 + q] = 0u;
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < TT; ++t) y[t] = 0.0f;
             }
-            buf ^= 1;
-            asm volatile("bar.sync 1, 128;" ::: "memory");        // the 4 epilogue warps only
+            if (++j == A.n_steps) {
+                j = 0;
+                ++rb;
+            }
         }
     }
 
-    if (aborted || *abort_flag) {
+    if (aborted || *abort_flag) {                  // let copies in flight land before the block exits
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == ALLOC_WARP) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc_1(tmem, TMEM_COLS);
     }

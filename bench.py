@@ -621,14 +621,13 @@ def run_qlinear(args):
         return statistics.median(ts)
 
     def path_and_launches(T):
-        # the library's dispatch.  Below 3 tokens: the x' kernel, then one pass of the
-        # CUDA-core kernel per 1 or 2 tokens.  From 3 tokens: the B-operand and
-        # group-sum kernels, then per pass of 5, 10 or 16 tokens the tensor-core kernel
-        # and (K split in chunks of 512 columns) the chunk reduction.
-        if T < 3:
-            return "cuda-core", 1 + -(-T // (1 if T == 1 else 2))
+        # the library's dispatch.  One token: the x' kernel, then one pass of the
+        # CUDA-core kernel.  From 2 tokens: the prep kernel (B operand, group sums),
+        # then one tensor-core pass per 5, 10 or 16 tokens.
+        if T < 2:
+            return "cuda-core", 2
         tt = 5 if T <= 5 else 10 if T <= 10 else 16
-        return "tensor-core", 2 + -(-T // tt) * (1 + (cfg.K > 512))
+        return "tensor-core", 1 + -(-T // tt)
 
     for T in [int(t) for t in args.tokens.split(",")]:
         Xt = Xd[:T].contiguous()

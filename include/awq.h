@@ -336,8 +336,8 @@ AWQ_API awq_status awq_get_status(void *stream);
  *       256-byte aligned (x' as binary32, partial sums of row blocks split
  *       across thread blocks, arrival counters); overwritten by every call
  * Requires K % 64 == 0.  Built for small T (decode), where streaming the
- * packed codes from HBM is the cost.  awq_qlinear runs awq_qlinear_cc below 3
- * tokens and awq_qlinear_tc from 3 tokens on; either may be called directly.
+ * packed codes from HBM is the cost.  awq_qlinear runs awq_qlinear_cc for one
+ * token and awq_qlinear_tc from 2 tokens on; either may be called directly.
  * Calls that share a workspace must be ordered (one stream). */
 AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
 AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
@@ -362,9 +362,11 @@ AWQ_API awq_status awq_qlinear_cc(const uint32_t *codes, const void *scales, con
  *         q is exact in bf16 and x' is split into three bf16 pieces whose sum
  *         is x' exactly, so every product is exact),
  *   S_g = RN32(sum_{k in g} x'[t, k]) in binary64.
- * Passes of up to 5, 10 or 16 tokens each read the codes once; K is split into
- * chunks whose partial sums are added in chunk order, so repeated calls on one
- * device give identical Y.  Calls that share a workspace must be ordered. */
+ * Passes of up to 5, 10 or 16 tokens each read the codes once.  The units (128
+ * rows x 256 columns) are dealt to the SMs in contiguous ranges; a row block
+ * split between two ranges is summed by the last to arrive, in range order, so
+ * repeated calls on one device give identical Y.  Calls that share a workspace
+ * must be ordered. */
 AWQ_API awq_status awq_qlinear_tc(const uint32_t *codes, const void *scales, const void *zeros,
                                   const float *s_best, int64_t N, int64_t K, awq_qcfg q,
                                   const void *X, int64_t T, int64_t ldx, float *Y,
