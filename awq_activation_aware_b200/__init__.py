@@ -82,6 +82,8 @@ def lib():
     L.awq_qlinear.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
     L.awq_qlinear_tc.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
     L.awq_qlinear_cc.argtypes = [P, P, P, P, i64, i64, QCfg, P, i64, i64, P, P, ctypes.c_size_t, P]
+    L.awq_qlinear_path.argtypes = [i64]
+    L.awq_qlinear_path.restype = ctypes.c_int32
     L.awq_qlinear.restype = ctypes.c_int
     L.awq_selftest_bounded_wait.argtypes = [P]
     L.awq_selftest_bounded_wait.restype = ctypes.c_int
@@ -271,6 +273,11 @@ def qlinear(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, s_be
               _dev(Y, torch.float32, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
               _stream(stream)), name)
     return Y
+
+
+def qlinear_path(T: int) -> str:
+    """The kernel qlinear(tensor_cores=None) runs for T tokens: "cuda_cores" or "tensor_cores"."""
+    return "tensor_cores" if lib().awq_qlinear_path(int(T)) == 1 else "cuda_cores"
 
 
 def quantize_shared_input(Ws, X: torch.Tensor, alphas: torch.Tensor | None = None, bits: int = 4,

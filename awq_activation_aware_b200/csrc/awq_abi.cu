@@ -943,10 +943,12 @@ awq_status awq_qlinear_tc(const uint32_t *codes, const void *scales, const void 
 
 // From kQlTcMinTokens tokens on, one tensor-core pass reads the codes once for
 // up to 16 tokens, where the CUDA-core kernel reads them once per 1, 2 or 4.
+int32_t awq_qlinear_path(int64_t T) { return T >= kQlTcMinTokens ? 1 : 0; }
+
 awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros, const float *s_best,
                        int64_t N, int64_t K, awq_qcfg q, const void *X, int64_t T, int64_t ldx, float *Y,
                        void *ws, size_t ws_bytes, void *stream) {
-    if (T >= kQlTcMinTokens)
+    if (awq_qlinear_path(T) == 1)
         return awq_qlinear_tc(codes, scales, zeros, s_best, N, K, q, X, T, ldx, Y, ws, ws_bytes, stream);
     return awq_qlinear_cc(codes, scales, zeros, s_best, N, K, q, X, T, ldx, Y, ws, ws_bytes, stream);
 }

@@ -340,6 +340,9 @@ AWQ_API awq_status awq_get_status(void *stream);
  * token and awq_qlinear_tc from 2 tokens on; either may be called directly.
  * Calls that share a workspace must be ordered (one stream). */
 AWQ_API size_t awq_qlinear_workspace_bytes(int64_t T, int64_t K, int64_t N);
+/* The kernel awq_qlinear runs for T tokens: 0 the CUDA-core kernel
+ * (awq_qlinear_cc), 1 the tensor-core kernel (awq_qlinear_tc).  Host only. */
+AWQ_API int32_t awq_qlinear_path(int64_t T);
 AWQ_API awq_status awq_qlinear(const uint32_t *codes, const void *scales, const void *zeros,
                                const float *s_best, int64_t N, int64_t K, awq_qcfg q,
                                const void *X, int64_t T, int64_t ldx, float *Y,

@@ -152,3 +152,11 @@ def test_gptq_entry_points_reject_bad_arguments():
     n = L.awq_output_error_workspace_bytes(256, 512, 512)
     assert L.awq_output_error(BOGUS, BOGUS, 256, 512, BOGUS, 512, 500, BOGUS, None, BOGUS, n, None) == 1   # ldx < K
     assert L.awq_output_error(BOGUS, BOGUS, 256, 512, BOGUS, 512, 512, BOGUS, None, BOGUS, n - 1, None) == 5
+
+
+def test_qlinear_dispatch_query():
+    # awq_qlinear runs the CUDA-core kernel for one token and the tensor-core
+    # kernel from two tokens on (host logic, no GPU needed)
+    assert awq.qlinear_path(1) == "cuda_cores"
+    for T in (2, 3, 5, 16, 17, 4096):
+        assert awq.qlinear_path(T) == "tensor_cores"

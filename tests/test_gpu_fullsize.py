@@ -133,3 +133,28 @@ def test_fullsize_qlinear(awq, name, T, tc):
     assert Y.shape == (T, cfg.N)
     assert np.all(np.abs(Y[:, rows] - ref) <= 2e-6 * bound + 1e-30)
     assert np.all(np.isfinite(Y))
+
+
+@pytest.mark.parametrize("name", ["attn4096", "mlp_up28672"])
+@pytest.mark.parametrize("T", [4, 16])
+def test_fullsize_tensor_core_decode_repeats(awq, name, T):
+    """Twenty more calls of the tensor-core decode at full size give the first
+    call's output bit for bit (its parity is checked by test_fullsize_qlinear):
+    a race in the kernel's hand-offs would show as a changed element."""
+    cfg = synth.CONFIGS[name]
+    W, X, _ = layer(name)
+    alphas = synth.default_alphas()
+    losses = np.linspace(1.0, 0.5, len(alphas))
+    Wd = torch.from_numpy(W).cuda()
+    a = awq.act_stats(torch.from_numpy(X).cuda())
+    out = awq.pack(Wd, a, torch.from_numpy(alphas).cuda(), torch.from_numpy(losses.astype(np.float32)).cuda(),
+                   cfg.bits, cfg.group)
+    del Wd
+    Xt = torch.from_numpy(np.ascontiguousarray(X[:T])).cuda()
+    first = awq.qlinear(out["codes"], out["scales"], out["zeros"], out["s_best"], Xt, cfg.bits, cfg.group,
+                        tensor_cores=True).cpu().numpy()
+    for _ in range(20):
+        Y = awq.qlinear(out["codes"], out["scales"], out["zeros"], out["s_best"], Xt, cfg.bits, cfg.group,
+                        tensor_cores=True).cpu().numpy()
+        assert np.array_equal(Y, first)
+    awq.get_status()

@@ -401,6 +401,28 @@ def test_qlinear(awq, N, K, T, bits, group, tc):
     assert np.array_equal(Y, Y2)
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("T", [1, 2, 4, 11, 16])
+def test_qlinear_dispatch_runs_the_named_kernel(awq, T):
+    # The two kernels sum in different orders, so their outputs differ in the
+    # last bits; the dispatched result is bit-identical to the kernel that
+    # awq_qlinear_path names and (on these inputs) differs from the other one.
+    N, K, bits, group = 2048, 3072, 4, 128
+    W, X = gen(N, K, T, bits=bits, group=group, seed=7 + T, outlier_frac=0.02)
+    a = oracle.act_stats(X)
+    alphas = synth.default_alphas()
+    losses = np.linspace(1.0, 0.5, 20).astype(np.float64)
+    pk = oracle.pack(W, a, bits, group, alphas, losses)
+    args = (dev(pk["codes"].view(np.int32)), dev(pk["scales"]), dev(pk["zeros"]), dev(pk["s_best"]), dev(X), bits, group)
+    y_auto = host(awq.qlinear(*args))
+    y_cc = host(awq.qlinear(*args, tensor_cores=False))
+    y_tc = host(awq.qlinear(*args, tensor_cores=True))
+    awq.get_status()
+    named, other = (y_tc, y_cc) if awq.qlinear_path(T) == "tensor_cores" else (y_cc, y_tc)
+    assert np.array_equal(y_auto, named)
+    assert not np.array_equal(y_auto, other)
+
+
 # ---------------------------------------------------------------------------
 # Quantizer variants and baselines: symmetric groups, channels held in fp16,
 # caller-given scale vectors, top-k channel selection
