@@ -739,14 +739,19 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 sv[1] = lds_f4(smem_u32(&S.sv[ws][c * 8 + 4]));
                 rv[0] = lds_f4(smem_u32(&S.rsv[ws][c * 8]));
                 rv[1] = lds_f4(smem_u32(&S.rsv[ws][c * 8 + 4]));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.w_empty[ws]);   // the stage's reads are done
-                if (++ws == WS) { ws = 0; wph ^= 1u; }
                 uint4 outv[4];
                 if (__any_sync(0xffffffffu, need))
                     compute_stage<true>(w, qp, sv, rv, A.qmax, outv);
                 else
                     compute_stage<false>(w, qp, sv, rv, A.qmax, outv);
+                // Release the stage only now: an issued shared-memory load is complete
+                // once an instruction has consumed its register, and every value read
+                // from the stage has been consumed by the arithmetic above.  (An arrive
+                // right after the loads could let the next tile's copy overwrite the
+                // stage under a load still in flight.)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.w_empty[ws]);
+                if (++ws == WS) { ws = 0; wph ^= 1u; }
                 if (!mbar_wait_warp(&S.a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
                 const uint32_t a_base = smem_u32(&S.a[as][0]);
 #pragma unroll
@@ -1416,9 +1421,9 @@ constexpr int THREADS = 16 * 32;
 // Token tiles: N = 16, 32 or 48 rows of x' pieces per pass (5, 10 or 16 tokens).
 __host__ __device__ constexpr int tile_tokens(int nr) { return nr == 16 ? 5 : nr == 32 ? 10 : 16; }
 template <int NR> __host__ __device__ constexpr int b_bytes() { return NR * SC * 2; }   // 4 swizzled boxes of NR x 64
-// Two rings: code tiles, freed as soon as the producers hold them in registers,
-// deep enough to cover the load latency of HBM under load; B tiles, freed when
-// the MMAs that read them complete.
+// Two rings: code tiles, freed once the producers have converted them, deep
+// enough to cover the load latency of HBM under load; B tiles, freed when the
+// MMAs that read them complete.
 template <int NR> __host__ __device__ constexpr int code_stages() { return NR == 16 ? 10 : NR == 32 ? 8 : 7; }
 constexpr int B_STAGES = 4;
 // Accumulator columns of one unit: one NR-wide block per group of the unit.
@@ -1589,7 +1594,7 @@ __global__ void qtc_prep_kernel(const __half *__restrict__ X, int64_t T, int64_t
 //   warp 14: the unit's B tile, 4 boxes of NR x 64 bf16 (128-byte swizzle);
 //   warps 0-7: producers; warp w converts columns 128 (w / 4) .. + 127 of the rows
 //            of lane quadrant w % 4 (one row per thread) into A slot as of tensor
-//            memory with tcgen05.st, after releasing the code tile;
+//            memory with tcgen05.st, then releases the code tile;
 //   warps 12 and 15: one thread each issues the 16 MMAs of every other unit (A
 //            from tensor memory, B from shared memory) into one accumulator per
 //            group, then commits;
@@ -1736,9 +1741,6 @@ qlinear_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_c
                                              : (uint32_t)rr * 64u + ((uint32_t)((2 * h + c) ^ ((rr >> 1) & 3)) << 4);
                 cw[c] = *reinterpret_cast<const uint4 *>(stage + off);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-            if (++st == CS) { st = 0; ph ^= 1u; }
             if (!mbar_wait_warp(&a_empty[as], aph ^ 1u, abort_flag, A.timeout_ns)) { aborted = true; break; }
             tc_fence_after();
 #pragma unroll
@@ -1760,8 +1762,16 @@ qlinear_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_c
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (lane == 0) {
+                mbar_arrive(&a_full[as]);
+                // the code tile is released only now that the conversion has consumed
+                // every value read from it: a load is complete once an instruction has
+                // read its register, so an arrive right after the loads could let the
+                // next tile's copy overwrite the stage under a load still in flight
+                mbar_arrive(&empty[st]);
+            }
             if (++as == AS) { as = 0; aph ^= 1u; }
+            if (++st == CS) { st = 0; ph ^= 1u; }
         }
     } else if (warp >= EWARP0 && warp < EWARP0 + 4) {   // epilogue: one row per thread
         const int q = warp - EWARP0;
