@@ -1826,42 +1826,67 @@ qlinear_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes, const __grid_c
                 sr.enter(j);
                 zr.enter(j);
             }
-            if (!mbar_wait_warp(&d_full[db], dph, abort_flag, A.timeout_ns, 64)) { aborted = true; break; }
+            if (!mbar_wait_warp(&d_full[db], dph, abort_flag, A.timeout_ns)) { aborted = true; break; }
             tc_fence_after();
+            const uint32_t dbase = tmem + lane_base + (uint32_t)(AS * A_COLS + db * D_COLS);
+            if constexpr (D_COLS == 32) {
+                // the whole unit's accumulators (two groups of 16 columns) in one load
+                // and one wait; the buffer is released before the arithmetic (a
+                // 64-column load measured slower, so wider units take the path below)
+                float dv[D_COLS];
+                tmem_ld_32x32b_x32_sync(dbase, dv);
+                tc_fence_before();
+                __syncwarp();                      // every lane's reads are complete (wait::ld)
+                if (lane == 0) mbar_arrive(&d_empty[db]);
 #pragma unroll
-            for (int g = 0; g < GPS; ++g) {
-                // dt[t] = (hi + mid) + lo: accumulator columns t, TT + t, 2 TT + t
-                float dt[TT];
-                const uint32_t dcol = tmem + lane_base + (uint32_t)(AS * A_COLS + db * D_COLS + g * NR);
-                if constexpr (NR == 48) {          // TT = 16: one 16-column load per piece
-                    float pc[16];
-                    tmem_ld_32x32b_x16_sync(dcol, pc);
+                for (int g = 0; g < GPS; ++g) {
+                    const int64_t gg = j * GPS + g;
+                    if (gg < A.G) {                // past G the codes and x' are zero: no term
+                        const float shg = sr.get(rb, j, g), zg = zr.get(rb, j, g);
 #pragma unroll
-                    for (int t = 0; t < TT; ++t) dt[t] = pc[t];
-                    tmem_ld_32x32b_x16_sync(dcol + 16, pc);
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
-                    tmem_ld_32x32b_x16_sync(dcol + 32, pc);
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
-                } else {
-                    float dv[NR];
-#pragma unroll
-                    for (int c = 0; c < NR; c += 16)
-                        tmem_ld_32x32b_x16_sync(dcol + c, *reinterpret_cast<float(*)[16]>(&dv[c]));
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(__fadd_rn(dv[t], dv[TT + t]), dv[2 * TT + t]);
+                        for (int t = 0; t < TT; ++t) {
+                            // (hi + mid) + lo: accumulator columns t, TT + t, 2 TT + t of the group
+                            const float dt = __fadd_rn(__fadd_rn(dv[g * NR + t], dv[g * NR + TT + t]), dv[g * NR + 2 * TT + t]);
+                            y[t] = __fmaf_rn(shg, __fmaf_rn(-zg, su[g * 16 + t], dt), y[t]);
+                        }
+                    }
                 }
-                const int64_t gg = j * GPS + g;
-                if (gg < A.G) {                    // past G the codes and x' are zero: no term
-                    const float shg = sr.get(rb, j, g), zg = zr.get(rb, j, g);
+            } else {
 #pragma unroll
-                    for (int t = 0; t < TT; ++t) y[t] = __fmaf_rn(shg, __fmaf_rn(-zg, su[g * 16 + t], dt[t]), y[t]);
+                for (int g = 0; g < GPS; ++g) {
+                    // dt[t] = (hi + mid) + lo: accumulator columns t, TT + t, 2 TT + t
+                    float dt[TT];
+                    const uint32_t dcol = dbase + (uint32_t)(g * NR);
+                    if constexpr (NR == 48) {      // TT = 16: one 16-column load per piece
+                        float pc[16];
+                        tmem_ld_32x32b_x16_sync(dcol, pc);
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) dt[t] = pc[t];
+                        tmem_ld_32x32b_x16_sync(dcol + 16, pc);
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
+                        tmem_ld_32x32b_x16_sync(dcol + 32, pc);
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(dt[t], pc[t]);
+                    } else {
+                        float dv[NR];
+#pragma unroll
+                        for (int c = 0; c < NR; c += 16)
+                            tmem_ld_32x32b_x16_sync(dcol + c, *reinterpret_cast<float(*)[16]>(&dv[c]));
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) dt[t] = __fadd_rn(__fadd_rn(dv[t], dv[TT + t]), dv[2 * TT + t]);
+                    }
+                    const int64_t gg = j * GPS + g;
+                    if (gg < A.G) {                // past G the codes and x' are zero: no term
+                        const float shg = sr.get(rb, j, g), zg = zr.get(rb, j, g);
+#pragma unroll
+                        for (int t = 0; t < TT; ++t) y[t] = __fmaf_rn(shg, __fmaf_rn(-zg, su[g * 16 + t], dt[t]), y[t]);
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();                      // every lane's reads are complete (wait::ld)
+                if (lane == 0) mbar_arrive(&d_empty[db]);
             }
-            tc_fence_before();
-            __syncwarp();                          // every lane's reads are complete (wait::ld)
-            if (lane == 0) mbar_arrive(&d_empty[db]);
             if (++db == DB) { db = 0; dph ^= 1u; }
             if (j == A.n_steps - 1 || u == u_end - 1) {
                 // row block rb's segment ends: Y, or a partial sum and the fixup
