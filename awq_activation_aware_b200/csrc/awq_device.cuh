@@ -308,7 +308,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+// Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                uint64_t limit_ns, uint32_t sleep_ns = 0) {
