@@ -65,6 +65,9 @@ def lib():
     L.awq_output_error_workspace_bytes.restype = ctypes.c_size_t
     L.awq_output_error.argtypes = [P, P, i64, i64, P, i64, i64, P, P, P, ctypes.c_size_t, P]
     L.awq_gptq_hessian.argtypes = [P, i64, i64, i64, P, P, P]
+    L.awq_gptq_hessian_workspace_bytes.argtypes = [i64, i64]
+    L.awq_gptq_hessian_workspace_bytes.restype = ctypes.c_size_t
+    L.awq_gptq_hessian_tc.argtypes = [P, i64, i64, i64, P, P, P, ctypes.c_size_t, P]
     L.awq_gptq_factor_workspace_bytes.argtypes = [i64]
     L.awq_gptq_factor_workspace_bytes.restype = ctypes.c_size_t
     L.awq_gptq_factor.argtypes = [P, i64, ctypes.c_float, P, P, ctypes.c_size_t, P]
@@ -93,7 +96,8 @@ def lib():
     L.awq_status_string.restype = ctypes.c_char_p
     for fn in ("awq_act_stats", "awq_alpha_scales", "awq_quant_dequant", "awq_search_layer", "awq_pack",
                "awq_get_status", "awq_quant_dequant_masked", "awq_search_scales", "awq_channel_topk",
-               "awq_pack_scales", "awq_salient_scales", "awq_output_error", "awq_gptq_hessian", "awq_gptq_factor",
+               "awq_pack_scales", "awq_salient_scales", "awq_output_error", "awq_gptq_hessian",
+               "awq_gptq_hessian_tc", "awq_gptq_factor",
                "awq_gptq_quantize", "awq_qlinear_tc", "awq_qlinear_cc"):
         getattr(L, fn).restype = ctypes.c_int
     _lib = L
@@ -399,14 +403,22 @@ def output_error(W: torch.Tensor, W_hat: torch.Tensor, X: torch.Tensor, row_loss
     return (loss[0], rl[0]) if row_losses else loss[0]
 
 
-def gptq_hessian(X: torch.Tensor, s: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """H = 2 X'^T X' (float32 [K, K]) of the input divided by s."""
+def gptq_hessian(X: torch.Tensor, s: torch.Tensor | None = None, stream=None,
+                 tensor_cores: bool = True) -> torch.Tensor:
+    """H = 2 X'^T X' (float32 [K, K]) of the input divided by s: awq_gptq_hessian_tc
+    (tcgen05), or awq_gptq_hessian (CUDA cores) with tensor_cores=False."""
     _rowmajor(X, "X")
     T, K = X.shape
     s = torch.ones(K, dtype=torch.float32, device=X.device) if s is None else s
     H = torch.empty((K, K), dtype=torch.float32, device=X.device)
-    _check(lib().awq_gptq_hessian(_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(s, torch.float32, "s"),
-                                  _dev(H, torch.float32, "H"), _stream(stream)), "awq_gptq_hessian")
+    args = (_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(s, torch.float32, "s"), _dev(H, torch.float32, "H"))
+    if tensor_cores:
+        need = int(lib().awq_gptq_hessian_workspace_bytes(T, K))
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+        _check(lib().awq_gptq_hessian_tc(*args, ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
+               "awq_gptq_hessian_tc")
+    else:
+        _check(lib().awq_gptq_hessian(*args, _stream(stream)), "awq_gptq_hessian")
     return H
 
 

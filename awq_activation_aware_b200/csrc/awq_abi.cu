@@ -146,6 +146,8 @@ awq_status device_info(DevInfo &out) {
             cudaFuncSetAttribute(awq::qlinear_gemv_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             !qtc_attrs<16>() || !qtc_attrs<32>() || !qtc_attrs<48>() ||
+            cudaFuncSetAttribute(awq::gptq_hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)awq::ghs::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<1, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  awq::qlv::SMEM_LIMIT) != cudaSuccess ||
             cudaFuncSetAttribute(awq::gptq_sweep_kernel<2, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -656,6 +658,37 @@ awq_status awq_gptq_hessian(const void *X, int64_t T, int64_t K, int64_t ldx, co
     if (awq_status e = device_info(d)) return e;
     const int nb = (int)(K / awq::kGb);
     awq::gptq_hessian_kernel<<<nb * (nb + 1) / 2, 256, 0, (cudaStream_t)stream>>>((const __half *)X, T, K, ldx, s, H);
+    return last_launch();
+}
+
+size_t awq_gptq_hessian_workspace_bytes(int64_t T, int64_t K) {
+    if (T < 1 || T > kMaxDim || K < 64 || K % 64 || K > kMaxGptqK) return 0;
+    const int64_t Tp = (T + awq::ghs::TS - 1) / awq::ghs::TS * awq::ghs::TS;
+    return round_up(2 * 3 * (size_t)K * (size_t)Tp, 256);
+}
+
+awq_status awq_gptq_hessian_tc(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s, float *H, void *ws,
+                               size_t ws_bytes, void *stream) {
+    if (!X || !s || !H || !aligned16(X) || !aligned16(s) || !aligned16(H)) return AWQ_ERR_INVALID_ARG;
+    if (T < 1 || T > kMaxDim || K < 64 || K > kMaxGptqK || K % 64 || ldx < K || ldx % 8) return AWQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < awq_gptq_hessian_workspace_bytes(T, K) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return AWQ_ERR_WORKSPACE;
+    DevInfo d;
+    if (awq_status e = device_info(d)) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t Tp = (T + awq::ghs::TS - 1) / awq::ghs::TS * awq::ghs::TS;
+    __nv_bfloat16 *xt = static_cast<__nv_bfloat16 *>(ws);
+    const dim3 pgrid((unsigned)((K + awq::ghs::XT_TILE - 1) / awq::ghs::XT_TILE),
+                     (unsigned)((Tp + awq::ghs::XT_TILE - 1) / awq::ghs::XT_TILE));
+    awq::gptq_hprep_kernel<<<pgrid, 256, 0, st>>>((const __half *)X, T, K, ldx, Tp, s, xt);
+    if (awq_status e = last_launch()) return e;
+    CUtensorMap tmap;
+    if (!encode_bf16_map(&tmap, xt, 3 * K, Tp, awq::ghs::TB)) return AWQ_ERR_CUDA;
+    const int nb = (int)((K + awq::ghs::TB - 1) / awq::ghs::TB);
+    const int n_tiles = nb * (nb + 1) / 2;
+    const int grid = n_tiles < d.sms ? n_tiles : d.sms;
+    awq::gptq_hessian_tc_kernel<<<grid, awq::ghs::THREADS, awq::ghs::SMEM_BYTES, st>>>(
+        tmap, K, Tp / awq::ghs::TS, H, (uint64_t)g_timeout_ms.load() * 1000000ull);
     return last_launch();
 }
 

@@ -2032,6 +2032,208 @@ gptq_hessian_kernel(const __half *__restrict__ X, int64_t T, int64_t K, int64_t 
         }
 }
 
+// H = 2 X'^T X' on the tensor cores.  x' = RN32(x RN32(1/s)) is split into
+// three bf16 pieces whose sum is x' exactly (hi = RN(x'), mid = RN(x' - hi),
+// lo = x' - hi - mid), so every product of pieces is exact in the fp32
+// accumulator, and H[i, j] = 2 sum_t sum_{p, q} P_p[t, i] P_q[t, j] differs from
+// the CUDA-core kernel's only in the order of its binary32 additions.
+namespace ghs {
+constexpr int TB = 128;                    // H tile: 128 x 128 (MMA M = N = 128)
+constexpr int TS = 64;                     // tokens per stage (one 128-byte swizzled row of bf16)
+constexpr int PIECE_BYTES = TB * TS * 2;   // 16 KiB: one piece of one operand
+constexpr int STAGE_BYTES = 6 * PIECE_BYTES;   // A pieces 0-2, B pieces 0-2
+constexpr int STAGES = 2;
+constexpr int THREADS = 256;               // warp 0 loads, warp 1 issues, warp 2 allocates, warps 4-7 store
+constexpr int TMEM_COLS = 256;             // two accumulators of 128 columns
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int XT_TILE = 32;                // transpose tile of the prep kernel
+}  // namespace ghs
+
+// xt[p][k][t] (bf16, t padded to Tp with zeros): piece p of x'[t, k], k-major
+// rows for the tensor-core Hessian, through a 32 x 32 shared-memory transpose.
+__global__ void __launch_bounds__(256) gptq_hprep_kernel(const __half *__restrict__ X, int64_t T, int64_t K,
+                                                         int64_t ldx, int64_t Tp, const float *__restrict__ s,
+                                                         __nv_bfloat16 *__restrict__ xt) {
+    using namespace ghs;
+    __shared__ __nv_bfloat16 tile[3][XT_TILE][XT_TILE + 2];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 8 rows of 32 a pass
+    const int64_t k0 = (int64_t)blockIdx.x * XT_TILE, t0 = (int64_t)blockIdx.y * XT_TILE;
+    for (int r = ty; r < XT_TILE; r += 8) {
+        const int64_t t = t0 + r, k = k0 + tx;
+        float hi = 0.0f, mid = 0.0f, lo = 0.0f;
+        if (t < T && k < K) {
+            const float xp = __fmul_rn(__half2float(X[t * ldx + k]), __frcp_rn(s[k]));
+            hi = __bfloat162float(__float2bfloat16_rn(xp));
+            const float r1 = __fsub_rn(xp, hi);                    // exact
+            mid = __bfloat162float(__float2bfloat16_rn(r1));
+            lo = __fsub_rn(r1, mid);                               // exact, at most 8 bits
+        }
+        tile[0][r][tx] = __float2bfloat16_rn(hi);
+        tile[1][r][tx] = __float2bfloat16_rn(mid);
+        tile[2][r][tx] = __float2bfloat16_rn(lo);
+    }
+    __syncthreads();
+    for (int r = ty; r < XT_TILE; r += 8) {
+        const int64_t k = k0 + r, t = t0 + tx;
+        if (k < K && t < Tp) {
+#pragma unroll
+            for (int p = 0; p < 3; ++p) xt[((int64_t)p * K + k) * Tp + t] = tile[p][tx][r];
+        }
+    }
+}
+
+// Persistent over the 128 x 128 tiles (bi >= bj) of H's lower block triangle.
+// Warp 0 loads, per stage of 64 tokens, the three pieces of rows bi (A) and bj
+// (B) with TMA; warp 1 issues the 9 piece pairs x 4 MMAs of K 16 into the tile's
+// accumulator (two in tensor memory, so one tile's stores overlap the next
+// tile's MMAs); warps 4-7 read the accumulator, one row of the tile per thread,
+// and store 2 D to H[i, j] and its mirror H[j, i] (the diagonal tile from its
+// lower half only), so H is exactly symmetric.
+__global__ void __launch_bounds__(ghs::THREADS, 1)
+gptq_hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap_xt, int64_t K, int64_t n_ts, float *__restrict__ H,
+                       uint64_t timeout_ns) {
+    using namespace ghs;
+    constexpr uint32_t IDESC = mma_idesc_bf16_f32(TB, TB);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES, *d_full = bars + 2 * STAGES, *d_empty = d_full + 2;
+    uint64_t *drain = d_empty + 2;
+    __shared__ uint32_t tmem_base_sm;
+    __shared__ int abort_sm;
+    volatile int *abort_flag = &abort_sm;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = (int)((K + TB - 1) / TB);
+    const int n_tiles = nb * (nb + 1) / 2;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&d_full[i], 1); mbar_init(&d_empty[i], 4); }
+        mbar_init(drain, 1);
+        abort_sm = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc_1(&tmem_base_sm, TMEM_COLS);
+        tmem_relinquish_1();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sm;
+    bool aborted = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_xt);
+            int st = 0;
+            uint32_t ph = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !aborted; tile += gridDim.x) {
+                int bi, bj;
+                lower_block(tile, bi, bj);
+                for (int64_t ts = 0; ts < n_ts; ++ts) {
+                    if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, timeout_ns)) { aborted = true; break; }
+                    mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+                    uint8_t *sb = base + st * STAGE_BYTES;
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        tma_load_2d(sb + p * PIECE_BYTES, &tmap_xt, (int32_t)(ts * TS), (int32_t)(p * K + bi * TB),
+                                    &full[st]);
+                        tma_load_2d(sb + (3 + p) * PIECE_BYTES, &tmap_xt, (int32_t)(ts * TS),
+                                    (int32_t)(p * K + bj * TB), &full[st]);
+                    }
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int st = 0, db = 0;
+            uint32_t ph = 0, dph = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !aborted; tile += gridDim.x) {
+                if (!mbar_wait_bounded(&d_empty[db], dph ^ 1u, abort_flag, timeout_ns)) { aborted = true; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(db * TB);
+                for (int64_t ts = 0; ts < n_ts; ++ts) {
+                    if (!mbar_wait_bounded(&full[st], ph, abort_flag, timeout_ns)) { aborted = true; break; }
+                    tc_fence_after();
+                    const uint64_t d0 = sw128_kmajor_desc(smem_u32(base + st * STAGE_BYTES));
+#pragma unroll
+                    for (int p = 0; p < 3; ++p)
+#pragma unroll
+                        for (int q = 0; q < 3; ++q)
+#pragma unroll
+                            for (int kk = 0; kk < TS / 16; ++kk)
+                                mma_f16_ss_1(d, d0 + (uint64_t)((p * PIECE_BYTES + kk * 32) >> 4),
+                                             d0 + (uint64_t)(((3 + q) * PIECE_BYTES + kk * 32) >> 4), IDESC,
+                                             (ts | p | q | kk) != 0 ? 1u : 0u);
+                    mma_commit_1(&empty[st]);
+                    if (++st == STAGES) { st = 0; ph ^= 1u; }
+                }
+                if (aborted) break;
+                mma_commit_1(&d_full[db]);
+                if (++db == 2) { db = 0; dph ^= 1u; }
+            }
+            mma_commit_1(drain);                   // every MMA issued has finished when this fires
+            mbar_wait_bounded(drain, 0, abort_flag, timeout_ns);
+        }
+    } else if (warp >= 4) {
+        const int q4 = warp - 4;
+        const int rr = 32 * q4 + lane;             // the thread's row of the tile
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        int db = 0;
+        uint32_t dph = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            int bi, bj;
+            lower_block(tile, bi, bj);
+            if (!mbar_wait_warp(&d_full[db], dph, abort_flag, timeout_ns)) { aborted = true; break; }
+            tc_fence_after();
+            const int64_t i = (int64_t)bi * TB + rr;
+            for (int c0 = 0; c0 < TB; c0 += 32) {
+                float v[32];
+                tmem_ld_32x32b_x32_sync(tmem + lane_base + (uint32_t)(db * TB + c0), v);
+                const int64_t j0 = (int64_t)bj * TB + c0;
+                // direct: H[i, j] for j <= i on the diagonal tile, all j off it
+                if (i < K) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        const int64_t j = j0 + c;
+                        if (j + 3 < K && (bi != bj || j + 3 <= i)) {
+                            *reinterpret_cast<float4 *>(H + i * K + j) =
+                                make_float4(2.0f * v[c], 2.0f * v[c + 1], 2.0f * v[c + 2], 2.0f * v[c + 3]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (j + e < K && (bi != bj || j + e <= i)) H[i * K + j + e] = 2.0f * v[c + e];
+                        }
+                    }
+                }
+                // mirror: H[j, i] for j < i on the diagonal tile, all j off it (coalesced over the warp's rows)
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int64_t j = j0 + c;
+                    if (i < K && j < K && (bi != bj || j < i)) H[j * K + i] = 2.0f * v[c];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();                          // every lane's reads are complete (wait::ld)
+            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (++db == 2) { db = 0; dph ^= 1u; }
+        }
+    }
+
+    if (aborted || *abort_flag) {                  // let copies in flight land before the block exits
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_1(tmem, TMEM_COLS);
+    }
+}
+
+
 // damp * mean(diag H), the damping term: one block, the diagonal summed in
 // index order in binary64 (the result does not depend on the launch).
 __global__ void __launch_bounds__(256)

@@ -283,6 +283,14 @@ AWQ_API awq_status awq_output_error(const void *W, const void *W_hat, int64_t N,
  * sweep); larger K returns AWQ_ERR_INVALID_ARG. */
 AWQ_API awq_status awq_gptq_hessian(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s,
                                     float *H, void *stream);
+/* The same H on the tensor cores (tcgen05): x' is split into three bf16 pieces
+ * whose sum is x' exactly, so every product is exact and only the binary32
+ * additions (in the tensor core's order, not token order) round; H is exactly
+ * symmetric.  ws >= awq_gptq_hessian_workspace_bytes(T, K) (the pieces, bf16
+ * [3][K][T rounded up to 64]), 256-byte aligned; overwritten by every call. */
+AWQ_API size_t awq_gptq_hessian_workspace_bytes(int64_t T, int64_t K);
+AWQ_API awq_status awq_gptq_hessian_tc(const void *X, int64_t T, int64_t K, int64_t ldx, const float *s,
+                                       float *H, void *ws, size_t ws_bytes, void *stream);
 AWQ_API size_t awq_gptq_factor_workspace_bytes(int64_t K);
 AWQ_API awq_status awq_gptq_factor(const float *H, int64_t K, float damp, float *U, void *ws,
                                    size_t ws_bytes, void *stream);

@@ -603,13 +603,15 @@ def test_output_error_equals_the_search_loss(awq):
     np.testing.assert_allclose(host(rows).astype(np.float64), ref["row_sums"], rtol=LOSS_RTOL)
 
 
-@pytest.mark.parametrize("T,K", [(512, 256), (700, 512), (64, 1024)])
-def test_gptq_hessian_matches_oracle(awq, T, K):
-    """binary32 accumulation in token order against the binary64 product:
+@pytest.mark.parametrize("T,K", [(512, 256), (700, 512), (64, 1024), (129, 320), (4096, 384)])
+@pytest.mark.parametrize("tc", [False, True], ids=["cuda_cores", "tensor_cores"])
+def test_gptq_hessian_matches_oracle(awq, T, K, tc):
+    """binary32 accumulation (in token order on the CUDA cores, of exact piece
+    products on the tensor cores) against the binary64 product:
     |H - H_oracle| <= T 2^-24 (2 |X'|^T |X'|) (the standard summation bound)."""
     W, X = gen(8, K, T, seed=112)
     s = oracle.scales(oracle.act_stats(X), 0.4)
-    H = host(awq.gptq_hessian(dev(X), dev(s))).astype(np.float64)
+    H = host(awq.gptq_hessian(dev(X), dev(s), tensor_cores=tc)).astype(np.float64)
     awq.get_status()
     ref = oracle.gptq_hessian(X, s)
     rs = (np.float32(1.0) / s).astype(np.float32)
