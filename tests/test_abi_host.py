@@ -141,6 +141,15 @@ def test_gptq_entry_points_reject_bad_arguments():
     assert L.awq_gptq_hessian(BOGUS, 16, 96, 96, BOGUS, BOGUS, None) == 1           # K % 64
     assert L.awq_gptq_hessian(BOGUS, 16, 16384, 16384, BOGUS, BOGUS, None) == 1     # K > 8192
     assert L.awq_gptq_hessian(MISALIGNED, 16, 128, 128, BOGUS, BOGUS, None) == 1
+    # the tensor-core form: pieces of x' as bf16 [3][K][T rounded up to 64]
+    assert L.awq_gptq_hessian_workspace_bytes(100, 128) == 2 * 3 * 128 * 128
+    assert L.awq_gptq_hessian_workspace_bytes(16, 96) == 0
+    assert L.awq_gptq_hessian_workspace_bytes(16, 16384) == 0
+    wh = L.awq_gptq_hessian_workspace_bytes(16, 128)
+    assert L.awq_gptq_hessian_tc(BOGUS, 16, 96, 96, BOGUS, BOGUS, BOGUS, wh, None) == 1        # K % 64
+    assert L.awq_gptq_hessian_tc(MISALIGNED, 16, 128, 128, BOGUS, BOGUS, BOGUS, wh, None) == 1
+    assert L.awq_gptq_hessian_tc(BOGUS, 16, 128, 128, BOGUS, BOGUS, BOGUS, wh - 1, None) == 5   # workspace
+    assert L.awq_gptq_hessian_tc(BOGUS, 16, 128, 128, BOGUS, BOGUS, MISALIGNED, wh, None) == 5  # ws alignment
     assert L.awq_gptq_factor_workspace_bytes(16384) == 0
     assert L.awq_gptq_factor_workspace_bytes(4096) >= 4 * 4096 * 4096
     ws = L.awq_gptq_factor_workspace_bytes(128)
