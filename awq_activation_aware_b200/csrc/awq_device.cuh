@@ -104,17 +104,6 @@ __device__ __forceinline__ QParams unpack_qparams(uint2 v) {
     return p;
 }
 
-// The integer code q = clamp(rint(w' r) + z, 0, qmax) (used by the packer).
-// v = RN32(w' r + kMagic) = kMagic + (q - z) once clamped; in [2^23, 2^24) the
-// spacing of binary32 is 1, so the bit pattern of v minus that of kMagic is
-// q - z exactly, and q = bits(v) - (bits(kMagic) - z).  `clamp` may be false
-// only when make_qparams found the group needs no clamping.
-__device__ __forceinline__ uint32_t quant_code(float wp, const QParams &p, float qmax, bool clamp) {
-    float v = __fmaf_rn(wp, p.r, kMagic);
-    if (clamp) v = fminf(fmaxf(v, __fsub_rn(kMagic, p.z)), __fadd_rn(kMagic, __fsub_rn(qmax, p.z)));
-    return (uint32_t)(__float_as_int(v) - (__float_as_int(kMagic) - (int)p.z));
-}
-
 // Three-input minimum / maximum (sm_100).
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
     float d;
@@ -374,9 +363,6 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
 // (.noinc: the barrier's expected count includes these arrivals).
 __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_8(void *smem_dst, const void *gsrc) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
 }
 __device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gsrc) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
