@@ -784,30 +784,48 @@ search_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 // a6 (reduction). losses[i] = RN32(sum over token blocks and rows of the
 // partials, in binary64 and a fixed order, / (R T)), R = N for a whole layer
 // or the layer's row count when these N rows are one part of it; optional
-// per-row sums.  One block per alpha.
+// per-row sums.  One block per alpha; thread t takes rows t, t + 1024, ... in
+// that order, kLossRows of them at a time so that all their loads of a batch
+// of 8 token blocks are in flight together.
 // ===========================================================================
 constexpr int kLossThreads = 1024;
+constexpr int kLossRows = 2;
 __global__ void __launch_bounds__(kLossThreads)
 loss_reduce_kernel(const float *__restrict__ partial, int64_t N, int64_t T, int n_tb, int64_t norm_rows,
                    float *__restrict__ losses, float *__restrict__ row_losses) {
     const int ai = blockIdx.x;
     const float *p = partial + (int64_t)ai * n_tb * N;
     double acc = 0.0;
-    for (int64_t n = threadIdx.x; n < N; n += kLossThreads) {
-        float rsum = 0.0f;
-        double dsum = 0.0;
+    for (int64_t nb = threadIdx.x; nb < N; nb += kLossRows * kLossThreads) {
+        float rsum[kLossRows];
+        double dsum[kLossRows];
+#pragma unroll
+        for (int i = 0; i < kLossRows; ++i) { rsum[i] = 0.0f; dsum[i] = 0.0; }
         for (int tb0 = 0; tb0 < n_tb; tb0 += 8) {
-            float v[8];
+            float v[kLossRows][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = tb0 + j < n_tb ? __ldg(p + (int64_t)(tb0 + j) * N + n) : 0.0f;
+            for (int i = 0; i < kLossRows; ++i) {
+                const int64_t n = nb + (int64_t)i * kLossThreads;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                rsum = __fadd_rn(rsum, v[j]);
-                dsum = __dadd_rn(dsum, (double)v[j]);
+                for (int j = 0; j < 8; ++j)
+                    v[i][j] = (n < N && tb0 + j < n_tb) ? __ldg(p + (int64_t)(tb0 + j) * N + n) : 0.0f;
+            }
+#pragma unroll
+            for (int i = 0; i < kLossRows; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    rsum[i] = __fadd_rn(rsum[i], v[i][j]);
+                    dsum[i] = __dadd_rn(dsum[i], (double)v[i][j]);
+                }
+        }
+#pragma unroll
+        for (int i = 0; i < kLossRows; ++i) {
+            const int64_t n = nb + (int64_t)i * kLossThreads;
+            if (n < N) {
+                if (row_losses) row_losses[(int64_t)ai * N + n] = rsum[i];
+                acc = __dadd_rn(acc, dsum[i]);
             }
         }
-        if (row_losses) row_losses[(int64_t)ai * N + n] = rsum;
-        acc = __dadd_rn(acc, dsum);
     }
     __shared__ double red[kLossThreads];
     red[threadIdx.x] = acc;
@@ -1352,42 +1370,20 @@ qlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes, const qlv::A
 }
 
 // ===========================================================================
-// The decode consumer on the tensor cores (row n1, any w_bit).  The same
-// definition as the CUDA-core kernel,
+// The decode consumer on the tensor cores ([AWQ-note] "Tiny Chat": the codes are
+// dequantized inside the kernel), any w_bit.  The same definition as the
+// CUDA-core kernel,
 //   Y[t, n] = sum_k x'[t, k] (q[n, k] - z[n, g]) sh[n, g],   x' = RN32(x RN32(1/s)),
 // evaluated as Y = sum_g sh (D_g - z S_g) with
 //   D_g[n, t] = sum_{k in g} q[n, k] x'[t, k]   on tcgen05 (kind::f16, bf16 operands, fp32 accumulate),
-//   S_g[t]    = RN32(sum_{k in g} x'[t, k])     in binary64 by the prep kernel.
+//   S_g[t]    = RN32(sum_{k in g} x'[t, k])     in binary64 by qtc_prep_kernel.
 // Both MMA operands hold exact values: A = q (an integer below 16, exact in
 // bf16) and B = x' split into three bf16 pieces whose sum is x' exactly
 // (8 + 8 + 8 significant bits), one B row per piece and token.  So every
 // product the tensor core forms is exact and only the fp32 accumulation
-// rounds; no step depends on the range of the zero point.
-//
-// Work unit: 128 weight rows x one chunk of K (a multiple of 512 columns);
-// the units go round-robin to one persistent CTA per SM.  A TMA warp loads
-// code stages of 128 bytes of every row of the unit (16 KiB: 256 columns at
-// 4-bit containers, 512 at 2-bit; a 6-deep ring keeps about 96 KiB in flight
-// per SM) and, per 64-column sub-stage, the B tile (NR = 16, 32 or 48 rows x
-// 64 bf16, 128-byte swizzle).  Eight producer warps turn each sub-stage's
-// codes into the bf16 A tile (128 x 64, 128-byte swizzle); one thread issues
-// the four MMAs of a sub-stage into the accumulator of its quantization group
-// (a ring of 4 in tensor memory); four epilogue warps (one row per thread)
-// read each finished group, add its three piece sums, and accumulate
-// sh (D - z S) per token.  A
-// unit's sums go to Y directly (one chunk) or to per-chunk partials that a
-// second kernel adds in chunk order, so Y does not depend on timing.
+// rounds; no step depends on the range of the zero point.  The work layout and
+// the roles of the warps are described at qlinear_tc_kernel.
 // ===========================================================================
-// ---------------------------------------------------------------------------
-// The decode consumer on the tensor cores (qlinear_tc_kernel), [AWQ-note]
-// "Tiny Chat" (dequantization inside the kernel) with reading 22's exact
-// products:
-//   Y[t, n] = sum_g sh[n, g] (D_g[n, t] - z[n, g] S_g[t]),
-//   D_g[n, t] = sum_{k in g} q[n, k] x'[t, k]   (tcgen05, bf16 operands, fp32 accumulation)
-//   S_g[t] = RN32(sum_{k in g} x'[t, k]) in binary64 (qtc_gsum_kernel).
-// q is exact in bf16 and x' = hi + mid + lo exactly (three bf16 pieces, the B
-// rows), so every product is exact and only the fp32 accumulation rounds.
-// ---------------------------------------------------------------------------
 
 // The 8 codes of one 8-column chunk (code e in bits CB e .. of x) as 4 bf16x2
 // words of A: word e holds (code e, code e + 4).  One mask places the two codes
