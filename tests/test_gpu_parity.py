@@ -581,6 +581,28 @@ def test_qlinear_on_symmetric_pack(awq):
     np.testing.assert_allclose(Y, ref, rtol=1e-4, atol=1e-4 * np.abs(ref).max())
 
 
+def test_saved_layer_reloads_for_decode(awq, tmp_path):
+    """A layer quantized on the GPU, saved and loaded back ([QAS-QA] §9:
+    save_quantized, then inference from the 4-bit model): the reloaded tensors
+    are bit-identical, and the decode from them gives the same Y."""
+    from awq_activation_aware_b200 import persist
+    W, X = gen(384, 512, 96, seed=131)
+    al = dev(synth.default_alphas())
+    res = awq.quantize_layer(dev(W), dev(X), al, 4, 128)
+    awq.get_status()
+    p = tmp_path / "layer.pt"
+    persist.save_quantized(p, res, 4, 128, alphas=al)
+    back = persist.load_quantized(p, device="cuda")
+    for k in ("codes", "scales", "zeros", "s_best", "best_idx", "losses", "a"):
+        assert torch.equal(back[k].view(torch.uint8), res[k].view(torch.uint8)), k
+    Xt = dev(X[:4])
+    Y0 = awq.qlinear(res["codes"], res["scales"], res["zeros"], res["s_best"], Xt, 4, 128)
+    Y1 = awq.qlinear(back["codes"], back["scales"], back["zeros"], back["s_best"], Xt,
+                     back["bits"], back["group_size"])
+    awq.get_status()
+    assert torch.equal(Y0, Y1)
+
+
 # ---------------------------------------------------------------------------
 # AWQ followed by GPTQ error compensation
 # ---------------------------------------------------------------------------
