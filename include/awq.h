@@ -30,8 +30,13 @@
  *     have stride ldx >= K elements, ldx a multiple of 8.
  *   - Sizes: 1 <= N, T <= 2^31 - 1; K a multiple of group_size.
  *   - Invalid arguments return AWQ_ERR_INVALID_ARG before anything is launched.
- *   - Calls are thread-safe and keep no state between calls, except the
- *     device error word read and cleared by awq_get_status().
+ *   - Calls are thread-safe.  What persists between calls: the device error
+ *     word (read and cleared by awq_get_status()); the wait limit, one value
+ *     for the process (awq_set_wait_timeout_ms); the event pair armed by
+ *     awq_profile_next_search, per host thread and used by that thread's next
+ *     search only; the per-device setup done once (shared-memory limits of the
+ *     kernels, the device properties, the scratch address of
+ *     awq_search_layer_noalloc).  No result of one call feeds another.
  */
 #ifndef AWQ_B200_AWQ_H
 #define AWQ_B200_AWQ_H
