@@ -45,7 +45,8 @@ def quantize_layer_rows(W_part: torch.Tensor, X: torch.Tensor, rows_total: int, 
     X: the full calibration input (fp16 [T, K], the same on every rank).
     Every rank of `process_group` must call this with the same rows_total,
     alphas and quantizer.  Returns the layer's losses (identical on every
-    rank), best_idx, s_best, and this part's codes, scales and zeros."""
+    rank) and a; a rank with rows also gets best_idx, s_best and its part's
+    codes, scales and zeros (a rank without rows has nothing to pack)."""
     import torch.distributed as dist
 
     dev = X.device
