@@ -114,11 +114,16 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _dev(t: torch.Tensor, dtype, name):
+def _dev(t: torch.Tensor, dtype, name, row_strided: bool = False):
+    """The device pointer of t.  The library reads every array densely packed,
+    except X, whose rows may sit ldx elements apart (row_strided: the caller
+    has checked the rows with _rowmajor and passes X.stride(0) as ldx)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not row_strided and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -141,7 +146,7 @@ def act_stats(X: torch.Tensor, stream=None) -> torch.Tensor:
     _rowmajor(X, "X")
     T, K = X.shape
     a = torch.empty(K, dtype=torch.float32, device=X.device)
-    _check(lib().awq_act_stats(_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(a, torch.float32, "a"),
+    _check(lib().awq_act_stats(_dev(X, torch.float16, "X", row_strided=True), T, K, X.stride(0), _dev(a, torch.float32, "a"),
                                _stream(stream)), "awq_act_stats")
     return a
 
@@ -200,7 +205,7 @@ def search_layer(W: torch.Tensor, X: torch.Tensor, a: torch.Tensor, alphas: torc
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     losses = losses_out if losses_out is not None else torch.empty(n, dtype=torch.float32, device=W.device)
     rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
-    rest = (_dev(X, torch.float16, "X"), T, X.stride(0), _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point),
+    rest = (_dev(X, torch.float16, "X", row_strided=True), T, X.stride(0), _dev(a, torch.float32, "a"), _qcfg(bits, group, zero_point),
             _dev(alphas, torch.float32, "alphas"), n, _dev(losses, torch.float32, "losses"),
             _dev(rl, torch.float32, "row_losses") if rl is not None else None,
             ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
@@ -273,7 +278,7 @@ def qlinear(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, s_be
     fn = getattr(lib(), name)
     _check(fn(_dev(codes, torch.int32, "codes"), _dev(scales, torch.float16, "scales"),
               _dev(zeros, torch.float16, "zeros"), _dev(s_best, torch.float32, "s_best"), N, K,
-              _qcfg(bits, group), _dev(X, torch.float16, "X"), T, X.stride(0),
+              _qcfg(bits, group), _dev(X, torch.float16, "X", row_strided=True), T, X.stride(0),
               _dev(Y, torch.float32, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
               _stream(stream)), name)
     return Y
@@ -325,7 +330,7 @@ def search_scales(W: torch.Tensor, X: torch.Tensor, s_table: torch.Tensor, bits:
     losses = torch.empty(n, dtype=torch.float32, device=W.device)
     rl = torch.empty((n, N), dtype=torch.float32, device=W.device) if row_losses else None
     _check(lib().awq_search_scales(
-        _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X"), T, X.stride(0), q,
+        _dev(W, torch.float16, "W"), N, K, _dev(X, torch.float16, "X", row_strided=True), T, X.stride(0), q,
         _dev(st, torch.float32, "s_table"), n, None if mask is None else _dev(mask, torch.uint8, "mask"),
         _dev(losses, torch.float32, "losses"), _dev(rl, torch.float32, "row_losses") if rl is not None else None,
         ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)), "awq_search_scales")
@@ -397,7 +402,7 @@ def output_error(W: torch.Tensor, W_hat: torch.Tensor, X: torch.Tensor, row_loss
     loss = torch.empty(1, dtype=torch.float32, device=W.device)
     rl = torch.empty((1, N), dtype=torch.float32, device=W.device) if row_losses else None
     _check(lib().awq_output_error(_dev(W.contiguous(), torch.float16, "W"), _dev(W_hat.contiguous(), torch.float16, "W_hat"),
-                                  N, K, _dev(X, torch.float16, "X"), T, X.stride(0), _dev(loss, torch.float32, "loss"),
+                                  N, K, _dev(X, torch.float16, "X", row_strided=True), T, X.stride(0), _dev(loss, torch.float32, "loss"),
                                   _dev(rl, torch.float32, "row_losses") if rl is not None else None,
                                   ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)), "awq_output_error")
     return (loss[0], rl[0]) if row_losses else loss[0]
@@ -411,7 +416,7 @@ def gptq_hessian(X: torch.Tensor, s: torch.Tensor | None = None, stream=None,
     T, K = X.shape
     s = torch.ones(K, dtype=torch.float32, device=X.device) if s is None else s
     H = torch.empty((K, K), dtype=torch.float32, device=X.device)
-    args = (_dev(X, torch.float16, "X"), T, K, X.stride(0), _dev(s, torch.float32, "s"), _dev(H, torch.float32, "H"))
+    args = (_dev(X, torch.float16, "X", row_strided=True), T, K, X.stride(0), _dev(s, torch.float32, "s"), _dev(H, torch.float32, "H"))
     if tensor_cores:
         need = int(lib().awq_gptq_hessian_workspace_bytes(T, K))
         ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)

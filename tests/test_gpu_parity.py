@@ -581,6 +581,27 @@ def test_qlinear_on_symmetric_pack(awq):
     np.testing.assert_allclose(Y, ref, rtol=1e-4, atol=1e-4 * np.abs(ref).max())
 
 
+def test_binding_rejects_non_contiguous_arrays(awq):
+    """Every array but X is read densely packed: a strided view is refused on
+    the host before anything is launched; X may have strided rows."""
+    W, X = gen(256, 256, 64, seed=141)
+    Xd = dev(X)
+    a = awq.act_stats(Xd)
+    al = dev(synth.default_alphas())
+    a_strided = torch.stack([a, a], dim=1)[:, 0]                   # stride 2
+    assert not a_strided.is_contiguous()
+    with pytest.raises(ValueError):
+        awq.alpha_scales(a_strided, al)
+    with pytest.raises(ValueError):
+        awq.alpha_scales(a, torch.stack([al, al], dim=1)[:, 0])
+    W_strided = dev(np.concatenate([W, W], axis=1))[:, :256]       # rows 512 apart
+    with pytest.raises(ValueError):
+        awq.search_layer(W_strided, Xd, a, al)
+    X_strided = dev(np.concatenate([X, X], axis=1))[:, :256]       # strided rows: accepted
+    assert torch.equal(awq.act_stats(X_strided), a)
+    awq.get_status()
+
+
 def test_saved_layer_reloads_for_decode(awq, tmp_path):
     """A layer quantized on the GPU, saved and loaded back ([QAS-QA] §9:
     save_quantized, then inference from the 4-bit model): the reloaded tensors
