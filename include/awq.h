@@ -378,7 +378,10 @@ AWQ_API awq_status awq_qlinear_cc(const uint32_t *codes, const void *scales, con
  *         q is exact in bf16 and x' is split into three bf16 pieces whose sum
  *         is x' exactly, so every product is exact),
  *   S_g = RN32(sum_{k in g} x'[t, k]) in binary64.
- * Passes of up to 5, 10 or 16 tokens each read the codes once.  The units (128
+ * Only the binary32 additions round, so the error of a group scales with
+ * sh (sum |q x'| + |z S_g|) where the CUDA-core form's scales with
+ * sum |x' (q - z)| sh; the two agree closely when a group's codes lie on both
+ * sides of z.  Passes of up to 5, 10 or 16 tokens each read the codes once.  The units (128
  * rows x 256 columns) are dealt to the SMs in contiguous ranges; a row block
  * split between two ranges is summed by the last to arrive, in range order, so
  * repeated calls on one device give identical Y.  Calls that share a workspace
