@@ -572,6 +572,40 @@ def test_gptq_with_uncorrelated_inputs_is_rtn(oracle_mod):
         assert np.array_equal(r["what"].view(np.uint16), ref["what"].view(np.uint16))
 
 
+def test_gptq_hessian_is_the_output_error_quadratic(oracle_mod):
+    """H is the curvature of the output error GPTQ compensates ([Notes-52] §4:
+    second-order statistics of the real input): with D = W_hat - W, the summed
+    squared output error sum_n ||D_n X^T||^2 equals (1/2) sum_n D_n H D_n^T.
+    The left side comes from output_error (a product with X^T, no Gram matrix),
+    so a transposed operand or a lost factor 2 in H fails here."""
+    rng = np.random.default_rng(103)
+    N, K, T = 5, 24, 37
+    W = (rng.standard_normal((N, K)) * 0.1).astype(np.float16)
+    step = (rng.integers(-3, 4, (N, K)) * 2.0 ** -8).astype(np.float32)
+    What = (W.astype(np.float32) + step).astype(np.float16)
+    X = (rng.standard_normal((T, K)) + rng.standard_normal((T, 1))).astype(np.float16)
+    lhs = oracle_mod.output_error(W, What, X)["loss"] * N * T
+    H = oracle_mod.gptq_hessian(X)
+    Dd = What.astype(np.float64) - W.astype(np.float64)            # exact: two fp16 values
+    assert np.count_nonzero(Dd) > N * K // 2
+    rhs = 0.5 * np.einsum("nk,kj,nj->", Dd, H, Dd)
+    assert lhs == pytest.approx(rhs, rel=1e-12)
+    assert H.shape == (K, K) and np.array_equal(H, H.T)
+
+
+def test_gptq_hessian_scales_with_the_input(oracle_mod):
+    """x' = x / s: with powers of two for s every x' is exact, so
+    H(s) = diag(1/s) H(1) diag(1/s) holds bit for bit."""
+    rng = np.random.default_rng(104)
+    K, T = 16, 50
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    s = (2.0 ** rng.integers(-3, 4, K)).astype(np.float32)
+    H1 = oracle_mod.gptq_hessian(X)
+    Hs = oracle_mod.gptq_hessian(X, s)
+    r = 1.0 / s.astype(np.float64)
+    assert np.array_equal(Hs, H1 * r[:, None] * r[None, :])
+
+
 def test_gptq_step_is_the_least_squares_correction(oracle_mod):
     """After the first column is rounded, the change the sweep makes to the
     remaining weights is the one that minimises the (damped) output error with
