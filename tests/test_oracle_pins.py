@@ -405,6 +405,34 @@ def test_qlinear_matches_dequantized_matmul(oracle_mod):
     assert np.linalg.norm(Y - Yh) / np.linalg.norm(Yh) < 2.0 ** -11
 
 
+def test_qlinear_against_exact_rationals(oracle_mod):
+    """Tiny case in exact arithmetic: r = RN32(1/s) and x' = RN32(x r) formed
+    from exact rationals with an explicit round-to-nearest-even, the sum
+    sum_k x' (q - z) sh kept exact.  s is not a power of two, so a division in
+    place of the reciprocal, or an x' left in binary64, moves Y off the exact
+    value by far more than the binary64 summation can."""
+    rng = np.random.default_rng(63)
+    N, K, T, bits, group = 3, 64, 2, 4, 32
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sh = (rng.uniform(0.001, 0.02, (N, K // group))).astype(np.float16)
+    z = rng.integers(-20, 36, (N, K // group)).astype(np.float16)
+    s = rng.uniform(0.3, 7.0, K).astype(np.float32)
+    X = (rng.standard_normal((T, K)) * 3).astype(np.float16)
+    codes = oracle_mod.pack_codes(q, bits)
+    Y = oracle_mod.qlinear(codes, sh, z, s, X, bits, group)
+    for t in range(T):
+        for n in range(N):
+            exact, absum = Fraction(0), Fraction(0)
+            for k in range(K):
+                r = _rn32_exact(Fraction(1) / Fraction(float(s[k])))
+                xp = _rn32_exact(Fraction(float(X[t, k])) * Fraction(float(r)))
+                term = Fraction(float(xp)) * (int(q[n, k]) - Fraction(float(z[n, k // group]))) \
+                    * Fraction(float(sh[n, k // group]))
+                exact += term
+                absum += abs(term)
+            assert abs(Fraction(float(Y[t, n])) - exact) <= Fraction(1, 10**12) * absum, (t, n)
+
+
 # ---------------------------------------------------------------------------
 # Quantizer variants and baselines: the symmetric absmax quantizer, channels
 # held in fp16, caller-given scale vectors, top-k channel selection
