@@ -224,6 +224,34 @@ def test_ties_round_to_even(oracle_mod):
     assert r["q"][0].tolist() == [0, 15, 0, 2, 2, 4, 10, 12]
 
 
+def test_scales_closed_forms(oracle_mod):
+    """s = RN32(a^alpha) ([AWQ-note] "Measures": a^alpha per candidate alpha)
+    at the exponents with closed forms: alpha = 1 gives a itself, alpha = 0
+    gives 1, and alpha = 1/2 gives the binary32 value nearest the exact square
+    root (chosen here by comparing squares of rationals, without pow); a dead
+    channel (a = 0) is lifted to FLT_MIN first."""
+    rng = np.random.default_rng(65)
+    a = np.concatenate([(10.0 ** rng.uniform(-6, 4, 400)).astype(np.float32),
+                        np.array([0.0, 1.0, 4.0, 2.0, 1e-30, 3.0e38], np.float32)])
+    fmin = np.float32(2.0 ** -126)
+    assert np.array_equal(oracle_mod.scales(a, 1.0), np.maximum(a, fmin))
+    assert np.all(oracle_mod.scales(a, 0.0) == 1.0)
+    half = oracle_mod.scales(a, 0.5)
+    for ai, si in zip(np.maximum(a, fmin), half):
+        A = Fraction(float(ai))
+        y = np.float32(math.sqrt(float(ai)))
+        cands = [np.nextafter(y, np.float32(0)), y, np.nextafter(y, np.float32(np.inf))]
+        best = y
+        for c in cands:                     # nearest: |sqrt(A) - c| smallest, via squares of midpoints
+            lo, hi = min(c, best), max(c, best)
+            if lo == hi:
+                continue
+            mid = (Fraction(float(lo)) + Fraction(float(hi))) / 2
+            nearer_lo = A < mid * mid
+            best = lo if nearer_lo else hi
+        assert si == best, (ai, si, best)
+
+
 def test_alpha_zero_is_plain_rtn(oracle_mod):
     """alpha = 0 gives s = 1 exactly, so the search's first candidate is plain
     group RTN; the brute force's RTN (binary32 hardware ops) must agree bit
