@@ -72,6 +72,8 @@ def _check_tensors(t: dict, bits: int, group: int):
     n = [t[k].numel() for k in ("losses", "alphas") if k in t]
     if len(n) == 2 and n[0] != n[1]:
         raise ValueError("losses and alphas have different lengths")
+    if n and not 0 <= int(t["best_idx"].reshape(-1)[0]) < n[0]:
+        raise ValueError(f"best_idx {int(t['best_idx'].reshape(-1)[0])} is outside the grid of {n[0]}")
 
 
 def save_quantized(path, result: dict, bits: int, group: int, zero_point: bool = True,

@@ -64,6 +64,8 @@ def test_save_rejects_inconsistent_results(tmp_path):
         persist.save_quantized(p, missing, 4, 128)
     with pytest.raises(ValueError):
         persist.save_quantized(p, r, 4, 128, alphas=torch.zeros(19))   # grid and losses differ in length
+    with pytest.raises(ValueError):
+        persist.save_quantized(p, dict(r, best_idx=torch.tensor([20], dtype=torch.int32)), 4, 128)
     assert not p.exists()
 
 
