@@ -169,3 +169,28 @@ def test_qlinear_dispatch_query():
     assert awq.qlinear_path(1) == "cuda_cores"
     for T in (2, 3, 5, 16, 17, 4096):
         assert awq.qlinear_path(T) == "tensor_cores"
+
+
+@pytest.mark.parametrize("fn", ["awq_qlinear", "awq_qlinear_cc", "awq_qlinear_tc"])
+def test_qlinear_entry_points_reject_bad_arguments(fn):
+    """Every decode entry point validates before touching the device."""
+    L = awq.lib()
+    f = getattr(L, fn)
+
+    def call(**kw):
+        a = dict(codes=BOGUS, scales=BOGUS, zeros=BOGUS, s_best=BOGUS, N=512, K=1024, q=QCfg(4, 128, 1),
+                 X=BOGUS, T=4, ldx=1024, Y=BOGUS, ws=BOGUS, ws_bytes=1 << 40, stream=None)
+        a.update(kw)
+        return f(*a.values())
+
+    bad_arg = [dict(codes=None), dict(scales=None), dict(zeros=None), dict(s_best=None), dict(X=None),
+               dict(Y=None), dict(codes=MISALIGNED), dict(X=MISALIGNED), dict(Y=MISALIGNED),
+               dict(N=0), dict(T=0), dict(K=1000), dict(K=32), dict(ldx=1000), dict(ldx=1028),
+               dict(q=QCfg(5, 128, 1)), dict(q=QCfg(4, 96, 1)), dict(K=1024 + 64, q=QCfg(4, 128, 1))]
+    for kw in bad_arg:
+        assert call(**kw) == 1, kw                          # AWQ_ERR_INVALID_ARG
+    need = awq.lib().awq_qlinear_workspace_bytes(4, 1024, 512)
+    assert need > 0
+    assert call(ws=None) == 5                               # AWQ_ERR_WORKSPACE
+    assert call(ws_bytes=need - 1) == 5
+    assert call(ws=ctypes.c_void_p(0x10010)) == 5           # not 256-byte aligned
