@@ -194,3 +194,32 @@ def test_qlinear_entry_points_reject_bad_arguments(fn):
     assert call(ws=None) == 5                               # AWQ_ERR_WORKSPACE
     assert call(ws_bytes=need - 1) == 5
     assert call(ws=ctypes.c_void_p(0x10010)) == 5           # not 256-byte aligned
+
+
+def test_row_part_and_noalloc_entry_points_reject_bad_arguments():
+    L = awq.lib()
+    L.awq_search_layer_part.restype = ctypes.c_int
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+
+    def part(**kw):
+        a = dict(W=BOGUS, N=256, rows_total=512, K=512, X=BOGUS, T=512, ldx=512, a=BOGUS, q=QCfg(4, 128, 1),
+                 alphas=BOGUS, n_alpha=20, losses=BOGUS, row_losses=None, ws=BOGUS, ws_bytes=1 << 40, stream=None)
+        a.update(kw)
+        return L.awq_search_layer_part(*a.values())
+
+    for kw in (dict(rows_total=255), dict(rows_total=(1 << 31)), dict(W=None), dict(losses=None),
+               dict(W=MISALIGNED), dict(row_losses=MISALIGNED), dict(K=500), dict(ldx=510),
+               dict(n_alpha=0), dict(n_alpha=65), dict(q=QCfg(4, 64, 2))):
+        assert part(**kw) == 1, kw
+    assert part(ws=None) == 5
+    assert part(ws_bytes=16) == 5
+
+    f = L.awq_search_layer_noalloc
+    f.argtypes = [P, i64, i64, P, i64, i64, P, QCfg, P, i32, P, P, P]
+    f.restype = ctypes.c_int
+    # no workspace size exists for these shapes: rejected before the device is touched
+    assert f(BOGUS, 256, 500, BOGUS, 512, 512, BOGUS, QCfg(4, 128, 1), BOGUS, 20, BOGUS, None, None) == 1
+    assert f(BOGUS, 256, 512, BOGUS, 512, 512, BOGUS, QCfg(4, 128, 1), BOGUS, 0, BOGUS, None, None) == 1
+    # a layer whose workspace exceeds the built-in scratch
+    assert awq.search_workspace_bytes(8192, 8192, 8192, 4, 128, 20) > 32 << 20
+    assert f(BOGUS, 8192, 8192, BOGUS, 8192, 8192, BOGUS, QCfg(4, 128, 1), BOGUS, 20, BOGUS, None, None) == 5
